@@ -1,0 +1,164 @@
+"""CPU oracle for the DCNv3 / DCNv4 core operator (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never does, and it
+shares no code with ``dcn_oracle.c``.
+
+Every function here is argument marshalling around the plain, single-threaded
+C loops of ``dcn_oracle.c`` (double accumulation); see that file for what is
+computed and for the page passages each step follows.  Inputs are converted
+to float64 exactly (fp32 and bf16 values are exactly representable).
+
+Parity status: every function is pinned by the closed forms, invariants and
+brute-force checks in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dcn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libdcnoracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc.  -ffp-contract=off keeps every fp32
+    multiply and add of the sampling location separately rounded."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + ".tmp.%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math",
+                               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        ci, cd, i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
+        shape = [ci] * 9 + [cd, ci, ci]
+        lib.oracle_output_extent.argtypes = [ci] * 5
+        lib.oracle_output_extent.restype = ci
+        lib.oracle_forward.argtypes = [dp] * 4 + shape
+        lib.oracle_forward.restype = ci
+        lib.oracle_forward_units.argtypes = [dp] * 3 + [i64p, i64, dp] + shape
+        lib.oracle_forward_units.restype = ci
+        lib.oracle_backward.argtypes = [dp] * 7 + shape
+        lib.oracle_backward.restype = ci
+        lib.oracle_backward_units.argtypes = [dp] * 4 + [i64p, i64, dp, dp] + shape
+        lib.oracle_backward_units.restype = ci
+        _lib = lib
+    return _lib
+
+
+def _d(a) -> np.ndarray:
+    """Exact float64 copy of a host array (numpy or CPU torch tensor)."""
+    if hasattr(a, "detach"):  # torch tensor: bf16 has no numpy dtype, widen via fp32
+        import torch
+        a = a.detach().to("cpu", torch.float32).numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def output_extent(n_in: int, K: int, stride: int, pad: int, dil: int) -> int:
+    return int(_load().oracle_output_extent(n_in, K, stride, pad, dil))
+
+
+def output_hw(H, W, K, stride, pad, dil):
+    return output_extent(H, K, stride, pad, dil), output_extent(W, K, stride, pad, dil)
+
+
+def _shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd):
+    return (int(N), int(H), int(W), int(G), int(Cg), int(K), int(stride), int(pad),
+            int(dil), float(offset_scale), int(softmax), int(bool(fd)))
+
+
+def forward(x, offset, mask, *, G, K=3, stride=1, pad=1, dil=1, offset_scale=1.0,
+            softmax=1, fd=False) -> np.ndarray:
+    """Forward of the whole problem.  x: (N,H,W,G*Cg), offset: (N,Ho,Wo,G*K*K*2),
+    mask: (N,Ho,Wo,G*K*K).  Returns float64 (N,Ho,Wo,G*Cg)."""
+    x, offset, mask = _d(x), _d(offset), _d(mask)
+    N, H, W, C = x.shape
+    Cg = C // G
+    Ho, Wo = output_hw(H, W, K, stride, pad, dil)
+    out = np.zeros((N, Ho, Wo, C), dtype=np.float64)
+    if out.size == 0:
+        return out
+    assert offset.shape == (N, Ho, Wo, G * K * K * 2), offset.shape
+    assert mask.shape == (N, Ho, Wo, G * K * K), mask.shape
+    rc = _load().oracle_forward(_p(x), _p(offset), _p(mask), _p(out),
+                                *_shape_args(N, H, W, G, Cg, K, stride, pad, dil,
+                                             offset_scale, softmax, fd))
+    assert rc == 0, rc
+    return out
+
+
+def forward_units(x, offset, mask, units, *, G, K=3, stride=1, pad=1, dil=1,
+                  offset_scale=1.0, softmax=1, fd=False) -> np.ndarray:
+    """Forward outputs of selected units u = ((n*Ho+ho)*Wo+wo)*G+g only.
+    Returns float64 (len(units), Cg)."""
+    x, offset, mask = _d(x), _d(offset), _d(mask)
+    N, H, W, C = x.shape
+    Cg = C // G
+    units = np.ascontiguousarray(np.asarray(units, dtype=np.int64))
+    out = np.zeros((units.size, Cg), dtype=np.float64)
+    rc = _load().oracle_forward_units(
+        _p(x), _p(offset), _p(mask), units.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        units.size, _p(out),
+        *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd))
+    assert rc == 0, rc
+    return out
+
+
+def backward(x, offset, mask, grad_out, *, G, K=3, stride=1, pad=1, dil=1,
+             offset_scale=1.0, softmax=1, fd=False):
+    """Returns float64 (grad_input, grad_offset, grad_mask); grad_mask is the
+    gradient with respect to the logits when softmax=1."""
+    x, offset, mask, grad_out = _d(x), _d(offset), _d(mask), _d(grad_out)
+    N, H, W, C = x.shape
+    Cg = C // G
+    gx = np.zeros_like(x)
+    goff = np.zeros_like(offset)
+    gm = np.zeros_like(mask)
+    rc = _load().oracle_backward(_p(x), _p(offset), _p(mask), _p(grad_out), _p(gx), _p(goff),
+                                 _p(gm), *_shape_args(N, H, W, G, Cg, K, stride, pad, dil,
+                                                      offset_scale, softmax, fd))
+    assert rc == 0, rc
+    return gx, goff, gm
+
+
+def backward_units(x, offset, mask, grad_out, units, *, G, K=3, stride=1, pad=1, dil=1,
+                   offset_scale=1.0, softmax=1, fd=False):
+    """Offset and mask gradients of selected units.  Returns float64
+    (goff (len, K*K*2), gmask (len, K*K))."""
+    x, offset, mask, grad_out = _d(x), _d(offset), _d(mask), _d(grad_out)
+    N, H, W, C = x.shape
+    Cg = C // G
+    KK = K * K
+    units = np.ascontiguousarray(np.asarray(units, dtype=np.int64))
+    goff = np.zeros((units.size, KK * 2), dtype=np.float64)
+    gm = np.zeros((units.size, KK), dtype=np.float64)
+    rc = _load().oracle_backward_units(
+        _p(x), _p(offset), _p(mask), _p(grad_out),
+        units.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), units.size, _p(goff), _p(gm),
+        *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd))
+    assert rc == 0, rc
+    return goff, gm
+
+
+def workload_kwargs(wl) -> dict:
+    """Keyword arguments of forward()/backward() for a gen.Workload."""
+    return dict(G=wl.G, K=wl.K, stride=wl.stride, pad=wl.pad, dil=wl.dilation,
+                offset_scale=wl.offset_scale, softmax=wl.softmax)
