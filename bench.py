@@ -1,0 +1,473 @@
+"""Benchmark of the DCNv3 core on B200: GB/s and Gsamples/s, fraction of HBM peak.
+
+A step is one pass of the whole hot path -- forward (offset/mask staging,
+softmax, bilinear gather, weighted sum, store) and backward (recompute,
+grad_mask, grad_offset, grad_input scatter) -- over one batch of the
+InternImage-L stage-1 shape (fp32, N=32, 96x96, C=160 = 10 groups x 16,
+3x3, offset_scale 2.0, softmax mask), inputs drawn from the seeded generator.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--no-sweep] [--no-cpu-baseline]
+
+Prints ONE JSON line (rank 0).  Multi-GPU runs (torchrun) are independent
+replicas, one per GPU, with no data-path collective (weak scaling); the step
+time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "DCNv3 core fwd/bwd GB/s and Gsamples/s on 1 B200; fraction of HBM peak"
+DEFAULT_WORKLOAD = "internimage_l_stage1_fp32_n32_96x96_c160"
+SWEEP = ["internimage_l_stage1_bf16_n64_96x96_c160", "internimage_l_stage2_bf16_n64_48x48_c320",
+         "internimage_l_stage3_bf16_n64_24x24_c640", "internimage_l_stage4_bf16_n64_12x12_c1280",
+         "dcnv4_hires_bf16_n2_256x256_c192_s1", "dcnv4_hires_bf16_n2_256x256_c192_s2",
+         "internimage_l_stage2_bwd_fp32_n32_48x48_c320"]
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel sources are unchanged since it was taken (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    csrc = os.path.join(ROOT, "deformable_convolution_core_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    for line in open(path):
+        parts = dict(p.split("=", 1) for p in line.split() if "=" in p)
+        if parts.get("kernel") == kernel and parts.get("src_sha") == sha:
+            return float(parts["bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.mark = 0
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def begin_region(self):
+        self.mark = len(self.lines)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r.split(", ") for r in self.lines[self.mark:]] or \
+               [r.split(", ") for r in self.lines]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------------------
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif args.impl == "ours":
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+class Step:
+    """Device buffers and the launches of one step of a workload."""
+
+    def __init__(self, wl, inputs, backward: bool):
+        import torch
+        import deformable_convolution_core_b200 as dcn
+        self.dcn = dcn
+        self.wl = wl
+        self.backward = backward
+        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        self.p = dcn.problem_for(wl)
+        dev = torch.device("cuda")
+        self.x = torch.from_numpy(inputs["x"]).to(dev).to(tdt)
+        self.off = torch.from_numpy(inputs["offset"]).to(dev).to(tdt)
+        self.mask = torch.from_numpy(inputs["mask"]).to(dev).to(tdt)
+        Ho, Wo = dcn.dcn_core_output_hw(self.p)
+        self.out = torch.empty((wl.N, Ho, Wo, wl.C), dtype=tdt, device=dev)
+        if backward:
+            self.gout = torch.from_numpy(inputs["grad_out"]).to(dev).to(tdt)
+            self.gx = torch.empty_like(self.x)
+            self.goff = torch.empty_like(self.off)
+            self.gm = torch.empty_like(self.mask)
+        self.stream = torch.cuda.Stream()
+        self.sh = self.stream.cuda_stream
+
+    def fwd(self):
+        self.dcn.dcn_core_forward(self.p, self.x, self.off, self.mask, self.out, self.sh)
+
+    def bwd(self):
+        self.dcn.dcn_core_backward(self.p, self.x, self.off, self.mask, self.gout, self.gx,
+                                   self.goff, self.gm, None, 0, self.sh)
+
+    def run(self):
+        if not (self.wl.backward and self.backward):
+            self.fwd()
+        if self.backward:
+            self.bwd()
+
+    def launches_per_step(self):
+        return (0 if (self.wl.backward and self.backward) else 1) + (1 if self.backward else 0)
+
+
+def timed(step, steps, warmup, barrier=None, ev_kernels=True):
+    """Time `steps` steps on the step's stream; also time each launch with
+    events on that stream.  Returns (total_ms, fwd_ms_avg, bwd_ms_avg)."""
+    import torch
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    s = step.stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fwd_only = not (step.wl.backward and step.backward)
+    t0.record(s)
+    for i in range(steps):
+        ev[i][0].record(s)
+        if fwd_only:
+            step.fwd()
+        ev[i][1].record(s)
+        if step.backward:
+            step.bwd()
+        ev[i][2].record(s)
+    t1.record(s)
+    torch.cuda.synchronize()
+    total = t0.elapsed_time(t1)
+    fw = sum(e[0].elapsed_time(e[1]) for e in ev) / steps if fwd_only else 0.0
+    bw = sum(e[1].elapsed_time(e[2]) for e in ev) / steps if step.backward else 0.0
+    return total, fw, bw
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    import gen
+    from deformable_convolution_core_b200 import build as lib_build
+
+    lib_build.build()
+    wl = gen.WORKLOADS[args.workload]
+    backward = wl.backward or wl.dtype == "f32"
+    inputs = gen.make_inputs(wl, with_grad_out=backward)
+    step = Step(wl, inputs, backward)
+
+    barrier = None
+    if world > 1:
+        import torch.distributed as dist
+        barrier = dist.barrier
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    clocks.begin_region()
+    total_ms, fwd_ms, bwd_ms = timed(step, args.steps, args.warmup, barrier)
+    time.sleep(0.25)
+    clock_summary = clocks.summary()
+    clocks.stop()
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms, fwd_ms, bwd_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, fwd_ms, bwd_ms = (float(v) for v in t.tolist())
+    ms_per_step = total_ms / args.steps
+
+    fwd_bytes = wl.forward_bytes() if not wl.backward else 0
+    bwd_bytes = wl.backward_bytes() if backward else 0
+    step_bytes = fwd_bytes + bwd_bytes
+    samples = wl.samples * ((0 if wl.backward else 1) + (1 if backward else 0))
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    # dominant launch: the longer of forward and backward
+    kernels = []
+    if fwd_ms > 0:
+        kernels.append(("dcn_forward_kernel", fwd_bytes, fwd_ms))
+    if bwd_ms > 0:
+        kernels.append(("dcn_backward_kernel", bwd_bytes, bwd_ms))
+    kname, kbytes, kms = max(kernels, key=lambda k: k[2])
+    achieved = kbytes / (kms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(kname),
+                "kernel": kname, "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": kbytes, "avg_launch_ms": round(kms, 4)}
+
+    # end to end through the public API: pinned host inputs -> device, step, results -> host
+    e2e = None
+    if rank == 0 or world > 1:
+        e2e = run_e2e(step, inputs, args, barrier, world)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": wl.dtype, "data": "synthetic (seeded counter-based generator)",
+        "config": {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
+                   "N": wl.N, "H": wl.H, "W": wl.W, "G": wl.G, "Cg": wl.Cg, "K": wl.K,
+                   "stride": wl.stride, "offset_scale": wl.offset_scale,
+                   "softmax": wl.softmax, "per_gpu_batch": wl.N,
+                   "parallelism": f"replicas x{world} (no collective)",
+                   "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB touched per step, "
+                         "no flush between steps"},
+        "gsamples_per_s": round(world * samples / (ms_per_step * 1e-3) / 1e9, 3),
+        "breakdown": {"forward": None if fwd_ms == 0 else {
+                          "ms": round(fwd_ms, 4),
+                          "GB/s": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9, 1),
+                          "Gsamples/s": round(wl.samples / (fwd_ms * 1e-3) / 1e9, 2),
+                          "frac_of_hbm": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9 / peak, 4)},
+                      "backward": None if bwd_ms == 0 else {
+                          "ms": round(bwd_ms, 4),
+                          "GB/s": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
+                          "Gsamples/s": round(wl.samples / (bwd_ms * 1e-3) / 1e9, 2),
+                          "frac_of_hbm": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peak, 4),
+                          "note": "includes the zero-fill of grad_input"}},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "clocks": clock_summary,
+    }
+    if rank == 0 and world == 1 and not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
+        result["sweep"] = run_sweep(gen, peak)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, inputs, backward)
+    del step
+    return result
+
+
+def run_e2e(step, inputs, args, barrier, world):
+    import torch
+    dcn = step.dcn
+    wl = step.wl
+    tdt = step.x.dtype
+    pin = lambda a: torch.from_numpy(a).to(tdt).pin_memory()
+    hx, ho, hm = pin(inputs["x"]), pin(inputs["offset"]), pin(inputs["mask"])
+    hout = torch.empty(step.out.shape, dtype=tdt).pin_memory()
+    h2d = (hx.numel() + ho.numel() + hm.numel()) * hx.element_size()
+    d2h = hout.numel() * hout.element_size()
+    if step.backward:
+        hg = pin(inputs["grad_out"])
+        hgx = torch.empty(step.gx.shape, dtype=tdt).pin_memory()
+        hgo = torch.empty(step.goff.shape, dtype=tdt).pin_memory()
+        hgm = torch.empty(step.gm.shape, dtype=tdt).pin_memory()
+        h2d += hg.numel() * hg.element_size()
+        d2h += (hgx.numel() + hgo.numel() + hgm.numel()) * hgx.element_size()
+    s = step.stream
+    fwd_only = not wl.backward
+
+    def one():
+        if fwd_only:
+            dcn.dcn_core_forward_host(step.p, hx, ho, hm, hout, step.x, step.off, step.mask,
+                                      step.out, step.sh)
+        else:
+            with torch.cuda.stream(s):
+                step.x.copy_(hx, non_blocking=True)
+                step.off.copy_(ho, non_blocking=True)
+                step.mask.copy_(hm, non_blocking=True)
+        if step.backward:
+            with torch.cuda.stream(s):
+                step.gout.copy_(hg, non_blocking=True)
+            step.bwd()
+            with torch.cuda.stream(s):
+                hgx.copy_(step.gx, non_blocking=True)
+                hgo.copy_(step.goff, non_blocking=True)
+                hgm.copy_(step.gm, non_blocking=True)
+
+    n = max(3, min(args.steps, 20))
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s)
+    for _ in range(n):
+        one()
+    t1.record(s)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    step_bytes = (wl.forward_bytes() if fwd_only else 0) + (wl.backward_bytes() if step.backward else 0)
+    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 3), "steps": n}
+
+
+def run_sweep(gen, peak):
+    """Forward GB/s of the other workloads (a few timed launches each)."""
+    import torch
+    out = {}
+    for name in SWEEP:
+        wl = gen.WORKLOADS[name]
+        inputs = gen.make_inputs(wl, with_grad_out=wl.backward)
+        step = Step(wl, inputs, backward=wl.backward)
+        total, fw, bw = timed(step, 20, 3)
+        ms = bw if wl.backward else fw
+        b = wl.backward_bytes() if wl.backward else wl.forward_bytes()
+        gbs = b / (ms * 1e-3) / 1e9
+        out[name] = {"pass": "backward" if wl.backward else "forward", "ms": round(ms, 4),
+                     "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
+                     "Gsamples/s": round(wl.samples / (ms * 1e-3) / 1e9, 2),
+                     "MB": round(b / 1e6, 1),
+                     "l2": "fits in L2" if b < L2_BYTES else "larger than L2"}
+        del step
+        torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(wl, inputs, backward, n_images=None):
+    """The CPU oracle, as it stands (single-threaded C, fp64), timed on the host."""
+    import oracle
+    oracle.build()
+    kw = oracle.workload_kwargs(wl)
+    n = wl.N if n_images is None else n_images
+    sl = {k: v[:n] for k, v in inputs.items()}
+    t0 = time.perf_counter()
+    if not wl.backward:
+        oracle.forward(sl["x"], sl["offset"], sl["mask"], **kw)
+    if backward:
+        oracle.backward(sl["x"], sl["offset"], sl["mask"], sl["grad_out"], **kw)
+    dt = time.perf_counter() - t0
+    frac = n / wl.N
+    b = ((0 if wl.backward else wl.forward_bytes()) + (wl.backward_bytes() if backward else 0)) * frac
+    return {"value": round(b / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"{n} of {wl.N} images of {wl.name}, "
+                      f"{'forward + backward' if backward and not wl.backward else 'one pass'}, "
+                      "including the float64 widening of the inputs"}
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: rank 0 only, on host cores, each step a
+    bounded sample (one image) of the workload."""
+    if rank != 0:
+        return None
+    import gen
+    wl = gen.WORKLOADS[args.workload]
+    backward = wl.backward or wl.dtype == "f32"
+    inputs = gen.make_inputs(wl, n_images=1, with_grad_out=backward)
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(wl, inputs, backward, n_images=1)
+    budget_s = 120.0
+    t_all = time.perf_counter()
+    vals, secs = [], []
+    steps = 0
+    for _ in range(args.steps):
+        r = cpu_baseline(wl, inputs, backward, n_images=1)
+        vals.append(r["value"])
+        secs.append(r["seconds"])
+        steps += 1
+        if time.perf_counter() - t_all > budget_s:
+            break
+    value = statistics.median(vals)
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * statistics.median(secs), 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded counter-based generator)",
+            "config": {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
+                       "sample": f"1 of {wl.N} images per step"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"1 of {wl.N} images of {wl.name} per step"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_ours(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

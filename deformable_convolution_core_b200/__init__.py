@@ -1,0 +1,184 @@
+"""Python binding of the B200 deformable-convolution core (DCNv3 / DCNv4).
+
+Argument marshalling only: every step of the operator runs in the CUDA
+kernels of ``libdcncore.so`` behind the C ABI declared in
+``include/dcn_core.h``.  The functions below carry the same names as the C
+entry points.  Tensors may be given as torch tensors (their device pointer is
+passed) or as raw integer addresses; streams as ``torch.cuda.Stream``, a raw
+handle or None (the current torch stream).
+
+There is no fallback: if the library is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdcncore.so")
+
+DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
+DCN_F32, DCN_BF16 = 0, 1
+
+# Every entry point of include/dcn_core.h.
+EXPORTED_SYMBOLS = (
+    "dcn_core_output_hw",
+    "dcn_core_forward",
+    "dcn_core_forward_host",
+    "dcn_core_backward_workspace",
+    "dcn_core_backward",
+    "dcn_core_sync_status",
+    "dcn_status_string",
+    "dcn_core_abi_version",
+)
+
+
+class DcnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {dcn_status_string(status)} (status {status})")
+
+
+class DcnProblem(ctypes.Structure):
+    """Mirror of ``dcn_problem`` in include/dcn_core.h."""
+    _fields_ = [("N", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("G", ctypes.c_int), ("Cg", ctypes.c_int), ("K", ctypes.c_int),
+                ("stride", ctypes.c_int), ("pad", ctypes.c_int), ("dilation", ctypes.c_int),
+                ("offset_scale", ctypes.c_float), ("softmax", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+    def __repr__(self):
+        return "DcnProblem(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_problem(N, H, W, G, Cg, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0,
+                 softmax=1, dtype="f32") -> DcnProblem:
+    if isinstance(dtype, str):
+        dtype = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16, "bfloat16": DCN_BF16}[dtype]
+    return DcnProblem(int(N), int(H), int(W), int(G), int(Cg), int(K), int(stride), int(pad),
+                      int(dilation), float(offset_scale), int(softmax), int(dtype))
+
+
+def problem_for(wl) -> DcnProblem:
+    """DcnProblem of a workload description (any object with the fields of
+    gen.workloads.Workload)."""
+    return make_problem(wl.N, wl.H, wl.W, wl.G, wl.Cg, wl.K, wl.stride, wl.pad, wl.dilation,
+                        wl.offset_scale, wl.softmax, wl.dtype)
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load libdcncore.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m deformable_convolution_core_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, pp = ctypes.c_void_p, ctypes.POINTER(DcnProblem)
+    ip = ctypes.POINTER(ctypes.c_int)
+    st = ctypes.c_int
+    lib.dcn_core_output_hw.argtypes = [pp, ip, ip]
+    lib.dcn_core_output_hw.restype = st
+    lib.dcn_core_forward.argtypes = [pp, vp, vp, vp, vp, vp]
+    lib.dcn_core_forward.restype = st
+    lib.dcn_core_forward_host.argtypes = [pp] + [vp] * 9
+    lib.dcn_core_forward_host.restype = st
+    lib.dcn_core_backward_workspace.argtypes = [pp]
+    lib.dcn_core_backward_workspace.restype = ctypes.c_size_t
+    lib.dcn_core_backward.argtypes = [pp] + [vp] * 8 + [ctypes.c_size_t, vp]
+    lib.dcn_core_backward.restype = st
+    lib.dcn_core_sync_status.argtypes = [vp]
+    lib.dcn_core_sync_status.restype = st
+    lib.dcn_status_string.argtypes = [st]
+    lib.dcn_status_string.restype = ctypes.c_char_p
+    lib.dcn_core_abi_version.argtypes = []
+    lib.dcn_core_abi_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        if not t.is_contiguous():
+            raise ValueError("tensors passed to the C ABI must be contiguous")
+        return t.data_ptr()
+    raise TypeError(f"cannot pass {type(t)} as a pointer")
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != DCN_OK:
+        raise DcnError(status, where)
+
+
+def dcn_status_string(status: int) -> str:
+    return load_library().dcn_status_string(int(status)).decode()
+
+
+def dcn_core_abi_version() -> int:
+    return int(load_library().dcn_core_abi_version())
+
+
+def dcn_core_output_hw(problem: DcnProblem) -> tuple[int, int]:
+    ho, wo = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load_library().dcn_core_output_hw(ctypes.byref(problem), ctypes.byref(ho),
+                                             ctypes.byref(wo)), "dcn_core_output_hw")
+    return ho.value, wo.value
+
+
+def dcn_core_forward(problem: DcnProblem, input, offset, mask, output, stream=None) -> None:
+    _check(load_library().dcn_core_forward(ctypes.byref(problem), _ptr(input), _ptr(offset),
+                                           _ptr(mask), _ptr(output), _stream(stream)),
+           "dcn_core_forward")
+
+
+def dcn_core_forward_host(problem: DcnProblem, h_input, h_offset, h_mask, h_output, d_input,
+                          d_offset, d_mask, d_output, stream=None) -> None:
+    _check(load_library().dcn_core_forward_host(
+        ctypes.byref(problem), _ptr(h_input), _ptr(h_offset), _ptr(h_mask), _ptr(h_output),
+        _ptr(d_input), _ptr(d_offset), _ptr(d_mask), _ptr(d_output), _stream(stream)),
+        "dcn_core_forward_host")
+
+
+def dcn_core_backward_workspace(problem: DcnProblem) -> int:
+    return int(load_library().dcn_core_backward_workspace(ctypes.byref(problem)))
+
+
+def dcn_core_backward(problem: DcnProblem, input, offset, mask, grad_out, grad_input,
+                      grad_offset, grad_mask, workspace=None, workspace_bytes=0,
+                      stream=None) -> None:
+    _check(load_library().dcn_core_backward(
+        ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
+        _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _ptr(workspace),
+        int(workspace_bytes), _stream(stream)), "dcn_core_backward")
+
+
+def dcn_core_sync_status(stream=None) -> None:
+    _check(load_library().dcn_core_sync_status(_stream(stream)), "dcn_core_sync_status")
+
+
+__all__ = ["DcnProblem", "DcnError", "make_problem", "problem_for", "load_library",
+           "library_path", "EXPORTED_SYMBOLS", *EXPORTED_SYMBOLS,
+           "DCN_OK", "DCN_ERR_INVALID_ARG", "DCN_ERR_UNSUPPORTED", "DCN_ERR_CUDA",
+           "DCN_ERR_TIMEOUT", "DCN_F32", "DCN_BF16"]

@@ -1,0 +1,369 @@
+// C ABI of the B200 deformable-convolution core: argument validation, tile
+// choice, kernel dispatch.  Declarations and the full contract are in
+// include/dcn_core.h.
+#include "dcn_core.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <cstdio>
+#include <cstdlib>
+
+#include "dcn_backward.cuh"
+#include "dcn_forward.cuh"
+
+namespace dcn {
+
+// Device error word: set by a kernel whose bounded wait gave up; read and
+// cleared by dcn_core_sync_status.
+__device__ unsigned int g_dcn_error_word = 0;
+
+namespace {
+
+// Shared memory a CTA may use for its staged offsets and mask, by default.
+constexpr int kDefaultSmemBudget = 40 * 1024;
+
+int64_t out_extent(int in, int K, int stride, int pad, int dil) {
+  const int64_t span = int64_t(in) + 2 * int64_t(pad) - int64_t(dil) * (K - 1) - 1;
+  if (span < 0 || stride < 1) return 0;
+  return span / stride + 1;
+}
+
+int esize(dcn_dtype d) { return d == DCN_BF16 ? 2 : 4; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Basic validity of the problem description.
+dcn_status check_problem(const dcn_problem* p, int64_t* Ho, int64_t* Wo) {
+  if (!p) return DCN_ERR_INVALID_ARG;
+  if (p->N < 1 || p->H < 1 || p->W < 1 || p->G < 1 || p->Cg < 1) return DCN_ERR_INVALID_ARG;
+  if (p->K < 1 || (p->K % 2) == 0) return DCN_ERR_INVALID_ARG;
+  if (p->stride < 1 || p->pad < 0 || p->dilation < 1) return DCN_ERR_INVALID_ARG;
+  if (p->softmax != 0 && p->softmax != 1) return DCN_ERR_INVALID_ARG;
+  if (p->dtype != DCN_F32 && p->dtype != DCN_BF16) return DCN_ERR_INVALID_ARG;
+  if (!(p->offset_scale == p->offset_scale)) return DCN_ERR_INVALID_ARG;  // NaN
+  const int64_t ho = out_extent(p->H, p->K, p->stride, p->pad, p->dilation);
+  const int64_t wo = out_extent(p->W, p->K, p->stride, p->pad, p->dilation);
+  if (ho < 1 || wo < 1) return DCN_ERR_INVALID_ARG;
+  const int64_t C = int64_t(p->G) * p->Cg;
+  const int64_t KK = int64_t(p->K) * p->K;
+  const int64_t n_in = int64_t(p->N) * p->H * p->W * C;
+  const int64_t n_out = int64_t(p->N) * ho * wo * C;
+  const int64_t n_off = int64_t(p->N) * ho * wo * p->G * KK * 2;
+  const int64_t lim = int64_t(INT_MAX);
+  if (C > lim || n_in > lim || n_out > lim || n_off > lim) return DCN_ERR_INVALID_ARG;
+  // Sampling coordinates are integers up to about H*stride + K*dilation in fp32.
+  if (int64_t(p->H) * p->stride + int64_t(p->K) * p->dilation > (int64_t(1) << 22) ||
+      int64_t(p->W) * p->stride + int64_t(p->K) * p->dilation > (int64_t(1) << 22))
+    return DCN_ERR_UNSUPPORTED;
+  *Ho = ho;
+  *Wo = wo;
+  return DCN_OK;
+}
+
+// Lane mapping for a channel width: bytes of one unit's channels UB =
+// Cg*sizeof(T) in {16, 32, 64, 128}; a lane gathers 16 (UB = 16) or 32 bytes.
+struct LaneMap {
+  int cpl, lanes;
+};
+
+bool lane_map(const dcn_problem* p, LaneMap* lm) {
+  const int ub = p->Cg * esize(p->dtype);
+  const int e = esize(p->dtype);
+  switch (ub) {
+    case 16: *lm = {16 / e, 1}; return true;
+    case 32: *lm = {32 / e, 1}; return true;
+    case 64: *lm = {32 / e, 2}; return true;
+    case 128: *lm = {32 / e, 4}; return true;
+    default: return false;
+  }
+}
+
+struct Plan {
+  TileParams t;
+  size_t smem;
+  unsigned grid;
+  LaneMap lm;
+};
+
+// Pick the tile (TH x TW output pixels, all groups).  The cost model counts
+// warp passes including those wasted on the ragged border, weighted by how
+// much of the gathered neighbourhood of a tile is halo (which costs L1 misses).
+void choose_tile(int Ho, int Wo, int G, int lanes, size_t entry_bytes, int KK, size_t budget,
+                 int* TH_out, int* TW_out) {
+  const int upw = 32 / lanes;
+  const size_t per_px = size_t(G) * KK * entry_bytes;
+  int max_px = int(std::max<size_t>(1, budget / per_px));
+  max_px = std::min(max_px, 1024);
+  const double halo = 3.0;
+  double best = 1e300;
+  int bth = 1, btw = 1;
+  for (int th = 1; th <= std::min(Ho, max_px); ++th) {
+    for (int tw = 1; tw <= std::min(Wo, max_px / th); ++tw) {
+      const int px = th * tw;
+      const int64_t tiles = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw);
+      const int64_t passes = tiles * ((int64_t(G) * px + upw - 1) / upw);
+      const double reach = (th + 2 * halo) * (tw + 2 * halo) / double(px);
+      const double cost = double(passes) * (1.0 + 0.25 * reach) + 4.0 * double(tiles);
+      if (cost < best) {
+        best = cost;
+        bth = th;
+        btw = tw;
+      }
+    }
+  }
+  *TH_out = bth;
+  *TW_out = btw;
+}
+
+dcn_status make_plan(const dcn_problem* p, int64_t Ho, int64_t Wo, size_t entry_bytes,
+                     Plan* plan) {
+  if (!lane_map(p, &plan->lm)) return DCN_ERR_UNSUPPORTED;
+  TileParams& t = plan->t;
+  t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
+  t.K = p->K; t.KK = p->K * p->K; t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation;
+  t.Ho = int(Ho); t.Wo = int(Wo); t.sigma = p->offset_scale;
+  size_t budget = kDefaultSmemBudget;
+  if (const char* s = std::getenv("DCN_CORE_SMEM_BUDGET")) budget = size_t(std::atol(s));
+  int TH = 0, TW = 0;
+  if (const char* s = std::getenv("DCN_CORE_TILE")) {  // "THxTW", for tuning sweeps
+    if (std::sscanf(s, "%dx%d", &TH, &TW) != 2 || TH < 1 || TW < 1) TH = TW = 0;
+    TH = std::min(TH, t.Ho);
+    TW = std::min(TW, t.Wo);
+  }
+  if (TH == 0) choose_tile(t.Ho, t.Wo, t.G, plan->lm.lanes, entry_bytes, t.KK, budget, &TH, &TW);
+  t.TH = TH; t.TW = TW;
+  t.nTY = (t.Ho + TH - 1) / TH;
+  t.nTX = (t.Wo + TW - 1) / TW;
+  t.tile_px = TH * TW;
+  t.P1 = t.tile_px | 1;
+  t.fd_tile_px = make_fastdiv(uint32_t(t.tile_px));
+  t.fd_TW = make_fastdiv(uint32_t(TW));
+  t.fd_GKK = make_fastdiv(uint32_t(t.G * t.KK));
+  t.fd_tiles_per_img = make_fastdiv(uint32_t(t.nTY * t.nTX));
+  t.fd_nTX = make_fastdiv(uint32_t(t.nTX));
+  plan->smem = size_t(t.G) * t.KK * t.P1 * entry_bytes;
+  const int64_t tiles = int64_t(t.N) * t.nTY * t.nTX;
+  if (tiles > INT_MAX) return DCN_ERR_UNSUPPORTED;
+  plan->grid = unsigned(tiles);
+  return DCN_OK;
+}
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+
+// Dynamic shared memory above 48 KB needs an opt-in per kernel and device.
+template <typename Kernel>
+dcn_status prepare_smem(Kernel k, size_t smem) {
+  if (smem <= 48 * 1024) return DCN_OK;
+  int dev = current_device();
+  int max_optin = 0;
+  if (cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+      cudaSuccess)
+    return DCN_ERR_CUDA;
+  if (smem > size_t(max_optin)) return DCN_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return DCN_ERR_CUDA;
+  return DCN_OK;
+}
+
+template <typename Kernel, typename Args>
+dcn_status launch(Kernel k, const Plan& plan, const Args& args, cudaStream_t stream) {
+  dcn_status st = prepare_smem(k, plan.smem);
+  if (st != DCN_OK) return st;
+  k<<<plan.grid, kThreads, plan.smem, stream>>>(args);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+template <typename T, int CPL, int LANES>
+dcn_status forward_dispatch_kk(const dcn_problem* p, const Plan& plan, const FwdArgs& args,
+                               cudaStream_t stream) {
+  const bool k3 = p->K == 3;
+  if (p->softmax) {
+    return k3 ? launch(dcn_forward_kernel<T, CPL, LANES, 9, true>, plan, args, stream)
+              : launch(dcn_forward_kernel<T, CPL, LANES, 0, true>, plan, args, stream);
+  }
+  return k3 ? launch(dcn_forward_kernel<T, CPL, LANES, 9, false>, plan, args, stream)
+            : launch(dcn_forward_kernel<T, CPL, LANES, 0, false>, plan, args, stream);
+}
+
+template <typename T>
+dcn_status forward_dispatch(const dcn_problem* p, const Plan& plan, const FwdArgs& args,
+                            cudaStream_t stream) {
+  constexpr int e = sizeof(T);
+  const int cpl = plan.lm.cpl, lanes = plan.lm.lanes;
+  if (cpl == 16 / e && lanes == 1) return forward_dispatch_kk<T, 16 / e, 1>(p, plan, args, stream);
+  if (cpl == 32 / e && lanes == 1) return forward_dispatch_kk<T, 32 / e, 1>(p, plan, args, stream);
+  if (cpl == 32 / e && lanes == 2) return forward_dispatch_kk<T, 32 / e, 2>(p, plan, args, stream);
+  if (cpl == 32 / e && lanes == 4) return forward_dispatch_kk<T, 32 / e, 4>(p, plan, args, stream);
+  return DCN_ERR_UNSUPPORTED;
+}
+
+template <int CPL, int LANES>
+dcn_status backward_dispatch_kk(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
+                                cudaStream_t stream) {
+  const bool k3 = p->K == 3;
+  if (p->softmax) {
+    return k3 ? launch(dcn_backward_kernel<CPL, LANES, 9, true>, plan, args, stream)
+              : launch(dcn_backward_kernel<CPL, LANES, 0, true>, plan, args, stream);
+  }
+  return k3 ? launch(dcn_backward_kernel<CPL, LANES, 9, false>, plan, args, stream)
+            : launch(dcn_backward_kernel<CPL, LANES, 0, false>, plan, args, stream);
+}
+
+dcn_status backward_dispatch(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
+                             cudaStream_t stream) {
+  const int cpl = plan.lm.cpl, lanes = plan.lm.lanes;
+  if (cpl == 4 && lanes == 1) return backward_dispatch_kk<4, 1>(p, plan, args, stream);
+  if (cpl == 8 && lanes == 1) return backward_dispatch_kk<8, 1>(p, plan, args, stream);
+  if (cpl == 8 && lanes == 2) return backward_dispatch_kk<8, 2>(p, plan, args, stream);
+  if (cpl == 8 && lanes == 4) return backward_dispatch_kk<8, 4>(p, plan, args, stream);
+  return DCN_ERR_UNSUPPORTED;
+}
+
+dcn_status check_forward_pointers(const dcn_problem* p, const void* x, const void* off,
+                                  const void* mask, const void* out) {
+  if (!x || !off || !mask || !out) return DCN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(off, 16) || !aligned(mask, 16) || !aligned(out, 16))
+    return DCN_ERR_UNSUPPORTED;
+  LaneMap lm;
+  if (!lane_map(p, &lm)) return DCN_ERR_UNSUPPORTED;
+  const size_t vb = size_t(lm.cpl) * esize(p->dtype);  // per-lane vector: 16 or 32 bytes
+  if (!aligned(x, vb) || !aligned(out, vb)) return DCN_ERR_UNSUPPORTED;
+  return DCN_OK;
+}
+
+}  // namespace
+}  // namespace dcn
+
+using namespace dcn;
+
+extern "C" {
+
+dcn_status dcn_core_output_hw(const dcn_problem* problem, int* Ho, int* Wo) {
+  if (!Ho || !Wo) return DCN_ERR_INVALID_ARG;
+  int64_t ho = 0, wo = 0;
+  dcn_status st = check_problem(problem, &ho, &wo);
+  if (st != DCN_OK && st != DCN_ERR_UNSUPPORTED) return st;
+  if (ho < 1 || wo < 1) {
+    ho = out_extent(problem->H, problem->K, problem->stride, problem->pad, problem->dilation);
+    wo = out_extent(problem->W, problem->K, problem->stride, problem->pad, problem->dilation);
+  }
+  *Ho = int(ho);
+  *Wo = int(wo);
+  return DCN_OK;
+}
+
+dcn_status dcn_core_forward(const dcn_problem* problem, const void* input, const void* offset,
+                            const void* mask, void* output, cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  st = check_forward_pointers(problem, input, offset, mask, output);
+  if (st != DCN_OK) return st;
+  Plan plan;
+  const size_t entry = problem->dtype == DCN_BF16 ? staged_bytes_per_entry<__nv_bfloat16>()
+                                                  : staged_bytes_per_entry<float>();
+  st = make_plan(problem, Ho, Wo, entry, &plan);
+  if (st != DCN_OK) return st;
+  FwdArgs args{input, offset, mask, output, plan.t};
+  return problem->dtype == DCN_BF16 ? forward_dispatch<__nv_bfloat16>(problem, plan, args, stream)
+                                    : forward_dispatch<float>(problem, plan, args, stream);
+}
+
+dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input,
+                                 const void* h_offset, const void* h_mask, void* h_output,
+                                 void* d_input, void* d_offset, void* d_mask, void* d_output,
+                                 cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!h_input || !h_offset || !h_mask || !h_output) return DCN_ERR_INVALID_ARG;
+  st = check_forward_pointers(problem, d_input, d_offset, d_mask, d_output);
+  if (st != DCN_OK) return st;
+  const size_t e = size_t(esize(problem->dtype));
+  const size_t C = size_t(problem->G) * problem->Cg, KK = size_t(problem->K) * problem->K;
+  const size_t b_in = size_t(problem->N) * problem->H * problem->W * C * e;
+  const size_t px = size_t(problem->N) * Ho * Wo;
+  const size_t b_off = px * problem->G * KK * 2 * e, b_msk = px * problem->G * KK * e;
+  const size_t b_out = px * C * e;
+  if (cudaMemcpyAsync(d_input, h_input, b_in, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_offset, h_offset, b_off, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaMemcpyAsync(d_mask, h_mask, b_msk, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return DCN_ERR_CUDA;
+  st = dcn_core_forward(problem, d_input, d_offset, d_mask, d_output, stream);
+  if (st != DCN_OK) return st;
+  if (cudaMemcpyAsync(h_output, d_output, b_out, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return DCN_ERR_CUDA;
+  return DCN_OK;
+}
+
+size_t dcn_core_backward_workspace(const dcn_problem* problem) {
+  (void)problem;
+  return 0;
+}
+
+dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, const void* offset,
+                             const void* mask, const void* grad_out, void* grad_input,
+                             void* grad_offset, void* grad_mask, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!input || !offset || !mask || !grad_out || !grad_input || !grad_offset || !grad_mask)
+    return DCN_ERR_INVALID_ARG;
+  if (problem->dtype != DCN_F32) return DCN_ERR_UNSUPPORTED;
+  st = check_forward_pointers(problem, input, offset, mask, grad_out);
+  if (st != DCN_OK) return st;
+  LaneMap lm;
+  lane_map(problem, &lm);
+  const size_t vb = size_t(lm.cpl) * 4;
+  if (!aligned(grad_input, vb) || !aligned(grad_offset, 16) || !aligned(grad_mask, 16))
+    return DCN_ERR_UNSUPPORTED;
+  Plan plan;
+  st = make_plan(problem, Ho, Wo, staged_bytes_per_entry<float>(), &plan);
+  if (st != DCN_OK) return st;
+  const size_t gx_bytes =
+      size_t(problem->N) * problem->H * problem->W * problem->G * problem->Cg * sizeof(float);
+  if (cudaMemsetAsync(grad_input, 0, gx_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
+  BwdArgs args{static_cast<const float*>(input), offset, mask,
+               static_cast<const float*>(grad_out), static_cast<float*>(grad_input),
+               static_cast<float*>(grad_offset), static_cast<float*>(grad_mask), plan.t};
+  return backward_dispatch(problem, plan, args, stream);
+}
+
+dcn_status dcn_core_sync_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return DCN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return DCN_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_dcn_error_word, sizeof(word)) != cudaSuccess)
+    return DCN_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_dcn_error_word, &zero, sizeof(zero));
+    return DCN_ERR_TIMEOUT;
+  }
+  return DCN_OK;
+}
+
+const char* dcn_status_string(dcn_status status) {
+  switch (status) {
+    case DCN_OK: return "ok";
+    case DCN_ERR_INVALID_ARG: return "invalid argument";
+    case DCN_ERR_UNSUPPORTED: return "unsupported argument (alignment, channel width or dtype)";
+    case DCN_ERR_CUDA: return "CUDA error";
+    case DCN_ERR_TIMEOUT: return "a bounded device wait gave up";
+    default: return "unknown status";
+  }
+}
+
+int dcn_core_abi_version(void) { return DCN_CORE_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,159 @@
+/*
+ * dcn_core.h -- C ABI of the B200 (sm_100a) deformable-convolution core.
+ *
+ * The operator (InternImage-L DCNv3 explainer (wmrh.cn), section 二 steps
+ * 2-4 and section 三): for every output pixel (n, ho, wo), group g and tap
+ * k = a*K + b of a K x K window, take the learned offset (dx, dy) of that
+ * tap, scale it by offset_scale, bilinearly sample the group's Cg input
+ * channels at
+ *     Y = ho*stride - pad + a*dilation + offset_scale*dy
+ *     X = wo*stride - pad + b*dilation + offset_scale*dx
+ * (integer coordinates are pixel centres; corners outside the image read as
+ * zero), and sum the K*K samples weighted by the mask of that (pixel, group):
+ * softmax-normalised over the taps for DCNv3, used as given for the DCNv4
+ * variant (DCNv4 speed-up write-up (pnsm.cn), sections 1-2).  Arithmetic is
+ * fp32 for both storage types; bf16 values are widened exactly on load and
+ * the output is rounded to nearest-even once.
+ *
+ * Layouts (all tensors dense, row-major, element indices; C = G*Cg, KK = K*K):
+ *   input   (N, H, W, C)            ((n*H + y)*W + x)*C + g*Cg + c
+ *   offset  (N, Ho, Wo, G*KK*2)     ((n*Ho + ho)*Wo + wo)*G*KK*2 + (g*KK + k)*2 + {0: dx, 1: dy}
+ *   mask    (N, Ho, Wo, G*KK)       ((n*Ho + ho)*Wo + wo)*G*KK + g*KK + k
+ *   output  (N, Ho, Wo, C)          ((n*Ho + ho)*Wo + wo)*C + g*Cg + c
+ *   Ho = floor((H + 2*pad - dilation*(K-1) - 1) / stride) + 1, Wo likewise.
+ *
+ * Ownership and execution: every pointer is owned by the caller.  Device
+ * pointers must stay valid until the enqueued work has finished.  All work is
+ * enqueued asynchronously on the caller's stream (NULL = the legacy default
+ * stream); the library never allocates device memory, never synchronises
+ * (except dcn_core_sync_status) and keeps no per-call state.
+ *
+ * Errors: arguments are validated on the host before anything is enqueued.
+ * Invalid arguments return DCN_ERR_INVALID_ARG, valid but unsupported ones
+ * (alignment, channel widths without a kernel, bf16 backward) return
+ * DCN_ERR_UNSUPPORTED, and a failed launch returns DCN_ERR_CUDA.  On any
+ * error nothing has been enqueued.  Device-side failures (a bounded wait
+ * that gave up) are reported by dcn_core_sync_status as DCN_ERR_TIMEOUT.
+ */
+#ifndef DCN_CORE_H_
+#define DCN_CORE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DCN_CORE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define DCN_API __attribute__((visibility("default")))
+#else
+#define DCN_API
+#endif
+
+typedef enum {
+  DCN_OK = 0,
+  DCN_ERR_INVALID_ARG = 1,
+  DCN_ERR_UNSUPPORTED = 2,
+  DCN_ERR_CUDA = 3,
+  DCN_ERR_TIMEOUT = 4
+} dcn_status;
+
+typedef enum {
+  DCN_F32 = 0,   /* fp32 storage                                    */
+  DCN_BF16 = 1   /* bf16 storage, fp32 arithmetic                   */
+} dcn_dtype;
+
+/*
+ * Problem description (the constructor arguments of the DCNv3/DCNv4 modules
+ * in the DCNv4 speed-up write-up (pnsm.cn), section 3.3: channels = G*Cg,
+ * kernel_size, stride, pad, dilation, group, offset_scale).
+ *   N, H, W      batch and input spatial size, >= 1
+ *   G, Cg        groups and channels per group, >= 1
+ *   K            kernel side, odd, >= 1 (taps = K*K)
+ *   stride >= 1, pad >= 0, dilation >= 1 (same for height and width)
+ *   offset_scale multiplies every offset (InternImage-L uses 2.0)
+ *   softmax      1: mask holds logits, softmax over the K*K taps of each
+ *                   (pixel, group) (DCNv3);  0: mask used as given (DCNv4)
+ *   dtype        storage type of input, offset, mask and output
+ */
+typedef struct {
+  int N, H, W, G, Cg;
+  int K;
+  int stride, pad, dilation;
+  float offset_scale;
+  int softmax;
+  dcn_dtype dtype;
+} dcn_problem;
+
+/* Output spatial size.  DCN_ERR_INVALID_ARG if the problem is invalid or the
+ * output would be empty. */
+DCN_API dcn_status dcn_core_output_hw(const dcn_problem* problem, int* Ho, int* Wo);
+
+/*
+ * Forward (explainer section 二 steps 2-4).  input, offset, mask: device
+ * pointers in the layouts above, of problem->dtype; output: device pointer,
+ * written entirely.  All four must be 16-byte aligned and must not overlap
+ * the output.  Supported channel widths: Cg*sizeof(dtype) a multiple of 16
+ * bytes and at most 128 bytes (Cg in {4, 8, 12, ..., 32} for fp32, {8, 16,
+ * ..., 64} for bf16); other widths return DCN_ERR_UNSUPPORTED.
+ */
+DCN_API dcn_status dcn_core_forward(const dcn_problem* problem, const void* input,
+                            const void* offset, const void* mask, void* output,
+                            cudaStream_t stream);
+
+/*
+ * Forward on HOST buffers: copies input, offset and mask from the host to the
+ * caller's device buffers, runs dcn_core_forward and copies the output back,
+ * all enqueued on `stream` (one cudaMemcpyAsync per tensor).  Host buffers
+ * should be pinned for the copies to be asynchronous; they must not be
+ * touched until the stream has reached this point.  Device buffers follow the
+ * rules of dcn_core_forward.
+ */
+DCN_API dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input,
+                                 const void* h_offset, const void* h_mask,
+                                 void* h_output, void* d_input, void* d_offset,
+                                 void* d_mask, void* d_output, cudaStream_t stream);
+
+/* Device workspace the backward needs, in bytes (0 for the current
+ * atomic-scatter backward). */
+DCN_API size_t dcn_core_backward_workspace(const dcn_problem* problem);
+
+/*
+ * Backward (gradients of the forward above).  grad_out: (N, Ho, Wo, C).
+ *   grad_input  (N, H, W, C)   OVERWRITTEN: zero-filled on the stream, then
+ *               accumulated by a vectorised atomic scatter (the order of
+ *               the additions, hence the last bits, may differ between runs)
+ *   grad_offset (N, Ho, Wo, G*KK*2), overwritten
+ *   grad_mask   (N, Ho, Wo, G*KK), overwritten; with softmax = 1 it is the
+ *               gradient with respect to the logits
+ * The gradient with respect to an offset at an integer sample coordinate is
+ * the one-sided derivative that floor() selects.  Only fp32 storage is
+ * supported (bf16 returns DCN_ERR_UNSUPPORTED); channel widths and alignment
+ * as for the forward.  workspace may be NULL when the workspace size is 0.
+ */
+DCN_API dcn_status dcn_core_backward(const dcn_problem* problem, const void* input,
+                             const void* offset, const void* mask,
+                             const void* grad_out, void* grad_input,
+                             void* grad_offset, void* grad_mask, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/* Synchronises `stream` and reports: DCN_ERR_CUDA if CUDA reports an error,
+ * DCN_ERR_TIMEOUT if a kernel of this library gave up a bounded wait since
+ * the last call (the device error word is then cleared), else DCN_OK. */
+DCN_API dcn_status dcn_core_sync_status(cudaStream_t stream);
+
+/* Static description of a status code. */
+DCN_API const char* dcn_status_string(dcn_status status);
+
+/* DCN_CORE_ABI_VERSION of the loaded library. */
+DCN_API int dcn_core_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN_CORE_H_ */

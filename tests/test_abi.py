@@ -1,0 +1,129 @@
+"""The C-ABI library builds, loads and exports every entry point its header
+declares; host-side validation rejects bad arguments before any launch.
+Runs without a GPU: no call here reaches a kernel."""
+import os
+import re
+
+import pytest
+
+import deformable_convolution_core_b200 as dcn
+from deformable_convolution_core_b200 import build as dcn_build
+from tests.conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dcn_build.build()
+    return dcn.load_library()
+
+
+def declared_symbols():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            text = open(os.path.join(inc, f)).read()
+            names += re.findall(r"DCN_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert set(dcn.EXPORTED_SYMBOLS) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert dcn.dcn_core_abi_version() == 1
+    for st in range(5):
+        assert dcn.dcn_status_string(st)
+    assert "unknown" in dcn.dcn_status_string(99)
+
+
+def test_output_hw(lib):
+    assert dcn.dcn_core_output_hw(dcn.make_problem(1, 96, 96, 10, 16)) == (96, 96)
+    assert dcn.dcn_core_output_hw(dcn.make_problem(2, 256, 256, 12, 16, stride=2)) == (128, 128)
+    assert dcn.dcn_core_output_hw(dcn.make_problem(1, 7, 9, 1, 8, K=5, pad=0, dilation=1)) == (3, 5)
+    with pytest.raises(dcn.DcnError):
+        dcn.dcn_core_output_hw(dcn.make_problem(1, 2, 2, 1, 8, K=5, pad=0))
+
+
+GOOD = dict(N=1, H=8, W=8, G=2, Cg=16, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0,
+            softmax=1, dtype="f32")
+FAKE = 1 << 20  # an address that is 16- and 32-byte aligned; never dereferenced here
+
+
+@pytest.mark.parametrize("change,status", [
+    (dict(N=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(H=-1), dcn.DCN_ERR_INVALID_ARG),
+    (dict(G=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(Cg=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(K=2), dcn.DCN_ERR_INVALID_ARG),
+    (dict(K=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(stride=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(pad=-1), dcn.DCN_ERR_INVALID_ARG),
+    (dict(dilation=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(softmax=2), dcn.DCN_ERR_INVALID_ARG),
+    (dict(dtype=7), dcn.DCN_ERR_INVALID_ARG),
+    (dict(offset_scale=float("nan")), dcn.DCN_ERR_INVALID_ARG),
+    (dict(H=2, W=2, K=5, pad=0), dcn.DCN_ERR_INVALID_ARG),     # empty output
+    (dict(N=1 << 16, H=1 << 8, W=1 << 8, G=16, Cg=16), dcn.DCN_ERR_INVALID_ARG),  # >= 2^31 elements
+    (dict(Cg=5), dcn.DCN_ERR_UNSUPPORTED),                      # 20 bytes: no kernel
+    (dict(Cg=48), dcn.DCN_ERR_UNSUPPORTED),                     # 192 bytes
+])
+def test_forward_rejects_before_launch(lib, change, status):
+    p = dcn.make_problem(**{**GOOD, **change})
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_forward(p, FAKE, FAKE, FAKE, FAKE, 0)
+    assert e.value.status == status
+
+
+def test_forward_rejects_null_and_misaligned(lib):
+    p = dcn.make_problem(**GOOD)
+    for args in [(0, FAKE, FAKE, FAKE), (FAKE, 0, FAKE, FAKE), (FAKE, FAKE, 0, FAKE),
+                 (FAKE, FAKE, FAKE, 0)]:
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_forward(p, *args, 0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    for args in [(FAKE + 4, FAKE, FAKE, FAKE), (FAKE, FAKE + 8, FAKE, FAKE),
+                 (FAKE, FAKE, FAKE + 2, FAKE), (FAKE, FAKE, FAKE, FAKE + 16)]:
+        with pytest.raises(dcn.DcnError) as e:   # Cg=16 fp32: 32-byte vectors on x and out
+            dcn.dcn_core_forward(p, *args, 0)
+        assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_before_launch(lib):
+    p = dcn.make_problem(**GOOD)
+    ptrs = [FAKE] * 7
+    for i in range(7):
+        bad = list(ptrs)
+        bad[i] = 0
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_backward(p, *bad, None, 0, 0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    pb = dcn.make_problem(**{**GOOD, "dtype": "bf16"})
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward(pb, *ptrs, None, 0, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    assert dcn.dcn_core_backward_workspace(p) == 0
+
+
+def test_forward_host_rejects_before_copy(lib):
+    p = dcn.make_problem(**GOOD)
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_forward_host(p, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0)
+    assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_forward_host(p, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+
+
+def test_library_has_no_oracle_dependency():
+    """The CUDA library and binding never reference the oracle."""
+    pkg = os.path.join(ROOT, "deformable_convolution_core_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in text.lower(), os.path.join(dirpath, f)

@@ -1,0 +1,109 @@
+"""Backward parity: grad_input, grad_offset and grad_mask (w.r.t. the logits
+when softmax is on) of the CUDA path against the CPU oracle, plus the
+adjoint identity and the softmax-Jacobian row sums at the full backward size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import deformable_convolution_core_b200 as dcn
+from gen.workloads import WORKLOADS
+from tests.dcn_testutil import assert_bwd, f64, gpu_backward, gpu_forward, problem_kwargs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(77)
+
+
+def near_kink_taps(p, off):
+    """Count taps whose sample coordinate lies within 1e-6 of an integer, where
+    the offset gradient switches between one-sided derivatives."""
+    N, Ho, Wo = off.shape[:3]
+    K = p.K
+    o = off.reshape(N, Ho, Wo, p.G, K * K, 2).astype(np.float32)
+    ho = np.arange(Ho).reshape(1, Ho, 1, 1, 1)
+    wo = np.arange(Wo).reshape(1, 1, Wo, 1, 1)
+    k = np.arange(K * K)
+    a, b = (k // K).reshape(1, 1, 1, 1, -1), (k % K).reshape(1, 1, 1, 1, -1)
+    s = np.float32(p.offset_scale)
+    Y = (ho * p.stride - p.pad + a * p.dilation).astype(np.float32) + s * o[..., 1]
+    X = (wo * p.stride - p.pad + b * p.dilation).astype(np.float32) + s * o[..., 0]
+    fy, fx = Y - np.floor(Y), X - np.floor(X)
+    near = (np.minimum(fy, 1 - fy) < 1e-6) | (np.minimum(fx, 1 - fx) < 1e-6)
+    return int(near.sum())
+
+
+def check(oracle_mod, p, x, off, mask, gout):
+    xd, od, md, gd = (to_dev(a, "f32") for a in (x, off, mask, gout))
+    gx, goff, gm = gpu_backward(p, xd, od, md, gd)
+    torch.cuda.synchronize()
+    rx, roff, rm = oracle_mod.backward(x, off, mask, gout, **problem_kwargs(p))
+    assert_bwd(f64(gx), rx, f"grad_input {p}")
+    assert_bwd(f64(goff), roff, f"grad_offset {p} (near-kink taps: {near_kink_taps(p, off)})")
+    assert_bwd(f64(gm), rm, f"grad_mask {p}")
+    return gx, goff, gm
+
+
+CASES = [
+    (2, 23, 29, 3, 16, dict()),
+    (2, 19, 17, 5, 16, dict(softmax=0)),
+    (2, 15, 21, 4, 4, dict()),
+    (2, 15, 21, 4, 8, dict()),
+    (2, 13, 14, 3, 32, dict()),
+    (2, 17, 19, 3, 16, dict(K=5, pad=2)),
+    (2, 17, 19, 3, 16, dict(K=1, pad=0)),
+    (2, 24, 26, 3, 16, dict(stride=2)),
+    (2, 21, 22, 3, 16, dict(dilation=2, pad=2)),
+    (1, 1, 1, 2, 16, dict()),
+    (1, 30, 3, 40, 16, dict()),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_" +
+                                             "_".join(f"{k}{v}" for k, v in c[5].items())
+                                             for c in CASES])
+def test_backward_matches_oracle(oracle_mod, case):
+    N, H, W, G, Cg, kw = case
+    kw = {"K": 3, "stride": 1, "pad": 1, "dilation": 1, "softmax": 1, **kw}
+    p = dcn.make_problem(N, H, W, G, Cg, kw["K"], kw["stride"], kw["pad"], kw["dilation"],
+                         2.0, kw["softmax"], "f32")
+    Ho, Wo = dcn.dcn_core_output_hw(p)
+    KK = kw["K"] ** 2
+    x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    off = (1.5 * RNG.standard_normal((N, Ho, Wo, G * KK * 2))).astype(np.float32)
+    mask = RNG.standard_normal((N, Ho, Wo, G * KK)).astype(np.float32)
+    gout = RNG.standard_normal((N, Ho, Wo, G * Cg)).astype(np.float32)
+    check(oracle_mod, p, x, off, mask, gout)
+
+
+def test_full_size_backward(gen_mod, oracle_mod):
+    wl = WORKLOADS["internimage_l_stage2_bwd_fp32_n32_48x48_c320"]
+    d = gen_mod.make_inputs(wl)
+    p = dcn.problem_for(wl)
+    gx, goff, gm = check(oracle_mod, p, d["x"], d["offset"], d["mask"], d["grad_out"])
+    # adjoint identity: <gout, F(v)> = <grad_input(gout), v>, v random
+    v = RNG.standard_normal(d["x"].shape).astype(np.float32)
+    xd, od, md = (to_dev(d[k], "f32") for k in ("x", "offset", "mask"))
+    gxv, _, _ = gpu_backward(p, to_dev(v, "f32"), od, md, to_dev(d["grad_out"], "f32"))
+    fv = gpu_forward(p, to_dev(v, "f32"), od, md)
+    torch.cuda.synchronize()
+    lhs = float((f64(fv) * d["grad_out"].astype(np.float64)).sum())
+    rhs = float((f64(gxv) * v.astype(np.float64)).sum())
+    assert abs(lhs - rhs) <= 1e-6 * max(abs(lhs), abs(rhs))
+    # softmax Jacobian rows: the logit gradients of every (pixel, group) sum to zero
+    rows = f64(gm).reshape(-1, 9)
+    assert np.abs(rows.sum(1)).max() <= 1e-5 * np.abs(rows).max()
+
+
+def test_backward_rerun_differs_only_by_rounding(gen_mod):
+    wl = WORKLOADS["internimage_l_stage2_bwd_fp32_n32_48x48_c320"]
+    d = gen_mod.make_inputs(wl, n_images=4)
+    p = dcn.make_problem(4, wl.H, wl.W, wl.G, wl.Cg, offset_scale=wl.offset_scale)
+    args = [to_dev(d[k], "f32") for k in ("x", "offset", "mask", "grad_out")]
+    a = gpu_backward(p, *args)
+    b = gpu_backward(p, *args)
+    torch.cuda.synchronize()
+    # offset and mask gradients are computed without atomics: bitwise equal
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    # the input gradient sums atomically: equal up to the order of additions
+    assert torch.allclose(a[0], b[0], rtol=0, atol=1e-5 * float(a[0].abs().max()))

@@ -1,0 +1,180 @@
+"""Forward parity: the CUDA path against the CPU oracle on the same seeded
+inputs, element by element, through the C ABI.
+
+Small and medium problems are compared in full (they span several tiles and
+ragged tile edges); the full-size workloads, in the launch configuration the
+benchmark times, are compared on sampled units the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import deformable_convolution_core_b200 as dcn
+from gen.workloads import WORKLOADS
+from tests.dcn_testutil import assert_fwd, f64, gpu_forward, problem_kwargs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(2024)
+
+
+def random_case(N, H, W, G, Cg, K=3, stride=1, pad=None, dil=1, sigma=2.0, softmax=1,
+                dtype="f32", off_sd=1.5, off_lo=None):
+    pad = (K // 2) * dil if pad is None else pad
+    p = dcn.make_problem(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, dtype)
+    Ho, Wo = dcn.dcn_core_output_hw(p)
+    x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    if off_lo is None:
+        off = (off_sd * RNG.standard_normal((N, Ho, Wo, G * K * K * 2))).astype(np.float32)
+    else:
+        off = RNG.uniform(off_lo, -off_lo, (N, Ho, Wo, G * K * K * 2)).astype(np.float32)
+    if softmax:
+        mask = RNG.standard_normal((N, Ho, Wo, G * K * K)).astype(np.float32)
+    else:
+        mask = RNG.uniform(-1, 1, (N, Ho, Wo, G * K * K)).astype(np.float32)
+    return p, x, off, mask
+
+
+def check_full(oracle_mod, p, x, off, mask, dtype):
+    xd, od, md = to_dev(x, dtype), to_dev(off, dtype), to_dev(mask, dtype)
+    out = gpu_forward(p, xd, od, md)
+    torch.cuda.synchronize()
+    ref = oracle_mod.forward(f64(xd), f64(od), f64(md), **problem_kwargs(p))
+    assert_fwd(f64(out), ref, f64(xd), dtype, repr(p))
+    return out
+
+
+CASES = [
+    # (N, H, W, G, Cg, dict)  -- ragged sizes, several tiles per image
+    (2, 23, 29, 3, 16, dict(dtype="f32")),
+    (2, 19, 27, 5, 16, dict(dtype="bf16")),
+    (1, 33, 17, 10, 16, dict(dtype="bf16", softmax=0)),
+    (3, 12, 12, 8, 16, dict(dtype="f32", softmax=0, sigma=1.0)),
+    (2, 15, 21, 4, 4, dict(dtype="f32")),        # 16-byte units, fp32
+    (2, 15, 21, 4, 8, dict(dtype="f32")),        # 32-byte units, fp32
+    (2, 13, 14, 3, 32, dict(dtype="f32")),       # 128-byte units, fp32 (4 lanes)
+    (2, 15, 21, 4, 8, dict(dtype="bf16")),       # 16-byte units, bf16
+    (2, 13, 14, 3, 32, dict(dtype="bf16")),      # 64-byte units, bf16 (2 lanes)
+    (1, 11, 10, 2, 64, dict(dtype="bf16")),      # 128-byte units, bf16 (4 lanes)
+    (2, 17, 19, 3, 16, dict(dtype="f32", K=1, pad=0)),
+    (2, 17, 19, 3, 16, dict(dtype="f32", K=5)),
+    (1, 17, 19, 2, 16, dict(dtype="bf16", K=7, softmax=0)),
+    (2, 24, 26, 3, 16, dict(dtype="f32", stride=2)),
+    (2, 25, 27, 3, 16, dict(dtype="bf16", stride=2, softmax=0)),
+    (2, 21, 22, 3, 16, dict(dtype="f32", dil=2)),
+    (2, 21, 22, 3, 16, dict(dtype="f32", pad=0)),
+    (1, 1, 1, 2, 16, dict(dtype="f32")),         # single pixel
+    (1, 1, 7, 2, 16, dict(dtype="bf16")),        # single row
+    (2, 3, 3, 2, 16, dict(dtype="f32", stride=5)),   # stride larger than the image
+    (1, 40, 3, 80, 16, dict(dtype="bf16")),      # many groups
+    (2, 20, 20, 2, 16, dict(dtype="f32", off_lo=-40.0)),   # most samples far outside
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_" +
+                                             "_".join(f"{k}{v}" for k, v in c[5].items())
+                                             for c in CASES])
+def test_forward_matches_oracle(oracle_mod, case):
+    N, H, W, G, Cg, kw = case
+    dtype = kw.get("dtype", "f32")
+    p, x, off, mask = random_case(N, H, W, G, Cg, **kw)
+    check_full(oracle_mod, p, x, off, mask, dtype)
+
+
+def test_identity_and_box_filter_on_gpu(oracle_mod):
+    # Zero offsets with a one-hot centre mask give the input back exactly; zero
+    # logits give the 3x3 box filter (the "plain 3x3 convolution" start state).
+    N, H, W, G, Cg = 2, 13, 17, 3, 16
+    x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    off = np.zeros((N, H, W, G * 18), np.float32)
+    onehot = np.zeros((N, H, W, G, 9), np.float32)
+    onehot[..., 4] = 1.0
+    p = dcn.make_problem(N, H, W, G, Cg, softmax=0)
+    out = gpu_forward(p, to_dev(x, "f32"), to_dev(off, "f32"), to_dev(onehot.reshape(N, H, W, -1), "f32"))
+    assert np.array_equal(f64(out), x.astype(np.float64))
+    p1 = dcn.make_problem(N, H, W, G, Cg, softmax=1)
+    logits = np.zeros((N, H, W, G * 9), np.float32)
+    out = gpu_forward(p1, to_dev(x, "f32"), to_dev(off, "f32"), to_dev(logits, "f32"))
+    xp = np.pad(x.astype(np.float64), ((0, 0), (1, 1), (1, 1), (0, 0)))
+    box = sum(xp[:, i:i + H, j:j + W, :] for i in range(3) for j in range(3)) / 9.0
+    np.testing.assert_allclose(f64(out), box, rtol=0, atol=1e-5 * np.abs(x).max())
+
+
+def test_nonfinite_and_border_offsets(oracle_mod):
+    N, H, W, G, Cg = 1, 9, 11, 2, 16
+    p, x, off, mask = random_case(N, H, W, G, Cg)
+    o = off.reshape(N, H, W, G, 9, 2)
+    o[0, 0, 0, 0, :, 0] = np.nan
+    o[0, 1, 1, 0, :, 1] = np.inf
+    o[0, 2, 2, 1, :, 0] = -np.inf
+    o[0, 3, 3, 0, :, :] = 1e30
+    # samples exactly on the borders -1, 0, W-1 and W (sigma = 2)
+    o[0, 4, :, 1, 4, 0] = (np.array([-1, 0, W - 1, W] * 3)[:W] - np.arange(W)) / 2.0
+    check_full(oracle_mod, p, x, off, mask, "f32")
+
+
+def test_forward_is_deterministic_and_stream_safe(oracle_mod):
+    p, x, off, mask = random_case(2, 31, 29, 6, 16, dtype="bf16")
+    xd, od, md = to_dev(x, "bf16"), to_dev(off, "bf16"), to_dev(mask, "bf16")
+    a = gpu_forward(p, xd, od, md)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = gpu_forward(p, xd, od, md, stream=s)
+    s.synchronize()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    dcn.dcn_core_sync_status(s)
+
+
+def test_forward_host_entry_point():
+    p, x, off, mask = random_case(2, 21, 23, 4, 16, dtype="f32")
+    Ho, Wo = dcn.dcn_core_output_hw(p)
+    hx = torch.from_numpy(x).pin_memory()
+    ho = torch.from_numpy(off).pin_memory()
+    hm = torch.from_numpy(mask).pin_memory()
+    hout = torch.empty((2, Ho, Wo, 64), dtype=torch.float32).pin_memory()
+    dx, do, dm = (torch.empty_like(t, device="cuda") for t in (hx, ho, hm))
+    dout = torch.empty(hout.shape, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    dcn.dcn_core_forward_host(p, hx, ho, hm, hout, dx, do, dm, dout, stream=s)
+    dcn.dcn_core_sync_status(s)
+    ref = gpu_forward(p, hx.cuda(), ho.cuda(), hm.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(hout, ref.cpu())
+
+
+# --- full-size workloads, sampled ----------------------------------------------------
+
+def sampled_units(wl, imgs, per_img=3000):
+    """Units u = ((n*Ho+ho)*Wo+wo)*G+g of a few images: random ones plus every
+    unit of the first and last output rows and columns (the image border)."""
+    Ho, Wo, G = wl.Ho, wl.Wo, wl.G
+    units = []
+    for j, _ in enumerate(imgs):
+        base = j * Ho * Wo * G
+        r = RNG.integers(0, Ho * Wo * G, size=per_img)
+        border = [((ho * Wo + wo) * G + g) for ho in (0, Ho - 1) for wo in range(Wo) for g in range(G)]
+        border += [((ho * Wo + wo) * G + g) for ho in range(Ho) for wo in (0, Wo - 1) for g in range(G)]
+        units.append(base + np.unique(np.concatenate([r, np.array(border)])))
+    return np.concatenate(units)
+
+
+FULL = [n for n, w in WORKLOADS.items() if not w.backward]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload_sampled(gen_mod, oracle_mod, name):
+    wl = WORKLOADS[name]
+    d = gen_mod.make_inputs(wl)
+    p = dcn.problem_for(wl)
+    xd, od, md = to_dev(d["x"], wl.dtype), to_dev(d["offset"], wl.dtype), to_dev(d["mask"], wl.dtype)
+    out = gpu_forward(p, xd, od, md)
+    torch.cuda.synchronize()
+    imgs = sorted({0, wl.N // 2, wl.N - 1})
+    units = sampled_units(wl, imgs)
+    xs, os_, ms = (f64(t[imgs]) for t in (xd, od, md))
+    ref = oracle_mod.forward_units(xs, os_, ms, units, **problem_kwargs(p))
+    got = f64(out[imgs]).reshape(-1, wl.Cg)[units]
+    assert_fwd(got, ref, xs, wl.dtype, name)
+    # the whole output is finite and, for bf16, every value is a rounded fp32
+    assert torch.isfinite(out).all()
