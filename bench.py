@@ -7,7 +7,7 @@ InternImage-L stage-1 shape (fp32, N=32, 96x96, C=160 = 10 groups x 16,
 3x3, offset_scale 2.0, softmax mask), inputs drawn from the seeded generator.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload NAME] [--no-sweep] [--no-cpu-baseline]
+                  [--workload NAME] [--no-sweep] [--no-cpu-baseline] [--no-e2e]
 
 Prints ONE JSON line (rank 0).  Multi-GPU runs (torchrun) are independent
 replicas, one per GPU, with no data-path collective (weak scaling); the step
@@ -262,7 +262,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API: pinned host inputs -> device, step, results -> host
     e2e = None
-    if rank == 0 or world > 1:
+    if not args.no_e2e:
         e2e = run_e2e(step, inputs, args, barrier, world)
 
     result = {
@@ -453,6 +453,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
