@@ -3,15 +3,19 @@
 // include/dcn_core.h.
 #include "dcn_core.h"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 #include <climits>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 
 #include "dcn_backward.cuh"
 #include "dcn_forward.cuh"
+#include "dcn_forward_tiled.cuh"
 
 namespace dcn {
 
@@ -80,6 +84,8 @@ bool lane_map(const dcn_problem* p, LaneMap* lm) {
   }
 }
 
+bool backward_lane_map(const dcn_problem* p, LaneMap* lm);
+
 struct Plan {
   TileParams t;
   size_t smem;
@@ -118,8 +124,9 @@ void choose_tile(int Ho, int Wo, int G, int lanes, size_t entry_bytes, int KK, s
 }
 
 dcn_status make_plan(const dcn_problem* p, int64_t Ho, int64_t Wo, size_t entry_bytes,
-                     Plan* plan) {
-  if (!lane_map(p, &plan->lm)) return DCN_ERR_UNSUPPORTED;
+                     Plan* plan, bool backward = false) {
+  if (!(backward ? backward_lane_map(p, &plan->lm) : lane_map(p, &plan->lm)))
+    return DCN_ERR_UNSUPPORTED;
   TileParams& t = plan->t;
   t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
   t.K = p->K; t.KK = p->K * p->K; t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation;
@@ -216,14 +223,28 @@ dcn_status backward_dispatch_kk(const dcn_problem* p, const Plan& plan, const Bw
             : launch(dcn_backward_kernel<CPL, LANES, 0, false>, plan, args, stream);
 }
 
+// The backward always gives a lane 4 channels (16 bytes), so that one warp
+// instruction covers a unit's whole corner chunk: a gather or a float4 atomic
+// touches one cache line per (unit, corner) instead of one per lane.
+bool backward_lane_map(const dcn_problem* p, LaneMap* lm) {
+  switch (p->Cg) {
+    case 4: *lm = {4, 1}; return true;
+    case 8: *lm = {4, 2}; return true;
+    case 16: *lm = {4, 4}; return true;
+    case 32: *lm = {4, 8}; return true;
+    default: return false;
+  }
+}
+
 dcn_status backward_dispatch(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                              cudaStream_t stream) {
-  const int cpl = plan.lm.cpl, lanes = plan.lm.lanes;
-  if (cpl == 4 && lanes == 1) return backward_dispatch_kk<4, 1>(p, plan, args, stream);
-  if (cpl == 8 && lanes == 1) return backward_dispatch_kk<8, 1>(p, plan, args, stream);
-  if (cpl == 8 && lanes == 2) return backward_dispatch_kk<8, 2>(p, plan, args, stream);
-  if (cpl == 8 && lanes == 4) return backward_dispatch_kk<8, 4>(p, plan, args, stream);
-  return DCN_ERR_UNSUPPORTED;
+  switch (plan.lm.lanes) {
+    case 1: return backward_dispatch_kk<4, 1>(p, plan, args, stream);
+    case 2: return backward_dispatch_kk<4, 2>(p, plan, args, stream);
+    case 4: return backward_dispatch_kk<4, 4>(p, plan, args, stream);
+    case 8: return backward_dispatch_kk<4, 8>(p, plan, args, stream);
+    default: return DCN_ERR_UNSUPPORTED;
+  }
 }
 
 dcn_status check_forward_pointers(const dcn_problem* p, const void* x, const void* off,
@@ -238,6 +259,206 @@ dcn_status check_forward_pointers(const dcn_problem* p, const void* x, const voi
   return DCN_OK;
 }
 
+
+// ---------------------------------------------------------------------------
+// Tiled forward (input box staged by TMA).
+// ---------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int smem_optin = 0;
+  unsigned int* error_word = nullptr;
+};
+
+// Per-device constants, looked up once per device.
+dcn_status device_info(DeviceInfo* out) {
+  constexpr int kMaxDev = 64;
+  static DeviceInfo cache[kMaxDev];
+  static bool ready[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DCN_ERR_CUDA;
+  if (!ready[dev]) {
+    DeviceInfo d;
+    void* ew = nullptr;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaGetSymbolAddress(&ew, g_dcn_error_word) != cudaSuccess)
+      return DCN_ERR_CUDA;
+    d.error_word = static_cast<unsigned int*>(ew);
+    cache[dev] = d;
+    ready[dev] = true;
+  }
+  *out = cache[dev];
+  return DCN_OK;
+}
+
+int env_int(const char* name, int dflt) {
+  const char* s = std::getenv(name);
+  return s ? std::atoi(s) : dflt;
+}
+
+bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
+  const char* mode = std::getenv("DCN_CORE_FORWARD");
+  if (mode && std::strcmp(mode, "direct") == 0) return false;
+  const int cs = p->Cg * esize(p->dtype);
+  if (p->K != 3 || (cs != 32 && cs != 64)) return false;
+  if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
+  return tensor_map_encoder() != nullptr;
+}
+
+// Box row pitch (pixels) that makes the footprint reads conflict-free: for
+// 32-byte groups the two rows of a footprint must fall into complementary
+// halves of the 32 banks (pitch = 2 mod 4); for 64-byte groups the pitch
+// must be even (the lanes' piece rotation does the rest).
+int box_pitch(int bw, int cs) {
+  if (cs == 32) return bw + (2 - bw % 4 + 4) % 4;
+  return bw + (bw & 1);
+}
+
+// Box extent along one axis for a tile of `tile` outputs.
+int box_extent(int tile, int stride, int dil, int halo) {
+  return (tile - 1) * stride + 2 * dil + 2 + 2 * halo;
+}
+
+// Pick the output tile: largest useful area under the shared-memory budget,
+// penalising ragged-edge waste, idle lanes and the halo the box carries.
+void choose_tiled_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, size_t box_budget,
+                       int* TH_out, int* TW_out) {
+  double best = 1e300;
+  int bth = 1, btw = 1;
+  for (int th = 1; th <= std::min(Ho, 64); ++th) {
+    for (int tw = 1; tw <= std::min(Wo, 64); ++tw) {
+      const int bh = box_extent(th, p->stride, p->dilation, halo);
+      int bw = box_extent(tw, p->stride, p->dilation, halo);
+      bw = box_pitch(bw, cs);
+      if (bh > 256 || bw > 256) continue;
+      const size_t bytes = size_t(bh) * bw * cs;
+      if (bytes > box_budget) continue;
+      const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * p->G;
+      const int px = th * tw;
+      const int64_t batches = (px + kTiledBatch - 1) / kTiledBatch;
+      const double per_item = double(batches) * kTiledBatch * kTiledKK  // unit-samples
+                              + 0.05 * double(bytes) / 32.0            // box fill
+                              + 300.0;                                 // item overhead
+      const double cost = double(items) * per_item;
+      if (cost < best) {
+        best = cost;
+        bth = th;
+        btw = tw;
+      }
+    }
+  }
+  *TH_out = bth;
+  *TW_out = btw;
+}
+
+template <typename T, int CS, bool SOFTMAX>
+dcn_status launch_tiled_kernel(const CUtensorMap& map, const TiledArgs& args, size_t smem,
+                               int sms, cudaStream_t stream) {
+  auto k = dcn_forward_tiled_kernel<T, CS, SOFTMAX>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return DCN_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kTiledThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return DCN_ERR_UNSUPPORTED;
+  const int64_t grid = std::min<int64_t>(args.t.items, int64_t(sms) * per_sm);
+  k<<<unsigned(grid), kTiledThreads, smem, stream>>>(map, args);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
+                         const void* off, const void* mask, void* out, cudaStream_t stream) {
+  DeviceInfo dev;
+  dcn_status st = device_info(&dev);
+  if (st != DCN_OK) return st;
+  const int e = esize(p->dtype);
+  const int cs = p->Cg * e;
+  const size_t slot_bytes = size_t(kTiledWarps) * kTiledBatch * kSlotBytes;
+  const size_t fixed = slot_bytes + 64;
+  if (size_t(dev.smem_optin) <= fixed + 2048) return DCN_ERR_UNSUPPORTED;
+  const size_t box_budget = (size_t(dev.smem_optin) - fixed) / 2 / 1024 * 1024;
+  const int halo = env_int("DCN_CORE_HALO", 5);
+  int TH = 0, TW = 0;
+  if (const char* s = std::getenv("DCN_CORE_TILED_TILE")) {
+    if (std::sscanf(s, "%dx%d", &TH, &TW) != 2 || TH < 1 || TW < 1) TH = TW = 0;
+  }
+  if (TH == 0) choose_tiled_tile(p, int(Ho), int(Wo), cs, halo, box_budget, &TH, &TW);
+  TH = std::min<int>(TH, int(Ho));
+  TW = std::min<int>(TW, int(Wo));
+
+  TiledArgs args;
+  TiledParams& t = args.t;
+  t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
+  t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation; t.Ho = int(Ho); t.Wo = int(Wo);
+  t.sigma = p->offset_scale; t.halo = halo; t.TH = TH; t.TW = TW;
+  t.nTY = (t.Ho + TH - 1) / TH;
+  t.nTX = (t.Wo + TW - 1) / TW;
+  t.BH = box_extent(TH, t.stride, t.dil, halo);
+  t.BW = box_extent(TW, t.stride, t.dil, halo);
+  t.BW = box_pitch(t.BW, cs);
+  if (t.BH > 256 || t.BW > 256) return DCN_ERR_UNSUPPORTED;
+  t.box_bytes = uint32_t(size_t(t.BH) * t.BW * cs);
+  t.box_stride = (t.box_bytes + 1023u) / 1024u * 1024u;
+  const int64_t items = int64_t(t.N) * t.nTY * t.nTX * t.G;
+  if (items > INT_MAX) return DCN_ERR_UNSUPPORTED;
+  t.items = int(items);
+  t.batches = (TH * TW + kTiledBatch - 1) / kTiledBatch;
+  t.fd_G = make_fastdiv(uint32_t(t.G));
+  t.fd_nTX = make_fastdiv(uint32_t(t.nTX));
+  t.fd_tiles = make_fastdiv(uint32_t(t.nTY * t.nTX));
+  t.fd_TW = make_fastdiv(uint32_t(TW));
+  const size_t smem = 2 * size_t(t.box_stride) + fixed;
+  if (smem > size_t(dev.smem_optin)) return DCN_ERR_UNSUPPORTED;
+  args.x = x; args.off = off; args.mask = mask; args.out = out;
+  args.error_word = dev.error_word;
+
+  // Tensor map of the input viewed as (C, W, H, N), innermost first; one box
+  // is (Cg, BW, BH, 1) starting at (g*Cg, X0, Y0, n).  Outside the tensor the
+  // box is zero filled, which is exactly the operator's zero padding.
+  CUtensorMap map;
+  const cuuint64_t dims[4] = {cuuint64_t(t.C), cuuint64_t(t.W), cuuint64_t(t.H),
+                              cuuint64_t(t.N)};
+  const cuuint64_t strides[3] = {cuuint64_t(t.C) * e, cuuint64_t(t.W) * t.C * e,
+                                 cuuint64_t(t.H) * t.W * t.C * e};
+  const cuuint32_t box[4] = {cuuint32_t(t.Cg), cuuint32_t(t.BW), cuuint32_t(t.BH), 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult cr = tensor_map_encoder()(
+      &map, p->dtype == DCN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+      4, const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return DCN_ERR_UNSUPPORTED;
+
+  if (p->dtype == DCN_BF16) {
+    if (cs == 32)
+      return p->softmax ? launch_tiled_kernel<__nv_bfloat16, 32, true>(map, args, smem, dev.sms, stream)
+                        : launch_tiled_kernel<__nv_bfloat16, 32, false>(map, args, smem, dev.sms, stream);
+    return p->softmax ? launch_tiled_kernel<__nv_bfloat16, 64, true>(map, args, smem, dev.sms, stream)
+                      : launch_tiled_kernel<__nv_bfloat16, 64, false>(map, args, smem, dev.sms, stream);
+  }
+  if (cs == 32)
+    return p->softmax ? launch_tiled_kernel<float, 32, true>(map, args, smem, dev.sms, stream)
+                      : launch_tiled_kernel<float, 32, false>(map, args, smem, dev.sms, stream);
+  return p->softmax ? launch_tiled_kernel<float, 64, true>(map, args, smem, dev.sms, stream)
+                    : launch_tiled_kernel<float, 64, false>(map, args, smem, dev.sms, stream);
+}
 }  // namespace
 }  // namespace dcn
 
@@ -266,6 +487,10 @@ dcn_status dcn_core_forward(const dcn_problem* problem, const void* input, const
   if (st != DCN_OK) return st;
   st = check_forward_pointers(problem, input, offset, mask, output);
   if (st != DCN_OK) return st;
+  if (tiled_eligible(problem, Ho, Wo)) {
+    st = forward_tiled(problem, Ho, Wo, input, offset, mask, output, stream);
+    if (st != DCN_ERR_UNSUPPORTED) return st;
+  }
   Plan plan;
   const size_t entry = problem->dtype == DCN_BF16 ? staged_bytes_per_entry<__nv_bfloat16>()
                                                   : staged_bytes_per_entry<float>();
@@ -322,13 +547,10 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
   if (problem->dtype != DCN_F32) return DCN_ERR_UNSUPPORTED;
   st = check_forward_pointers(problem, input, offset, mask, grad_out);
   if (st != DCN_OK) return st;
-  LaneMap lm;
-  lane_map(problem, &lm);
-  const size_t vb = size_t(lm.cpl) * 4;
-  if (!aligned(grad_input, vb) || !aligned(grad_offset, 16) || !aligned(grad_mask, 16))
+  if (!aligned(grad_input, 16) || !aligned(grad_offset, 16) || !aligned(grad_mask, 16))
     return DCN_ERR_UNSUPPORTED;
   Plan plan;
-  st = make_plan(problem, Ho, Wo, staged_bytes_per_entry<float>(), &plan);
+  st = make_plan(problem, Ho, Wo, staged_bytes_per_entry<float>(), &plan, true);
   if (st != DCN_OK) return st;
   const size_t gx_bytes =
       size_t(problem->N) * problem->H * problem->W * problem->G * problem->Cg * sizeof(float);

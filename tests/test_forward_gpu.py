@@ -5,6 +5,9 @@ Small and medium problems are compared in full (they span several tiles and
 ragged tile edges); the full-size workloads, in the launch configuration the
 benchmark times, are compared on sampled units the oracle computes one by one.
 """
+import contextlib
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -33,6 +36,24 @@ def random_case(N, H, W, G, Cg, K=3, stride=1, pad=None, dil=1, sigma=2.0, softm
     else:
         mask = RNG.uniform(-1, 1, (N, Ho, Wo, G * K * K)).astype(np.float32)
     return p, x, off, mask
+
+
+@contextlib.contextmanager
+def forward_path(path):
+    """Select the forward kernel: "auto" (the library's choice: the TMA-tiled
+    kernel where it applies) or "direct" (the direct-gather kernel)."""
+    old = os.environ.get("DCN_CORE_FORWARD")
+    if path == "direct":
+        os.environ["DCN_CORE_FORWARD"] = "direct"
+    else:
+        os.environ.pop("DCN_CORE_FORWARD", None)
+    try:
+        yield
+    finally:
+        if old is None:
+            os.environ.pop("DCN_CORE_FORWARD", None)
+        else:
+            os.environ["DCN_CORE_FORWARD"] = old
 
 
 def check_full(oracle_mod, p, x, off, mask, dtype):
@@ -71,14 +92,36 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["auto", "direct"])
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_" +
                                              "_".join(f"{k}{v}" for k, v in c[5].items())
                                              for c in CASES])
-def test_forward_matches_oracle(oracle_mod, case):
+def test_forward_matches_oracle(oracle_mod, case, path):
     N, H, W, G, Cg, kw = case
     dtype = kw.get("dtype", "f32")
     p, x, off, mask = random_case(N, H, W, G, Cg, **kw)
-    check_full(oracle_mod, p, x, off, mask, dtype)
+    with forward_path(path):
+        check_full(oracle_mod, p, x, off, mask, dtype)
+
+
+@pytest.mark.parametrize("halo,tile", [("0", "1x1"), ("2", "3x5"), ("9", "32x32"), ("5", "7x64")])
+def test_tiled_kernel_tile_and_halo_settings(oracle_mod, halo, tile):
+    """Every tile shape and halo width of the tiled kernel gives the same
+    operator (only the split between box reads and global reads changes)."""
+    old = {k: os.environ.get(k) for k in ("DCN_CORE_HALO", "DCN_CORE_TILED_TILE")}
+    os.environ["DCN_CORE_HALO"], os.environ["DCN_CORE_TILED_TILE"] = halo, tile
+    try:
+        for dtype in ("f32", "bf16"):
+            p, x, off, mask = random_case(2, 37, 41, 3, 16, dtype=dtype, off_sd=3.0)
+            check_full(oracle_mod, p, x, off, mask, dtype)
+            p, x, off, mask = random_case(1, 40, 36, 2, 16, dtype=dtype, stride=2, softmax=0)
+            check_full(oracle_mod, p, x, off, mask, dtype)
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
 
 
 def test_identity_and_box_filter_on_gpu(oracle_mod):
@@ -162,13 +205,15 @@ def sampled_units(wl, imgs, per_img=3000):
 FULL = [n for n, w in WORKLOADS.items() if not w.backward]
 
 
+@pytest.mark.parametrize("path", ["auto", "direct"])
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_workload_sampled(gen_mod, oracle_mod, name):
+def test_full_size_workload_sampled(gen_mod, oracle_mod, name, path):
     wl = WORKLOADS[name]
     d = gen_mod.make_inputs(wl)
     p = dcn.problem_for(wl)
     xd, od, md = to_dev(d["x"], wl.dtype), to_dev(d["offset"], wl.dtype), to_dev(d["mask"], wl.dtype)
-    out = gpu_forward(p, xd, od, md)
+    with forward_path(path):
+        out = gpu_forward(p, xd, od, md)
     torch.cuda.synchronize()
     imgs = sorted({0, wl.N // 2, wl.N - 1})
     units = sampled_units(wl, imgs)
