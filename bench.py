@@ -250,7 +250,10 @@ def run_ours(args, world, rank, local):
     # dominant launch: the longer of forward and backward
     kernels = []
     if fwd_ms > 0:
-        kernels.append(("dcn_forward_kernel", fwd_bytes, fwd_ms))
+        tiled = (os.environ.get("DCN_CORE_FORWARD") != "direct" and wl.K == 3
+                 and wl.Cg * wl.esize in (32, 64))
+        kernels.append(("dcn_forward_tiled_kernel" if tiled else "dcn_forward_kernel",
+                        fwd_bytes, fwd_ms))
     if bwd_ms > 0:
         kernels.append(("dcn_backward_kernel", bwd_bytes, bwd_ms))
     kname, kbytes, kms = max(kernels, key=lambda k: k[2])
