@@ -314,8 +314,9 @@ int env_int(const char* name, int dflt) {
 bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
   const char* mode = std::getenv("DCN_CORE_FORWARD");
   if (mode && std::strcmp(mode, "direct") == 0) return false;
-  const int cs = p->Cg * esize(p->dtype);
-  if (p->K != 3 || (cs != 32 && cs != 64)) return false;
+  // 16 channels per group in either storage type: 32-byte bf16 groups or
+  // 64-byte fp32 groups (eight accumulated values per phase-B lane).
+  if (p->K != 3 || p->Cg != 16) return false;
   if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
   return tensor_map_encoder() != nullptr;
 }
@@ -446,16 +447,9 @@ dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return DCN_ERR_UNSUPPORTED;
 
-  if (p->dtype == DCN_BF16) {
-    if (cs == 32)
-      return p->softmax ? launch_tiled_kernel<__nv_bfloat16, 32, true>(map, args, smem, dev.sms, stream)
-                        : launch_tiled_kernel<__nv_bfloat16, 32, false>(map, args, smem, dev.sms, stream);
-    return p->softmax ? launch_tiled_kernel<__nv_bfloat16, 64, true>(map, args, smem, dev.sms, stream)
-                      : launch_tiled_kernel<__nv_bfloat16, 64, false>(map, args, smem, dev.sms, stream);
-  }
-  if (cs == 32)
-    return p->softmax ? launch_tiled_kernel<float, 32, true>(map, args, smem, dev.sms, stream)
-                      : launch_tiled_kernel<float, 32, false>(map, args, smem, dev.sms, stream);
+  if (p->dtype == DCN_BF16)
+    return p->softmax ? launch_tiled_kernel<__nv_bfloat16, 32, true>(map, args, smem, dev.sms, stream)
+                      : launch_tiled_kernel<__nv_bfloat16, 32, false>(map, args, smem, dev.sms, stream);
   return p->softmax ? launch_tiled_kernel<float, 64, true>(map, args, smem, dev.sms, stream)
                     : launch_tiled_kernel<float, 64, false>(map, args, smem, dev.sms, stream);
 }

@@ -26,7 +26,7 @@
 
 namespace dcn {
 
-constexpr int kTiledWarps = 16;                       // consumer warps
+constexpr int kTiledWarps = 15;  // consumer warps: with the producer, 4 warps per SM sub-partition
 constexpr int kTiledThreads = (kTiledWarps + 1) * 32;  // + one TMA producer warp
 constexpr int kTiledBatch = 32;                       // units per warp batch
 constexpr int kTiledKK = 9;  // the tiled kernel serves 3x3 windows
@@ -222,7 +222,8 @@ __device__ __forceinline__ int far_code(int y0, int x0) {
 constexpr int kSlotBytes = 184;
 constexpr int kCodeAt = kTiledKK * 16;
 constexpr int kLogitAt = 80;               // staged mask values (before the records)
-static_assert(kSlotBytes % 8 == 0 && kCodeAt + kTiledKK * 4 <= kSlotBytes, "slot layout");
+constexpr int kFarMaskAt = kCodeAt + kTiledKK * 4;  // 180: bit k = tap k is read from global
+static_assert(kSlotBytes % 8 == 0 && kFarMaskAt + 4 <= kSlotBytes, "slot layout");
 
 // Phase-B lane roles: 8 lanes per unit, lane li = (corner r = li >> 1, q = li & 1).
 // A 32-byte group (bf16 x 16) is one 16-byte piece per lane: piece q.  A
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         __syncwarp();  // every lane has read its staged inputs
         float* wsl = reinterpret_cast<float*>(sl);
         int* csl = reinterpret_cast<int*>(sl + kCodeAt);
+        unsigned farmask = 0u;
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
           const int ka = k / K, kb = k % K;
@@ -440,7 +442,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           if (!live) code = far_code(kFarCell, kFarCell);
           else if (by >= 0 && by + 1 < t.BH && bx >= 0 && bx + 1 < t.BW)
             code = (by * t.BW + bx) * CS;
-          else code = far_code(f.y0, f.x0);
+          else {
+            code = far_code(f.y0, f.x0);
+            farmask |= 1u << k;
+          }
           const float mk = live ? m[k] : 0.f;
           const float hy = 1.f - f.ly, hx = 1.f - f.lx;
           wsl[4 * k + 0] = hy * hx * mk;
@@ -449,76 +454,129 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           wsl[4 * k + 3] = f.ly * f.lx * mk;
           csl[k] = code;
         }
+        *reinterpret_cast<unsigned*>(sl + kFarMaskAt) = farmask;
       }
       __syncwarp();
       // The next batch's inputs are loaded while this one is gathered.
       if (beta + kTiledWarps < total_batches) prefetch(beta + kTiledWarps);
 
-      // Phase B: UPW units per step, eight lanes each.
+      // Phase B: UPW units per step, eight lanes each.  Box taps are
+      // branch-free (predicated shared-memory reads); a unit's taps whose
+      // footprint leaves the box ("far" taps) read global memory: the first
+      // one of each unit is fetched a step ahead, any further ones in a
+      // warp-uniform loop.
       const int v0 = (beta - il * nb) * kTiledBatch;
+      // Global read of this lane's corner piece(s) for tap k of the unit in slot sl.
+      auto far_fetch = [&](const unsigned char* sl, int k, uint4 (&fv)[NP], float& fw) {
+        const int code = reinterpret_cast<const int*>(sl + kCodeAt)[k];
+        fw = reinterpret_cast<const float*>(sl)[4 * k + r];
+        const int yc = ((code >> 15) & 0x7FFF) - 1 + dyc;
+        const int xc = (code & 0x7FFF) - 1 + dxc;
+        const bool in = unsigned(yc) < unsigned(t.H) && unsigned(xc) < unsigned(t.W);
+        const char* gp = ximg + (size_t(in ? yc : 0) * t.W + (in ? xc : 0)) * pixB;
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          fv[j] = in ? ldg128(gp + Role::piece(j, q, dyc) * 16) : make_uint4(0u, 0u, 0u, 0u);
+        if (!in) fw = 0.f;
+      };
+      auto far_first = [&](int u, uint4 (&fv)[NP], float& fw) {
+        const unsigned char* sl = myslots + u * kSlotBytes;
+        const unsigned fm = *reinterpret_cast<const unsigned*>(sl + kFarMaskAt);
+        fw = 0.f;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) fv[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (fm) far_fetch(sl, __ffs(fm) - 1, fv, fw);
+      };
+      uint4 fv_cur[NP], fv_nxt[NP];
+      float fw_cur, fw_nxt;
+      far_first(ul, fv_cur, fw_cur);
 #pragma unroll 1
       for (int s = 0; s < kTiledBatch / UPW; ++s) {
         const int u = s * UPW + ul;
         const unsigned char* sl = myslots + u * kSlotBytes;
         const float* wsl = reinterpret_cast<const float*>(sl) + r;
         const int* csl = reinterpret_cast<const int*>(sl + kCodeAt);
-        float acc[NP][EPC];
+        if (s + 1 < kTiledBatch / UPW) far_first(u + UPW, fv_nxt, fw_nxt);
+        float acc[NP * EPC];
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-#pragma unroll
-          for (int e = 0; e < EPC; ++e) acc[j][e] = 0.f;
+        for (int e = 0; e < NP * EPC; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
           const int code = csl[k];
           const float w = wsl[4 * k];
-          uint4 val[NP];
-          if (code >= 0) {
+          const bool inbox = code >= 0;
 #pragma unroll
-            for (int j = 0; j < NP; ++j) val[j] = lds128(box + code + cdelta[j]);
-          } else {
-            const int yc = ((code >> 15) & 0x7FFF) - 1 + dyc;
-            const int xc = (code & 0x7FFF) - 1 + dxc;
-            const bool in = unsigned(yc) < unsigned(t.H) && unsigned(xc) < unsigned(t.W);
-            const char* gp = ximg + (size_t(yc) * t.W + xc) * pixB;
+          for (int j = 0; j < NP; ++j) {
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (inbox) val = lds128(box + code + cdelta[j]);
+            IO::fma16(*reinterpret_cast<float(*)[EPC]>(acc + j * EPC), w, val);
+          }
+        }
+        // First far tap (fetched during the previous step), then any others.
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          IO::fma16(*reinterpret_cast<float(*)[EPC]>(acc + j * EPC), fw_cur, fv_cur[j]);
+        unsigned more = *reinterpret_cast<const unsigned*>(sl + kFarMaskAt);
+        more &= more - 1u;
+        while (__any_sync(0xFFFFFFFFu, more != 0u)) {
+          if (more) {
+            uint4 fv[NP];
+            float fw;
+            far_fetch(sl, __ffs(more) - 1, fv, fw);
 #pragma unroll
             for (int j = 0; j < NP; ++j)
-              val[j] = in ? ldg128(gp + Role::piece(j, q, dyc) * 16) : make_uint4(0u, 0u, 0u, 0u);
+              IO::fma16(*reinterpret_cast<float(*)[EPC]>(acc + j * EPC), fw, fv[j]);
+            more &= more - 1u;
           }
-#pragma unroll
-          for (int j = 0; j < NP; ++j) IO::fma16(acc[j], w, val[j]);
         }
         // Lanes with dy = 1 hold their pieces in the other order (fp32 only).
         if (NP == 2 && dyc) {
 #pragma unroll
           for (int e = 0; e < EPC; ++e) {
-            const float tmp = acc[0][e];
-            acc[0][e] = acc[NP - 1][e];
-            acc[NP - 1][e] = tmp;
+            const float tmp = acc[e];
+            acc[e] = acc[EPC + e];
+            acc[EPC + e] = tmp;
           }
         }
-        // Sum the four corner lanes of each piece.
+        // Reduce-scatter over the four corner lanes of each piece: the dx pair
+        // splits the 8 values in halves, the dy pair splits those again, so each
+        // lane ends with 2 summed values: acc index 4*dxc + 2*dyc + {0, 1}.
+        constexpr int NV = NP * EPC;  // 8 values per lane
+        static_assert(NV == 8, "eight accumulated values per lane");
+        float h4[4], h2[2];
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
+        for (int i = 0; i < 4; ++i) {
+          const float keep = dxc ? acc[4 + i] : acc[i];
+          const float send = dxc ? acc[i] : acc[4 + i];
+          h4[i] = keep + __shfl_xor_sync(umask, send, 2);
+        }
 #pragma unroll
-          for (int e = 0; e < EPC; ++e) {
-            acc[j][e] += __shfl_xor_sync(umask, acc[j][e], 2);
-            acc[j][e] += __shfl_xor_sync(umask, acc[j][e], 4);
-          }
+        for (int i = 0; i < 2; ++i) {
+          const float keep = dyc ? h4[2 + i] : h4[i];
+          const float send = dyc ? h4[i] : h4[2 + i];
+          h2[i] = keep + __shfl_xor_sync(umask, send, 4);
+        }
         const int v = v0 + u;
         const int rr = int(fdiv(uint32_t(v), t.fd_TW));
         const int uho = c.ho0 + rr, uwo = c.wo0 + (v - rr * t.TW);
-        if (r == 0 && v < npx && uho < t.Ho && uwo < t.Wo) {
+        if (v < npx && uho < t.Ho && uwo < t.Wo) {
           const size_t pix = size_t(c.n * t.Ho + uho) * t.Wo + uwo;
           char* op = reinterpret_cast<char*>(a.out) + (pix * t.C + size_t(c.g) * t.Cg) * sizeof(T);
-#pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            const uint4 o = IO::pack(acc[j]);
-            asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(
-                             op + Role::piece(j, q, 0) * 16),
-                         "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
+          // channel of h2[0]: piece p, element 2*dyc (+ 4*dxc for bf16's 8-wide pieces)
+          if (CS == 32) {
+            const int ch = 8 * q + 4 * dxc + 2 * dyc;
+            const uint32_t w = pack_bf16x2(h2[0], h2[1]);
+            asm volatile("st.global.b32 [%0], %1;" ::"l"(op + ch * 2), "r"(w) : "memory");
+          } else {
+            const int ch = 4 * (q + 2 * dxc) + 2 * dyc;
+            asm volatile("st.global.v2.f32 [%0], {%1, %2};" ::"l"(op + ch * 4), "f"(h2[0]),
+                         "f"(h2[1])
                          : "memory");
           }
         }
+#pragma unroll
+        for (int j = 0; j < NP; ++j) fv_cur[j] = fv_nxt[j];
+        fw_cur = fw_nxt;
       }
       __syncwarp();  // slots are rewritten by the next batch
     }
