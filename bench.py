@@ -33,7 +33,8 @@ DEFAULT_WORKLOAD = "internimage_l_stage1_fp32_n32_96x96_c160"
 SWEEP = ["internimage_l_stage1_bf16_n64_96x96_c160", "internimage_l_stage2_bf16_n64_48x48_c320",
          "internimage_l_stage3_bf16_n64_24x24_c640", "internimage_l_stage4_bf16_n64_12x12_c1280",
          "dcnv4_hires_bf16_n2_256x256_c192_s1", "dcnv4_hires_bf16_n2_256x256_c192_s2",
-         "internimage_l_stage2_bwd_fp32_n32_48x48_c320"]
+         "internimage_l_stage2_bwd_fp32_n32_48x48_c320",
+         "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 
@@ -159,6 +160,9 @@ class Step:
             self.gx = torch.empty_like(self.x)
             self.goff = torch.empty_like(self.off)
             self.gm = torch.empty_like(self.mask)
+            self.ws_bytes = dcn.dcn_core_backward_workspace(self.p)
+            self.ws = (torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+                       if self.ws_bytes else None)
         self.stream = torch.cuda.Stream()
         self.sh = self.stream.cuda_stream
 
@@ -167,7 +171,7 @@ class Step:
 
     def bwd(self):
         self.dcn.dcn_core_backward(self.p, self.x, self.off, self.mask, self.gout, self.gx,
-                                   self.goff, self.gm, None, 0, self.sh)
+                                   self.goff, self.gm, self.ws, self.ws_bytes, self.sh)
 
     def run(self):
         if not (self.wl.backward and self.backward):

@@ -1,4 +1,5 @@
-// Backward kernel of the deformable-convolution core (sm_100a, fp32).
+// Backward kernel of the deformable-convolution core (sm_100a; fp32 or bf16
+// storage, fp32 arithmetic).
 //
 // Gradients of the forward (InternImage-L DCNv3 explainer (wmrh.cn), section
 // 二 steps 2-4; the DCNv3 extension build guide (trdm.cn), section 2.1, names
@@ -20,15 +21,62 @@
 namespace dcn {
 
 struct BwdArgs {
-  const float* x;
+  const void* x;
   const void* off;
   const void* mask;
-  const float* gout;
-  float* gx;
-  float* goff;
-  float* gmask;
+  const void* gout;
+  float* gx;     // fp32 input-gradient accumulator: grad_input itself for fp32
+                 // storage, the caller's workspace for bf16 storage
+  void* goff;
+  void* gmask;
   TileParams t;
 };
+
+// Four channels of storage type T <-> four floats.
+template <typename T>
+struct Quad;
+template <>
+struct Quad<float> {
+  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
+    Vec<16> w;
+    ldg_nc(w, p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(w.w[i]);
+  }
+  __device__ __forceinline__ static void store_pair(void* base, size_t i, float a, float b) {
+    reinterpret_cast<float2*>(base)[i] = make_float2(a, b);
+  }
+  __device__ __forceinline__ static void store_one(void* base, size_t i, float a) {
+    reinterpret_cast<float*>(base)[i] = a;
+  }
+};
+template <>
+struct Quad<__nv_bfloat16> {
+  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
+    uint32_t w0, w1;
+    asm("ld.global.nc.v2.b32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "l"(p));
+    v[0] = bf16lo_to_f32(w0);
+    v[1] = bf16hi_to_f32(w0);
+    v[2] = bf16lo_to_f32(w1);
+    v[3] = bf16hi_to_f32(w1);
+  }
+  __device__ __forceinline__ static void store_pair(void* base, size_t i, float a, float b) {
+    reinterpret_cast<uint32_t*>(base)[i] = pack_bf16x2(a, b);
+  }
+  __device__ __forceinline__ static void store_one(void* base, size_t i, float a) {
+    reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(a);
+  }
+};
+
+// fp32 accumulator -> bf16 grad_input, rounded to nearest even once.
+__global__ void dcn_round_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out,
+                                         size_t n4) {
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += size_t(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(in + i);
+    out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
 
 template <int LANES>
 __device__ __forceinline__ float unit_sum(float v, unsigned mask) {
@@ -37,12 +85,11 @@ __device__ __forceinline__ float unit_sum(float v, unsigned mask) {
   return v;
 }
 
-template <int CPL, int LANES, int KKS, bool SOFTMAX>
+// A lane owns 4 channels of its unit: LANES = Cg / 4 lanes per unit.
+template <typename T, int LANES, int KKS, bool SOFTMAX>
 __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a) {
-  using St = Staged<float>;
-  constexpr int VB = CPL * 4;
-  static_assert(VB == 16 || VB == 32, "a lane gathers 16 or 32 bytes per corner");
-  using V = Vec<VB>;
+  using St = Staged<T>;
+  constexpr int CPL = 4;
   constexpr int UPW = 32 / LANES;
 
   const TileParams& t = a.t;
@@ -50,11 +97,12 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
   const int GKK = t.G * KK;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  auto* s_off = reinterpret_cast<float2*>(smem_raw);
-  auto* s_msk = reinterpret_cast<float*>(smem_raw + size_t(GKK) * t.P1 * sizeof(float2));
+  auto* s_off = reinterpret_cast<typename St::Pair*>(smem_raw);
+  auto* s_msk = reinterpret_cast<typename St::One*>(smem_raw + size_t(GKK) * t.P1 *
+                                                                   sizeof(typename St::Pair));
 
   const TileCoord tc = tile_coord(t, blockIdx.x);
-  stage_tile<float>(t, tc, KK, a.off, a.mask, s_off, s_msk);
+  stage_tile<T>(t, tc, KK, a.off, a.mask, s_off, s_msk);
   __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -65,25 +113,22 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
   const size_t pixE = size_t(t.C);
   const size_t rowE = size_t(t.W) * pixE;
   const size_t img_off = size_t(tc.n) * t.H * rowE + size_t(sub) * CPL;
+  const char* xbytes = reinterpret_cast<const char*>(a.x);
+  const char* gobytes = reinterpret_cast<const char*>(a.gout);
 
   for (int v0 = warp * UPW; v0 < units; v0 += kWarps * UPW) {
     const UnitCoord u = unit_coord(t, tc, v0 + lane / LANES);
     if (!u.valid) continue;
     const int row0 = u.g * KK;
     const size_t g_off = img_off + size_t(u.g) * t.Cg;
-    const float* xg = a.x + g_off;
+    const char* xg = xbytes + g_off * sizeof(T);
     float* gxg = a.gx + g_off;
     const size_t upix = size_t(tc.n * t.Ho + u.ho) * t.Wo + u.wo;
     const size_t unit = upix * t.G + u.g;
     const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride - t.pad;
 
     float go[CPL];
-    {
-      V gv;
-      ldg_nc(gv, a.gout + upix * t.C + size_t(u.g) * t.Cg + size_t(sub) * CPL);
-#pragma unroll
-      for (int j = 0; j < CPL; ++j) go[j] = __uint_as_float(gv.w[j]);
-    }
+    Quad<T>::load(gobytes + (upix * t.C + size_t(u.g) * t.Cg + size_t(sub) * CPL) * sizeof(T), go);
 
     // One tap: returns s_k (reduced over the unit's lanes) and writes the
     // offset gradient of the tap.
@@ -103,13 +148,11 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
         float dc[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          V cv;
-#pragma unroll
-          for (int i = 0; i < CPL; ++i) cv.w[i] = 0u;
-          if (cval[c]) ldg_nc(cv, xg + cofs[c]);
+          float cv[CPL] = {0.f, 0.f, 0.f, 0.f};
+          if (cval[c]) Quad<T>::load(xg + cofs[c] * ptrdiff_t(sizeof(T)), cv);
           float dsum = 0.f;
 #pragma unroll
-          for (int j = 0; j < CPL; ++j) dsum = fmaf(go[j], __uint_as_float(cv.w[j]), dsum);
+          for (int j = 0; j < CPL; ++j) dsum = fmaf(go[j], cv[j], dsum);
           dc[c] = dsum;
           if (cval[c]) {
             const float wv = mk * cw[c];
@@ -132,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
       }
       if (sub == 0) {
         const float sc = t.sigma * mk;
-        reinterpret_cast<float2*>(a.goff)[unit * KK + k] = make_float2(sc * gX, sc * gY);
+        Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
       }
       return s;
     };
@@ -141,7 +184,7 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
       constexpr int K = KKS == 1 ? 1 : (KKS == 9 ? 3 : (KKS == 25 ? 5 : 7));
       static_assert(K * K == KKS, "compile-time tap counts are odd squares");
       float m[KKS], s[KKS];
-      mask_weights<float, KKS, SOFTMAX>(s_msk, row0, t.P1, u.pix, m);
+      mask_weights<T, KKS, SOFTMAX>(s_msk, row0, t.P1, u.pix, m);
 #pragma unroll
       for (int k = 0; k < KKS; ++k) s[k] = tap(k, k / K, k % K, m[k]);
       if (sub == 0) {
@@ -152,30 +195,35 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
         }
 #pragma unroll
         for (int k = 0; k < KKS; ++k)
-          a.gmask[unit * KK + k] = SOFTMAX ? m[k] * (s[k] - ms) : s[k];
+          Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? m[k] * (s[k] - ms) : s[k]);
       }
     } else {
-      // Runtime tap count: keep (s_k, m_k) in the tap's staged offset slot,
-      // which no other unit reads and this unit no longer needs.
+      // Runtime tap count: keep s_k in the tap's staged offset slot, which no
+      // other unit reads and this unit no longer needs (its mask weight m_k is
+      // recomputed from the staged logit).
       float mx, inv;
-      mask_stats<float, SOFTMAX>(s_msk, row0, t.P1, u.pix, KK, mx, inv);
+      mask_stats<T, SOFTMAX>(s_msk, row0, t.P1, u.pix, KK, mx, inv);
       for (int k = 0, ka = 0, kb = 0; k < KK; ++k) {
-        const float mk = mask_weight_at<float, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv);
+        const float mk = mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv);
         const float sk = tap(k, ka, kb, mk);
         if (LANES > 1) __syncwarp(umask);
-        if (sub == 0) s_off[(row0 + k) * t.P1 + u.pix] = make_float2(sk, mk);
+        if (sub == 0)  // first 4 bytes of the tap's staged pair
+          *reinterpret_cast<float*>(s_off + (row0 + k) * t.P1 + u.pix) = sk;
         if (++kb == t.K) { kb = 0; ++ka; }
       }
       if (sub == 0) {
+        auto s_at = [&](int k) {
+          return *reinterpret_cast<const float*>(s_off + (row0 + k) * t.P1 + u.pix);
+        };
         float ms = 0.f;
         if (SOFTMAX)
-          for (int k = 0; k < KK; ++k) {
-            const float2 sm = s_off[(row0 + k) * t.P1 + u.pix];
-            ms = fmaf(sm.y, sm.x, ms);
-          }
+          for (int k = 0; k < KK; ++k)
+            ms = fmaf(mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv),
+                      s_at(k), ms);
         for (int k = 0; k < KK; ++k) {
-          const float2 sm = s_off[(row0 + k) * t.P1 + u.pix];
-          a.gmask[unit * KK + k] = SOFTMAX ? sm.y * (sm.x - ms) : sm.x;
+          const float sk = s_at(k);
+          const float mk = mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv);
+          Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? mk * (sk - ms) : sk);
         }
       }
     }

@@ -211,16 +211,16 @@ dcn_status forward_dispatch(const dcn_problem* p, const Plan& plan, const FwdArg
   return DCN_ERR_UNSUPPORTED;
 }
 
-template <int CPL, int LANES>
+template <typename T, int LANES>
 dcn_status backward_dispatch_kk(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                                 cudaStream_t stream) {
   const bool k3 = p->K == 3;
   if (p->softmax) {
-    return k3 ? launch(dcn_backward_kernel<CPL, LANES, 9, true>, plan, args, stream)
-              : launch(dcn_backward_kernel<CPL, LANES, 0, true>, plan, args, stream);
+    return k3 ? launch(dcn_backward_kernel<T, LANES, 9, true>, plan, args, stream)
+              : launch(dcn_backward_kernel<T, LANES, 0, true>, plan, args, stream);
   }
-  return k3 ? launch(dcn_backward_kernel<CPL, LANES, 9, false>, plan, args, stream)
-            : launch(dcn_backward_kernel<CPL, LANES, 0, false>, plan, args, stream);
+  return k3 ? launch(dcn_backward_kernel<T, LANES, 9, false>, plan, args, stream)
+            : launch(dcn_backward_kernel<T, LANES, 0, false>, plan, args, stream);
 }
 
 // The backward always gives a lane 4 channels (16 bytes), so that one warp
@@ -236,15 +236,27 @@ bool backward_lane_map(const dcn_problem* p, LaneMap* lm) {
   }
 }
 
-dcn_status backward_dispatch(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
-                             cudaStream_t stream) {
+template <typename T>
+dcn_status backward_dispatch_t(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
+                               cudaStream_t stream) {
   switch (plan.lm.lanes) {
-    case 1: return backward_dispatch_kk<4, 1>(p, plan, args, stream);
-    case 2: return backward_dispatch_kk<4, 2>(p, plan, args, stream);
-    case 4: return backward_dispatch_kk<4, 4>(p, plan, args, stream);
-    case 8: return backward_dispatch_kk<4, 8>(p, plan, args, stream);
+    case 1: return backward_dispatch_kk<T, 1>(p, plan, args, stream);
+    case 2: return backward_dispatch_kk<T, 2>(p, plan, args, stream);
+    case 4: return backward_dispatch_kk<T, 4>(p, plan, args, stream);
+    case 8: return backward_dispatch_kk<T, 8>(p, plan, args, stream);
     default: return DCN_ERR_UNSUPPORTED;
   }
+}
+
+dcn_status backward_dispatch(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
+                             cudaStream_t stream) {
+  return p->dtype == DCN_BF16 ? backward_dispatch_t<__nv_bfloat16>(p, plan, args, stream)
+                              : backward_dispatch_t<float>(p, plan, args, stream);
+}
+
+// Bytes of the fp32 grad_input accumulator that bf16 storage needs.
+size_t bf16_accumulator_bytes(const dcn_problem* p) {
+  return size_t(p->N) * p->H * p->W * p->G * p->Cg * sizeof(float);
 }
 
 dcn_status check_forward_pointers(const dcn_problem* p, const void* x, const void* off,
@@ -523,36 +535,45 @@ dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input
 }
 
 size_t dcn_core_backward_workspace(const dcn_problem* problem) {
-  (void)problem;
-  return 0;
+  int64_t Ho, Wo;
+  if (check_problem(problem, &Ho, &Wo) != DCN_OK) return 0;
+  return problem->dtype == DCN_BF16 ? bf16_accumulator_bytes(problem) : 0;
 }
 
 dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, const void* offset,
                              const void* mask, const void* grad_out, void* grad_input,
                              void* grad_offset, void* grad_mask, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   int64_t Ho, Wo;
   dcn_status st = check_problem(problem, &Ho, &Wo);
   if (st != DCN_OK) return st;
   if (!input || !offset || !mask || !grad_out || !grad_input || !grad_offset || !grad_mask)
     return DCN_ERR_INVALID_ARG;
-  if (problem->dtype != DCN_F32) return DCN_ERR_UNSUPPORTED;
-  st = check_forward_pointers(problem, input, offset, mask, grad_out);
-  if (st != DCN_OK) return st;
-  if (!aligned(grad_input, 16) || !aligned(grad_offset, 16) || !aligned(grad_mask, 16))
+  const bool bf16 = problem->dtype == DCN_BF16;
+  const size_t acc_bytes = bf16_accumulator_bytes(problem);
+  if (bf16 && (!workspace || workspace_bytes < acc_bytes)) return DCN_ERR_INVALID_ARG;
+  if (!aligned(input, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
+      !aligned(grad_out, 16) || !aligned(grad_input, 16) || !aligned(grad_offset, 16) ||
+      !aligned(grad_mask, 16) || (bf16 && !aligned(workspace, 16)))
     return DCN_ERR_UNSUPPORTED;
   Plan plan;
-  st = make_plan(problem, Ho, Wo, staged_bytes_per_entry<float>(), &plan, true);
+  st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
+                                       : staged_bytes_per_entry<float>(),
+                 &plan, true);
   if (st != DCN_OK) return st;
-  const size_t gx_bytes =
-      size_t(problem->N) * problem->H * problem->W * problem->G * problem->Cg * sizeof(float);
-  if (cudaMemsetAsync(grad_input, 0, gx_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
-  BwdArgs args{static_cast<const float*>(input), offset, mask,
-               static_cast<const float*>(grad_out), static_cast<float*>(grad_input),
-               static_cast<float*>(grad_offset), static_cast<float*>(grad_mask), plan.t};
-  return backward_dispatch(problem, plan, args, stream);
+  float* acc = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(grad_input);
+  if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
+  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, plan.t};
+  st = backward_dispatch(problem, plan, args, stream);
+  if (st != DCN_OK || !bf16) return st;
+  // bf16: round the fp32 accumulator once into grad_input.
+  const size_t n4 = acc_bytes / 16;
+  DeviceInfo dev;
+  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
+  const unsigned grid = unsigned(std::min<size_t>((n4 + 255) / 256, size_t(dev.sms) * 8));
+  dcn_round_to_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
+                                                     static_cast<uint2*>(grad_input), n4);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
 }
 
 dcn_status dcn_core_sync_status(cudaStream_t stream) {

@@ -121,6 +121,9 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     # Backward at InternImage-L stage-2 shape, fp32.
     _wl(name="internimage_l_stage2_bwd_fp32_n32_48x48_c320", cfg=5, N=32, H=48, W=48, G=20,
         dtype="f32", Ho=48, Wo=48, backward=True, **_STAGE),
+    # The same backward with bf16 storage (fp32 arithmetic, grad_input accumulated in fp32).
+    _wl(name="internimage_l_stage2_bwd_bf16_n32_48x48_c320", cfg=5, N=32, H=48, W=48, G=20,
+        dtype="bf16", Ho=48, Wo=48, backward=True, **_STAGE),
 ]}
 
 

@@ -30,7 +30,7 @@
  *
  * Errors: arguments are validated on the host before anything is enqueued.
  * Invalid arguments return DCN_ERR_INVALID_ARG, valid but unsupported ones
- * (alignment, channel widths without a kernel, bf16 backward) return
+ * (alignment, channel widths without a kernel) return
  * DCN_ERR_UNSUPPORTED, and a failed launch returns DCN_ERR_CUDA.  On any
  * error nothing has been enqueued.  Device-side failures (a bounded wait
  * that gave up) are reported by dcn_core_sync_status as DCN_ERR_TIMEOUT.
@@ -98,8 +98,8 @@ DCN_API dcn_status dcn_core_output_hw(const dcn_problem* problem, int* Ho, int* 
  * pointers in the layouts above, of problem->dtype; output: device pointer,
  * written entirely.  All four must be 16-byte aligned and must not overlap
  * the output.  Supported channel widths: Cg*sizeof(dtype) a multiple of 16
- * bytes and at most 128 bytes (Cg in {4, 8, 12, ..., 32} for fp32, {8, 16,
- * ..., 64} for bf16); other widths return DCN_ERR_UNSUPPORTED.
+ * bytes and at most 128 bytes: Cg in {4, 8, 16, 32} for fp32, {8, 16, 32,
+ * 64} for bf16; other widths return DCN_ERR_UNSUPPORTED.
  */
 DCN_API dcn_status dcn_core_forward(const dcn_problem* problem, const void* input,
                             const void* offset, const void* mask, void* output,
@@ -118,8 +118,8 @@ DCN_API dcn_status dcn_core_forward_host(const dcn_problem* problem, const void*
                                  void* h_output, void* d_input, void* d_offset,
                                  void* d_mask, void* d_output, cudaStream_t stream);
 
-/* Device workspace the backward needs, in bytes (0 for the current
- * atomic-scatter backward). */
+/* Device workspace the backward needs, in bytes: 0 for fp32 storage; for
+ * bf16 storage an fp32 accumulator for grad_input, N*H*W*G*Cg*4 bytes. */
 DCN_API size_t dcn_core_backward_workspace(const dcn_problem* problem);
 
 /*
@@ -131,9 +131,13 @@ DCN_API size_t dcn_core_backward_workspace(const dcn_problem* problem);
  *   grad_mask   (N, Ho, Wo, G*KK), overwritten; with softmax = 1 it is the
  *               gradient with respect to the logits
  * The gradient with respect to an offset at an integer sample coordinate is
- * the one-sided derivative that floor() selects.  Only fp32 storage is
- * supported (bf16 returns DCN_ERR_UNSUPPORTED); channel widths and alignment
- * as for the forward.  workspace may be NULL when the workspace size is 0.
+ * the one-sided derivative that floor() selects.  All gradients are computed
+ * in fp32.  With bf16 storage the input gradient is accumulated in the
+ * caller's workspace (dcn_core_backward_workspace bytes, 16-byte aligned,
+ * contents on entry irrelevant) and rounded to bf16 once at the end; grad
+ * offset and grad mask are rounded once.  Cg must be 4, 8, 16 or 32; all
+ * pointers 16-byte aligned.  workspace may be NULL when the workspace size
+ * is 0; a missing or short workspace returns DCN_ERR_INVALID_ARG.
  */
 DCN_API dcn_status dcn_core_backward(const dcn_problem* problem, const void* input,
                              const void* offset, const void* mask,

@@ -103,10 +103,17 @@ def test_backward_rejects_before_launch(lib):
             dcn.dcn_core_backward(p, *bad, None, 0, 0)
         assert e.value.status == dcn.DCN_ERR_INVALID_ARG
     pb = dcn.make_problem(**{**GOOD, "dtype": "bf16"})
-    with pytest.raises(dcn.DcnError) as e:
-        dcn.dcn_core_backward(pb, *ptrs, None, 0, 0)
-    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    need = dcn.dcn_core_backward_workspace(pb)
+    assert need == 1 * 8 * 8 * 2 * 16 * 4          # fp32 accumulator for grad_input
+    for ws, nbytes in [(None, 0), (FAKE, need - 16)]:  # bf16 needs the full workspace
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_backward(pb, *ptrs, ws, nbytes, 0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
     assert dcn.dcn_core_backward_workspace(p) == 0
+    pc = dcn.make_problem(**{**GOOD, "Cg": 12})
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward(pc, *ptrs, None, 0, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
 
 
 def test_forward_host_rejects_before_copy(lib):

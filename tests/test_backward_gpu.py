@@ -33,14 +33,16 @@ def near_kink_taps(p, off):
     return int(near.sum())
 
 
-def check(oracle_mod, p, x, off, mask, gout):
-    xd, od, md, gd = (to_dev(a, "f32") for a in (x, off, mask, gout))
+def check(oracle_mod, p, x, off, mask, gout, dtype="f32"):
+    xd, od, md, gd = (to_dev(a, dtype) for a in (x, off, mask, gout))
     gx, goff, gm = gpu_backward(p, xd, od, md, gd)
     torch.cuda.synchronize()
-    rx, roff, rm = oracle_mod.backward(x, off, mask, gout, **problem_kwargs(p))
-    assert_bwd(f64(gx), rx, f"grad_input {p}")
-    assert_bwd(f64(goff), roff, f"grad_offset {p} (near-kink taps: {near_kink_taps(p, off)})")
-    assert_bwd(f64(gm), rm, f"grad_mask {p}")
+    # the oracle sees exactly the values the GPU saw (bf16-rounded for bf16)
+    rx, roff, rm = oracle_mod.backward(f64(xd), f64(od), f64(md), f64(gd), **problem_kwargs(p))
+    assert_bwd(f64(gx), rx, f"grad_input {p}", dtype)
+    assert_bwd(f64(goff), roff, f"grad_offset {p} (near-kink taps: {near_kink_taps(p, f64(od))})",
+               dtype)
+    assert_bwd(f64(gm), rm, f"grad_mask {p}", dtype)
     return gx, goff, gm
 
 
@@ -59,21 +61,24 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_" +
                                              "_".join(f"{k}{v}" for k, v in c[5].items())
                                              for c in CASES])
-def test_backward_matches_oracle(oracle_mod, case):
+def test_backward_matches_oracle(oracle_mod, case, dtype):
     N, H, W, G, Cg, kw = case
+    if dtype == "bf16" and Cg * 2 < 16:
+        pytest.skip("bf16 needs Cg >= 8")
     kw = {"K": 3, "stride": 1, "pad": 1, "dilation": 1, "softmax": 1, **kw}
     p = dcn.make_problem(N, H, W, G, Cg, kw["K"], kw["stride"], kw["pad"], kw["dilation"],
-                         2.0, kw["softmax"], "f32")
+                         2.0, kw["softmax"], dtype)
     Ho, Wo = dcn.dcn_core_output_hw(p)
     KK = kw["K"] ** 2
     x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
     off = (1.5 * RNG.standard_normal((N, Ho, Wo, G * KK * 2))).astype(np.float32)
     mask = RNG.standard_normal((N, Ho, Wo, G * KK)).astype(np.float32)
     gout = RNG.standard_normal((N, Ho, Wo, G * Cg)).astype(np.float32)
-    check(oracle_mod, p, x, off, mask, gout)
+    check(oracle_mod, p, x, off, mask, gout, dtype)
 
 
 def test_full_size_backward(gen_mod, oracle_mod):
@@ -107,3 +112,10 @@ def test_backward_rerun_differs_only_by_rounding(gen_mod):
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     # the input gradient sums atomically: equal up to the order of additions
     assert torch.allclose(a[0], b[0], rtol=0, atol=1e-5 * float(a[0].abs().max()))
+
+
+def test_full_size_backward_bf16(gen_mod, oracle_mod):
+    wl = WORKLOADS["internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
+    d = gen_mod.make_inputs(wl)
+    p = dcn.problem_for(wl)
+    check(oracle_mod, p, d["x"], d["offset"], d["mask"], d["grad_out"], "bf16")
