@@ -19,6 +19,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdcncore.so")
 
 DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
+# Scratch the allocation-free backward owns per GPU (DCN_CORE_NOALLOC_SCRATCH_BYTES).
+DCN_CORE_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 DCN_F32, DCN_BF16 = 0, 1
 
 # Every entry point of include/dcn_core.h.
@@ -28,6 +30,7 @@ EXPORTED_SYMBOLS = (
     "dcn_core_forward_host",
     "dcn_core_backward_workspace",
     "dcn_core_backward",
+    "dcn_core_backward_noalloc",
     "dcn_core_sync_status",
     "dcn_status_string",
     "dcn_core_abi_version",
@@ -96,6 +99,8 @@ def load_library():
     lib.dcn_core_backward_workspace.restype = ctypes.c_size_t
     lib.dcn_core_backward.argtypes = [pp] + [vp] * 8 + [ctypes.c_size_t, vp]
     lib.dcn_core_backward.restype = st
+    lib.dcn_core_backward_noalloc.argtypes = [pp] + [vp] * 8
+    lib.dcn_core_backward_noalloc.restype = st
     lib.dcn_core_sync_status.argtypes = [vp]
     lib.dcn_core_sync_status.restype = st
     lib.dcn_status_string.argtypes = [st]
@@ -174,11 +179,30 @@ def dcn_core_backward(problem: DcnProblem, input, offset, mask, grad_out, grad_i
         int(workspace_bytes), _stream(stream)), "dcn_core_backward")
 
 
+def dcn_core_backward_noalloc(problem: DcnProblem, input, offset, mask, grad_out, grad_input,
+                              grad_offset, grad_mask, stream=None) -> None:
+    """Backward without a workspace, for callers that cannot allocate device
+    memory (see include/dcn_core.h).  For bf16 storage the fp32 grad_input
+    accumulator must fit the library's fixed DCN_CORE_NOALLOC_SCRATCH_BYTES
+    array; calls that may overlap on the GPU must be serialised."""
+    status = load_library().dcn_core_backward_noalloc(
+        ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
+        _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _stream(stream))
+    if status == DCN_ERR_UNSUPPORTED and problem.dtype == DCN_BF16:
+        need = problem.N * problem.H * problem.W * problem.G * problem.Cg * 4
+        if need > DCN_CORE_NOALLOC_SCRATCH_BYTES:
+            raise DcnError(status, f"dcn_core_backward_noalloc: the bf16 accumulator needs {need} "
+                                   f"bytes, more than the {DCN_CORE_NOALLOC_SCRATCH_BYTES} bytes "
+                                   "of scratch this entry point owns")
+    _check(status, "dcn_core_backward_noalloc")
+
+
 def dcn_core_sync_status(stream=None) -> None:
     _check(load_library().dcn_core_sync_status(_stream(stream)), "dcn_core_sync_status")
 
 
 __all__ = ["DcnProblem", "DcnError", "make_problem", "problem_for", "load_library",
            "library_path", "EXPORTED_SYMBOLS", *EXPORTED_SYMBOLS,
+           "DCN_CORE_NOALLOC_SCRATCH_BYTES",
            "DCN_OK", "DCN_ERR_INVALID_ARG", "DCN_ERR_UNSUPPORTED", "DCN_ERR_CUDA",
            "DCN_ERR_TIMEOUT", "DCN_F32", "DCN_BF16"]

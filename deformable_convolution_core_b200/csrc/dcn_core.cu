@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "dcn_backward.cuh"
 #include "dcn_forward.cuh"
@@ -604,3 +605,83 @@ const char* dcn_status_string(dcn_status status) {
 int dcn_core_abi_version(void) { return DCN_CORE_ABI_VERSION; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free backward (dcn_core_backward_noalloc in include/dcn_core.h).
+// ---------------------------------------------------------------------------
+namespace dcn {
+namespace {
+
+// The bf16 backward's fp32 grad_input accumulator, owned by the library.  In
+// host code this name is only a stand-in for the device array: the kernels
+// get the device address that cudaGetSymbolAddress returns for the current
+// device.
+static __device__ __align__(256) float
+    g_noalloc_scratch[DCN_CORE_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+dcn_status noalloc_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices)
+    return DCN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return DCN_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return DCN_OK;
+}
+
+}  // namespace
+}  // namespace dcn
+
+extern "C" dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, const void* input,
+                                                const void* offset, const void* mask,
+                                                const void* grad_out, void* grad_input,
+                                                void* grad_offset, void* grad_mask,
+                                                cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!input || !offset || !mask || !grad_out || !grad_input || !grad_offset || !grad_mask)
+    return DCN_ERR_INVALID_ARG;
+  if (!aligned(input, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
+      !aligned(grad_out, 16) || !aligned(grad_input, 16) || !aligned(grad_offset, 16) ||
+      !aligned(grad_mask, 16))
+    return DCN_ERR_UNSUPPORTED;
+  const bool bf16 = problem->dtype == DCN_BF16;
+  const size_t acc_bytes = bf16_accumulator_bytes(problem);  // fp32 grad_input size
+  if (bf16 && acc_bytes > size_t(DCN_CORE_NOALLOC_SCRATCH_BYTES)) return DCN_ERR_UNSUPPORTED;
+  Plan plan;
+  st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
+                                       : staged_bytes_per_entry<float>(),
+                 &plan, true);
+  if (st != DCN_OK) return st;
+  float* acc = static_cast<float*>(grad_input);
+  if (bf16) {
+    void* scratch = nullptr;
+    st = noalloc_scratch_address(&scratch);
+    if (st != DCN_OK) return st;
+    acc = static_cast<float*>(scratch);
+  }
+  // The shared array keeps the previous call's sums: clear it first.
+  if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
+  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, plan.t};
+  st = backward_dispatch(problem, plan, args, stream);
+  if (st != DCN_OK || !bf16) return st;
+  const size_t n4 = acc_bytes / 16;
+  DeviceInfo dev;
+  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
+  const unsigned grid = unsigned(std::min<size_t>((n4 + 255) / 256, size_t(dev.sms) * 8));
+  dcn_round_to_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
+                                                     static_cast<uint2*>(grad_input), n4);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}

@@ -145,6 +145,36 @@ DCN_API dcn_status dcn_core_backward(const dcn_problem* problem, const void* inp
                              void* grad_offset, void* grad_mask, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream);
 
+/* Scratch bytes the allocation-free backward below owns, per GPU (16 MiB). */
+#define DCN_CORE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * Backward that allocates nothing and takes no workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory where they run the backward -- plugin hosts and inference
+ * runtimes that give a custom operator only its input and output buffers
+ * (the runtime owns every other byte of device memory), and latency-critical
+ * code that may not call cudaMalloc because it synchronises the device.
+ *
+ * Arguments and results are those of dcn_core_backward without the
+ * workspace.  fp32 storage needs no scratch.  For bf16 storage the fp32
+ * grad_input accumulator (N*H*W*G*Cg*4 bytes) lives in a fixed array inside
+ * the library of DCN_CORE_NOALLOC_SCRATCH_BYTES; every GPU that loads the
+ * library holds that array until the process exits, and a bf16 problem whose
+ * accumulator is larger returns DCN_ERR_UNSUPPORTED without enqueuing work.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current): make that first call before any stream
+ * capture.  Every call shares the one array and each call clears it on its
+ * stream before use; calls whose work can overlap on the GPU (other streams,
+ * other host threads on the same device) race on it and must be serialised
+ * by the caller.  Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+DCN_API dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, const void* input,
+                                             const void* offset, const void* mask,
+                                             const void* grad_out, void* grad_input,
+                                             void* grad_offset, void* grad_mask,
+                                             cudaStream_t stream);
+
 /* Synchronises `stream` and reports: DCN_ERR_CUDA if CUDA reports an error,
  * DCN_ERR_TIMEOUT if a kernel of this library gave up a bounded wait since
  * the last call (the device error word is then cleared), else DCN_OK. */
