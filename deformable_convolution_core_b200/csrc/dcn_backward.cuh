@@ -87,7 +87,7 @@ __device__ __forceinline__ float unit_sum(float v, unsigned mask) {
 
 // A lane owns 4 channels of its unit: LANES = Cg / 4 lanes per unit.
 template <typename T, int LANES, int KKS, bool SOFTMAX>
-__global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs a) {
   using St = Staged<T>;
   constexpr int CPL = 4;
   constexpr int UPW = 32 / LANES;
@@ -185,8 +185,74 @@ __global__ void __launch_bounds__(kThreads) dcn_backward_kernel(const BwdArgs a)
       static_assert(K * K == KKS, "compile-time tap counts are odd squares");
       float m[KKS], s[KKS];
       mask_weights<T, KKS, SOFTMAX>(s_msk, row0, t.P1, u.pix, m);
+      // Taps in groups of three, without branches: the group's twelve corner
+      // gathers are issued together (predicated on the corner lying in the
+      // image), then reduced; the per-tap partial sums stay in registers and
+      // are summed over the unit's lanes once, after the last tap.
+      constexpr int GRP = 3;
+      static_assert(KKS % GRP == 0, "taps come in groups of three");
 #pragma unroll
-      for (int k = 0; k < KKS; ++k) s[k] = tap(k, k / K, k % K, m[k]);
+      for (int k0 = 0; k0 < KKS; k0 += GRP) {
+        Footprint f[GRP];
+        float cv[GRP][4][CPL];
+        int cofs[GRP][4];  // element offsets within the image (< 2^31)
+        bool cval[GRP][4];
+#pragma unroll
+        for (int j = 0; j < GRP; ++j) {
+          const int k = k0 + j;
+          const float2 d = St::pair(s_off[(row0 + k) * t.P1 + u.pix]);
+          const float Y = tap_coord(by + (k / K) * t.dil, t.sigma, d.y);
+          const float X = tap_coord(bx + (k % K) * t.dil, t.sigma, d.x);
+          f[j] = footprint(Y, X, t.H, t.W);
+          const int base = f[j].y0 * int(rowE) + f[j].x0 * int(pixE);
+          cofs[j][0] = base;
+          cofs[j][1] = base + int(pixE);
+          cofs[j][2] = base + int(rowE);
+          cofs[j][3] = base + int(rowE + pixE);
+          cval[j][0] = f[j].v00;
+          cval[j][1] = f[j].v01;
+          cval[j][2] = f[j].v10;
+          cval[j][3] = f[j].v11;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int e = 0; e < CPL; ++e) cv[j][c][e] = 0.f;
+            if (cval[j][c]) Quad<T>::load(xg + ptrdiff_t(cofs[j][c]) * ptrdiff_t(sizeof(T)), cv[j][c]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < GRP; ++j) {
+          const int k = k0 + j;
+          const float hy = 1.f - f[j].ly, hx = 1.f - f[j].lx;
+          const float cw[4] = {hy * hx, hy * f[j].lx, f[j].ly * hx, f[j].ly * f[j].lx};
+          float dc[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float dsum = 0.f;
+#pragma unroll
+            for (int e = 0; e < CPL; ++e) dsum = fmaf(go[e], cv[j][c][e], dsum);
+            dc[c] = dsum;
+            if (cval[j][c]) {
+              const float wv = m[k] * cw[c];
+              atomicAdd(reinterpret_cast<float4*>(gxg + ptrdiff_t(cofs[j][c])),
+                        make_float4(wv * go[0], wv * go[1], wv * go[2], wv * go[3]));
+            }
+          }
+          // out-of-support samples have no valid corner: every dc is 0
+          s[k] = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];
+          float gX = hy * (dc[1] - dc[0]) + f[j].ly * (dc[3] - dc[2]);
+          float gY = hx * (dc[2] - dc[0]) + f[j].lx * (dc[3] - dc[1]);
+          if (LANES > 1) {
+            s[k] = unit_sum<LANES>(s[k], umask);
+            gX = unit_sum<LANES>(gX, umask);
+            gY = unit_sum<LANES>(gY, umask);
+          }
+          if (sub == 0) {
+            const float sc = t.sigma * m[k];
+            Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
+          }
+        }
+      }
       if (sub == 0) {
         float ms = 0.f;
         if (SOFTMAX) {

@@ -145,14 +145,6 @@ __device__ __forceinline__ ItemCoord item_coord(const TiledParams& t, int item) 
   return c;
 }
 
-// acc.lo += w * x0, acc.hi += w * x1 as one packed fp32x2 FMA (sm_100).
-__device__ __forceinline__ void fma2(float& a0, float& a1, float w, float x0, float x1) {
-  asm("{\n .reg .b64 ra, rx, rw;\n mov.b64 ra, {%0, %1};\n mov.b64 rx, {%2, %3};\n"
-      " mov.b64 rw, {%4, %4};\n fma.rn.f32x2 ra, rx, rw, ra;\n mov.b64 {%0, %1}, ra;\n}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(x0), "f"(x1), "f"(w));
-}
-
 template <typename T>
 struct TiledIO;
 template <>
@@ -168,9 +160,10 @@ struct TiledIO<float> {
   }
   __device__ __forceinline__ static float2 pair(Pair p) { return p; }
   __device__ __forceinline__ static float one(One v) { return v; }
-  __device__ __forceinline__ static void fma16(float (&acc)[4], float w, const uint4& v) {
-    fma2(acc[0], acc[1], w, __uint_as_float(v.x), __uint_as_float(v.y));
-    fma2(acc[2], acc[3], w, __uint_as_float(v.z), __uint_as_float(v.w));
+  // acc += w * (the piece's 4 channels), as two packed fp32x2 FMAs.
+  __device__ __forceinline__ static void fma16(float2* acc, float2 w, const uint4& v) {
+    acc[0] = __ffma2_rn(make_float2(__uint_as_float(v.x), __uint_as_float(v.y)), w, acc[0]);
+    acc[1] = __ffma2_rn(make_float2(__uint_as_float(v.z), __uint_as_float(v.w)), w, acc[1]);
   }
   __device__ __forceinline__ static uint4 pack(const float (&acc)[4]) {
     return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
@@ -192,11 +185,12 @@ struct TiledIO<__nv_bfloat16> {
     return make_float2(bf16lo_to_f32(p), bf16hi_to_f32(p));
   }
   __device__ __forceinline__ static float one(One v) { return __uint_as_float(uint32_t(v) << 16); }
-  __device__ __forceinline__ static void fma16(float (&acc)[8], float w, const uint4& v) {
-    fma2(acc[0], acc[1], w, bf16lo_to_f32(v.x), bf16hi_to_f32(v.x));
-    fma2(acc[2], acc[3], w, bf16lo_to_f32(v.y), bf16hi_to_f32(v.y));
-    fma2(acc[4], acc[5], w, bf16lo_to_f32(v.z), bf16hi_to_f32(v.z));
-    fma2(acc[6], acc[7], w, bf16lo_to_f32(v.w), bf16hi_to_f32(v.w));
+  // acc += w * (the piece's 8 channels, widened), as four packed fp32x2 FMAs.
+  __device__ __forceinline__ static void fma16(float2* acc, float2 w, const uint4& v) {
+    acc[0] = __ffma2_rn(make_float2(bf16lo_to_f32(v.x), bf16hi_to_f32(v.x)), w, acc[0]);
+    acc[1] = __ffma2_rn(make_float2(bf16lo_to_f32(v.y), bf16hi_to_f32(v.y)), w, acc[1]);
+    acc[2] = __ffma2_rn(make_float2(bf16lo_to_f32(v.z), bf16hi_to_f32(v.z)), w, acc[2]);
+    acc[3] = __ffma2_rn(make_float2(bf16lo_to_f32(v.w), bf16hi_to_f32(v.w)), w, acc[3]);
   }
   __device__ __forceinline__ static uint4 pack(const float (&acc)[8]) {
     return make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
@@ -497,25 +491,28 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         const float* wsl = reinterpret_cast<const float*>(sl) + r;
         const int* csl = reinterpret_cast<const int*>(sl + kCodeAt);
         if (s + 1 < kTiledBatch / UPW) far_first(u + UPW, fv_nxt, fw_nxt);
-        float acc[NP * EPC];
+        constexpr int NV = NP * EPC;  // 8 values per lane, as 4 packed pairs
+        static_assert(NV == 8, "eight accumulated values per lane");
+        float2 acc[NV / 2];
 #pragma unroll
-        for (int e = 0; e < NP * EPC; ++e) acc[e] = 0.f;
+        for (int e = 0; e < NV / 2; ++e) acc[e] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
           const int code = csl[k];
           const float w = wsl[4 * k];
+          const float2 w2 = make_float2(w, w);
           const bool inbox = code >= 0;
 #pragma unroll
           for (int j = 0; j < NP; ++j) {
             uint4 val = make_uint4(0u, 0u, 0u, 0u);
             if (inbox) val = lds128(box + code + cdelta[j]);
-            IO::fma16(*reinterpret_cast<float(*)[EPC]>(acc + j * EPC), w, val);
+            IO::fma16(acc + j * (EPC / 2), w2, val);
           }
         }
         // First far tap (fetched during the previous step), then any others.
 #pragma unroll
         for (int j = 0; j < NP; ++j)
-          IO::fma16(*reinterpret_cast<float(*)[EPC]>(acc + j * EPC), fw_cur, fv_cur[j]);
+          IO::fma16(acc + j * (EPC / 2), make_float2(fw_cur, fw_cur), fv_cur[j]);
         unsigned more = *reinterpret_cast<const unsigned*>(sl + kFarMaskAt);
         more &= more - 1u;
         while (__any_sync(0xFFFFFFFFu, more != 0u)) {
@@ -524,30 +521,29 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
             float fw;
             far_fetch(sl, __ffs(more) - 1, fv, fw);
 #pragma unroll
-            for (int j = 0; j < NP; ++j)
-              IO::fma16(*reinterpret_cast<float(*)[EPC]>(acc + j * EPC), fw, fv[j]);
+            for (int j = 0; j < NP; ++j) IO::fma16(acc + j * (EPC / 2), make_float2(fw, fw), fv[j]);
             more &= more - 1u;
           }
         }
         // Lanes with dy = 1 hold their pieces in the other order (fp32 only).
         if (NP == 2 && dyc) {
 #pragma unroll
-          for (int e = 0; e < EPC; ++e) {
-            const float tmp = acc[e];
-            acc[e] = acc[EPC + e];
-            acc[EPC + e] = tmp;
+          for (int e = 0; e < EPC / 2; ++e) {
+            const float2 tmp = acc[e];
+            acc[e] = acc[EPC / 2 + e];
+            acc[EPC / 2 + e] = tmp;
           }
         }
         // Reduce-scatter over the four corner lanes of each piece: the dx pair
         // splits the 8 values in halves, the dy pair splits those again, so each
-        // lane ends with 2 summed values: acc index 4*dxc + 2*dyc + {0, 1}.
-        constexpr int NV = NP * EPC;  // 8 values per lane
-        static_assert(NV == 8, "eight accumulated values per lane");
+        // lane ends with 2 summed values: value index 4*dxc + 2*dyc + {0, 1}.
         float h4[4], h2[2];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float keep = dxc ? acc[4 + i] : acc[i];
-          const float send = dxc ? acc[i] : acc[4 + i];
+          const float lo = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;           // value i
+          const float hi = (i & 1) ? acc[2 + (i >> 1)].y : acc[2 + (i >> 1)].x;  // value 4 + i
+          const float keep = dxc ? hi : lo;
+          const float send = dxc ? lo : hi;
           h4[i] = keep + __shfl_xor_sync(umask, send, 2);
         }
 #pragma unroll
