@@ -121,6 +121,18 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------------------
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings over the process group (the
+    identity at one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def dist_setup(args):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -237,11 +249,7 @@ def run_ours(args, world, rank, local):
     time.sleep(0.25)
     clock_summary = clocks.summary()
     clocks.stop()
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms, fwd_ms, bwd_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, fwd_ms, bwd_ms = (float(v) for v in t.tolist())
+    total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], "cuda")
     ms_per_step = total_ms / args.steps
 
     fwd_bytes = wl.forward_bytes() if not wl.backward else 0
@@ -359,12 +367,7 @@ def run_e2e(step, inputs, args, barrier, world):
         one()
     t1.record(s)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / n
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([t0.elapsed_time(t1) / n], "cuda")[0]
     step_bytes = (wl.forward_bytes() if fwd_only else 0) + (wl.backward_bytes() if step.backward else 0)
     return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
