@@ -99,8 +99,8 @@ def draw(seed: int, tensor_id: int, shape, dist) -> np.ndarray:
 def make_inputs(wl: Workload | str, seed: int | None = None, n_images: int | None = None,
                 with_grad_out: bool | None = None) -> dict:
     """Host float32 arrays for one workload: x (N,H,W,G*Cg), offset
-    (N,Ho,Wo,G*K*K*2) as (dx, dy) pairs, mask (N,Ho,Wo,G*K*K) and, for
-    backward workloads, grad_out (N,Ho,Wo,G*Cg).
+    (N,Ho,Wo,G*T*2) as (dx, dy) pairs, mask (N,Ho,Wo,G*T) with T = wl.KK taps
+    per (pixel, group), and, for backward workloads, grad_out (N,Ho,Wo,G*Cg).
 
     ``n_images`` generates only the first n images of the batch; because the
     generator is counter-based these are bit-identical to the leading images
@@ -111,7 +111,7 @@ def make_inputs(wl: Workload | str, seed: int | None = None, n_images: int | Non
     seed = wl.seed if seed is None else seed
     N = wl.N if n_images is None else n_images
     Ho, Wo = output_hw(wl)
-    C, KK = wl.G * wl.Cg, wl.K * wl.K
+    C, KK = wl.G * wl.Cg, wl.KK
 
     def gen_prefix(tid, full_shape, dist):
         # Draw the full tensor's first N images only: same values as the full draw.

@@ -38,6 +38,7 @@ class Workload:
     mask_dist: tuple = ("normal", 0.0, 1.0)
     far: tuple | None = None  # (fraction of (dx,dy) pairs, lo, hi) redrawn from U(lo, hi)
     backward: bool = False
+    remove_center: int = 0    # 1: the window's centre is not sampled (DCNv4), K*K - 1 taps
     seed_base: int = 1000
     tags: tuple = field(default_factory=tuple)
 
@@ -51,7 +52,8 @@ class Workload:
 
     @property
     def KK(self) -> int:
-        return self.K * self.K
+        """Taps per (pixel, group): the K x K window, less its centre with remove_center."""
+        return self.K * self.K - self.remove_center
 
     @property
     def units(self) -> int:
@@ -118,6 +120,11 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     _wl(name="dcnv4_hires_bf16_n2_256x256_c192_s2", cfg=4, N=2, H=256, W=256, G=12, Cg=16,
         K=3, stride=2, pad=1, dilation=1, offset_scale=1.0, softmax=0, dtype="bf16",
         Ho=128, Wo=128, offset_dist=("normal", 0.0, 2.0), mask_dist=("uniform", -1.0, 1.0)),
+    # The same forward without the centre tap (DCNv4's remove_center: 8 taps).
+    _wl(name="dcnv4_hires_bf16_n2_256x256_c192_s1_remove_center", cfg=4, N=2, H=256, W=256,
+        G=12, Cg=16, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0, softmax=0,
+        dtype="bf16", Ho=256, Wo=256, offset_dist=("normal", 0.0, 2.0),
+        mask_dist=("uniform", -1.0, 1.0), remove_center=1),
     # Backward at InternImage-L stage-2 shape, fp32.
     _wl(name="internimage_l_stage2_bwd_fp32_n32_48x48_c320", cfg=5, N=32, H=48, W=48, G=20,
         dtype="f32", Ho=48, Wo=48, backward=True, **_STAGE),

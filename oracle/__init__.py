@@ -45,7 +45,7 @@ def _load():
         dp = ctypes.POINTER(ctypes.c_double)
         i64p = ctypes.POINTER(ctypes.c_int64)
         ci, cd, i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
-        shape = [ci] * 9 + [cd, ci, ci]
+        shape = [ci] * 9 + [cd, ci, ci, ci]
         lib.oracle_output_extent.argtypes = [ci] * 5
         lib.oracle_output_extent.restype = ci
         lib.oracle_forward.argtypes = [dp] * 4 + shape
@@ -80,15 +80,23 @@ def output_hw(H, W, K, stride, pad, dil):
     return output_extent(H, K, stride, pad, dil), output_extent(W, K, stride, pad, dil)
 
 
-def _shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd):
+def taps(K: int, remove_center=0) -> int:
+    """Taps per (pixel, group): the K x K window, less its centre with
+    remove_center (DCNv4 speed-up write-up (pnsm.cn), section 3.3)."""
+    return K * K - (1 if remove_center else 0)
+
+
+def _shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd, remove_center):
     return (int(N), int(H), int(W), int(G), int(Cg), int(K), int(stride), int(pad),
-            int(dil), float(offset_scale), int(softmax), int(bool(fd)))
+            int(dil), float(offset_scale), int(softmax), int(bool(fd)),
+            int(bool(remove_center)))
 
 
 def forward(x, offset, mask, *, G, K=3, stride=1, pad=1, dil=1, offset_scale=1.0,
-            softmax=1, fd=False) -> np.ndarray:
-    """Forward of the whole problem.  x: (N,H,W,G*Cg), offset: (N,Ho,Wo,G*K*K*2),
-    mask: (N,Ho,Wo,G*K*K).  Returns float64 (N,Ho,Wo,G*Cg)."""
+            softmax=1, fd=False, remove_center=0) -> np.ndarray:
+    """Forward of the whole problem.  x: (N,H,W,G*Cg), offset: (N,Ho,Wo,G*T*2),
+    mask: (N,Ho,Wo,G*T) with T = taps(K, remove_center).  Returns float64
+    (N,Ho,Wo,G*Cg)."""
     x, offset, mask = _d(x), _d(offset), _d(mask)
     N, H, W, C = x.shape
     Cg = C // G
@@ -96,17 +104,18 @@ def forward(x, offset, mask, *, G, K=3, stride=1, pad=1, dil=1, offset_scale=1.0
     out = np.zeros((N, Ho, Wo, C), dtype=np.float64)
     if out.size == 0:
         return out
-    assert offset.shape == (N, Ho, Wo, G * K * K * 2), offset.shape
-    assert mask.shape == (N, Ho, Wo, G * K * K), mask.shape
+    T = taps(K, remove_center)
+    assert offset.shape == (N, Ho, Wo, G * T * 2), offset.shape
+    assert mask.shape == (N, Ho, Wo, G * T), mask.shape
     rc = _load().oracle_forward(_p(x), _p(offset), _p(mask), _p(out),
                                 *_shape_args(N, H, W, G, Cg, K, stride, pad, dil,
-                                             offset_scale, softmax, fd))
+                                             offset_scale, softmax, fd, remove_center))
     assert rc == 0, rc
     return out
 
 
 def forward_units(x, offset, mask, units, *, G, K=3, stride=1, pad=1, dil=1,
-                  offset_scale=1.0, softmax=1, fd=False) -> np.ndarray:
+                  offset_scale=1.0, softmax=1, fd=False, remove_center=0) -> np.ndarray:
     """Forward outputs of selected units u = ((n*Ho+ho)*Wo+wo)*G+g only.
     Returns float64 (len(units), Cg)."""
     x, offset, mask = _d(x), _d(offset), _d(mask)
@@ -117,13 +126,14 @@ def forward_units(x, offset, mask, units, *, G, K=3, stride=1, pad=1, dil=1,
     rc = _load().oracle_forward_units(
         _p(x), _p(offset), _p(mask), units.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
         units.size, _p(out),
-        *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd))
+        *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd,
+                     remove_center))
     assert rc == 0, rc
     return out
 
 
 def backward(x, offset, mask, grad_out, *, G, K=3, stride=1, pad=1, dil=1,
-             offset_scale=1.0, softmax=1, fd=False):
+             offset_scale=1.0, softmax=1, fd=False, remove_center=0):
     """Returns float64 (grad_input, grad_offset, grad_mask); grad_mask is the
     gradient with respect to the logits when softmax=1."""
     x, offset, mask, grad_out = _d(x), _d(offset), _d(mask), _d(grad_out)
@@ -134,26 +144,27 @@ def backward(x, offset, mask, grad_out, *, G, K=3, stride=1, pad=1, dil=1,
     gm = np.zeros_like(mask)
     rc = _load().oracle_backward(_p(x), _p(offset), _p(mask), _p(grad_out), _p(gx), _p(goff),
                                  _p(gm), *_shape_args(N, H, W, G, Cg, K, stride, pad, dil,
-                                                      offset_scale, softmax, fd))
+                                                      offset_scale, softmax, fd, remove_center))
     assert rc == 0, rc
     return gx, goff, gm
 
 
 def backward_units(x, offset, mask, grad_out, units, *, G, K=3, stride=1, pad=1, dil=1,
-                   offset_scale=1.0, softmax=1, fd=False):
+                   offset_scale=1.0, softmax=1, fd=False, remove_center=0):
     """Offset and mask gradients of selected units.  Returns float64
-    (goff (len, K*K*2), gmask (len, K*K))."""
+    (goff (len, T*2), gmask (len, T)), T = taps(K, remove_center)."""
     x, offset, mask, grad_out = _d(x), _d(offset), _d(mask), _d(grad_out)
     N, H, W, C = x.shape
     Cg = C // G
-    KK = K * K
+    KK = taps(K, remove_center)
     units = np.ascontiguousarray(np.asarray(units, dtype=np.int64))
     goff = np.zeros((units.size, KK * 2), dtype=np.float64)
     gm = np.zeros((units.size, KK), dtype=np.float64)
     rc = _load().oracle_backward_units(
         _p(x), _p(offset), _p(mask), _p(grad_out),
         units.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), units.size, _p(goff), _p(gm),
-        *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd))
+        *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd,
+                     remove_center))
     assert rc == 0, rc
     return goff, gm
 
@@ -161,4 +172,5 @@ def backward_units(x, offset, mask, grad_out, units, *, G, K=3, stride=1, pad=1,
 def workload_kwargs(wl) -> dict:
     """Keyword arguments of forward()/backward() for a gen.Workload."""
     return dict(G=wl.G, K=wl.K, stride=wl.stride, pad=wl.pad, dil=wl.dilation,
-                offset_scale=wl.offset_scale, softmax=wl.softmax)
+                offset_scale=wl.offset_scale, softmax=wl.softmax,
+                remove_center=getattr(wl, "remove_center", 0))

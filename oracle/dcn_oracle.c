@@ -35,15 +35,20 @@
  *    CUDA path does, so both land in the same floor cell; in "fd" mode
  *    (fd = 1) everything is double, for finite differences;
  *  - the gradient at an integer coordinate is the one-sided derivative that
- *    floor() selects (corners x0 = X and X + 1).
+ *    floor() selects (corners x0 = X and X + 1);
+ *  - remove_center (a DCNv4 module argument, DCNv4 speed-up write-up
+ *    (pnsm.cn), section 3.3, which drops the centre sampling point): the taps
+ *    are the K x K window positions in row-major order with the centre
+ *    position (K/2, K/2) left out, so there are T = K*K - 1 of them and
+ *    offset and mask carry T entries per group; without it T = K*K.
  *
  * All accumulation is in double.  Inputs are double arrays holding the exact
  * values of the fp32 / bf16 tensors the CUDA path sees.
  *
- * Layouts (element indices, C = G*Cg, KK = K*K):
+ * Layouts (element indices, C = G*Cg, T taps per group):
  *   x      ((n*H + y)*W + x)*C + g*Cg + c
- *   offset ((n*Ho + ho)*Wo + wo)*(G*KK*2) + (g*KK + k)*2 + {0: dx, 1: dy}
- *   mask   ((n*Ho + ho)*Wo + wo)*(G*KK) + g*KK + k
+ *   offset ((n*Ho + ho)*Wo + wo)*(G*T*2) + (g*T + k)*2 + {0: dx, 1: dy}
+ *   mask   ((n*Ho + ho)*Wo + wo)*(G*T) + g*T + k
  *   out    ((n*Ho + ho)*Wo + wo)*C + g*Cg + c
  */
 #include <math.h>
@@ -53,8 +58,9 @@
 
 typedef struct {
   int64_t N, H, W, G, Cg, K, stride, pad, dil, Ho, Wo;
+  int64_t T; /* taps per (pixel, group) */
   double sigma;
-  int softmax, fd;
+  int softmax, fd, remove_center;
 } prob_t;
 
 /* Output extent of a convolution grid; 0 when no tap window fits. */
@@ -65,17 +71,42 @@ int oracle_output_extent(int in, int K, int stride, int pad, int dil) {
 }
 
 static prob_t make_prob(int N, int H, int W, int G, int Cg, int K, int stride,
-                        int pad, int dil, double sigma, int softmax, int fd) {
+                        int pad, int dil, double sigma, int softmax, int fd,
+                        int remove_center) {
   prob_t p;
   p.N = N; p.H = H; p.W = W; p.G = G; p.Cg = Cg; p.K = K;
   p.stride = stride; p.pad = pad; p.dil = dil;
   p.Ho = oracle_output_extent(H, K, stride, pad, dil);
   p.Wo = oracle_output_extent(W, K, stride, pad, dil);
   p.sigma = sigma; p.softmax = softmax; p.fd = fd;
+  p.remove_center = remove_center != 0;
+  p.T = (int64_t)K * K - p.remove_center;
   return p;
 }
 
-/* Mask weights of one (pixel, group): softmax over the KK taps (DCNv3,
+/* A problem the oracle can evaluate: a non-empty output and at least one tap. */
+static int usable(const prob_t* p) { return p->Ho > 0 && p->Wo > 0 && p->T > 0; }
+
+/* Window position (a, b) of tap j: the K x K positions are listed row by
+ * row, skipping the centre when remove_center is set, and tap j is the j-th
+ * entry of that list. */
+static void tap_position(const prob_t* p, int64_t j, int64_t* a, int64_t* b) {
+  int64_t listed = 0;
+  *a = *b = 0;
+  for (int64_t r = 0; r < p->K; ++r) {
+    for (int64_t c = 0; c < p->K; ++c) {
+      if (p->remove_center && r == p->K / 2 && c == p->K / 2) continue;
+      if (listed == j) {
+        *a = r;
+        *b = c;
+        return;
+      }
+      ++listed;
+    }
+  }
+}
+
+/* Mask weights of one (pixel, group): softmax over its KK taps (DCNv3,
  * explainer section 二 step 3) or the raw values (DCNv4). */
 static void mask_weights(const double* logits, int64_t KK, int softmax, double* m) {
   if (!softmax) {
@@ -123,7 +154,7 @@ static const double* pixel_ptr(const prob_t* p, const double* t, int64_t n,
 static void forward_unit(const prob_t* p, const double* x, const double* off,
                          const double* mask, int64_t n, int64_t ho, int64_t wo,
                          int64_t g, double* out_c) {
-  const int64_t KK = p->K * p->K;
+  const int64_t KK = p->T;
   const int64_t pix = (n * p->Ho + ho) * p->Wo + wo;
   const double* o = off + pix * (p->G * KK * 2) + g * KK * 2;
   const double* l = mask + pix * (p->G * KK) + g * KK;
@@ -131,7 +162,8 @@ static void forward_unit(const prob_t* p, const double* x, const double* off,
   mask_weights(l, KK, p->softmax, m);
   for (int64_t c = 0; c < p->Cg; ++c) out_c[c] = 0.0;
   for (int64_t k = 0; k < KK; ++k) {
-    const int64_t a = k / p->K, b = k % p->K;
+    int64_t a, b;
+    tap_position(p, k, &a, &b);
     double Y, X;
     location(p, ho, wo, a, b, o[2 * k], o[2 * k + 1], &Y, &X);
     if (!in_support(p, Y, X)) continue;
@@ -152,15 +184,16 @@ static void forward_unit(const prob_t* p, const double* x, const double* off,
 }
 
 /*
- * Full forward.  x: (N,H,W,G*Cg); offset: (N,Ho,Wo,G*K*K*2);
- * mask: (N,Ho,Wo,G*K*K); out: (N,Ho,Wo,G*Cg).  Returns 0, or -1 when the
- * output would be empty.
+ * Full forward.  x: (N,H,W,G*Cg); offset: (N,Ho,Wo,G*T*2); mask: (N,Ho,Wo,G*T)
+ * with T = K*K - remove_center; out: (N,Ho,Wo,G*Cg).  Returns 0, or -1 when
+ * the output would be empty or there is no tap.
  */
 int oracle_forward(const double* x, const double* offset, const double* mask,
                    double* out, int N, int H, int W, int G, int Cg, int K,
-                   int stride, int pad, int dil, double sigma, int softmax, int fd) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd);
-  if (p.Ho <= 0 || p.Wo <= 0) return -1;
+                   int stride, int pad, int dil, double sigma, int softmax, int fd,
+                   int remove_center) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+  if (!usable(&p)) return -1;
   for (int64_t n = 0; n < p.N; ++n)
     for (int64_t ho = 0; ho < p.Ho; ++ho)
       for (int64_t wo = 0; wo < p.Wo; ++wo)
@@ -177,9 +210,9 @@ int oracle_forward(const double* x, const double* offset, const double* mask,
 int oracle_forward_units(const double* x, const double* offset, const double* mask,
                          const int64_t* units, int64_t n_units, double* out, int N,
                          int H, int W, int G, int Cg, int K, int stride, int pad,
-                         int dil, double sigma, int softmax, int fd) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd);
-  if (p.Ho <= 0 || p.Wo <= 0) return -1;
+                         int dil, double sigma, int softmax, int fd, int remove_center) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+  if (!usable(&p)) return -1;
   for (int64_t i = 0; i < n_units; ++i) {
     int64_t u = units[i];
     int64_t g = u % p.G, pix = u / p.G;
@@ -193,7 +226,7 @@ int oracle_forward_units(const double* x, const double* offset, const double* ma
 
 /*
  * Backward of one unit.  Writes the unit's offset and mask gradients
- * (goff: KK*2 values, gmask: KK values) and, when gx != NULL, adds the
+ * (goff: T*2 values, gmask: T values) and, when gx != NULL, adds the
  * unit's contribution to the input gradient.
  *
  *   v_k[c]   = B(x[.,.,g,c]; Y_k, X_k)                      (unweighted sample)
@@ -208,7 +241,7 @@ static void backward_unit(const prob_t* p, const double* x, const double* off,
                           const double* mask, const double* gout, int64_t n,
                           int64_t ho, int64_t wo, int64_t g, double* gx,
                           double* goff_u, double* gmask_u) {
-  const int64_t KK = p->K * p->K, C = p->G * p->Cg;
+  const int64_t KK = p->T, C = p->G * p->Cg;
   const int64_t pix = (n * p->Ho + ho) * p->Wo + wo;
   const double* o = off + pix * (p->G * KK * 2) + g * KK * 2;
   const double* l = mask + pix * (p->G * KK) + g * KK;
@@ -217,7 +250,8 @@ static void backward_unit(const prob_t* p, const double* x, const double* off,
   double* s = (double*)malloc(sizeof(double) * (size_t)KK);
   mask_weights(l, KK, p->softmax, m);
   for (int64_t k = 0; k < KK; ++k) {
-    const int64_t a = k / p->K, b = k % p->K;
+    int64_t a, b;
+    tap_position(p, k, &a, &b);
     double Y, X;
     location(p, ho, wo, a, b, o[2 * k], o[2 * k + 1], &Y, &X);
     s[k] = 0.0;
@@ -269,10 +303,11 @@ static void backward_unit(const prob_t* p, const double* x, const double* off,
 int oracle_backward(const double* x, const double* offset, const double* mask,
                     const double* grad_out, double* grad_input, double* grad_offset,
                     double* grad_mask, int N, int H, int W, int G, int Cg, int K,
-                    int stride, int pad, int dil, double sigma, int softmax, int fd) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd);
-  if (p.Ho <= 0 || p.Wo <= 0) return -1;
-  const int64_t KK = p.K * p.K;
+                    int stride, int pad, int dil, double sigma, int softmax, int fd,
+                    int remove_center) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+  if (!usable(&p)) return -1;
+  const int64_t KK = p.T;
   memset(grad_input, 0, sizeof(double) * (size_t)(p.N * p.H * p.W * p.G * p.Cg));
   for (int64_t n = 0; n < p.N; ++n)
     for (int64_t ho = 0; ho < p.Ho; ++ho)
@@ -286,15 +321,15 @@ int oracle_backward(const double* x, const double* offset, const double* mask,
 }
 
 /* Offset and mask gradients of selected units (no input gradient).
- * goff: (n_units, KK*2), gmask: (n_units, KK). */
+ * goff: (n_units, T*2), gmask: (n_units, T). */
 int oracle_backward_units(const double* x, const double* offset, const double* mask,
                           const double* grad_out, const int64_t* units, int64_t n_units,
                           double* goff, double* gmask, int N, int H, int W, int G,
                           int Cg, int K, int stride, int pad, int dil, double sigma,
-                          int softmax, int fd) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd);
-  if (p.Ho <= 0 || p.Wo <= 0) return -1;
-  const int64_t KK = p.K * p.K;
+                          int softmax, int fd, int remove_center) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+  if (!usable(&p)) return -1;
+  const int64_t KK = p.T;
   for (int64_t i = 0; i < n_units; ++i) {
     int64_t u = units[i];
     int64_t g = u % p.G, pix = u / p.G;

@@ -82,6 +82,63 @@ def test_zero_init_is_box_filter(oracle_mod):
     np.testing.assert_allclose(out, box, rtol=0, atol=1e-14)
 
 
+@pytest.mark.parametrize("K", [3, 5])
+def test_zero_init_without_centre_is_ring_mean(oracle_mod, K):
+    # With remove_center (DCNv4 speed-up write-up (pnsm.cn), section 3.3) the
+    # centre point is not sampled: zero offsets and equal logits average the
+    # K*K - 1 other window positions, zero-padded.
+    N, H, W, G, Cg = 2, 6, 5, 2, 3
+    r = K // 2
+    x = rand(N, H, W, G * Cg)
+    T = K * K - 1
+    off = np.zeros((N, H, W, G * T * 2))
+    logits = np.full((N, H, W, G * T), 0.3)
+    out = oracle_mod.forward(x, off, logits, G=G, K=K, pad=r, softmax=1, offset_scale=2.0,
+                             remove_center=1)
+    xp = np.pad(x, ((0, 0), (r, r), (r, r), (0, 0)))
+    ring = sum(xp[:, i:i + H, j:j + W, :] for i in range(K) for j in range(K)
+               if (i, j) != (r, r)) / T
+    np.testing.assert_allclose(out, ring, rtol=0, atol=1e-14)
+    # the raw-mask variant with weight 1 per tap: the ring sum
+    out4 = oracle_mod.forward(x, off, np.ones_like(logits), G=G, K=K, pad=r, softmax=0,
+                              offset_scale=2.0, remove_center=1)
+    np.testing.assert_allclose(out4, ring * T, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("softmax", [0, 1])
+def test_remove_center_is_full_window_with_centre_weight_zero(oracle_mod, softmax):
+    # Dropping the centre tap equals keeping it with a zero weight: a raw
+    # mask of 0 (DCNv4) or a logit of -inf (DCNv3 softmax), whatever its offset.
+    N, H, W, G, Cg, K = 2, 7, 6, 3, 4, 3
+    c = (K * K) // 2
+    x = rand(N, H, W, G * Cg)
+    off8 = rand(N, H, W, G, K * K - 1, 2, lo=-2.5, hi=2.5)
+    m8 = rand(N, H, W, G, K * K - 1, lo=-2, hi=2)
+    gout = rand(N, H, W, G * Cg)
+    off9 = np.insert(off8, c, rand(N, H, W, G, 2, lo=-3, hi=3), axis=4)
+    m9 = np.insert(m8, c, -np.inf if softmax else 0.0, axis=4)
+    kw = dict(G=G, K=K, offset_scale=2.0, softmax=softmax)
+    a8 = (off8.reshape(N, H, W, -1), m8.reshape(N, H, W, -1))
+    a9 = (off9.reshape(N, H, W, -1), m9.reshape(N, H, W, -1))
+    f8 = oracle_mod.forward(x, *a8, remove_center=1, **kw)
+    f9 = oracle_mod.forward(x, *a9, **kw)
+    assert np.array_equal(f8, f9)
+    gx8, go8, gm8 = oracle_mod.backward(x, *a8, gout, remove_center=1, **kw)
+    gx9, go9, gm9 = oracle_mod.backward(x, *a9, gout, **kw)
+    assert np.array_equal(gx8, gx9)
+    keep = [k for k in range(K * K) if k != c]
+    assert np.array_equal(go8.reshape(N, H, W, G, -1, 2), go9.reshape(N, H, W, G, -1, 2)[..., keep, :])
+    assert np.array_equal(gm8.reshape(N, H, W, G, -1), gm9.reshape(N, H, W, G, -1)[..., keep])
+
+
+def test_remove_center_needs_a_tap(oracle_mod):
+    # K = 1 without its centre has no tap left: the oracle refuses it.
+    x = np.zeros((1, 3, 3, 2))
+    with pytest.raises(AssertionError):
+        oracle_mod.forward(x, np.zeros((1, 3, 3, 0)), np.zeros((1, 3, 3, 0)), G=1, K=1, pad=0,
+                           remove_center=1)
+
+
 # --- P3 integer offsets = exact shifts ---------------------------------------------
 
 @pytest.mark.parametrize("stride,dil,sigma", [(1, 1, 2.0), (2, 1, 1.0), (1, 2, 1.0), (2, 2, 2.0)])
@@ -144,19 +201,27 @@ def test_half_pixel_is_mean_of_neighbours(oracle_mod):
 
 # --- P6 brute force through torch grid_sample -------------------------------------
 
-@pytest.mark.parametrize("softmax,stride", [(1, 1), (0, 1), (1, 2)])
-def test_grid_sample_brute_force(oracle_mod, softmax, stride):
-    N, H, W, G, Cg, K = 2, 7, 8, 2, 3, 3
-    pad, dil, sigma = 1, 1, 2.0
+@pytest.mark.parametrize("softmax,stride,K,remove_center",
+                         [(1, 1, 3, 0), (0, 1, 3, 0), (1, 2, 3, 0), (1, 1, 3, 1), (0, 2, 3, 1),
+                          (1, 1, 5, 1)])
+def test_grid_sample_brute_force(oracle_mod, softmax, stride, K, remove_center):
+    N, H, W, G, Cg = 2, 7, 8, 2, 3
+    pad, dil, sigma = K // 2, 1, 2.0
+    # The window positions, row-major; remove_center (DCNv4 speed-up write-up
+    # (pnsm.cn), section 3.3) leaves the centre out of the list.
+    window = [(a, b) for a in range(K) for b in range(K)
+              if not (remove_center and a == K // 2 and b == K // 2)]
+    T = len(window)
     Ho, Wo = oracle_mod.output_hw(H, W, K, stride, pad, dil)
     x = rand(N, H, W, G * Cg)
-    off = rand(N, Ho, Wo, G * K * K * 2, lo=-2.5, hi=2.5)   # many samples cross the border
-    mask = rand(N, Ho, Wo, G * K * K, lo=-2, hi=2)
+    off = rand(N, Ho, Wo, G * T * 2, lo=-2.5, hi=2.5)   # many samples cross the border
+    mask = rand(N, Ho, Wo, G * T, lo=-2, hi=2)
     got = oracle_mod.forward(x, off, mask, G=G, K=K, stride=stride, pad=pad, dil=dil,
-                             offset_scale=sigma, softmax=softmax, fd=True)
+                             offset_scale=sigma, softmax=softmax, fd=True,
+                             remove_center=remove_center)
     xt = torch.from_numpy(x).reshape(N, H, W, G, Cg)
-    o = torch.from_numpy(off).reshape(N, Ho, Wo, G, K * K, 2)
-    m = torch.from_numpy(mask).reshape(N, Ho, Wo, G, K * K)
+    o = torch.from_numpy(off).reshape(N, Ho, Wo, G, T, 2)
+    m = torch.from_numpy(mask).reshape(N, Ho, Wo, G, T)
     if softmax:
         m = torch.softmax(m, dim=-1)
     ref = torch.zeros(N, Ho, Wo, G, Cg, dtype=torch.float64)
@@ -164,8 +229,7 @@ def test_grid_sample_brute_force(oracle_mod, softmax, stride):
     ww = torch.arange(Wo, dtype=torch.float64).view(1, Wo)
     for g in range(G):
         img = xt[:, :, :, g, :].permute(0, 3, 1, 2)          # (N, Cg, H, W)
-        for k in range(K * K):
-            a, b = divmod(k, K)
+        for k, (a, b) in enumerate(window):
             Y = hh * stride - pad + a * dil + sigma * o[:, :, :, g, k, 1]
             X = ww * stride - pad + b * dil + sigma * o[:, :, :, g, k, 0]
             grid = torch.stack([(2 * X + 1) / W - 1, (2 * Y + 1) / H - 1], dim=-1)
@@ -229,31 +293,28 @@ def test_groups_are_independent(oracle_mod):
 
 # --- P10 finite differences ---------------------------------------------------------
 
-def kink_free_offsets(N, Ho, Wo, G, K, stride, pad, dil, sigma, H, W):
-    """Offsets whose sample coordinates have fractional parts in [0.05, 0.95]
-    and stay at least one pixel inside... or outside... the image border, so
-    that no finite-difference stencil crosses a floor() boundary."""
-    KK = K * K
-    off = np.zeros((N, Ho, Wo, G, KK, 2))
-    for idx in np.ndindex(N, Ho, Wo, G, KK):
-        n, ho, wo, g, k = idx
-        a, b = divmod(k, K)
-        for comp, base in ((0, wo * stride - pad + b * dil), (1, ho * stride - pad + a * dil)):
-            shift = RNG.integers(-2, 3) + RNG.uniform(0.05, 0.95)
-            off[idx + (comp,)] = (shift) / sigma
-    return off.reshape(N, Ho, Wo, -1)
+def kink_free_offsets(N, Ho, Wo, G, T, sigma):
+    """Offsets of T taps whose sample coordinates have fractional parts in
+    [0.05, 0.95] (grid points are integers, so the offset alone sets the
+    fraction), so that no finite-difference stencil crosses a floor()
+    boundary."""
+    shift = RNG.integers(-2, 3, size=(N, Ho, Wo, G, T, 2)) + \
+        RNG.uniform(0.05, 0.95, size=(N, Ho, Wo, G, T, 2))
+    return (shift / sigma).reshape(N, Ho, Wo, -1)
 
 
-@pytest.mark.parametrize("softmax,stride", [(1, 1), (0, 1), (1, 2)])
-def test_backward_matches_finite_differences(oracle_mod, softmax, stride):
+@pytest.mark.parametrize("softmax,stride,remove_center",
+                         [(1, 1, 0), (0, 1, 0), (1, 2, 0), (1, 1, 1), (0, 2, 1)])
+def test_backward_matches_finite_differences(oracle_mod, softmax, stride, remove_center):
     N, H, W, G, Cg, K, pad, dil, sigma = 1, 5, 5, 2, 4, 3, 1, 1, 2.0
+    T = K * K - remove_center
     Ho, Wo = oracle_mod.output_hw(H, W, K, stride, pad, dil)
     x = rand(N, H, W, G * Cg)
-    off = kink_free_offsets(N, Ho, Wo, G, K, stride, pad, dil, sigma, H, W)
-    m = rand(N, Ho, Wo, G * K * K, lo=-1.5, hi=1.5)
+    off = kink_free_offsets(N, Ho, Wo, G, T, sigma)
+    m = rand(N, Ho, Wo, G * T, lo=-1.5, hi=1.5)
     gout = rand(N, Ho, Wo, G * Cg)
     kw = dict(G=G, K=K, stride=stride, pad=pad, dil=dil, offset_scale=sigma,
-              softmax=softmax, fd=True)
+              softmax=softmax, fd=True, remove_center=remove_center)
     gx, goff, gm = oracle_mod.backward(x, off, m, gout, **kw)
 
     def L(xx, oo, mm):
