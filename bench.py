@@ -33,6 +33,7 @@ DEFAULT_WORKLOAD = "internimage_l_stage1_fp32_n32_96x96_c160"
 SWEEP = ["internimage_l_stage1_bf16_n64_96x96_c160", "internimage_l_stage2_bf16_n64_48x48_c320",
          "internimage_l_stage3_bf16_n64_24x24_c640", "internimage_l_stage4_bf16_n64_12x12_c1280",
          "dcnv4_hires_bf16_n2_256x256_c192_s1", "dcnv4_hires_bf16_n2_256x256_c192_s2",
+         "dcnv4_hires_bf16_n2_256x256_c192_s1_remove_center",
          "internimage_l_stage2_bwd_fp32_n32_48x48_c320",
          "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
 FALLBACK_HBM_GBS = 6650.0
@@ -263,7 +264,7 @@ def run_ours(args, world, rank, local):
     kernels = []
     if fwd_ms > 0:
         tiled = (os.environ.get("DCN_CORE_FORWARD") != "direct" and wl.K == 3
-                 and wl.Cg * wl.esize in (32, 64))
+                 and wl.Cg == 16 and not wl.remove_center)
         kernels.append(("dcn_forward_tiled_kernel" if tiled else "dcn_forward_kernel",
                         fwd_bytes, fwd_ms))
     if bwd_ms > 0:
@@ -288,7 +289,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
                    "N": wl.N, "H": wl.H, "W": wl.W, "G": wl.G, "Cg": wl.Cg, "K": wl.K,
                    "stride": wl.stride, "offset_scale": wl.offset_scale,
-                   "softmax": wl.softmax, "per_gpu_batch": wl.N,
+                   "softmax": wl.softmax, "remove_center": wl.remove_center,
+                   "per_gpu_batch": wl.N,
                    "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB touched per step, "
                          "no flush between steps"},

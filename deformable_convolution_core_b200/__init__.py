@@ -18,6 +18,8 @@ import os
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdcncore.so")
 
+# DCN_CORE_ABI_VERSION of include/dcn_core.h that DcnProblem mirrors.
+ABI_VERSION = 2
 DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
 # Scratch the allocation-free backward owns per GPU (DCN_CORE_NOALLOC_SCRATCH_BYTES).
 DCN_CORE_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -49,25 +51,32 @@ class DcnProblem(ctypes.Structure):
                 ("G", ctypes.c_int), ("Cg", ctypes.c_int), ("K", ctypes.c_int),
                 ("stride", ctypes.c_int), ("pad", ctypes.c_int), ("dilation", ctypes.c_int),
                 ("offset_scale", ctypes.c_float), ("softmax", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("remove_center", ctypes.c_int)]
 
     def __repr__(self):
         return "DcnProblem(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
 def make_problem(N, H, W, G, Cg, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0,
-                 softmax=1, dtype="f32") -> DcnProblem:
+                 softmax=1, dtype="f32", remove_center=0) -> DcnProblem:
     if isinstance(dtype, str):
         dtype = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16, "bfloat16": DCN_BF16}[dtype]
     return DcnProblem(int(N), int(H), int(W), int(G), int(Cg), int(K), int(stride), int(pad),
-                      int(dilation), float(offset_scale), int(softmax), int(dtype))
+                      int(dilation), float(offset_scale), int(softmax), int(dtype),
+                      int(remove_center))
 
 
 def problem_for(wl) -> DcnProblem:
     """DcnProblem of a workload description (any object with the fields of
     gen.workloads.Workload)."""
     return make_problem(wl.N, wl.H, wl.W, wl.G, wl.Cg, wl.K, wl.stride, wl.pad, wl.dilation,
-                        wl.offset_scale, wl.softmax, wl.dtype)
+                        wl.offset_scale, wl.softmax, wl.dtype,
+                        getattr(wl, "remove_center", 0))
+
+
+def taps(problem: DcnProblem) -> int:
+    """Taps per (pixel, group): K*K, or K*K - 1 with remove_center."""
+    return problem.K * problem.K - (1 if problem.remove_center else 0)
 
 
 _lib = None
@@ -107,6 +116,9 @@ def load_library():
     lib.dcn_status_string.restype = ctypes.c_char_p
     lib.dcn_core_abi_version.argtypes = []
     lib.dcn_core_abi_version.restype = ctypes.c_int
+    if lib.dcn_core_abi_version() != ABI_VERSION:
+        raise ImportError(f"{LIB_PATH} has ABI version {lib.dcn_core_abi_version()}, this binding "
+                          f"expects {ABI_VERSION}: rebuild it")
     _lib = lib
     return lib
 
@@ -201,8 +213,8 @@ def dcn_core_sync_status(stream=None) -> None:
     _check(load_library().dcn_core_sync_status(_stream(stream)), "dcn_core_sync_status")
 
 
-__all__ = ["DcnProblem", "DcnError", "make_problem", "problem_for", "load_library",
-           "library_path", "EXPORTED_SYMBOLS", *EXPORTED_SYMBOLS,
+__all__ = ["DcnProblem", "DcnError", "make_problem", "problem_for", "taps", "load_library",
+           "library_path", "EXPORTED_SYMBOLS", *EXPORTED_SYMBOLS, "ABI_VERSION",
            "DCN_CORE_NOALLOC_SCRATCH_BYTES",
            "DCN_OK", "DCN_ERR_INVALID_ARG", "DCN_ERR_UNSUPPORTED", "DCN_ERR_CUDA",
            "DCN_ERR_TIMEOUT", "DCN_F32", "DCN_BF16"]

@@ -181,16 +181,14 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
     };
 
     if constexpr (KKS > 0) {
-      constexpr int K = KKS == 1 ? 1 : (KKS == 9 ? 3 : (KKS == 25 ? 5 : 7));
-      static_assert(K * K == KKS, "compile-time tap counts are odd squares");
+      constexpr int K = tap_side(KKS);
       float m[KKS], s[KKS];
       mask_weights<T, KKS, SOFTMAX>(s_msk, row0, t.P1, u.pix, m);
-      // Taps in groups of three, without branches: the group's twelve corner
-      // gathers are issued together (predicated on the corner lying in the
-      // image), then reduced; the per-tap partial sums stay in registers and
-      // are summed over the unit's lanes once, after the last tap.
-      constexpr int GRP = 3;
-      static_assert(KKS % GRP == 0, "taps come in groups of three");
+      // Taps in groups of three (two for the 8-tap set), without branches:
+      // the group's corner gathers are issued together (predicated on the
+      // corner lying in the image), then reduced and scattered.
+      constexpr int GRP = KKS % 3 == 0 ? 3 : 2;
+      static_assert(KKS % GRP == 0, "the tap set splits into whole groups");
 #pragma unroll
       for (int k0 = 0; k0 < KKS; k0 += GRP) {
         Footprint f[GRP];
@@ -201,8 +199,9 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
         for (int j = 0; j < GRP; ++j) {
           const int k = k0 + j;
           const float2 d = St::pair(s_off[(row0 + k) * t.P1 + u.pix]);
-          const float Y = tap_coord(by + (k / K) * t.dil, t.sigma, d.y);
-          const float X = tap_coord(bx + (k % K) * t.dil, t.sigma, d.x);
+          const int q = tap_pos(KKS, k);  // window position of tap k
+          const float Y = tap_coord(by + (q / K) * t.dil, t.sigma, d.y);
+          const float X = tap_coord(bx + (q % K) * t.dil, t.sigma, d.x);
           f[j] = footprint(Y, X, t.H, t.W);
           const int base = f[j].y0 * int(rowE) + f[j].x0 * int(pixE);
           cofs[j][0] = base;
@@ -270,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
       float mx, inv;
       mask_stats<T, SOFTMAX>(s_msk, row0, t.P1, u.pix, KK, mx, inv);
       for (int k = 0, ka = 0, kb = 0; k < KK; ++k) {
+        skip_removed_tap(t, ka, kb);
         const float mk = mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv);
         const float sk = tap(k, ka, kb, mk);
         if (LANES > 1) __syncwarp(umask);

@@ -39,6 +39,16 @@ int esize(dcn_dtype d) { return d == DCN_BF16 ? 2 : 4; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Taps per (pixel, group): the K x K window, less its centre with remove_center.
+int taps(const dcn_problem* p) { return p->K * p->K - (p->remove_center ? 1 : 0); }
+
+// Compile-time tap set of a problem: 9 (3 x 3 window), 8 (3 x 3 without its
+// centre), or 0 (any other window, counted at run time).
+int compile_time_taps(const dcn_problem* p) {
+  if (p->K != 3) return 0;
+  return p->remove_center ? 8 : 9;
+}
+
 // Basic validity of the problem description.
 dcn_status check_problem(const dcn_problem* p, int64_t* Ho, int64_t* Wo) {
   if (!p) return DCN_ERR_INVALID_ARG;
@@ -46,13 +56,15 @@ dcn_status check_problem(const dcn_problem* p, int64_t* Ho, int64_t* Wo) {
   if (p->K < 1 || (p->K % 2) == 0) return DCN_ERR_INVALID_ARG;
   if (p->stride < 1 || p->pad < 0 || p->dilation < 1) return DCN_ERR_INVALID_ARG;
   if (p->softmax != 0 && p->softmax != 1) return DCN_ERR_INVALID_ARG;
+  if (p->remove_center != 0 && p->remove_center != 1) return DCN_ERR_INVALID_ARG;
+  if (p->remove_center && p->K < 3) return DCN_ERR_INVALID_ARG;  // no tap would be left
   if (p->dtype != DCN_F32 && p->dtype != DCN_BF16) return DCN_ERR_INVALID_ARG;
   if (!(p->offset_scale == p->offset_scale)) return DCN_ERR_INVALID_ARG;  // NaN
   const int64_t ho = out_extent(p->H, p->K, p->stride, p->pad, p->dilation);
   const int64_t wo = out_extent(p->W, p->K, p->stride, p->pad, p->dilation);
   if (ho < 1 || wo < 1) return DCN_ERR_INVALID_ARG;
   const int64_t C = int64_t(p->G) * p->Cg;
-  const int64_t KK = int64_t(p->K) * p->K;
+  const int64_t KK = taps(p);
   const int64_t n_in = int64_t(p->N) * p->H * p->W * C;
   const int64_t n_out = int64_t(p->N) * ho * wo * C;
   const int64_t n_off = int64_t(p->N) * ho * wo * p->G * KK * 2;
@@ -130,7 +142,8 @@ dcn_status make_plan(const dcn_problem* p, int64_t Ho, int64_t Wo, size_t entry_
     return DCN_ERR_UNSUPPORTED;
   TileParams& t = plan->t;
   t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
-  t.K = p->K; t.KK = p->K * p->K; t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation;
+  t.K = p->K; t.KK = taps(p); t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation;
+  t.kc = p->remove_center ? (p->K * p->K) / 2 : -1;
   t.Ho = int(Ho); t.Wo = int(Wo); t.sigma = p->offset_scale;
   size_t budget = kDefaultSmemBudget;
   if (const char* s = std::getenv("DCN_CORE_SMEM_BUDGET")) budget = size_t(std::atol(s));
@@ -188,16 +201,21 @@ dcn_status launch(Kernel k, const Plan& plan, const Args& args, cudaStream_t str
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
 }
 
+template <typename T, int CPL, int LANES, bool SOFTMAX>
+dcn_status forward_dispatch_sm(const dcn_problem* p, const Plan& plan, const FwdArgs& args,
+                               cudaStream_t stream) {
+  switch (compile_time_taps(p)) {
+    case 9: return launch(dcn_forward_kernel<T, CPL, LANES, 9, SOFTMAX>, plan, args, stream);
+    case 8: return launch(dcn_forward_kernel<T, CPL, LANES, 8, SOFTMAX>, plan, args, stream);
+    default: return launch(dcn_forward_kernel<T, CPL, LANES, 0, SOFTMAX>, plan, args, stream);
+  }
+}
+
 template <typename T, int CPL, int LANES>
 dcn_status forward_dispatch_kk(const dcn_problem* p, const Plan& plan, const FwdArgs& args,
                                cudaStream_t stream) {
-  const bool k3 = p->K == 3;
-  if (p->softmax) {
-    return k3 ? launch(dcn_forward_kernel<T, CPL, LANES, 9, true>, plan, args, stream)
-              : launch(dcn_forward_kernel<T, CPL, LANES, 0, true>, plan, args, stream);
-  }
-  return k3 ? launch(dcn_forward_kernel<T, CPL, LANES, 9, false>, plan, args, stream)
-            : launch(dcn_forward_kernel<T, CPL, LANES, 0, false>, plan, args, stream);
+  return p->softmax ? forward_dispatch_sm<T, CPL, LANES, true>(p, plan, args, stream)
+                    : forward_dispatch_sm<T, CPL, LANES, false>(p, plan, args, stream);
 }
 
 template <typename T>
@@ -212,16 +230,21 @@ dcn_status forward_dispatch(const dcn_problem* p, const Plan& plan, const FwdArg
   return DCN_ERR_UNSUPPORTED;
 }
 
+template <typename T, int LANES, bool SOFTMAX>
+dcn_status backward_dispatch_sm(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
+                                cudaStream_t stream) {
+  switch (compile_time_taps(p)) {
+    case 9: return launch(dcn_backward_kernel<T, LANES, 9, SOFTMAX>, plan, args, stream);
+    case 8: return launch(dcn_backward_kernel<T, LANES, 8, SOFTMAX>, plan, args, stream);
+    default: return launch(dcn_backward_kernel<T, LANES, 0, SOFTMAX>, plan, args, stream);
+  }
+}
+
 template <typename T, int LANES>
 dcn_status backward_dispatch_kk(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                                 cudaStream_t stream) {
-  const bool k3 = p->K == 3;
-  if (p->softmax) {
-    return k3 ? launch(dcn_backward_kernel<T, LANES, 9, true>, plan, args, stream)
-              : launch(dcn_backward_kernel<T, LANES, 0, true>, plan, args, stream);
-  }
-  return k3 ? launch(dcn_backward_kernel<T, LANES, 9, false>, plan, args, stream)
-            : launch(dcn_backward_kernel<T, LANES, 0, false>, plan, args, stream);
+  return p->softmax ? backward_dispatch_sm<T, LANES, true>(p, plan, args, stream)
+                    : backward_dispatch_sm<T, LANES, false>(p, plan, args, stream);
 }
 
 // The backward always gives a lane 4 channels (16 bytes), so that one warp
@@ -329,7 +352,7 @@ bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
   if (mode && std::strcmp(mode, "direct") == 0) return false;
   // 16 channels per group in either storage type: 32-byte bf16 groups or
   // 64-byte fp32 groups (eight accumulated values per phase-B lane).
-  if (p->K != 3 || p->Cg != 16) return false;
+  if (p->K != 3 || p->Cg != 16 || p->remove_center) return false;
   if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
   return tensor_map_encoder() != nullptr;
 }
@@ -519,7 +542,7 @@ dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input
   st = check_forward_pointers(problem, d_input, d_offset, d_mask, d_output);
   if (st != DCN_OK) return st;
   const size_t e = size_t(esize(problem->dtype));
-  const size_t C = size_t(problem->G) * problem->Cg, KK = size_t(problem->K) * problem->K;
+  const size_t C = size_t(problem->G) * problem->Cg, KK = size_t(taps(problem));
   const size_t b_in = size_t(problem->N) * problem->H * problem->W * C * e;
   const size_t px = size_t(problem->N) * Ho * Wo;
   const size_t b_off = px * problem->G * KK * 2 * e, b_msk = px * problem->G * KK * e;

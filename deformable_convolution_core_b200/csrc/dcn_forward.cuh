@@ -100,14 +100,14 @@ __global__ void __launch_bounds__(kThreads) dcn_forward_kernel(const FwdArgs a) 
     if constexpr (KKS > 0) {
       float m[KKS];
       mask_weights<T, KKS, SOFTMAX>(s_msk, row0, t.P1, u.pix, m);
-      constexpr int K = KKS == 1 ? 1 : (KKS == 9 ? 3 : (KKS == 25 ? 5 : 7));
-      static_assert(K * K == KKS, "compile-time tap counts are odd squares");
+      constexpr int K = tap_side(KKS);
 #pragma unroll
-      for (int k = 0; k < KKS; ++k) tap(k, k / K, k % K, m[k]);
+      for (int k = 0; k < KKS; ++k) tap(k, tap_pos(KKS, k) / K, tap_pos(KKS, k) % K, m[k]);
     } else {
       float mx, inv;
       mask_stats<T, SOFTMAX>(s_msk, row0, t.P1, u.pix, KK, mx, inv);
       for (int k = 0, ka = 0, kb = 0; k < KK; ++k) {
+        skip_removed_tap(t, ka, kb);
         tap(k, ka, kb, mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv));
         if (++kb == t.K) { kb = 0; ++ka; }
       }

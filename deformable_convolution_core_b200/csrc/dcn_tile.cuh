@@ -17,6 +17,7 @@ constexpr int kWarps = kThreads / 32;
 
 struct TileParams {
   int N, H, W, G, Cg, C, K, KK, stride, pad, dil, Ho, Wo;
+  int kc;       // window position (a*K + b) left out by remove_center, else -1
   float sigma;
   int TH, TW, nTY, nTX;
   int tile_px;  // TH * TW
@@ -62,6 +63,28 @@ struct Staged<__nv_bfloat16> {
 template <typename T>
 __host__ __device__ constexpr int staged_bytes_per_entry() {
   return int(sizeof(typename Staged<T>::Pair) + sizeof(typename Staged<T>::One));
+}
+
+// Compile-time tap sets: KKS = K*K taps of a K x K window, or 8 for the 3 x 3
+// window without its centre (DCNv4's remove_center, DCNv4 speed-up write-up
+// (pnsm.cn), section 3.3).  Tap k sits at window position tap_pos(KKS, k).
+__host__ __device__ constexpr int tap_side(int kks) {
+  return kks == 8 || kks == 9 ? 3 : (kks == 25 ? 5 : (kks == 49 ? 7 : 1));
+}
+__host__ __device__ constexpr int tap_pos(int kks, int k) {
+  return (tap_side(kks) * tap_side(kks) != kks && k >= kks / 2) ? k + 1 : k;
+}
+static_assert(tap_pos(8, 3) == 3 && tap_pos(8, 4) == 5 && tap_pos(8, 7) == 8 &&
+                  tap_pos(9, 4) == 4,
+              "the 8-tap set skips window position 4");
+
+// Runtime tap sets: step (ka, kb) over the window row by row, skipping the
+// position kc (remove_center; kc = -1 skips nothing).
+__device__ __forceinline__ void skip_removed_tap(const TileParams& t, int& ka, int& kb) {
+  if (ka * t.K + kb == t.kc && ++kb == t.K) {
+    kb = 0;
+    ++ka;
+  }
 }
 
 struct TileCoord {

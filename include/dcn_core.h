@@ -3,19 +3,24 @@
  *
  * The operator (InternImage-L DCNv3 explainer (wmrh.cn), section 二 steps
  * 2-4 and section 三): for every output pixel (n, ho, wo), group g and tap
- * k = a*K + b of a K x K window, take the learned offset (dx, dy) of that
- * tap, scale it by offset_scale, bilinearly sample the group's Cg input
- * channels at
+ * k of a K x K window (position (a, b), k = a*K + b), take the learned
+ * offset (dx, dy) of that tap, scale it by offset_scale, bilinearly sample
+ * the group's Cg input channels at
  *     Y = ho*stride - pad + a*dilation + offset_scale*dy
  *     X = wo*stride - pad + b*dilation + offset_scale*dx
  * (integer coordinates are pixel centres; corners outside the image read as
  * zero), and sum the K*K samples weighted by the mask of that (pixel, group):
  * softmax-normalised over the taps for DCNv3, used as given for the DCNv4
- * variant (DCNv4 speed-up write-up (pnsm.cn), sections 1-2).  Arithmetic is
- * fp32 for both storage types; bf16 values are widened exactly on load and
- * the output is rounded to nearest-even once.
+ * variant (DCNv4 speed-up write-up (pnsm.cn), sections 1-2).  With
+ * remove_center (a DCNv4 module argument, same write-up, section 3.3) the
+ * window's centre position (K/2, K/2) is not sampled: the KK = K*K - 1 taps
+ * are the other positions in row-major order, tap k at position k for
+ * k < (K*K)/2 and at k + 1 after it.  Arithmetic is fp32 for both storage
+ * types; bf16 values are widened exactly on load and the output is rounded to
+ * nearest-even once.
  *
- * Layouts (all tensors dense, row-major, element indices; C = G*Cg, KK = K*K):
+ * Layouts (all tensors dense, row-major, element indices; C = G*Cg, KK = taps
+ * = K*K, or K*K - 1 with remove_center):
  *   input   (N, H, W, C)            ((n*H + y)*W + x)*C + g*Cg + c
  *   offset  (N, Ho, Wo, G*KK*2)     ((n*Ho + ho)*Wo + wo)*G*KK*2 + (g*KK + k)*2 + {0: dx, 1: dy}
  *   mask    (N, Ho, Wo, G*KK)       ((n*Ho + ho)*Wo + wo)*G*KK + g*KK + k
@@ -46,7 +51,7 @@
 extern "C" {
 #endif
 
-#define DCN_CORE_ABI_VERSION 1
+#define DCN_CORE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define DCN_API __attribute__((visibility("default")))
@@ -70,15 +75,17 @@ typedef enum {
 /*
  * Problem description (the constructor arguments of the DCNv3/DCNv4 modules
  * in the DCNv4 speed-up write-up (pnsm.cn), section 3.3: channels = G*Cg,
- * kernel_size, stride, pad, dilation, group, offset_scale).
+ * kernel_size, stride, pad, dilation, group, offset_scale, remove_center).
  *   N, H, W      batch and input spatial size, >= 1
  *   G, Cg        groups and channels per group, >= 1
  *   K            kernel side, odd, >= 1 (taps = K*K)
  *   stride >= 1, pad >= 0, dilation >= 1 (same for height and width)
  *   offset_scale multiplies every offset (InternImage-L uses 2.0)
- *   softmax      1: mask holds logits, softmax over the K*K taps of each
+ *   softmax      1: mask holds logits, softmax over the KK taps of each
  *                   (pixel, group) (DCNv3);  0: mask used as given (DCNv4)
  *   dtype        storage type of input, offset, mask and output
+ *   remove_center  0: all K*K window positions are taps;  1: the centre
+ *                position is left out (KK = K*K - 1 taps; needs K >= 3)
  */
 typedef struct {
   int N, H, W, G, Cg;
@@ -87,6 +94,7 @@ typedef struct {
   float offset_scale;
   int softmax;
   dcn_dtype dtype;
+  int remove_center;
 } dcn_problem;
 
 /* Output spatial size.  DCN_ERR_INVALID_ARG if the problem is invalid or the

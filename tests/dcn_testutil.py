@@ -66,4 +66,5 @@ def assert_bwd(got, ref, what="", dtype="f32"):
 
 def problem_kwargs(problem) -> dict:
     return dict(G=problem.G, K=problem.K, stride=problem.stride, pad=problem.pad,
-                dil=problem.dilation, offset_scale=problem.offset_scale, softmax=problem.softmax)
+                dil=problem.dilation, offset_scale=problem.offset_scale, softmax=problem.softmax,
+                remove_center=problem.remove_center)

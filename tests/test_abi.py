@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert dcn.dcn_core_abi_version() == 1
+    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 2
     for st in range(5):
         assert dcn.dcn_status_string(st)
     assert "unknown" in dcn.dcn_status_string(99)
@@ -47,6 +47,20 @@ def test_output_hw(lib):
     assert dcn.dcn_core_output_hw(dcn.make_problem(1, 7, 9, 1, 8, K=5, pad=0, dilation=1)) == (3, 5)
     with pytest.raises(dcn.DcnError):
         dcn.dcn_core_output_hw(dcn.make_problem(1, 2, 2, 1, 8, K=5, pad=0))
+    # removing the centre tap leaves the output grid unchanged
+    assert dcn.dcn_core_output_hw(dcn.make_problem(1, 7, 9, 1, 8, K=3, remove_center=1)) == (7, 9)
+
+
+def test_problem_mirrors_header_struct():
+    """DcnProblem has the fields of dcn_problem, in order."""
+    text = open(os.path.join(ROOT, "include", "dcn_core.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} dcn_problem;", text, re.S).group(1)
+    names = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            names += [n.strip().lstrip("*") for n in decl.split(None, 1)[1].split(",")]
+    assert names == [n for n, _ in dcn.DcnProblem._fields_]
 
 
 GOOD = dict(N=1, H=8, W=8, G=2, Cg=16, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0,
@@ -65,6 +79,8 @@ FAKE = 1 << 20  # an address that is 16- and 32-byte aligned; never dereferenced
     (dict(pad=-1), dcn.DCN_ERR_INVALID_ARG),
     (dict(dilation=0), dcn.DCN_ERR_INVALID_ARG),
     (dict(softmax=2), dcn.DCN_ERR_INVALID_ARG),
+    (dict(remove_center=2), dcn.DCN_ERR_INVALID_ARG),
+    (dict(remove_center=1, K=1, pad=0), dcn.DCN_ERR_INVALID_ARG),  # no tap left
     (dict(dtype=7), dcn.DCN_ERR_INVALID_ARG),
     (dict(offset_scale=float("nan")), dcn.DCN_ERR_INVALID_ARG),
     (dict(H=2, W=2, K=5, pad=0), dcn.DCN_ERR_INVALID_ARG),     # empty output

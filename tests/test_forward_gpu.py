@@ -22,19 +22,21 @@ RNG = np.random.default_rng(2024)
 
 
 def random_case(N, H, W, G, Cg, K=3, stride=1, pad=None, dil=1, sigma=2.0, softmax=1,
-                dtype="f32", off_sd=1.5, off_lo=None):
+                dtype="f32", off_sd=1.5, off_lo=None, remove_center=0):
     pad = (K // 2) * dil if pad is None else pad
-    p = dcn.make_problem(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, dtype)
+    p = dcn.make_problem(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, dtype,
+                         remove_center)
     Ho, Wo = dcn.dcn_core_output_hw(p)
+    T = dcn.taps(p)
     x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
     if off_lo is None:
-        off = (off_sd * RNG.standard_normal((N, Ho, Wo, G * K * K * 2))).astype(np.float32)
+        off = (off_sd * RNG.standard_normal((N, Ho, Wo, G * T * 2))).astype(np.float32)
     else:
-        off = RNG.uniform(off_lo, -off_lo, (N, Ho, Wo, G * K * K * 2)).astype(np.float32)
+        off = RNG.uniform(off_lo, -off_lo, (N, Ho, Wo, G * T * 2)).astype(np.float32)
     if softmax:
-        mask = RNG.standard_normal((N, Ho, Wo, G * K * K)).astype(np.float32)
+        mask = RNG.standard_normal((N, Ho, Wo, G * T)).astype(np.float32)
     else:
-        mask = RNG.uniform(-1, 1, (N, Ho, Wo, G * K * K)).astype(np.float32)
+        mask = RNG.uniform(-1, 1, (N, Ho, Wo, G * T)).astype(np.float32)
     return p, x, off, mask
 
 
@@ -89,6 +91,13 @@ CASES = [
     (2, 3, 3, 2, 16, dict(dtype="f32", stride=5)),   # stride larger than the image
     (1, 40, 3, 80, 16, dict(dtype="bf16")),      # many groups
     (2, 20, 20, 2, 16, dict(dtype="f32", off_lo=-40.0)),   # most samples far outside
+    # remove_center: the window without its centre (8 taps at K = 3, 24 at K = 5, 48 at K = 7)
+    (2, 23, 29, 3, 16, dict(dtype="f32", remove_center=1)),
+    (1, 33, 17, 10, 16, dict(dtype="bf16", softmax=0, remove_center=1)),
+    (2, 25, 27, 4, 8, dict(dtype="bf16", stride=2, remove_center=1)),
+    (2, 13, 14, 3, 32, dict(dtype="f32", softmax=0, remove_center=1)),
+    (2, 17, 19, 3, 16, dict(dtype="f32", K=5, remove_center=1)),
+    (1, 17, 19, 2, 16, dict(dtype="bf16", K=7, softmax=0, dil=2, remove_center=1)),
 ]
 
 
@@ -141,6 +150,23 @@ def test_identity_and_box_filter_on_gpu(oracle_mod):
     xp = np.pad(x.astype(np.float64), ((0, 0), (1, 1), (1, 1), (0, 0)))
     box = sum(xp[:, i:i + H, j:j + W, :] for i in range(3) for j in range(3)) / 9.0
     np.testing.assert_allclose(f64(out), box, rtol=0, atol=1e-5 * np.abs(x).max())
+
+
+@pytest.mark.parametrize("K", [3, 5])
+def test_remove_center_ring_mean_on_gpu(K):
+    # Zero offsets and equal logits without the centre tap: the zero-padded
+    # mean of the other K*K - 1 window positions.
+    N, H, W, G, Cg = 2, 14, 11, 3, 16
+    r, T = K // 2, K * K - 1
+    x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    p = dcn.make_problem(N, H, W, G, Cg, K, pad=r, softmax=1, remove_center=1)
+    off = np.zeros((N, H, W, G * T * 2), np.float32)
+    logits = np.full((N, H, W, G * T), 0.25, np.float32)
+    out = gpu_forward(p, to_dev(x, "f32"), to_dev(off, "f32"), to_dev(logits, "f32"))
+    xp = np.pad(x.astype(np.float64), ((0, 0), (r, r), (r, r), (0, 0)))
+    ring = sum(xp[:, i:i + H, j:j + W, :] for i in range(K) for j in range(K)
+               if (i, j) != (r, r)) / T
+    np.testing.assert_allclose(f64(out), ring, rtol=0, atol=1e-5 * np.abs(x).max())
 
 
 def test_nonfinite_and_border_offsets(oracle_mod):
