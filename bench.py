@@ -264,7 +264,7 @@ def run_ours(args, world, rank, local):
     kernels = []
     if fwd_ms > 0:
         tiled = (os.environ.get("DCN_CORE_FORWARD") != "direct" and wl.K == 3
-                 and wl.Cg == 16 and not wl.remove_center)
+                 and wl.Cg == 16)
         kernels.append(("dcn_forward_tiled_kernel" if tiled else "dcn_forward_kernel",
                         fwd_bytes, fwd_ms))
     if bwd_ms > 0:

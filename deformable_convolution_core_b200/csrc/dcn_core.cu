@@ -352,7 +352,7 @@ bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
   if (mode && std::strcmp(mode, "direct") == 0) return false;
   // 16 channels per group in either storage type: 32-byte bf16 groups or
   // 64-byte fp32 groups (eight accumulated values per phase-B lane).
-  if (p->K != 3 || p->Cg != 16 || p->remove_center) return false;
+  if (p->K != 3 || p->Cg != 16) return false;
   if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
   return tensor_map_encoder() != nullptr;
 }
@@ -388,7 +388,7 @@ void choose_tiled_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, s
       const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * p->G;
       const int px = th * tw;
       const int64_t batches = (px + kTiledBatch - 1) / kTiledBatch;
-      const double per_item = double(batches) * kTiledBatch * kTiledKK  // unit-samples
+      const double per_item = double(batches) * kTiledBatch * taps(p)  // unit-samples
                               + 0.05 * double(bytes) / 32.0            // box fill
                               + 300.0;                                 // item overhead
       const double cost = double(items) * per_item;
@@ -403,10 +403,10 @@ void choose_tiled_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, s
   *TW_out = btw;
 }
 
-template <typename T, int CS, bool SOFTMAX>
+template <typename T, int CS, int KKS, bool SOFTMAX>
 dcn_status launch_tiled_kernel(const CUtensorMap& map, const TiledArgs& args, size_t smem,
                                int sms, cudaStream_t stream) {
-  auto k = dcn_forward_tiled_kernel<T, CS, SOFTMAX>;
+  auto k = dcn_forward_tiled_kernel<T, CS, KKS, SOFTMAX>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return DCN_ERR_CUDA;
@@ -418,6 +418,16 @@ dcn_status launch_tiled_kernel(const CUtensorMap& map, const TiledArgs& args, si
   const int64_t grid = std::min<int64_t>(args.t.items, int64_t(sms) * per_sm);
   k<<<unsigned(grid), kTiledThreads, smem, stream>>>(map, args);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+template <typename T, int CS>
+dcn_status tiled_dispatch(const dcn_problem* p, const CUtensorMap& map, const TiledArgs& args,
+                          size_t smem, int sms, cudaStream_t stream) {
+  if (p->remove_center)
+    return p->softmax ? launch_tiled_kernel<T, CS, 8, true>(map, args, smem, sms, stream)
+                      : launch_tiled_kernel<T, CS, 8, false>(map, args, smem, sms, stream);
+  return p->softmax ? launch_tiled_kernel<T, CS, 9, true>(map, args, smem, sms, stream)
+                    : launch_tiled_kernel<T, CS, 9, false>(map, args, smem, sms, stream);
 }
 
 dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
@@ -483,11 +493,8 @@ dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return DCN_ERR_UNSUPPORTED;
 
-  if (p->dtype == DCN_BF16)
-    return p->softmax ? launch_tiled_kernel<__nv_bfloat16, 32, true>(map, args, smem, dev.sms, stream)
-                      : launch_tiled_kernel<__nv_bfloat16, 32, false>(map, args, smem, dev.sms, stream);
-  return p->softmax ? launch_tiled_kernel<float, 64, true>(map, args, smem, dev.sms, stream)
-                    : launch_tiled_kernel<float, 64, false>(map, args, smem, dev.sms, stream);
+  if (p->dtype == DCN_BF16) return tiled_dispatch<__nv_bfloat16, 32>(p, map, args, smem, dev.sms, stream);
+  return tiled_dispatch<float, 64>(p, map, args, smem, dev.sms, stream);
 }
 }  // namespace
 }  // namespace dcn

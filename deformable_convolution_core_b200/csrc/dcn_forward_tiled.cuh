@@ -29,7 +29,7 @@ namespace dcn {
 constexpr int kTiledWarps = 15;  // consumer warps: with the producer, 4 warps per SM sub-partition
 constexpr int kTiledThreads = (kTiledWarps + 1) * 32;  // + one TMA producer warp
 constexpr int kTiledBatch = 32;                       // units per warp batch
-constexpr int kTiledKK = 9;  // the tiled kernel serves 3x3 windows
+constexpr int kTiledMaxTaps = 9;  // the tiled kernel serves 3x3 windows (9 or 8 taps)
 
 struct TiledParams {
   int N, H, W, G, Cg, C, stride, pad, dil, Ho, Wo;
@@ -200,7 +200,8 @@ struct TiledIO<__nv_bfloat16> {
 
 // Tap records, written by the unit's owner lane in phase A and read by the
 // unit's eight lanes in phase B.  A unit slot holds w[9][4] (the tap's four
-// corner weights, mask weight folded in) followed by code[9].  code >= 0 is
+// corner weights, mask weight folded in) followed by code[9], of which the
+// 8-tap set (remove_center) uses the first eight.  code >= 0 is
 // the byte offset in the box of corner (y0, x0) when the whole 2x2 footprint
 // lies in the box; otherwise code = INT_MIN | (y0 + 1) << 15 | (x0 + 1), and
 // the corners are read from global memory ((y0, x0) = (32766, 32766) marks a
@@ -214,9 +215,9 @@ __device__ __forceinline__ int far_code(int y0, int x0) {
 // 46 words per slot also keeps both the 32-lane phase-A reads and the
 // four-unit phase-B reads free of bank conflicts.
 constexpr int kSlotBytes = 184;
-constexpr int kCodeAt = kTiledKK * 16;
+constexpr int kCodeAt = kTiledMaxTaps * 16;
 constexpr int kLogitAt = 80;               // staged mask values (before the records)
-constexpr int kFarMaskAt = kCodeAt + kTiledKK * 4;  // 180: bit k = tap k is read from global
+constexpr int kFarMaskAt = kCodeAt + kTiledMaxTaps * 4;  // 180: bit k = tap k is read from global
 static_assert(kSlotBytes % 8 == 0 && kFarMaskAt + 4 <= kSlotBytes, "slot layout");
 
 // Phase-B lane roles: 8 lanes per unit, lane li = (corner r = li >> 1, q = li & 1).
@@ -232,14 +233,16 @@ struct LaneRole {
   }
 };
 
-template <typename T, int CS, bool SOFTMAX>
+// KKS: 9 (the 3x3 window) or 8 (the window without its centre).
+template <typename T, int CS, int KKS, bool SOFTMAX>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     dcn_forward_tiled_kernel(const __grid_constant__ CUtensorMap xmap, const TiledArgs a) {
   using IO = TiledIO<T>;
   using Pair = typename IO::Pair;
   using One = typename IO::One;
   using Role = LaneRole<CS>;
-  constexpr int KK = kTiledKK, K = 3;
+  constexpr int KK = KKS, K = tap_side(KKS);
+  static_assert(K == 3 && KK <= kTiledMaxTaps, "the tiled kernel serves 3x3 tap sets");
   constexpr int LU = 8;            // phase-B lanes per unit
   constexpr int UPW = 32 / LU;     // units per phase-B step
   constexpr int NP = Role::kPieces;
@@ -426,7 +429,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         unsigned farmask = 0u;
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          const int ka = k / K, kb = k % K;
+          const int ka = tap_pos(KK, k) / K, kb = tap_pos(KK, k) % K;
           const float Y = tap_coord(ho * t.stride - t.pad + ka * t.dil, t.sigma, d[k].y);
           const float X = tap_coord(wo * t.stride - t.pad + kb * t.dil, t.sigma, d[k].x);
           const Footprint f = footprint(Y, X, t.H, t.W);

@@ -125,6 +125,9 @@ def test_tiled_kernel_tile_and_halo_settings(oracle_mod, halo, tile):
             check_full(oracle_mod, p, x, off, mask, dtype)
             p, x, off, mask = random_case(1, 40, 36, 2, 16, dtype=dtype, stride=2, softmax=0)
             check_full(oracle_mod, p, x, off, mask, dtype)
+            p, x, off, mask = random_case(2, 29, 31, 3, 16, dtype=dtype, off_sd=3.0,
+                                          remove_center=1)
+            check_full(oracle_mod, p, x, off, mask, dtype)
     finally:
         for k, v in old.items():
             if v is None:
