@@ -268,7 +268,10 @@ def run_ours(args, world, rank, local):
         kernels.append(("dcn_forward_tiled_kernel" if tiled else "dcn_forward_kernel",
                         fwd_bytes, fwd_ms))
     if bwd_ms > 0:
-        kernels.append(("dcn_backward_kernel", bwd_bytes, bwd_ms))
+        tiled_bwd = (os.environ.get("DCN_CORE_BACKWARD") != "direct" and wl.K == 3
+                     and wl.Cg == 16)
+        kernels.append(("dcn_backward_tiled_kernel" if tiled_bwd else "dcn_backward_kernel",
+                        bwd_bytes, bwd_ms))
     kname, kbytes, kms = max(kernels, key=lambda k: k[2])
     achieved = kbytes / (kms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",

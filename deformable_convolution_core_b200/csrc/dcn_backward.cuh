@@ -43,6 +43,15 @@ struct Quad<float> {
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(w.w[i]);
   }
+  // Zeros unless `pred`; a false predicate issues no memory access (p may then
+  // point anywhere).
+  __device__ __forceinline__ static void load_pred(const void* p, bool pred, float (&v)[4]) {
+    asm("{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
+        " mov.b32 %0, 0;\n mov.b32 %1, 0;\n mov.b32 %2, 0;\n mov.b32 %3, 0;\n"
+        " @q ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];\n}"
+        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+        : "l"(p), "r"(int(pred)));
+  }
   __device__ __forceinline__ static void store_pair(void* base, size_t i, float a, float b) {
     reinterpret_cast<float2*>(base)[i] = make_float2(a, b);
   }
@@ -55,6 +64,17 @@ struct Quad<__nv_bfloat16> {
   __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
     uint32_t w0, w1;
     asm("ld.global.nc.v2.b32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "l"(p));
+    v[0] = bf16lo_to_f32(w0);
+    v[1] = bf16hi_to_f32(w0);
+    v[2] = bf16lo_to_f32(w1);
+    v[3] = bf16hi_to_f32(w1);
+  }
+  __device__ __forceinline__ static void load_pred(const void* p, bool pred, float (&v)[4]) {
+    uint32_t w0, w1;
+    asm("{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n mov.b32 %0, 0;\n mov.b32 %1, 0;\n"
+        " @q ld.global.nc.v2.b32 {%0, %1}, [%2];\n}"
+        : "=r"(w0), "=r"(w1)
+        : "l"(p), "r"(int(pred)));
     v[0] = bf16lo_to_f32(w0);
     v[1] = bf16hi_to_f32(w0);
     v[2] = bf16lo_to_f32(w1);
@@ -76,6 +96,15 @@ __global__ void dcn_round_to_bf16_kernel(const float4* __restrict__ in, uint2* _
     const float4 v = __ldg(in + i);
     out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
   }
+}
+
+// grad_input[p .. p+3] += v, as one 16-byte vector reduction, only if `pred`
+// (a false predicate issues no memory access).
+__device__ __forceinline__ void red_add_v4_pred(float* p, float2 lo, float2 hi, bool pred) {
+  asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
+               " @q red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n}" ::"l"(p),
+               "f"(lo.x), "f"(lo.y), "f"(hi.x), "f"(hi.y), "r"(int(pred))
+               : "memory");
 }
 
 template <int LANES>
@@ -184,9 +213,11 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
       constexpr int K = tap_side(KKS);
       float m[KKS], s[KKS];
       mask_weights<T, KKS, SOFTMAX>(s_msk, row0, t.P1, u.pix, m);
+      const float2 g01 = make_float2(go[0], go[1]), g23 = make_float2(go[2], go[3]);
       // Taps in groups of three (two for the 8-tap set), without branches:
-      // the group's corner gathers are issued together (predicated on the
-      // corner lying in the image), then reduced and scattered.
+      // the group's corner gathers are issued together, then reduced and
+      // scattered; loads and reductions are predicated on the corner lying in
+      // the image, and the products run as packed fp32 pairs.
       constexpr int GRP = KKS % 3 == 0 ? 3 : 2;
       static_assert(KKS % GRP == 0, "the tap set splits into whole groups");
 #pragma unroll
@@ -213,11 +244,9 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
           cval[j][2] = f[j].v10;
           cval[j][3] = f[j].v11;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-#pragma unroll
-            for (int e = 0; e < CPL; ++e) cv[j][c][e] = 0.f;
-            if (cval[j][c]) Quad<T>::load(xg + ptrdiff_t(cofs[j][c]) * ptrdiff_t(sizeof(T)), cv[j][c]);
-          }
+          for (int c = 0; c < 4; ++c)
+            Quad<T>::load_pred(xg + ptrdiff_t(cofs[j][c]) * ptrdiff_t(sizeof(T)), cval[j][c],
+                               cv[j][c]);
         }
 #pragma unroll
         for (int j = 0; j < GRP; ++j) {
@@ -227,15 +256,14 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
           float dc[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            float dsum = 0.f;
-#pragma unroll
-            for (int e = 0; e < CPL; ++e) dsum = fmaf(go[e], cv[j][c][e], dsum);
-            dc[c] = dsum;
-            if (cval[j][c]) {
-              const float wv = m[k] * cw[c];
-              atomicAdd(reinterpret_cast<float4*>(gxg + ptrdiff_t(cofs[j][c])),
-                        make_float4(wv * go[0], wv * go[1], wv * go[2], wv * go[3]));
-            }
+            // <g, x[corner]> over the lane's four channels, as two packed pairs
+            float2 pd = __fmul2_rn(make_float2(cv[j][c][0], cv[j][c][1]), g01);
+            pd = __ffma2_rn(make_float2(cv[j][c][2], cv[j][c][3]), g23, pd);
+            dc[c] = pd.x + pd.y;
+            const float wv = m[k] * cw[c];
+            const float2 w2 = make_float2(wv, wv);
+            red_add_v4_pred(gxg + ptrdiff_t(cofs[j][c]), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23),
+                            cval[j][c]);
           }
           // out-of-support samples have no valid corner: every dc is 0
           s[k] = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];

@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "dcn_backward.cuh"
+#include "dcn_backward_tiled.cuh"
 #include "dcn_forward.cuh"
 #include "dcn_forward_tiled.cuh"
 
@@ -403,10 +404,11 @@ void choose_tiled_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, s
   *TW_out = btw;
 }
 
-template <typename T, int CS, int KKS, bool SOFTMAX>
-dcn_status launch_tiled_kernel(const CUtensorMap& map, const TiledArgs& args, size_t smem,
-                               int sms, cudaStream_t stream) {
-  auto k = dcn_forward_tiled_kernel<T, CS, KKS, SOFTMAX>;
+// Launch a persistent tiled kernel: as many CTAs as fit on the GPU at once,
+// never more than there are items.
+template <typename Kernel, typename Args>
+dcn_status launch_persistent(Kernel k, const CUtensorMap& map, const Args& args, size_t smem,
+                             int sms, cudaStream_t stream) {
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return DCN_ERR_CUDA;
@@ -421,37 +423,61 @@ dcn_status launch_tiled_kernel(const CUtensorMap& map, const TiledArgs& args, si
 }
 
 template <typename T, int CS>
-dcn_status tiled_dispatch(const dcn_problem* p, const CUtensorMap& map, const TiledArgs& args,
-                          size_t smem, int sms, cudaStream_t stream) {
+dcn_status forward_tiled_dispatch(const dcn_problem* p, const CUtensorMap& map,
+                                  const TiledArgs& args, size_t smem, int sms,
+                                  cudaStream_t stream) {
   if (p->remove_center)
-    return p->softmax ? launch_tiled_kernel<T, CS, 8, true>(map, args, smem, sms, stream)
-                      : launch_tiled_kernel<T, CS, 8, false>(map, args, smem, sms, stream);
-  return p->softmax ? launch_tiled_kernel<T, CS, 9, true>(map, args, smem, sms, stream)
-                    : launch_tiled_kernel<T, CS, 9, false>(map, args, smem, sms, stream);
+    return p->softmax
+               ? launch_persistent(dcn_forward_tiled_kernel<T, CS, 8, true>, map, args, smem, sms, stream)
+               : launch_persistent(dcn_forward_tiled_kernel<T, CS, 8, false>, map, args, smem, sms, stream);
+  return p->softmax
+             ? launch_persistent(dcn_forward_tiled_kernel<T, CS, 9, true>, map, args, smem, sms, stream)
+             : launch_persistent(dcn_forward_tiled_kernel<T, CS, 9, false>, map, args, smem, sms, stream);
 }
 
-dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
-                         const void* off, const void* mask, void* out, cudaStream_t stream) {
+template <typename T, int CS>
+dcn_status backward_tiled_dispatch(const dcn_problem* p, const CUtensorMap& map,
+                                   const TiledBwdArgs& args, size_t smem, int sms,
+                                   cudaStream_t stream) {
+  if (p->remove_center)
+    return p->softmax
+               ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, true>, map, args, smem, sms, stream)
+               : launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, false>, map, args, smem, sms, stream);
+  return p->softmax
+             ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, true>, map, args, smem, sms, stream)
+             : launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, false>, map, args, smem, sms, stream);
+}
+
+// Everything a tiled launch needs: the tile and box geometry, the shared
+// memory size and the input's tensor map.  `tile_env` names the variable that
+// may force the tile ("THxTW", for tuning sweeps).
+struct TiledLaunch {
+  TiledParams t;
+  CUtensorMap map;
+  size_t smem;
   DeviceInfo dev;
-  dcn_status st = device_info(&dev);
+};
+
+dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
+                         const char* tile_env, TiledLaunch* L) {
+  dcn_status st = device_info(&L->dev);
   if (st != DCN_OK) return st;
   const int e = esize(p->dtype);
   const int cs = p->Cg * e;
   const size_t slot_bytes = size_t(kTiledWarps) * kTiledBatch * kSlotBytes;
   const size_t fixed = slot_bytes + 64;
-  if (size_t(dev.smem_optin) <= fixed + 2048) return DCN_ERR_UNSUPPORTED;
-  const size_t box_budget = (size_t(dev.smem_optin) - fixed) / 2 / 1024 * 1024;
+  if (size_t(L->dev.smem_optin) <= fixed + 2048) return DCN_ERR_UNSUPPORTED;
+  const size_t box_budget = (size_t(L->dev.smem_optin) - fixed) / 2 / 1024 * 1024;
   const int halo = env_int("DCN_CORE_HALO", 5);
   int TH = 0, TW = 0;
-  if (const char* s = std::getenv("DCN_CORE_TILED_TILE")) {
+  if (const char* s = std::getenv(tile_env)) {
     if (std::sscanf(s, "%dx%d", &TH, &TW) != 2 || TH < 1 || TW < 1) TH = TW = 0;
   }
   if (TH == 0) choose_tiled_tile(p, int(Ho), int(Wo), cs, halo, box_budget, &TH, &TW);
   TH = std::min<int>(TH, int(Ho));
   TW = std::min<int>(TW, int(Wo));
 
-  TiledArgs args;
-  TiledParams& t = args.t;
+  TiledParams& t = L->t;
   t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
   t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation; t.Ho = int(Ho); t.Wo = int(Wo);
   t.sigma = p->offset_scale; t.halo = halo; t.TH = TH; t.TW = TW;
@@ -471,15 +497,12 @@ dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   t.fd_nTX = make_fastdiv(uint32_t(t.nTX));
   t.fd_tiles = make_fastdiv(uint32_t(t.nTY * t.nTX));
   t.fd_TW = make_fastdiv(uint32_t(TW));
-  const size_t smem = 2 * size_t(t.box_stride) + fixed;
-  if (smem > size_t(dev.smem_optin)) return DCN_ERR_UNSUPPORTED;
-  args.x = x; args.off = off; args.mask = mask; args.out = out;
-  args.error_word = dev.error_word;
+  L->smem = 2 * size_t(t.box_stride) + fixed;
+  if (L->smem > size_t(L->dev.smem_optin)) return DCN_ERR_UNSUPPORTED;
 
   // Tensor map of the input viewed as (C, W, H, N), innermost first; one box
   // is (Cg, BW, BH, 1) starting at (g*Cg, X0, Y0, n).  Outside the tensor the
   // box is zero filled, which is exactly the operator's zero padding.
-  CUtensorMap map;
   const cuuint64_t dims[4] = {cuuint64_t(t.C), cuuint64_t(t.W), cuuint64_t(t.H),
                               cuuint64_t(t.N)};
   const cuuint64_t strides[3] = {cuuint64_t(t.C) * e, cuuint64_t(t.W) * t.C * e,
@@ -487,14 +510,65 @@ dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   const cuuint32_t box[4] = {cuuint32_t(t.Cg), cuuint32_t(t.BW), cuuint32_t(t.BH), 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUresult cr = tensor_map_encoder()(
-      &map, p->dtype == DCN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+      &L->map,
+      p->dtype == DCN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
       4, const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
       CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return DCN_ERR_UNSUPPORTED;
+  return cr == CUDA_SUCCESS ? DCN_OK : DCN_ERR_UNSUPPORTED;
+}
 
-  if (p->dtype == DCN_BF16) return tiled_dispatch<__nv_bfloat16, 32>(p, map, args, smem, dev.sms, stream);
-  return tiled_dispatch<float, 64>(p, map, args, smem, dev.sms, stream);
+dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
+                         const void* off, const void* mask, void* out, cudaStream_t stream) {
+  TiledLaunch L;
+  dcn_status st = tiled_prepare(p, Ho, Wo, x, "DCN_CORE_TILED_TILE", &L);
+  if (st != DCN_OK) return st;
+  TiledArgs args;
+  args.t = L.t;
+  args.x = x; args.off = off; args.mask = mask; args.out = out;
+  args.error_word = L.dev.error_word;
+  if (p->dtype == DCN_BF16)
+    return forward_tiled_dispatch<__nv_bfloat16, 32>(p, L.map, args, L.smem, L.dev.sms, stream);
+  return forward_tiled_dispatch<float, 64>(p, L.map, args, L.smem, L.dev.sms, stream);
+}
+
+// The tiled backward applies where the tiled forward does (3x3 tap sets,
+// 16 channels per group); DCN_CORE_BACKWARD=direct selects the direct kernel.
+bool backward_tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
+  const char* mode = std::getenv("DCN_CORE_BACKWARD");
+  if (mode && std::strcmp(mode, "direct") == 0) return false;
+  if (p->K != 3 || p->Cg != 16) return false;
+  if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
+  return tensor_map_encoder() != nullptr;
+}
+
+// Launch the tiled backward on a zero-filled fp32 accumulator `acc`.
+dcn_status backward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
+                          const void* off, const void* mask, const void* gout, float* acc,
+                          void* goff, void* gmask, cudaStream_t stream) {
+  TiledLaunch L;
+  dcn_status st = tiled_prepare(p, Ho, Wo, x, "DCN_CORE_BWD_TILED_TILE", &L);
+  if (st != DCN_OK) return st;
+  TiledBwdArgs args;
+  args.t = L.t;
+  args.x = x; args.off = off; args.mask = mask; args.gout = gout;
+  args.gx = acc; args.goff = goff; args.gmask = gmask;
+  args.error_word = L.dev.error_word;
+  if (p->dtype == DCN_BF16)
+    return backward_tiled_dispatch<__nv_bfloat16, 32>(p, L.map, args, L.smem, L.dev.sms, stream);
+  return backward_tiled_dispatch<float, 64>(p, L.map, args, L.smem, L.dev.sms, stream);
+}
+
+// The backward's kernel launch on a zero-filled accumulator: the tiled kernel
+// where it applies, else (or when it cannot be configured) the direct one.
+dcn_status backward_launch(const dcn_problem* p, int64_t Ho, int64_t Wo, const Plan& plan,
+                           const BwdArgs& a, cudaStream_t stream) {
+  if (backward_tiled_eligible(p, Ho, Wo)) {
+    const dcn_status st = backward_tiled(p, Ho, Wo, a.x, a.off, a.mask, a.gout, a.gx, a.goff,
+                                         a.gmask, stream);
+    if (st != DCN_ERR_UNSUPPORTED) return st;
+  }
+  return backward_dispatch(p, plan, a, stream);
 }
 }  // namespace
 }  // namespace dcn
@@ -595,7 +669,7 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
   float* acc = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(grad_input);
   if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
   BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, plan.t};
-  st = backward_dispatch(problem, plan, args, stream);
+  st = backward_launch(problem, Ho, Wo, plan, args, stream);
   if (st != DCN_OK || !bf16) return st;
   // bf16: round the fp32 accumulator once into grad_input.
   const size_t n4 = acc_bytes / 16;
@@ -705,7 +779,7 @@ extern "C" dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, cons
   // The shared array keeps the previous call's sums: clear it first.
   if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
   BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, plan.t};
-  st = backward_dispatch(problem, plan, args, stream);
+  st = backward_launch(problem, Ho, Wo, plan, args, stream);
   if (st != DCN_OK || !bf16) return st;
   const size_t n4 = acc_bytes / 16;
   DeviceInfo dev;

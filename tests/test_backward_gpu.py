@@ -2,6 +2,9 @@
 when softmax is on) of the CUDA path against the CPU oracle, plus the
 adjoint identity and the softmax-Jacobian row sums at the full backward size.
 """
+import contextlib
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -13,6 +16,31 @@ from tests.dcn_testutil import assert_bwd, f64, gpu_backward, gpu_forward, probl
 pytestmark = pytest.mark.gpu
 
 RNG = np.random.default_rng(77)
+
+
+@contextlib.contextmanager
+def env(**kv):
+    """Set (value) or clear (None) environment variables for the block."""
+    old = {k: os.environ.get(k) for k in kv}
+    for k, v in kv.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
+    try:
+        yield
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
+def backward_path(path):
+    """"auto": the library's choice (the TMA-tiled kernel where it applies);
+    "direct": the direct-gather kernel."""
+    return env(DCN_CORE_BACKWARD="direct" if path == "direct" else None)
 
 
 def near_kink_taps(p, off):
@@ -66,11 +94,12 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["auto", "direct"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_" +
                                              "_".join(f"{k}{v}" for k, v in c[5].items())
                                              for c in CASES])
-def test_backward_matches_oracle(oracle_mod, case, dtype):
+def test_backward_matches_oracle(oracle_mod, case, dtype, path):
     N, H, W, G, Cg, kw = case
     if dtype == "bf16" and Cg * 2 < 16:
         pytest.skip("bf16 needs Cg >= 8")
@@ -83,7 +112,55 @@ def test_backward_matches_oracle(oracle_mod, case, dtype):
     off = (1.5 * RNG.standard_normal((N, Ho, Wo, G * KK * 2))).astype(np.float32)
     mask = RNG.standard_normal((N, Ho, Wo, G * KK)).astype(np.float32)
     gout = RNG.standard_normal((N, Ho, Wo, G * Cg)).astype(np.float32)
-    check(oracle_mod, p, x, off, mask, gout, dtype)
+    with backward_path(path):
+        check(oracle_mod, p, x, off, mask, gout, dtype)
+
+
+@pytest.mark.parametrize("halo,tile", [("0", "1x1"), ("2", "3x5"), ("9", "32x32"), ("5", "7x64")])
+def test_tiled_backward_tile_and_halo_settings(oracle_mod, halo, tile):
+    """Every tile shape and halo width of the tiled backward gives the same
+    gradients (only the split between box reads and global reads changes)."""
+    with env(DCN_CORE_HALO=halo, DCN_CORE_BWD_TILED_TILE=tile):
+        for dtype in ("f32", "bf16"):
+            for kw in (dict(), dict(stride=2, softmax=0), dict(remove_center=1)):
+                kw = {"stride": 1, "softmax": 1, "remove_center": 0, **kw}
+                N, H, W, G, Cg = 2, 29, 31, 3, 16
+                p = dcn.make_problem(N, H, W, G, Cg, 3, kw["stride"], 1, 1, 2.0, kw["softmax"],
+                                     dtype, kw["remove_center"])
+                Ho, Wo = dcn.dcn_core_output_hw(p)
+                T = dcn.taps(p)
+                x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+                off = (3.0 * RNG.standard_normal((N, Ho, Wo, G * T * 2))).astype(np.float32)
+                mask = RNG.standard_normal((N, Ho, Wo, G * T)).astype(np.float32)
+                gout = RNG.standard_normal((N, Ho, Wo, G * Cg)).astype(np.float32)
+                check(oracle_mod, p, x, off, mask, gout, dtype)
+
+
+def test_backward_paths_agree_on_nonfinite_and_border_offsets(oracle_mod):
+    """NaN, infinite, huge and exact-border offsets: both backward kernels
+    match the oracle."""
+    N, H, W, G, Cg = 1, 9, 11, 2, 16
+    p = dcn.make_problem(N, H, W, G, Cg, offset_scale=2.0)
+    x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    off = (1.5 * RNG.standard_normal((N, H, W, G, 9, 2))).astype(np.float32)
+    off[0, 0, 0, 0, :, 0] = np.nan
+    off[0, 1, 1, 0, :, 1] = np.inf
+    off[0, 2, 2, 1, :, 0] = -np.inf
+    off[0, 3, 3, 0, :, :] = 1e30
+    off[0, 4, :, 1, 4, 0] = (np.array([-1, 0, W - 1, W] * 3)[:W] - np.arange(W)) / 2.0
+    off = off.reshape(N, H, W, -1)
+    mask = RNG.standard_normal((N, H, W, G * 9)).astype(np.float32)
+    gout = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    for path in ("auto", "direct"):
+        with backward_path(path):
+            xd, od, md, gd = (to_dev(a, "f32") for a in (x, off, mask, gout))
+            gx, goff, gm = gpu_backward(p, xd, od, md, gd)
+            torch.cuda.synchronize()
+        rx, roff, rm = oracle_mod.backward(x, off, mask, gout, **problem_kwargs(p))
+        # NaN / inf offsets give NaN-free zeros on both sides
+        assert_bwd(f64(gx), rx, f"grad_input {path}")
+        assert_bwd(f64(goff), roff, f"grad_offset {path}")
+        assert_bwd(f64(gm), rm, f"grad_mask {path}")
 
 
 def test_full_size_backward(gen_mod, oracle_mod):
