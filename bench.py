@@ -36,6 +36,9 @@ SWEEP = ["internimage_l_stage1_bf16_n64_96x96_c160", "internimage_l_stage2_bf16_
          "dcnv4_hires_bf16_n2_256x256_c192_s1_remove_center",
          "internimage_l_stage2_bwd_fp32_n32_48x48_c320",
          "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
+# The same backward workloads through dcn_core_backward_deterministic.
+DETERMINISTIC_SWEEP = ["internimage_l_stage2_bwd_fp32_n32_48x48_c320",
+                       "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1024 * 1024
 
@@ -154,12 +157,13 @@ def dist_setup(args):
 class Step:
     """Device buffers and the launches of one step of a workload."""
 
-    def __init__(self, wl, inputs, backward: bool):
+    def __init__(self, wl, inputs, backward: bool, deterministic: bool = False):
         import torch
         import deformable_convolution_core_b200 as dcn
         self.dcn = dcn
         self.wl = wl
         self.backward = backward
+        self.deterministic = deterministic
         tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
         self.p = dcn.problem_for(wl)
         dev = torch.device("cuda")
@@ -173,7 +177,8 @@ class Step:
             self.gx = torch.empty_like(self.x)
             self.goff = torch.empty_like(self.off)
             self.gm = torch.empty_like(self.mask)
-            self.ws_bytes = dcn.dcn_core_backward_workspace(self.p)
+            self.ws_bytes = (dcn.dcn_core_backward_deterministic_workspace(self.p)
+                             if deterministic else dcn.dcn_core_backward_workspace(self.p))
             self.ws = (torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
                        if self.ws_bytes else None)
         self.stream = torch.cuda.Stream()
@@ -183,8 +188,10 @@ class Step:
         self.dcn.dcn_core_forward(self.p, self.x, self.off, self.mask, self.out, self.sh)
 
     def bwd(self):
-        self.dcn.dcn_core_backward(self.p, self.x, self.off, self.mask, self.gout, self.gx,
-                                   self.goff, self.gm, self.ws, self.ws_bytes, self.sh)
+        call = (self.dcn.dcn_core_backward_deterministic if self.deterministic
+                else self.dcn.dcn_core_backward)
+        call(self.p, self.x, self.off, self.mask, self.gout, self.gx, self.goff, self.gm,
+             self.ws, self.ws_bytes, self.sh)
 
     def run(self):
         if not (self.wl.backward and self.backward):
@@ -383,15 +390,18 @@ def run_sweep(gen, peak):
     """Forward GB/s of the other workloads (a few timed launches each)."""
     import torch
     out = {}
-    for name in SWEEP:
+    runs = [(name, False) for name in SWEEP] + [(name, True) for name in DETERMINISTIC_SWEEP]
+    for name, det in runs:
         wl = gen.WORKLOADS[name]
         inputs = gen.make_inputs(wl, with_grad_out=wl.backward)
-        step = Step(wl, inputs, backward=wl.backward)
+        step = Step(wl, inputs, backward=wl.backward, deterministic=det)
         total, fw, bw = timed(step, 20, 3)
         ms = bw if wl.backward else fw
         b = wl.backward_bytes() if wl.backward else wl.forward_bytes()
         gbs = b / (ms * 1e-3) / 1e9
-        out[name] = {"pass": "backward" if wl.backward else "forward", "ms": round(ms, 4),
+        key = name + (" deterministic" if det else "")
+        out[key] = {"pass": ("deterministic backward" if det else "backward") if wl.backward
+                    else "forward", "ms": round(ms, 4),
                      "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
                      "Gsamples/s": round(wl.samples / (ms * 1e-3) / 1e9, 2),
                      "MB": round(b / 1e6, 1),

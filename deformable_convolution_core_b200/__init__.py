@@ -33,6 +33,8 @@ EXPORTED_SYMBOLS = (
     "dcn_core_backward_workspace",
     "dcn_core_backward",
     "dcn_core_backward_noalloc",
+    "dcn_core_backward_deterministic_workspace",
+    "dcn_core_backward_deterministic",
     "dcn_core_sync_status",
     "dcn_status_string",
     "dcn_core_abi_version",
@@ -110,6 +112,10 @@ def load_library():
     lib.dcn_core_backward.restype = st
     lib.dcn_core_backward_noalloc.argtypes = [pp] + [vp] * 8
     lib.dcn_core_backward_noalloc.restype = st
+    lib.dcn_core_backward_deterministic_workspace.argtypes = [pp]
+    lib.dcn_core_backward_deterministic_workspace.restype = ctypes.c_size_t
+    lib.dcn_core_backward_deterministic.argtypes = [pp] + [vp] * 8 + [ctypes.c_size_t, vp]
+    lib.dcn_core_backward_deterministic.restype = st
     lib.dcn_core_sync_status.argtypes = [vp]
     lib.dcn_core_sync_status.restype = st
     lib.dcn_status_string.argtypes = [st]
@@ -207,6 +213,21 @@ def dcn_core_backward_noalloc(problem: DcnProblem, input, offset, mask, grad_out
                                    f"bytes, more than the {DCN_CORE_NOALLOC_SCRATCH_BYTES} bytes "
                                    "of scratch this entry point owns")
     _check(status, "dcn_core_backward_noalloc")
+
+
+def dcn_core_backward_deterministic_workspace(problem: DcnProblem) -> int:
+    return int(load_library().dcn_core_backward_deterministic_workspace(ctypes.byref(problem)))
+
+
+def dcn_core_backward_deterministic(problem: DcnProblem, input, offset, mask, grad_out,
+                                    grad_input, grad_offset, grad_mask, workspace,
+                                    workspace_bytes, stream=None) -> None:
+    """Bitwise-reproducible backward (see include/dcn_core.h): grad_input is
+    accumulated exactly in 64-bit fixed point inside `workspace`."""
+    _check(load_library().dcn_core_backward_deterministic(
+        ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
+        _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _ptr(workspace),
+        int(workspace_bytes), _stream(stream)), "dcn_core_backward_deterministic")
 
 
 def dcn_core_sync_status(stream=None) -> None:

@@ -25,10 +25,13 @@ struct BwdArgs {
   const void* off;
   const void* mask;
   const void* gout;
-  float* gx;     // fp32 input-gradient accumulator: grad_input itself for fp32
-                 // storage, the caller's workspace for bf16 storage
+  void* gx;      // input-gradient accumulator: fp32 (grad_input itself for fp32
+                 // storage, the caller's workspace for bf16 storage) or, for the
+                 // deterministic backward, 64-bit fixed point
   void* goff;
   void* gmask;
+  const unsigned int* det_hdr;  // deterministic backward: the pre-pass bounds
+  int det_cbits;                // ... and ceil(log2(contributions per element))
   TileParams t;
 };
 
@@ -107,6 +110,106 @@ __device__ __forceinline__ void red_add_v4_pred(float* p, float2 lo, float2 hi, 
                : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// grad_input accumulation.
+//
+// GxScatter<false>: fp32 vector reductions; the order of the additions, hence
+// the last bits of the sum, may differ between runs.
+// GxScatter<true> (deterministic backward): each fp32 contribution v is turned
+// into the 64-bit integer round(v * 2^S) and added exactly, so the sum does not
+// depend on the order.  S is chosen so that no partial sum can overflow: a
+// pre-pass stores max|grad_out| (and, for a raw mask, max|mask|) in the
+// header; every contribution is at most their product P in magnitude (bilinear
+// weights and softmax weights are <= 1), an element receives at most
+// 2^cbits contributions, hence |sum| * 2^S < 2^(cbits + e + S) <= 2^62 with
+// P < 2^e and S = 62 - cbits - e (clamped to [-120, 120]).
+// ---------------------------------------------------------------------------
+constexpr int kDetHeaderBytes = 256;  // header in front of the 64-bit accumulator
+
+// The fixed-point exponent S; false when the bounds are not finite (then the
+// result is NaN: the conversion writes NaN into every element).
+__device__ __forceinline__ bool det_exponent(const unsigned int* hdr, bool softmax, int cbits,
+                                             int* S) {
+  const unsigned gb = __ldg(hdr), mb = softmax ? 0x3f800000u : __ldg(hdr + 1);
+  if (gb >= 0x7f800000u || mb >= 0x7f800000u) return false;  // inf or NaN met
+  const double P = double(__uint_as_float(gb)) * double(__uint_as_float(mb));
+  int e = 0;
+  if (P > 0.0) (void)frexp(P, &e);  // P = f * 2^e, 0.5 <= f < 1
+  int s = 62 - cbits - e;
+  s = s > 120 ? 120 : s;
+  if (s < -120) return false;
+  *S = s;
+  return true;
+}
+
+template <bool DET>
+struct GxScatter;
+template <>
+struct GxScatter<false> {
+  float* p;
+  __device__ __forceinline__ GxScatter(void* base, const unsigned int*, bool, int)
+      : p(static_cast<float*>(base)) {}
+  // accumulator[e .. e+3] += (lo, hi) if pred
+  __device__ __forceinline__ void add(size_t e, float2 lo, float2 hi, bool pred) const {
+    red_add_v4_pred(p + e, lo, hi, pred);
+  }
+};
+template <>
+struct GxScatter<true> {
+  unsigned long long* p;
+  float scale;  // 2^S, or 0 when the bounds are not finite
+  __device__ __forceinline__ GxScatter(void* base, const unsigned int* hdr, bool softmax,
+                                       int cbits)
+      : p(static_cast<unsigned long long*>(base)) {
+    int S = 0;
+    scale = det_exponent(hdr, softmax, cbits, &S) ? __int_as_float((S + 127) << 23) : 0.f;
+  }
+  __device__ __forceinline__ void add(size_t e, float2 lo, float2 hi, bool pred) const {
+    // v * 2^S is exact (a power-of-two scaling below 2^62); the conversion rounds
+    // it to the nearest integer.
+    const long long a = __float2ll_rn(lo.x * scale), b = __float2ll_rn(lo.y * scale);
+    const long long c = __float2ll_rn(hi.x * scale), d = __float2ll_rn(hi.y * scale);
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
+        " @q red.global.add.u64 [%0], %1;\n @q red.global.add.u64 [%0+8], %2;\n"
+        " @q red.global.add.u64 [%0+16], %3;\n @q red.global.add.u64 [%0+24], %4;\n}" ::"l"(p + e),
+        "l"(a), "l"(b), "l"(c), "l"(d), "r"(int(pred))
+        : "memory");
+  }
+};
+
+// max |v| over n values, as float bits, into *out (atomicMax; *out starts at 0).
+// NaN compares above +inf, so a non-finite input shows as bits >= 0x7f800000.
+template <typename T>
+__global__ void dcn_absmax_kernel(const T* __restrict__ v, size_t n, unsigned int* out) {
+  unsigned m = 0;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += size_t(gridDim.x) * blockDim.x) {
+    const float f = Storage<T>::to_float(v[i]);
+    m = max(m, __float_as_uint(f) & 0x7fffffffu);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(out, m);
+}
+
+// 64-bit fixed-point accumulator -> grad_input: sum * 2^-S, rounded once to
+// fp32 (then to nearest-even bf16 for bf16 storage); NaN everywhere when the
+// bounds were not finite.
+template <typename T>
+__global__ void dcn_fixed_to_grad_kernel(const long long* __restrict__ acc, T* __restrict__ out,
+                                         size_t n, const unsigned int* hdr, int softmax,
+                                         int cbits) {
+  int S = 0;
+  const bool ok = det_exponent(hdr, softmax != 0, cbits, &S);
+  const double inv = ok ? ldexp(1.0, -S) : 0.0;
+  for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += size_t(gridDim.x) * blockDim.x) {
+    const float f = ok ? float(double(acc[i]) * inv) : __int_as_float(0x7fc00000);
+    Storage<T>::store_float(out + i, f);
+  }
+}
+
 template <int LANES>
 __device__ __forceinline__ float unit_sum(float v, unsigned mask) {
 #pragma unroll
@@ -115,7 +218,7 @@ __device__ __forceinline__ float unit_sum(float v, unsigned mask) {
 }
 
 // A lane owns 4 channels of its unit: LANES = Cg / 4 lanes per unit.
-template <typename T, int LANES, int KKS, bool SOFTMAX>
+template <typename T, int LANES, int KKS, bool SOFTMAX, bool DET>
 __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs a) {
   using St = Staged<T>;
   constexpr int CPL = 4;
@@ -144,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
   const size_t img_off = size_t(tc.n) * t.H * rowE + size_t(sub) * CPL;
   const char* xbytes = reinterpret_cast<const char*>(a.x);
   const char* gobytes = reinterpret_cast<const char*>(a.gout);
+  const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits);
 
   for (int v0 = warp * UPW; v0 < units; v0 += kWarps * UPW) {
     const UnitCoord u = unit_coord(t, tc, v0 + lane / LANES);
@@ -151,7 +255,6 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
     const int row0 = u.g * KK;
     const size_t g_off = img_off + size_t(u.g) * t.Cg;
     const char* xg = xbytes + g_off * sizeof(T);
-    float* gxg = a.gx + g_off;
     const size_t upix = size_t(tc.n * t.Ho + u.ho) * t.Wo + u.wo;
     const size_t unit = upix * t.G + u.g;
     const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride - t.pad;
@@ -183,15 +286,9 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
 #pragma unroll
           for (int j = 0; j < CPL; ++j) dsum = fmaf(go[j], cv[j], dsum);
           dc[c] = dsum;
-          if (cval[c]) {
-            const float wv = mk * cw[c];
-            float* gp = gxg + cofs[c];
-#pragma unroll
-            for (int q = 0; q < CPL / 4; ++q)
-              atomicAdd(reinterpret_cast<float4*>(gp) + q,
-                        make_float4(wv * go[4 * q], wv * go[4 * q + 1], wv * go[4 * q + 2],
-                                    wv * go[4 * q + 3]));
-          }
+          const float wv = mk * cw[c];
+          gxs.add(size_t(ptrdiff_t(g_off) + cofs[c]), make_float2(wv * go[0], wv * go[1]),
+                  make_float2(wv * go[2], wv * go[3]), cval[c]);
         }
         s = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];
         gX = hy * (dc[1] - dc[0]) + f.ly * (dc[3] - dc[2]);
@@ -262,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
             dc[c] = pd.x + pd.y;
             const float wv = m[k] * cw[c];
             const float2 w2 = make_float2(wv, wv);
-            red_add_v4_pred(gxg + ptrdiff_t(cofs[j][c]), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23),
-                            cval[j][c]);
+            gxs.add(size_t(ptrdiff_t(g_off) + cofs[j][c]), __fmul2_rn(w2, g01),
+                    __fmul2_rn(w2, g23), cval[j][c]);
           }
           // out-of-support samples have no valid corner: every dc is 0
           s[k] = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];

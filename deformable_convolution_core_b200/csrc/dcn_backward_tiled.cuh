@@ -35,9 +35,11 @@ struct TiledBwdArgs {
   const void* off;
   const void* mask;
   const void* gout;
-  float* gx;  // fp32 grad_input accumulator, zero-filled before the launch
+  void* gx;  // grad_input accumulator (fp32, or 64-bit fixed point), zero-filled first
   void* goff;
   void* gmask;
+  const unsigned int* det_hdr;  // deterministic backward: the pre-pass bounds
+  int det_cbits;
   unsigned int* error_word;
   TiledParams t;
 };
@@ -87,8 +89,9 @@ struct BwdPiece<__nv_bfloat16> {
 };
 
 // KKS: 9 (the 3x3 window) or 8 (the window without its centre).  CS = the
-// group's bytes per pixel = 16 channels.
-template <typename T, int CS, int KKS, bool SOFTMAX>
+// group's bytes per pixel = 16 channels.  DET: exact fixed-point accumulation
+// of grad_input (GxScatter).
+template <typename T, int CS, int KKS, bool SOFTMAX, bool DET>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     dcn_backward_tiled_kernel(const __grid_constant__ CUtensorMap xmap, const TiledBwdArgs a) {
   using IO = TiledIO<T>;
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const int X0 = c.wo0 * t.stride - t.pad - t.halo;
     const size_t img = size_t(c.n) * t.H * t.W * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4;
     const char* xg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
-    float* gxg = a.gx + img;
+    const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits);
 
     for (; beta < (il + 1) * nb; beta += kTiledWarps) {
       // Staging: the prefetched inputs go to the unit slots.
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
             dc[cc] = pd.x + pd.y;
             const float wv = mk * cw[cc];
             const float2 w2 = make_float2(wv, wv);
-            red_add_v4_pred(gxg + ptrdiff_t(e), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23), in);
+            gxs.add(img + size_t(e), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23), in);
           }
           // a sample that contributes nothing has no corner in the image: every dc is 0
           float sv = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];

@@ -93,6 +93,8 @@ struct Storage;
 template <>
 struct Storage<float> {
   static constexpr int kSize = 4;
+  __device__ __forceinline__ static float to_float(float v) { return v; }
+  __device__ __forceinline__ static void store_float(float* p, float v) { *p = v; }
   // Widen the j-th channel held in a vector of words.
   template <int N>
   __device__ __forceinline__ static float chan(const uint32_t (&w)[N], int j) {
@@ -108,6 +110,11 @@ struct Storage<float> {
 template <>
 struct Storage<__nv_bfloat16> {
   static constexpr int kSize = 2;
+  __device__ __forceinline__ static float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+  // round to nearest even
+  __device__ __forceinline__ static void store_float(__nv_bfloat16* p, float v) {
+    *p = __float2bfloat16_rn(v);
+  }
   template <int N>
   __device__ __forceinline__ static float chan(const uint32_t (&w)[N], int j) {
     return (j & 1) ? bf16hi_to_f32(w[j >> 1]) : bf16lo_to_f32(w[j >> 1]);

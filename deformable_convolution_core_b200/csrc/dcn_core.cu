@@ -231,21 +231,21 @@ dcn_status forward_dispatch(const dcn_problem* p, const Plan& plan, const FwdArg
   return DCN_ERR_UNSUPPORTED;
 }
 
-template <typename T, int LANES, bool SOFTMAX>
+template <typename T, int LANES, bool SOFTMAX, bool DET>
 dcn_status backward_dispatch_sm(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                                 cudaStream_t stream) {
   switch (compile_time_taps(p)) {
-    case 9: return launch(dcn_backward_kernel<T, LANES, 9, SOFTMAX>, plan, args, stream);
-    case 8: return launch(dcn_backward_kernel<T, LANES, 8, SOFTMAX>, plan, args, stream);
-    default: return launch(dcn_backward_kernel<T, LANES, 0, SOFTMAX>, plan, args, stream);
+    case 9: return launch(dcn_backward_kernel<T, LANES, 9, SOFTMAX, DET>, plan, args, stream);
+    case 8: return launch(dcn_backward_kernel<T, LANES, 8, SOFTMAX, DET>, plan, args, stream);
+    default: return launch(dcn_backward_kernel<T, LANES, 0, SOFTMAX, DET>, plan, args, stream);
   }
 }
 
-template <typename T, int LANES>
+template <typename T, int LANES, bool DET>
 dcn_status backward_dispatch_kk(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                                 cudaStream_t stream) {
-  return p->softmax ? backward_dispatch_sm<T, LANES, true>(p, plan, args, stream)
-                    : backward_dispatch_sm<T, LANES, false>(p, plan, args, stream);
+  return p->softmax ? backward_dispatch_sm<T, LANES, true, DET>(p, plan, args, stream)
+                    : backward_dispatch_sm<T, LANES, false, DET>(p, plan, args, stream);
 }
 
 // The backward always gives a lane 4 channels (16 bytes), so that one warp
@@ -261,22 +261,26 @@ bool backward_lane_map(const dcn_problem* p, LaneMap* lm) {
   }
 }
 
-template <typename T>
+template <typename T, bool DET>
 dcn_status backward_dispatch_t(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                                cudaStream_t stream) {
   switch (plan.lm.lanes) {
-    case 1: return backward_dispatch_kk<T, 1>(p, plan, args, stream);
-    case 2: return backward_dispatch_kk<T, 2>(p, plan, args, stream);
-    case 4: return backward_dispatch_kk<T, 4>(p, plan, args, stream);
-    case 8: return backward_dispatch_kk<T, 8>(p, plan, args, stream);
+    case 1: return backward_dispatch_kk<T, 1, DET>(p, plan, args, stream);
+    case 2: return backward_dispatch_kk<T, 2, DET>(p, plan, args, stream);
+    case 4: return backward_dispatch_kk<T, 4, DET>(p, plan, args, stream);
+    case 8: return backward_dispatch_kk<T, 8, DET>(p, plan, args, stream);
     default: return DCN_ERR_UNSUPPORTED;
   }
 }
 
+// det: the accumulator is 64-bit fixed point (the deterministic backward).
 dcn_status backward_dispatch(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
-                             cudaStream_t stream) {
-  return p->dtype == DCN_BF16 ? backward_dispatch_t<__nv_bfloat16>(p, plan, args, stream)
-                              : backward_dispatch_t<float>(p, plan, args, stream);
+                             bool det, cudaStream_t stream) {
+  if (det)
+    return p->dtype == DCN_BF16 ? backward_dispatch_t<__nv_bfloat16, true>(p, plan, args, stream)
+                                : backward_dispatch_t<float, true>(p, plan, args, stream);
+  return p->dtype == DCN_BF16 ? backward_dispatch_t<__nv_bfloat16, false>(p, plan, args, stream)
+                              : backward_dispatch_t<float, false>(p, plan, args, stream);
 }
 
 // Bytes of the fp32 grad_input accumulator that bf16 storage needs.
@@ -435,17 +439,17 @@ dcn_status forward_tiled_dispatch(const dcn_problem* p, const CUtensorMap& map,
              : launch_persistent(dcn_forward_tiled_kernel<T, CS, 9, false>, map, args, smem, sms, stream);
 }
 
-template <typename T, int CS>
+template <typename T, int CS, bool DET>
 dcn_status backward_tiled_dispatch(const dcn_problem* p, const CUtensorMap& map,
                                    const TiledBwdArgs& args, size_t smem, int sms,
                                    cudaStream_t stream) {
   if (p->remove_center)
     return p->softmax
-               ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, true>, map, args, smem, sms, stream)
-               : launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, false>, map, args, smem, sms, stream);
+               ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, true, DET>, map, args, smem, sms, stream)
+               : launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, false, DET>, map, args, smem, sms, stream);
   return p->softmax
-             ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, true>, map, args, smem, sms, stream)
-             : launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, false>, map, args, smem, sms, stream);
+             ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, true, DET>, map, args, smem, sms, stream)
+             : launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, false, DET>, map, args, smem, sms, stream);
 }
 
 // Everything a tiled launch needs: the tile and box geometry, the shared
@@ -542,33 +546,37 @@ bool backward_tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
   return tensor_map_encoder() != nullptr;
 }
 
-// Launch the tiled backward on a zero-filled fp32 accumulator `acc`.
-dcn_status backward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
-                          const void* off, const void* mask, const void* gout, float* acc,
-                          void* goff, void* gmask, cudaStream_t stream) {
+// Launch the tiled backward on the zero-filled accumulator a.gx.
+dcn_status backward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const BwdArgs& a,
+                          bool det, cudaStream_t stream) {
   TiledLaunch L;
-  dcn_status st = tiled_prepare(p, Ho, Wo, x, "DCN_CORE_BWD_TILED_TILE", &L);
+  dcn_status st = tiled_prepare(p, Ho, Wo, a.x, "DCN_CORE_BWD_TILED_TILE", &L);
   if (st != DCN_OK) return st;
   TiledBwdArgs args;
   args.t = L.t;
-  args.x = x; args.off = off; args.mask = mask; args.gout = gout;
-  args.gx = acc; args.goff = goff; args.gmask = gmask;
+  args.x = a.x; args.off = a.off; args.mask = a.mask; args.gout = a.gout;
+  args.gx = a.gx; args.goff = a.goff; args.gmask = a.gmask;
+  args.det_hdr = a.det_hdr; args.det_cbits = a.det_cbits;
   args.error_word = L.dev.error_word;
-  if (p->dtype == DCN_BF16)
-    return backward_tiled_dispatch<__nv_bfloat16, 32>(p, L.map, args, L.smem, L.dev.sms, stream);
-  return backward_tiled_dispatch<float, 64>(p, L.map, args, L.smem, L.dev.sms, stream);
+  const int sms = L.dev.sms;
+  if (det)
+    return p->dtype == DCN_BF16
+               ? backward_tiled_dispatch<__nv_bfloat16, 32, true>(p, L.map, args, L.smem, sms, stream)
+               : backward_tiled_dispatch<float, 64, true>(p, L.map, args, L.smem, sms, stream);
+  return p->dtype == DCN_BF16
+             ? backward_tiled_dispatch<__nv_bfloat16, 32, false>(p, L.map, args, L.smem, sms, stream)
+             : backward_tiled_dispatch<float, 64, false>(p, L.map, args, L.smem, sms, stream);
 }
 
 // The backward's kernel launch on a zero-filled accumulator: the tiled kernel
 // where it applies, else (or when it cannot be configured) the direct one.
 dcn_status backward_launch(const dcn_problem* p, int64_t Ho, int64_t Wo, const Plan& plan,
-                           const BwdArgs& a, cudaStream_t stream) {
+                           const BwdArgs& a, bool det, cudaStream_t stream) {
   if (backward_tiled_eligible(p, Ho, Wo)) {
-    const dcn_status st = backward_tiled(p, Ho, Wo, a.x, a.off, a.mask, a.gout, a.gx, a.goff,
-                                         a.gmask, stream);
+    const dcn_status st = backward_tiled(p, Ho, Wo, a, det, stream);
     if (st != DCN_ERR_UNSUPPORTED) return st;
   }
-  return backward_dispatch(p, plan, a, stream);
+  return backward_dispatch(p, plan, a, det, stream);
 }
 }  // namespace
 }  // namespace dcn
@@ -668,8 +676,8 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
   if (st != DCN_OK) return st;
   float* acc = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(grad_input);
   if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
-  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, plan.t};
-  st = backward_launch(problem, Ho, Wo, plan, args, stream);
+  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, nullptr, 0, plan.t};
+  st = backward_launch(problem, Ho, Wo, plan, args, false, stream);
   if (st != DCN_OK || !bf16) return st;
   // bf16: round the fp32 accumulator once into grad_input.
   const size_t n4 = acc_bytes / 16;
@@ -778,8 +786,8 @@ extern "C" dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, cons
   }
   // The shared array keeps the previous call's sums: clear it first.
   if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
-  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, plan.t};
-  st = backward_launch(problem, Ho, Wo, plan, args, stream);
+  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, nullptr, 0, plan.t};
+  st = backward_launch(problem, Ho, Wo, plan, args, false, stream);
   if (st != DCN_OK || !bf16) return st;
   const size_t n4 = acc_bytes / 16;
   DeviceInfo dev;
@@ -788,4 +796,92 @@ extern "C" dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, cons
   dcn_round_to_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
                                                      static_cast<uint2*>(grad_input), n4);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Deterministic backward (dcn_core_backward_deterministic in include/dcn_core.h).
+// ---------------------------------------------------------------------------
+namespace dcn {
+namespace {
+
+int ceil_log2(int64_t n) {
+  int b = 0;
+  while ((int64_t(1) << b) < n) ++b;
+  return b;
+}
+
+size_t det_workspace_bytes(const dcn_problem* p) {
+  return size_t(kDetHeaderBytes) + size_t(p->N) * p->H * p->W * p->G * p->Cg * 8;
+}
+
+unsigned grid_for(size_t n, int sms) {
+  return unsigned(std::max<size_t>(1, std::min<size_t>((n + 255) / 256, size_t(sms) * 8)));
+}
+
+template <typename T>
+dcn_status det_passes(const dcn_problem* p, int64_t Ho, int64_t Wo, const Plan& plan,
+                      const void* input, const void* offset, const void* mask,
+                      const void* grad_out, void* grad_input, void* grad_offset,
+                      void* grad_mask, unsigned char* ws, int sms, cudaStream_t stream) {
+  unsigned int* hdr = reinterpret_cast<unsigned int*>(ws);
+  void* acc = ws + kDetHeaderBytes;
+  const size_t n_out = size_t(p->N) * Ho * Wo * p->G * p->Cg;
+  const size_t n_msk = size_t(p->N) * Ho * Wo * p->G * taps(p);
+  const size_t n_in = size_t(p->N) * p->H * p->W * p->G * p->Cg;
+  dcn_absmax_kernel<T><<<grid_for(n_out, sms), 256, 0, stream>>>(static_cast<const T*>(grad_out),
+                                                                 n_out, hdr);
+  if (!p->softmax)
+    dcn_absmax_kernel<T><<<grid_for(n_msk, sms), 256, 0, stream>>>(static_cast<const T*>(mask),
+                                                                   n_msk, hdr + 1);
+  if (cudaGetLastError() != cudaSuccess) return DCN_ERR_CUDA;
+  // An element of grad_input receives at most one contribution per (output
+  // pixel, tap) of its image and group.
+  const int cbits = ceil_log2(int64_t(Ho) * Wo * taps(p));
+  BwdArgs args{input, offset, mask, grad_out, acc, grad_offset, grad_mask, hdr, cbits, plan.t};
+  dcn_status st = backward_launch(p, Ho, Wo, plan, args, true, stream);
+  if (st != DCN_OK) return st;
+  dcn_fixed_to_grad_kernel<T><<<grid_for(n_in, sms), 256, 0, stream>>>(
+      static_cast<const long long*>(acc), static_cast<T*>(grad_input), n_in, hdr, p->softmax,
+      cbits);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace dcn
+
+extern "C" size_t dcn_core_backward_deterministic_workspace(const dcn_problem* problem) {
+  int64_t Ho, Wo;
+  if (check_problem(problem, &Ho, &Wo) != DCN_OK) return 0;
+  return det_workspace_bytes(problem);
+}
+
+extern "C" dcn_status dcn_core_backward_deterministic(
+    const dcn_problem* problem, const void* input, const void* offset, const void* mask,
+    const void* grad_out, void* grad_input, void* grad_offset, void* grad_mask, void* workspace,
+    size_t workspace_bytes, cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!input || !offset || !mask || !grad_out || !grad_input || !grad_offset || !grad_mask)
+    return DCN_ERR_INVALID_ARG;
+  const size_t ws_bytes = det_workspace_bytes(problem);
+  if (!workspace || workspace_bytes < ws_bytes) return DCN_ERR_INVALID_ARG;
+  if (!aligned(input, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
+      !aligned(grad_out, 16) || !aligned(grad_input, 16) || !aligned(grad_offset, 16) ||
+      !aligned(grad_mask, 16) || !aligned(workspace, 256))
+    return DCN_ERR_UNSUPPORTED;
+  const bool bf16 = problem->dtype == DCN_BF16;
+  Plan plan;
+  st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
+                                       : staged_bytes_per_entry<float>(),
+                 &plan, true);
+  if (st != DCN_OK) return st;
+  DeviceInfo dev;
+  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, ws_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  return bf16 ? det_passes<__nv_bfloat16>(problem, Ho, Wo, plan, input, offset, mask, grad_out,
+                                          grad_input, grad_offset, grad_mask, ws, dev.sms, stream)
+              : det_passes<float>(problem, Ho, Wo, plan, input, offset, mask, grad_out,
+                                  grad_input, grad_offset, grad_mask, ws, dev.sms, stream);
 }

@@ -183,6 +183,40 @@ DCN_API dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, const v
                                              void* grad_offset, void* grad_mask,
                                              cudaStream_t stream);
 
+/* Device workspace dcn_core_backward_deterministic needs, in bytes:
+ * 256 + N*H*W*G*Cg*8 (0 for an invalid problem). */
+DCN_API size_t dcn_core_backward_deterministic_workspace(const dcn_problem* problem);
+
+/*
+ * Backward whose results are bitwise reproducible: run after run, whatever the
+ * stream, the launch configuration or the scheduling, the same inputs give the
+ * same grad_input, grad_offset and grad_mask bits.  (The pages' backward, DCNv3
+ * extension build guide (trdm.cn), section 2.1, accumulates with atomics; this
+ * entry point trades speed for reproducibility.)
+ *
+ * Arguments and results are those of dcn_core_backward; the workspace
+ * (dcn_core_backward_deterministic_workspace bytes, 256-byte aligned, contents
+ * on entry irrelevant) replaces the bf16 accumulator.  grad_offset and
+ * grad_mask are computed exactly as by dcn_core_backward.  grad_input is
+ * accumulated exactly in 64-bit fixed point: every fp32 contribution
+ * m_k * w_corner * grad_out[c] is rounded to an integer multiple of 2^-S and
+ * the integers are summed, so the order of the additions does not matter; the
+ * sum is then rounded once to fp32 (and to nearest-even bf16 for bf16
+ * storage).  S is chosen on the device from max|grad_out| (and max|mask| for
+ * a raw mask) so that no sum can overflow: 2^-S is about 2^-62 times
+ * (max|grad_out| * max|mask weight| * Ho*Wo*KK), far below fp32 resolution
+ * for every element except those many orders of magnitude smaller than the
+ * largest.  A non-finite grad_out (or raw mask) makes every grad_input
+ * element NaN.  Cg must be 4, 8, 16 or 32; all pointers 16-byte aligned.
+ * Slower than dcn_core_backward: the 64-bit reductions are scalar.
+ */
+DCN_API dcn_status dcn_core_backward_deterministic(const dcn_problem* problem, const void* input,
+                                                   const void* offset, const void* mask,
+                                                   const void* grad_out, void* grad_input,
+                                                   void* grad_offset, void* grad_mask,
+                                                   void* workspace, size_t workspace_bytes,
+                                                   cudaStream_t stream);
+
 /* Synchronises `stream` and reports: DCN_ERR_CUDA if CUDA reports an error,
  * DCN_ERR_TIMEOUT if a kernel of this library gave up a bounded wait since
  * the last call (the device error word is then cleared), else DCN_OK. */

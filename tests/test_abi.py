@@ -132,6 +132,31 @@ def test_backward_rejects_before_launch(lib):
     assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
 
 
+def test_deterministic_backward_rejects_before_launch(lib):
+    p = dcn.make_problem(**GOOD)
+    need = dcn.dcn_core_backward_deterministic_workspace(p)
+    assert need == 256 + 1 * 8 * 8 * 2 * 16 * 8   # header + 64-bit accumulator
+    ptrs = [FAKE] * 7
+    for i in range(7):
+        bad = list(ptrs)
+        bad[i] = 0
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_backward_deterministic(p, *bad, FAKE, need, 0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    for ws, nbytes in [(None, need), (FAKE, need - 8)]:
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_backward_deterministic(p, *ptrs, ws, nbytes, 0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    with pytest.raises(dcn.DcnError) as e:   # the workspace must be 256-byte aligned
+        dcn.dcn_core_backward_deterministic(p, *ptrs, FAKE + 16, need, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    pc = dcn.make_problem(**{**GOOD, "Cg": 12})
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward_deterministic(pc, *ptrs, FAKE, 1 << 20, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    assert dcn.dcn_core_backward_deterministic_workspace(dcn.make_problem(**{**GOOD, "N": 0})) == 0
+
+
 def test_forward_host_rejects_before_copy(lib):
     p = dcn.make_problem(**GOOD)
     with pytest.raises(dcn.DcnError) as e:
