@@ -35,6 +35,7 @@ EXPORTED_SYMBOLS = (
     "dcn_core_backward_noalloc",
     "dcn_core_backward_deterministic_workspace",
     "dcn_core_backward_deterministic",
+    "dcn_core_offset_mask_projection",
     "dcn_core_sync_status",
     "dcn_status_string",
     "dcn_core_abi_version",
@@ -116,6 +117,8 @@ def load_library():
     lib.dcn_core_backward_deterministic_workspace.restype = ctypes.c_size_t
     lib.dcn_core_backward_deterministic.argtypes = [pp] + [vp] * 8 + [ctypes.c_size_t, vp]
     lib.dcn_core_backward_deterministic.restype = st
+    lib.dcn_core_offset_mask_projection.argtypes = [pp, vp, ctypes.c_int, vp, vp, vp, vp, vp]
+    lib.dcn_core_offset_mask_projection.restype = st
     lib.dcn_core_sync_status.argtypes = [vp]
     lib.dcn_core_sync_status.restype = st
     lib.dcn_status_string.argtypes = [st]
@@ -228,6 +231,17 @@ def dcn_core_backward_deterministic(problem: DcnProblem, input, offset, mask, gr
         ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
         _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _ptr(workspace),
         int(workspace_bytes), _stream(stream)), "dcn_core_backward_deterministic")
+
+
+def dcn_core_offset_mask_projection(problem: DcnProblem, query, Cq: int, weight, bias, offset,
+                                    mask, stream=None) -> None:
+    """offset / mask = query @ weight.T + bias on the tensor cores (see
+    include/dcn_core.h).  query (N, Ho, Wo, Cq) and weight (G*KK*3, Cq) are
+    bf16; bias (G*KK*3) fp32 or None; offset and mask are written in the
+    problem's storage type and the layouts dcn_core_forward reads."""
+    _check(load_library().dcn_core_offset_mask_projection(
+        ctypes.byref(problem), _ptr(query), int(Cq), _ptr(weight), _ptr(bias), _ptr(offset),
+        _ptr(mask), _stream(stream)), "dcn_core_offset_mask_projection")
 
 
 def dcn_core_sync_status(stream=None) -> None:

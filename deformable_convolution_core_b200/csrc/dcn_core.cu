@@ -18,6 +18,7 @@
 #include "dcn_backward_tiled.cuh"
 #include "dcn_forward.cuh"
 #include "dcn_forward_tiled.cuh"
+#include "dcn_projection.cuh"
 
 namespace dcn {
 
@@ -884,4 +885,81 @@ extern "C" dcn_status dcn_core_backward_deterministic(
                                           grad_input, grad_offset, grad_mask, ws, dev.sms, stream)
               : det_passes<float>(problem, Ho, Wo, plan, input, offset, mask, grad_out,
                                   grad_input, grad_offset, grad_mask, ws, dev.sms, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Offset / mask projection (dcn_core_offset_mask_projection in include/dcn_core.h).
+// ---------------------------------------------------------------------------
+namespace dcn {
+namespace {
+
+// 2-D bf16 tensor map (inner, outer) with a (64, 128) box and 128-byte swizzle.
+dcn_status bf16_kmajor_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer) {
+  const cuuint64_t dims[2] = {cuuint64_t(inner), cuuint64_t(outer)};
+  const cuuint64_t strides[1] = {cuuint64_t(inner) * 2};
+  const cuuint32_t box[2] = {cuuint32_t(kPjBK), cuuint32_t(kPjBM)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult cr = tensor_map_encoder()(
+      map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return cr == CUDA_SUCCESS ? DCN_OK : DCN_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+dcn_status launch_projection(const CUtensorMap& qmap, const CUtensorMap& wmap,
+                             const ProjArgs& args, int sms, cudaStream_t stream) {
+  auto k = dcn_projection_kernel<T>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(kPjSmemBytes)) != cudaSuccess)
+    return DCN_ERR_CUDA;
+  const int grid = std::min(args.tiles, sms);
+  k<<<unsigned(grid), kPjThreads, kPjSmemBytes, stream>>>(qmap, wmap, args);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace dcn
+
+extern "C" dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem,
+                                                      const void* query, int Cq,
+                                                      const void* weight, const float* bias,
+                                                      void* offset, void* mask,
+                                                      cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!query || !weight || !offset || !mask || Cq < 1) return DCN_ERR_INVALID_ARG;
+  if (Cq % 8 != 0) return DCN_ERR_UNSUPPORTED;  // TMA rows must be 16-byte multiples
+  if (!aligned(query, 16) || !aligned(weight, 16) || !aligned(offset, 16) ||
+      !aligned(mask, 16) || (bias && !aligned(bias, 4)))
+    return DCN_ERR_UNSUPPORTED;
+  const int64_t M = int64_t(problem->N) * Ho * Wo;
+  const int64_t KK = taps(problem);
+  const int64_t nout = int64_t(problem->G) * KK * 3;
+  if (M * Cq > INT_MAX || M * nout > INT_MAX || nout > INT_MAX) return DCN_ERR_INVALID_ARG;
+  if (tensor_map_encoder() == nullptr) return DCN_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
+  if (size_t(dev.smem_optin) < kPjSmemBytes) return DCN_ERR_UNSUPPORTED;
+
+  ProjArgs args;
+  args.M = int(M);
+  args.Nout = int(nout);
+  args.n_off = int(problem->G * KK * 2);
+  args.k_blocks = (Cq + kPjBK - 1) / kPjBK;
+  args.m_tiles = int((M + kPjBM - 1) / kPjBM);
+  args.n_tiles = int((nout + kPjBN - 1) / kPjBN);
+  if (int64_t(args.m_tiles) * args.n_tiles > INT_MAX) return DCN_ERR_UNSUPPORTED;
+  args.tiles = args.m_tiles * args.n_tiles;
+  args.bias = bias;
+  args.offset = offset;
+  args.mask = mask;
+  args.error_word = dev.error_word;
+  CUtensorMap qmap, wmap;
+  if ((st = bf16_kmajor_map(&qmap, query, uint64_t(Cq), uint64_t(M))) != DCN_OK) return st;
+  if ((st = bf16_kmajor_map(&wmap, weight, uint64_t(Cq), uint64_t(nout))) != DCN_OK) return st;
+  return problem->dtype == DCN_BF16
+             ? launch_projection<__nv_bfloat16>(qmap, wmap, args, dev.sms, stream)
+             : launch_projection<float>(qmap, wmap, args, dev.sms, stream);
 }

@@ -217,6 +217,33 @@ DCN_API dcn_status dcn_core_backward_deterministic(const dcn_problem* problem, c
                                                    void* workspace, size_t workspace_bytes,
                                                    cudaStream_t stream);
 
+/*
+ * Offset and mask projection of the DCNv3 block on the tensor cores.  The
+ * block predicts each (pixel, group, tap)'s offset pair and mask logit with
+ * linear layers on its query features (InternImage-L DCNv3 explainer
+ * (wmrh.cn), section 二 steps 1-3); with the two layers' weights stacked
+ * row-wise this is one GEMM:
+ *     P[pixel, j] = sum_c query[pixel, c] * weight[j, c] + bias[j],
+ *     j in [0, G*KK*3),  pixel = (n*Ho + ho)*Wo + wo.
+ * Columns j < G*KK*2 are written to `offset` (element j of the pixel, i.e.
+ * (g*KK + k)*2 + {dx, dy}), the others to `mask` (element j - G*KK*2), in
+ * the layouts dcn_core_forward reads and in problem->dtype.
+ *   query   device, bf16, (N, Ho, Wo, Cq), dense; Cq >= 8 and a multiple of 8
+ *   weight  device, bf16, (G*KK*3, Cq) row-major (a linear layer's weight)
+ *   bias    device, fp32, (G*KK*3), or NULL for none
+ *   offset  device, (N, Ho, Wo, G*KK*2); mask device, (N, Ho, Wo, G*KK);
+ *           both written entirely, must not overlap the inputs
+ * bf16 products are exact in fp32 and are summed in fp32 (tensor-core
+ * accumulation in tensor memory, order of the K sum unspecified); each
+ * output is rounded once to the storage type.  All pointers 16-byte aligned
+ * (bias 4-byte).  Cq not a multiple of 8 or unaligned pointers return
+ * DCN_ERR_UNSUPPORTED; the usual problem checks apply.
+ */
+DCN_API dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem, const void* query,
+                                                   int Cq, const void* weight, const float* bias,
+                                                   void* offset, void* mask,
+                                                   cudaStream_t stream);
+
 /* Synchronises `stream` and reports: DCN_ERR_CUDA if CUDA reports an error,
  * DCN_ERR_TIMEOUT if a kernel of this library gave up a bounded wait since
  * the last call (the device error word is then cleared), else DCN_OK. */

@@ -169,6 +169,26 @@ def backward_units(x, offset, mask, grad_out, units, *, G, K=3, stride=1, pad=1,
     return goff, gm
 
 
+def projection(query, weight, bias=None, *, G, K=3, remove_center=0):
+    """Offset and mask projection of the DCNv3 block (InternImage-L DCNv3
+    explainer (wmrh.cn), section 二 steps 1-3: linear layers on the query
+    features predict each group's and tap's offset pair and mask logit).  With
+    the two layers' weights stacked row-wise:
+        P[pixel, j] = sum_c query[pixel, c] * weight[j, c] + bias[j]
+    in float64 (a matrix product).  query (..., Cq), weight (G*T*3, Cq), bias
+    (G*T*3) or None.  Returns (offset (..., G*T*2), mask (..., G*T)): the first
+    G*T*2 columns in the order (g, k, {dx, dy}), then the G*T mask logits."""
+    T = taps(K, remove_center)
+    q = _d(query)
+    w = _d(weight)
+    assert w.shape == (G * T * 3, q.shape[-1]), (w.shape, q.shape)
+    P = q.reshape(-1, q.shape[-1]) @ w.T
+    if bias is not None:
+        P = P + _d(bias)[None, :]
+    P = P.reshape(q.shape[:-1] + (G * T * 3,))
+    return P[..., :G * T * 2], P[..., G * T * 2:]
+
+
 def workload_kwargs(wl) -> dict:
     """Keyword arguments of forward()/backward() for a gen.Workload."""
     return dict(G=wl.G, K=wl.K, stride=wl.stride, pad=wl.pad, dil=wl.dilation,

@@ -397,3 +397,34 @@ def test_far_and_nonfinite_samples_contribute_zero(oracle_mod):
     assert np.array_equal(oracle_mod.forward(x, off, mask, G=1, softmax=0), np.zeros_like(x))
     off[..., 0::2] = -np.inf
     assert np.array_equal(oracle_mod.forward(x, off, mask, G=1, softmax=0), np.zeros_like(x))
+
+
+# --- offset / mask projection -------------------------------------------------------
+
+def test_projection_matches_explicit_sums(oracle_mod):
+    # the stacked linear layers written out as loops, on a tiny case
+    G, K, Cq = 2, 3, 5
+    q = rand(2, 3, Cq)
+    w = rand(G * 9 * 3, Cq)
+    b = rand(G * 9 * 3)
+    off, msk = oracle_mod.projection(q, w, b, G=G, K=K)
+    for i in range(2):
+        for j in range(3):
+            for col in range(G * 27):
+                v = b[col] + sum(q[i, j, c] * w[col, c] for c in range(Cq))
+                got = off[i, j, col] if col < G * 18 else msk[i, j, col - G * 18]
+                assert abs(got - v) <= 1e-14
+
+
+def test_projection_identity_and_bias(oracle_mod):
+    # identity weight: the offsets and mask are the query's columns, split at G*T*2;
+    # zero weight: the bias everywhere
+    G, K, rc = 1, 3, 1
+    T = 8
+    q = rand(4, T * 3)
+    off, msk = oracle_mod.projection(q, np.eye(T * 3), None, G=G, K=K, remove_center=rc)
+    assert np.array_equal(off, q[:, :T * 2]) and np.array_equal(msk, q[:, T * 2:])
+    b = rand(T * 3)
+    off, msk = oracle_mod.projection(q, np.zeros((T * 3, T * 3)), b, G=G, K=K, remove_center=rc)
+    assert np.array_equal(off, np.broadcast_to(b[:T * 2], off.shape))
+    assert np.array_equal(msk, np.broadcast_to(b[T * 2:], msk.shape))
