@@ -40,7 +40,23 @@ SWEEP = ["internimage_l_stage1_bf16_n64_96x96_c160", "internimage_l_stage2_bf16_
 DETERMINISTIC_SWEEP = ["internimage_l_stage2_bwd_fp32_n32_48x48_c320",
                        "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# Offset / mask projections timed next to the sweep: (workload, query channels).
+PROJECTION_SWEEP = [("internimage_l_stage1_fp32_n32_96x96_c160", 160),
+                    ("internimage_l_stage1_bf16_n64_96x96_c160", 160),
+                    ("internimage_l_stage2_bf16_n64_48x48_c320", 320)]
 L2_BYTES = 126 * 1024 * 1024
+
+
+def bf16_peak():
+    """Dense bf16 tensor throughput (TFLOP/s): the burst cuBLAS figure of
+    MEASURED_PEAKS.json, for a kernel timed on its own."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def hbm_peak():
@@ -323,6 +339,7 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0 and world == 1 and not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
         result["sweep"] = run_sweep(gen, peak)
+        result["projection"] = run_projection(gen, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, inputs, backward)
     del step
@@ -384,6 +401,51 @@ def run_e2e(step, inputs, args, barrier, world):
     return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 3), "steps": n}
+
+
+def run_projection(gen, peak, launches=20):
+    """dcn_core_offset_mask_projection (tcgen05 GEMM) on the stage shapes:
+    bytes = query + weight + bias read, offset + mask written; flops = 2 M N K."""
+    import torch
+    import deformable_convolution_core_b200 as dcn
+    tflops_peak, tf_kind = bf16_peak()
+    out = {}
+    for name, cq in PROJECTION_SWEEP:
+        wl = gen.WORKLOADS[name]
+        d = gen.make_projection_inputs(wl, cq)
+        p = dcn.problem_for(wl)
+        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        q = torch.from_numpy(d["query"]).cuda().to(torch.bfloat16)
+        w = torch.from_numpy(d["weight"]).cuda().to(torch.bfloat16)
+        b = torch.from_numpy(d["bias"]).cuda()
+        M = wl.N * wl.Ho * wl.Wo
+        nout = wl.G * wl.KK * 3
+        off = torch.empty((M, wl.G * wl.KK * 2), dtype=tdt, device="cuda")
+        msk = torch.empty((M, wl.G * wl.KK), dtype=tdt, device="cuda")
+        s = torch.cuda.Stream()
+        for _ in range(3):
+            dcn.dcn_core_offset_mask_projection(p, q, cq, w, b, off, msk, s)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(launches):
+            dcn.dcn_core_offset_mask_projection(p, q, cq, w, b, off, msk, s)
+        e1.record(s)
+        torch.cuda.synchronize()
+        dcn.dcn_core_sync_status(s)
+        ms = e0.elapsed_time(e1) / launches
+        nbytes = M * cq * 2 + nout * cq * 2 + nout * 4 + M * nout * wl.esize
+        flops = 2.0 * M * nout * cq
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tfs = flops / (ms * 1e-3) / 1e12
+        out[f"{name} Cq={cq}"] = {
+            "ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
+            "TFLOP/s": round(tfs, 1), "frac_of_bf16_tensor": round(tfs / tflops_peak, 4),
+            "bound": "hbm" if nbytes / (peak * 1e9) > flops / (tflops_peak * 1e12) else "tensor",
+            "MB": round(nbytes / 1e6, 1), "out_dtype": wl.dtype, "tensor_peak_source": tf_kind}
+        del q, w, b, off, msk
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_sweep(gen, peak):

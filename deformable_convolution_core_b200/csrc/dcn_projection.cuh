@@ -14,8 +14,9 @@
 // streams 64-wide K blocks of the query and weight tiles into a 4-stage
 // shared-memory ring with TMA (128-byte swizzle); warp 1 allocates 256 TMEM
 // columns (two 128-column accumulators) and one of its threads issues
-// tcgen05.mma (M = 128, N = 128, K = 16) and tcgen05.commit; warps 2-5 drain
-// an accumulator with tcgen05.ld, add the bias and store, staging each 32x32
+// tcgen05.mma (M = 128, N = 128, K = 16) and tcgen05.commit; warps 2-9 drain
+// an accumulator with tcgen05.ld (two warps per 32-lane quarter of TMEM, each
+// taking 64 of the 128 columns), add the bias and store, staging each 32x32
 // block through shared memory so that every store instruction writes one
 // pixel's contiguous columns.  The epilogue of one tile overlaps the MMAs of
 // the next.  Every mbarrier wait is bounded; on expiry the kernel sets the
@@ -33,12 +34,14 @@ constexpr int kPjBM = 128;      // pixels per tile (MMA M, TMEM lanes)
 constexpr int kPjBN = 128;      // columns per tile (MMA N)
 constexpr int kPjBK = 64;       // K block: one 128-byte swizzle atom of bf16
 constexpr int kPjStages = 4;
-constexpr int kPjThreads = 192; // 6 warps: TMA, MMA, 4 x epilogue
+constexpr int kPjEpiWarps = 8;   // two per TMEM lane quarter, each draining half the columns
+constexpr int kPjThreads = (2 + kPjEpiWarps) * 32;  // TMA warp, MMA warp, epilogue warps
 constexpr uint32_t kPjTmemCols = 256;
 constexpr uint32_t kPjStageBytes = (kPjBM + kPjBN) * kPjBK * 2;  // A + B, 32 KB
 constexpr int kPjEpiPitch = 33;  // floats per staged row (conflict-free transpose)
 constexpr size_t kPjSmemBytes = 1024 /* alignment slack */ + size_t(kPjStages) * kPjStageBytes +
-                                4 * 32 * kPjEpiPitch * 4 + 256 /* barriers, TMEM address */;
+                                size_t(kPjEpiWarps) * 32 * kPjEpiPitch * 4 +
+                                256 /* barriers, TMEM address */;
 
 struct ProjArgs {
   int M;         // pixels N*Ho*Wo
@@ -130,11 +133,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-template <typename T>
-__device__ __forceinline__ void store_out(void* base, size_t i, float v) {
-  Storage<T>::store_float(static_cast<T*>(base) + i, v);
-}
-
 // T: storage type of the offset and mask outputs (fp32 or bf16).
 template <typename T>
 __global__ void __launch_bounds__(kPjThreads, 1)
@@ -147,7 +145,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
   unsigned char* stage_a = smem;
   unsigned char* stage_b = smem + size_t(kPjStages) * kPjBM * kPjBK * 2;
   float* epi = reinterpret_cast<float*>(smem + size_t(kPjStages) * kPjStageBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(epi + 4 * 32 * kPjEpiPitch);
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi + kPjEpiWarps * 32 * kPjEpiPitch);
   uint64_t* empty = full + kPjStages;
   uint64_t* tfull = empty + kPjStages;  // accumulator ready (2)
   uint64_t* tempty = tfull + 2;         // accumulator drained (2)
@@ -163,7 +161,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[b], kPjEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(mma_done, 1);
     *s_abort = 0;
@@ -253,8 +251,9 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       (void)mbar_wait_bounded(mma_done, 0);
     }
   } else {
-    // ---- epilogue: warps 2-5, TMEM lanes 32 * (warp % 4) ... + 31 ----
+    // ---- epilogue: warps 2-9; TMEM lanes 32 * (warp % 4) ... + 31, columns of half h ----
     const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
     float* st = epi + (warp - 2) * 32 * kPjEpiPitch;
     const int n_mask = a.Nout - a.n_off;
     uint32_t li = 0;
@@ -266,26 +265,33 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       }
       tc_fence_after();
       const int mt = tile / a.n_tiles, nt = tile - mt * a.n_tiles;
+      const int row0 = mt * kPjBM + q * 32;
+      const int rows = a.M - row0;  // rows of this quarter inside the image batch
 #pragma unroll 1
-      for (int c = 0; c < kPjBN / 32; ++c) {
+      for (int c = 2 * h; c < 2 * h + 2; ++c) {
         float v[32];
         tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kPjBN + c * 32), v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) st[lane * kPjEpiPitch + i] = v[i];  // row = lane
         __syncwarp();
+        // this lane's column, its tensor and that tensor's row pitch
         const int col = nt * kPjBN + c * 32 + lane;
         const bool cin = col < a.Nout;
         const float b = (a.bias != nullptr && cin) ? a.bias[col] : 0.f;
-#pragma unroll 4
+        T* dst;
+        size_t pitch;
+        if (col < a.n_off) {
+          dst = static_cast<T*>(a.offset) + col;
+          pitch = size_t(a.n_off);
+        } else {
+          dst = static_cast<T*>(a.mask) + (col - a.n_off);
+          pitch = size_t(n_mask);
+        }
+        dst += size_t(row0) * pitch;
+#pragma unroll 8
         for (int r = 0; r < 32; ++r) {
-          const int pixel = mt * kPjBM + q * 32 + r;
-          if (cin && pixel < a.M) {
-            const float val = st[r * kPjEpiPitch + lane] + b;
-            if (col < a.n_off)
-              store_out<T>(a.offset, size_t(pixel) * a.n_off + col, val);
-            else
-              store_out<T>(a.mask, size_t(pixel) * n_mask + (col - a.n_off), val);
-          }
+          if (cin && r < rows) Storage<T>::store_float(dst, st[r * kPjEpiPitch + lane] + b);
+          dst += pitch;
         }
         __syncwarp();
       }

@@ -24,6 +24,8 @@ _SRC = os.path.join(_HERE, "dcn_gen.c")
 _LIB_PATH = os.path.join(_HERE, "libdcngen.so")
 
 TID_X, TID_OFFSET, TID_MASK, TID_GRAD_OUT, TID_FAR_SELECT, TID_FAR_VALUE = 1, 2, 3, 4, 5, 6
+# inputs of the offset / mask projection: query features, weight, bias
+TID_QUERY, TID_WEIGHT, TID_BIAS = 7, 8, 9
 
 _lib = None
 
@@ -138,5 +140,19 @@ def make_inputs(wl: Workload | str, seed: int | None = None, n_images: int | Non
     return out
 
 
-__all__ = ["WORKLOADS", "Workload", "output_hw", "make_inputs", "uniform", "normal",
+def make_projection_inputs(wl, Cq: int, seed=None) -> dict:
+    """Host float32 arrays for the offset / mask projection of a workload:
+    query (N, Ho, Wo, Cq) ~ N(0, 1), weight (G*KK*3, Cq) ~ N(0, 1/Cq) (unit
+    output variance) and bias (G*KK*3) ~ N(0, 1)."""
+    if isinstance(wl, str):
+        wl = WORKLOADS[wl]
+    seed = wl.seed if seed is None else seed
+    Ho, Wo = output_hw(wl)
+    nout = wl.G * wl.KK * 3
+    return {"query": normal(seed, TID_QUERY, (wl.N, Ho, Wo, Cq), 0.0, 1.0),
+            "weight": normal(seed, TID_WEIGHT, (nout, Cq), 0.0, float(Cq) ** -0.5),
+            "bias": normal(seed, TID_BIAS, (nout,), 0.0, 1.0)}
+
+
+__all__ = ["WORKLOADS", "Workload", "output_hw", "make_inputs", "make_projection_inputs", "uniform", "normal",
            "redraw_pairs", "raw_hash", "draw", "build"]
