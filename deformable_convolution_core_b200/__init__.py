@@ -36,6 +36,7 @@ EXPORTED_SYMBOLS = (
     "dcn_core_backward_deterministic_workspace",
     "dcn_core_backward_deterministic",
     "dcn_core_offset_mask_projection",
+    "dcn_core_linear_bf16",
     "dcn_core_sync_status",
     "dcn_status_string",
     "dcn_core_abi_version",
@@ -119,6 +120,9 @@ def load_library():
     lib.dcn_core_backward_deterministic.restype = st
     lib.dcn_core_offset_mask_projection.argtypes = [pp, vp, ctypes.c_int, vp, vp, vp, vp, vp]
     lib.dcn_core_offset_mask_projection.restype = st
+    lib.dcn_core_linear_bf16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, vp, vp,
+                                         ctypes.c_int, vp]
+    lib.dcn_core_linear_bf16.restype = st
     lib.dcn_core_sync_status.argtypes = [vp]
     lib.dcn_core_sync_status.restype = st
     lib.dcn_status_string.argtypes = [st]
@@ -242,6 +246,18 @@ def dcn_core_offset_mask_projection(problem: DcnProblem, query, Cq: int, weight,
     _check(load_library().dcn_core_offset_mask_projection(
         ctypes.byref(problem), _ptr(query), int(Cq), _ptr(weight), _ptr(bias), _ptr(offset),
         _ptr(mask), _stream(stream)), "dcn_core_offset_mask_projection")
+
+
+def dcn_core_linear_bf16(input, M: int, K: int, weight, Nout: int, bias, output,
+                         out_dtype="f32", stream=None) -> None:
+    """output (M, Nout) = input (M, K) @ weight (Nout, K).T + bias on the tensor
+    cores; bf16 operands, fp32 accumulation, output in out_dtype."""
+    if isinstance(out_dtype, str):
+        out_dtype = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16,
+                     "bfloat16": DCN_BF16}[out_dtype]
+    _check(load_library().dcn_core_linear_bf16(
+        _ptr(input), int(M), int(K), _ptr(weight), int(Nout), _ptr(bias), _ptr(output),
+        int(out_dtype), _stream(stream)), "dcn_core_linear_bf16")
 
 
 def dcn_core_sync_status(stream=None) -> None:

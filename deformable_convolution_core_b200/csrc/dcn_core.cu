@@ -921,6 +921,47 @@ dcn_status launch_projection(const CUtensorMap& qmap, const CUtensorMap& wmap,
 }  // namespace
 }  // namespace dcn
 
+namespace dcn {
+namespace {
+
+// out0[m, j] (j < n_split) / out1[m, j - n_split] (j >= n_split) =
+//     sum_c a[m, c] * w[j, c] + bias[j]  on the tensor cores.
+dcn_status bf16_gemm(const void* a, int64_t M, int K, const void* w, int64_t nout,
+                     int64_t n_split, const float* bias, void* out0, void* out1, bool bf16_out,
+                     cudaStream_t stream) {
+  if (K % 8 != 0) return DCN_ERR_UNSUPPORTED;  // TMA rows must be 16-byte multiples
+  if (!aligned(a, 16) || !aligned(w, 16) || !aligned(out0, 16) || !aligned(out1, 16) ||
+      (bias && !aligned(bias, 4)))
+    return DCN_ERR_UNSUPPORTED;
+  if (M * K > INT_MAX || M * nout > INT_MAX || nout > INT_MAX) return DCN_ERR_INVALID_ARG;
+  if (tensor_map_encoder() == nullptr) return DCN_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
+  if (size_t(dev.smem_optin) < kPjSmemBytes) return DCN_ERR_UNSUPPORTED;
+  ProjArgs args;
+  args.M = int(M);
+  args.Nout = int(nout);
+  args.n_off = int(n_split);
+  args.k_blocks = (K + kPjBK - 1) / kPjBK;
+  args.m_tiles = int((M + kPjBM - 1) / kPjBM);
+  args.n_tiles = int((nout + kPjBN - 1) / kPjBN);
+  if (int64_t(args.m_tiles) * args.n_tiles > INT_MAX) return DCN_ERR_UNSUPPORTED;
+  args.tiles = args.m_tiles * args.n_tiles;
+  args.bias = bias;
+  args.offset = out0;
+  args.mask = out1;
+  args.error_word = dev.error_word;
+  CUtensorMap amap, wmap;
+  dcn_status st;
+  if ((st = bf16_kmajor_map(&amap, a, uint64_t(K), uint64_t(M))) != DCN_OK) return st;
+  if ((st = bf16_kmajor_map(&wmap, w, uint64_t(K), uint64_t(nout))) != DCN_OK) return st;
+  return bf16_out ? launch_projection<__nv_bfloat16>(amap, wmap, args, dev.sms, stream)
+                  : launch_projection<float>(amap, wmap, args, dev.sms, stream);
+}
+
+}  // namespace
+}  // namespace dcn
+
 extern "C" dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem,
                                                       const void* query, int Cq,
                                                       const void* weight, const float* bias,
@@ -930,36 +971,18 @@ extern "C" dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem
   dcn_status st = check_problem(problem, &Ho, &Wo);
   if (st != DCN_OK) return st;
   if (!query || !weight || !offset || !mask || Cq < 1) return DCN_ERR_INVALID_ARG;
-  if (Cq % 8 != 0) return DCN_ERR_UNSUPPORTED;  // TMA rows must be 16-byte multiples
-  if (!aligned(query, 16) || !aligned(weight, 16) || !aligned(offset, 16) ||
-      !aligned(mask, 16) || (bias && !aligned(bias, 4)))
-    return DCN_ERR_UNSUPPORTED;
   const int64_t M = int64_t(problem->N) * Ho * Wo;
   const int64_t KK = taps(problem);
-  const int64_t nout = int64_t(problem->G) * KK * 3;
-  if (M * Cq > INT_MAX || M * nout > INT_MAX || nout > INT_MAX) return DCN_ERR_INVALID_ARG;
-  if (tensor_map_encoder() == nullptr) return DCN_ERR_UNSUPPORTED;
-  DeviceInfo dev;
-  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
-  if (size_t(dev.smem_optin) < kPjSmemBytes) return DCN_ERR_UNSUPPORTED;
+  return bf16_gemm(query, M, Cq, weight, int64_t(problem->G) * KK * 3,
+                   int64_t(problem->G) * KK * 2, bias, offset, mask,
+                   problem->dtype == DCN_BF16, stream);
+}
 
-  ProjArgs args;
-  args.M = int(M);
-  args.Nout = int(nout);
-  args.n_off = int(problem->G * KK * 2);
-  args.k_blocks = (Cq + kPjBK - 1) / kPjBK;
-  args.m_tiles = int((M + kPjBM - 1) / kPjBM);
-  args.n_tiles = int((nout + kPjBN - 1) / kPjBN);
-  if (int64_t(args.m_tiles) * args.n_tiles > INT_MAX) return DCN_ERR_UNSUPPORTED;
-  args.tiles = args.m_tiles * args.n_tiles;
-  args.bias = bias;
-  args.offset = offset;
-  args.mask = mask;
-  args.error_word = dev.error_word;
-  CUtensorMap qmap, wmap;
-  if ((st = bf16_kmajor_map(&qmap, query, uint64_t(Cq), uint64_t(M))) != DCN_OK) return st;
-  if ((st = bf16_kmajor_map(&wmap, weight, uint64_t(Cq), uint64_t(nout))) != DCN_OK) return st;
-  return problem->dtype == DCN_BF16
-             ? launch_projection<__nv_bfloat16>(qmap, wmap, args, dev.sms, stream)
-             : launch_projection<float>(qmap, wmap, args, dev.sms, stream);
+extern "C" dcn_status dcn_core_linear_bf16(const void* input, int M, int K, const void* weight,
+                                           int Nout, const float* bias, void* output,
+                                           dcn_dtype out_dtype, cudaStream_t stream) {
+  if (!input || !weight || !output || M < 1 || K < 1 || Nout < 1) return DCN_ERR_INVALID_ARG;
+  if (out_dtype != DCN_F32 && out_dtype != DCN_BF16) return DCN_ERR_INVALID_ARG;
+  return bf16_gemm(input, M, K, weight, Nout, Nout, bias, output, output, out_dtype == DCN_BF16,
+                   stream);
 }

@@ -244,6 +244,22 @@ DCN_API dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem, c
                                                    void* offset, void* mask,
                                                    cudaStream_t stream);
 
+/*
+ * The linear layers on either side of the core operator in the DCNv3 block
+ * (InternImage-L DCNv3 explainer (wmrh.cn), section 二: input_proj before it,
+ * output_proj after it), as one tensor-core GEMM with bf16 operands:
+ *     output[m, j] = sum_c input[m, c] * weight[j, c] + bias[j]
+ *   input   device, bf16, (M, K) row-major; K >= 8 and a multiple of 8
+ *   weight  device, bf16, (Nout, K) row-major (a linear layer's weight)
+ *   bias    device, fp32, (Nout), or NULL
+ *   output  device, (M, Nout) in out_dtype (fp32 or bf16), written entirely
+ * Same arithmetic, alignment rules and errors as
+ * dcn_core_offset_mask_projection (M*K and M*Nout below 2^31).
+ */
+DCN_API dcn_status dcn_core_linear_bf16(const void* input, int M, int K, const void* weight,
+                                        int Nout, const float* bias, void* output,
+                                        dcn_dtype out_dtype, cudaStream_t stream);
+
 /* Synchronises `stream` and reports: DCN_ERR_CUDA if CUDA reports an error,
  * DCN_ERR_TIMEOUT if a kernel of this library gave up a bounded wait since
  * the last call (the device error word is then cleared), else DCN_OK. */

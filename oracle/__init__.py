@@ -189,6 +189,19 @@ def projection(query, weight, bias=None, *, G, K=3, remove_center=0):
     return P[..., :G * T * 2], P[..., G * T * 2:]
 
 
+def linear(x, weight, bias=None):
+    """A linear layer in float64: x (..., K) @ weight (Nout, K)^T + bias (Nout).
+    The DCNv3 block's input_proj and output_proj around the core operator
+    (InternImage-L DCNv3 explainer (wmrh.cn), section 二)."""
+    a = _d(x)
+    w = _d(weight)
+    assert w.shape[1] == a.shape[-1], (w.shape, a.shape)
+    y = a.reshape(-1, a.shape[-1]) @ w.T
+    if bias is not None:
+        y = y + _d(bias)[None, :]
+    return y.reshape(a.shape[:-1] + (w.shape[0],))
+
+
 def workload_kwargs(wl) -> dict:
     """Keyword arguments of forward()/backward() for a gen.Workload."""
     return dict(G=wl.G, K=wl.K, stride=wl.stride, pad=wl.pad, dil=wl.dilation,

@@ -175,3 +175,29 @@ def test_library_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in text.lower(), os.path.join(dirpath, f)
+
+
+def test_projection_and_linear_reject_before_launch(lib):
+    p = dcn.make_problem(**GOOD)
+    for args in [(0, 64, FAKE, None, FAKE, FAKE), (FAKE, 64, 0, None, FAKE, FAKE),
+                 (FAKE, 64, FAKE, None, 0, FAKE), (FAKE, 64, FAKE, None, FAKE, 0),
+                 (FAKE, 0, FAKE, None, FAKE, FAKE)]:
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_offset_mask_projection(p, *args, stream=0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    for args in [(FAKE, 60, FAKE, None, FAKE, FAKE),        # Cq not a multiple of 8
+                 (FAKE + 8, 64, FAKE, None, FAKE, FAKE),    # unaligned query
+                 (FAKE, 64, FAKE, FAKE + 2, FAKE, FAKE)]:   # unaligned bias
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_offset_mask_projection(p, *args, stream=0)
+        assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    for args, status in [((0, 16, 64, FAKE, 32, None, FAKE), dcn.DCN_ERR_INVALID_ARG),
+                         ((FAKE, 0, 64, FAKE, 32, None, FAKE), dcn.DCN_ERR_INVALID_ARG),
+                         ((FAKE, 16, 60, FAKE, 32, None, FAKE), dcn.DCN_ERR_UNSUPPORTED),
+                         ((FAKE, 16, 64, FAKE, 32, None, FAKE + 4), dcn.DCN_ERR_UNSUPPORTED)]:
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_linear_bf16(*args, stream=0)
+        assert e.value.status == status
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_linear_bf16(FAKE, 16, 64, FAKE, 32, None, FAKE, out_dtype=7, stream=0)
+    assert e.value.status == dcn.DCN_ERR_INVALID_ARG

@@ -428,3 +428,14 @@ def test_projection_identity_and_bias(oracle_mod):
     off, msk = oracle_mod.projection(q, np.zeros((T * 3, T * 3)), b, G=G, K=K, remove_center=rc)
     assert np.array_equal(off, np.broadcast_to(b[:T * 2], off.shape))
     assert np.array_equal(msk, np.broadcast_to(b[T * 2:], msk.shape))
+
+
+def test_linear_matches_explicit_sums(oracle_mod):
+    x = rand(3, 2, 4)
+    w = rand(5, 4)
+    b = rand(5)
+    y = oracle_mod.linear(x, w, b)
+    for idx in np.ndindex(3, 2):
+        for j in range(5):
+            assert abs(y[idx + (j,)] - (b[j] + sum(x[idx + (c,)] * w[j, c] for c in range(4)))) <= 1e-14
+    assert np.array_equal(oracle_mod.linear(x, np.eye(4)), x)

@@ -112,3 +112,41 @@ def test_projection_feeds_the_forward(oracle_mod):
     torch.cuda.synchronize()
     ref = oracle_mod.forward(x, f64(off), f64(msk), **problem_kwargs(p))
     assert np.abs(f64(out) - ref).max() <= 1e-5 * np.abs(x).max()
+
+
+@pytest.mark.parametrize("M,K,Nout,out_dtype", [(300, 160, 160, "f32"), (1000, 320, 320, "bf16"),
+                                                (129, 64, 40, "f32"), (77, 8, 130, "bf16")])
+def test_linear_matches_oracle(oracle_mod, M, K, Nout, out_dtype):
+    x = bf16_round(RNG.standard_normal((M, K)))
+    w = bf16_round(RNG.standard_normal((Nout, K)) / np.sqrt(K))
+    b = torch.from_numpy(RNG.standard_normal(Nout).astype(np.float32))
+    y = torch.empty((M, Nout), dtype=torch.float32 if out_dtype == "f32" else torch.bfloat16,
+                    device="cuda")
+    dcn.dcn_core_linear_bf16(x.cuda(), M, K, w.cuda(), Nout, b.cuda(), y, out_dtype)
+    torch.cuda.synchronize()
+    xf, wf, bf = f64(x), f64(w), b.numpy().astype(np.float64)
+    ref = oracle_mod.linear(xf, wf, bf)
+    bound = 4 * K * 2.0 ** -24 * (np.abs(xf) @ np.abs(wf).T + np.abs(bf)[None, :])
+    if out_dtype == "bf16":
+        bound = bound + 2.0 ** -8 * np.abs(ref)
+    assert (np.abs(f64(y) - ref) <= bound).all()
+
+
+def test_dcnv3_block_core_path_bf16(oracle_mod):
+    """The block around the core operator, bf16 activations: offset / mask
+    projection (tensor cores) -> core forward -> output_proj (tensor cores).
+    Each GPU stage is checked against the oracle fed that stage's GPU inputs."""
+    N, H, W, G, Cg = 2, 24, 20, 4, 16
+    C = G * Cg
+    p, off, msk = run_case(oracle_mod, N, H, W, G, C, dtype="bf16", scale=0.5)
+    x = bf16_round(RNG.standard_normal((N, H, W, C))).cuda()
+    core = gpu_forward(p, x, off, msk)
+    w_out = bf16_round(RNG.standard_normal((C, C)) / np.sqrt(C))
+    b_out = torch.from_numpy(RNG.standard_normal(C).astype(np.float32))
+    y = torch.empty((N * H * W, C), dtype=torch.bfloat16, device="cuda")
+    dcn.dcn_core_linear_bf16(core, N * H * W, C, w_out.cuda(), C, b_out.cuda(), y, "bf16")
+    torch.cuda.synchronize()
+    ref_core = oracle_mod.forward(f64(x), f64(off), f64(msk), **problem_kwargs(p))
+    assert np.abs(f64(core) - ref_core).max() <= 1e-2 * np.abs(ref_core).max()
+    ref_y = oracle_mod.linear(f64(core).reshape(-1, C), f64(w_out), b_out.numpy())
+    assert np.abs(f64(y) - ref_y).max() <= 1e-2 * np.abs(ref_y).max()
