@@ -115,7 +115,8 @@ def test_projection_feeds_the_forward(oracle_mod):
 
 
 @pytest.mark.parametrize("M,K,Nout,out_dtype", [(300, 160, 160, "f32"), (1000, 320, 320, "bf16"),
-                                                (129, 64, 40, "f32"), (77, 8, 130, "bf16")])
+                                                (129, 64, 40, "f32"), (77, 8, 130, "bf16"),
+                                                (50, 16, 33, "bf16"), (70, 24, 33, "f32")])
 def test_linear_matches_oracle(oracle_mod, M, K, Nout, out_dtype):
     x = bf16_round(RNG.standard_normal((M, K)))
     w = bf16_round(RNG.standard_normal((Nout, K)) / np.sqrt(K))
