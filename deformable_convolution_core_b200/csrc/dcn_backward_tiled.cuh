@@ -71,6 +71,28 @@ struct BwdPiece<float> {
         : "memory");
   }
 };
+// The same four channels from the box in shared memory (always in bounds).
+template <typename T>
+struct BoxPiece;
+template <>
+struct BoxPiece<float> {
+  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+                 : "r"(smem_addr(p)));
+  }
+};
+template <>
+struct BoxPiece<__nv_bfloat16> {
+  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
+    uint32_t w0, w1;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(smem_addr(p)));
+    v[0] = bf16lo_to_f32(w0);
+    v[1] = bf16hi_to_f32(w0);
+    v[2] = bf16lo_to_f32(w1);
+    v[3] = bf16hi_to_f32(w1);
+  }
+};
 template <>
 struct BwdPiece<__nv_bfloat16> {
   __device__ __forceinline__ static void load(const void* p, bool pred, float (&v)[4]) {
@@ -278,15 +300,18 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           const float X = tap_coord(wo * t.stride - t.pad + (q % K) * t.dil, t.sigma, d[k].x);
           const Footprint f = footprint(Y, X, t.H, t.W);
           const bool live = valid && f.in_support;
-          uint32_t code = kBwdFar;
+          // a sample that contributes nothing keeps code 0: box offset 0, no corner
+          uint32_t code = 0;
           int ce = 0;
           if (live) {
-            code |= (uint32_t(f.v00) | uint32_t(f.v01) << 1 | uint32_t(f.v10) << 2 |
-                     uint32_t(f.v11) << 3)
-                    << 24;
+            code = (uint32_t(f.v00) | uint32_t(f.v01) << 1 | uint32_t(f.v10) << 2 |
+                    uint32_t(f.v11) << 3)
+                   << 24;
             const int by = f.y0 - Y0, bx = f.x0 - X0;
             if (by >= 0 && by + 1 < t.BH && bx >= 0 && bx + 1 < t.BW)
-              code = (code & ~kBwdFar) | uint32_t((by * t.BW + bx) * CS);
+              code |= uint32_t((by * t.BW + bx) * CS);
+            else
+              code |= kBwdFar;
             ce = f.y0 * rowE + f.x0 * pixE;
           }
           // slots are 8-byte aligned (184-byte stride): two 8-byte stores
@@ -330,19 +355,36 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           const unsigned char* bp = box_lane + (code & 0xFFFFFFu);
           const float hy = 1.f - ly, hx = 1.f - lx;
           const float cw[4] = {hy * hx, hy * lx, ly * hx, ly * lx};
+          float cv[4][4];
+          if (__any_sync(0xFFFFFFFFu, far)) {
+            // some footprint of this step lies outside the box: box or global
+            // memory per lane through a generic address, predicated per corner
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int dy = cc >> 1, dx = cc & 1;
+              const bool in = ((code >> (24 + cc)) & 1u) != 0u;
+              const int e = ce + dy * rowE + dx * pixE;
+              const void* src =
+                  far ? static_cast<const void*>(xg + ptrdiff_t(e) * ptrdiff_t(sizeof(T)))
+                      : static_cast<const void*>(bp + (dy * t.BW + dx) * CS);
+              BwdPiece<T>::load(src, in, cv[cc]);
+            }
+          } else {
+            // every footprint is in the box: plain shared loads (corners outside
+            // the image read the box's zero fill, and dc is masked below anyway)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              BoxPiece<T>::load(bp + ((cc >> 1) * t.BW + (cc & 1)) * CS, cv[cc]);
+          }
           float dc[4];
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             const int dy = cc >> 1, dx = cc & 1;
             const bool in = ((code >> (24 + cc)) & 1u) != 0u;
             const int e = ce + dy * rowE + dx * pixE;  // element offset of the corner
-            const void* src = far ? static_cast<const void*>(xg + ptrdiff_t(e) * ptrdiff_t(sizeof(T)))
-                                  : static_cast<const void*>(bp + (dy * t.BW + dx) * CS);
-            float cv[4];
-            BwdPiece<T>::load(src, in, cv);
-            float2 pd = __fmul2_rn(make_float2(cv[0], cv[1]), g01);
-            pd = __ffma2_rn(make_float2(cv[2], cv[3]), g23, pd);
-            dc[cc] = pd.x + pd.y;
+            float2 pd = __fmul2_rn(make_float2(cv[cc][0], cv[cc][1]), g01);
+            pd = __ffma2_rn(make_float2(cv[cc][2], cv[cc][3]), g23, pd);
+            dc[cc] = in ? pd.x + pd.y : 0.f;
             const float wv = mk * cw[cc];
             const float2 w2 = make_float2(wv, wv);
             gxs.add(img + size_t(e), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23), in);
