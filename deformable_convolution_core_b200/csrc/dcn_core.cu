@@ -325,13 +325,16 @@ struct DeviceInfo {
   unsigned int* error_word = nullptr;
 };
 
-// Per-device constants, looked up once per device.
+// Per-device constants, looked up once per device (under a lock: calls may
+// come from several host threads).
 dcn_status device_info(DeviceInfo* out) {
   constexpr int kMaxDev = 64;
   static DeviceInfo cache[kMaxDev];
   static bool ready[kMaxDev] = {};
+  static std::mutex lock;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DCN_ERR_CUDA;
+  std::lock_guard<std::mutex> guard(lock);
   if (!ready[dev]) {
     DeviceInfo d;
     void* ew = nullptr;
