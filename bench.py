@@ -232,6 +232,7 @@ def timed(step, steps, warmup, barrier=None, ev_kernels=True):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     fwd_only = not (step.wl.backward and step.backward)
+    torch.cuda.nvtx.range_push(f"dcn {step.wl.name}: {steps} timed steps")
     t0.record(s)
     for i in range(steps):
         ev[i][0].record(s)
@@ -242,6 +243,7 @@ def timed(step, steps, warmup, barrier=None, ev_kernels=True):
             step.bwd()
         ev[i][2].record(s)
     t1.record(s)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     total = t0.elapsed_time(t1)
     fw = sum(e[0].elapsed_time(e[1]) for e in ev) / steps if fwd_only else 0.0
@@ -475,6 +477,7 @@ def run_sweep(gen, peak, reps=30, warmup=3):
             launch()
         torch.cuda.synchronize()
         times = []
+        torch.cuda.nvtx.range_push(f"dcn sweep {name}{' deterministic' if det else ''}")
         with torch.cuda.stream(step.stream):
             for _ in range(reps):
                 flush.fill_(1.0)  # evicts the inputs from L2 (not timed)
@@ -483,6 +486,7 @@ def run_sweep(gen, peak, reps=30, warmup=3):
                 launch()
                 e1.record(step.stream)
                 times.append((e0, e1))
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         ms_all = np.array([a.elapsed_time(b) for a, b in times])
         ms = float(np.median(ms_all))

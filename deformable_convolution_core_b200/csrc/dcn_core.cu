@@ -489,6 +489,10 @@ dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
   t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation; t.Ho = int(Ho); t.Wo = int(Wo);
   t.sigma = p->offset_scale; t.halo = halo; t.TH = TH; t.TW = TW;
+  // Test knob for the failure path: DCN_CORE_TEST_STALL=1 makes the first box
+  // of every CTA never arrive; the bounded waits then give up and
+  // dcn_core_sync_status reports DCN_ERR_TIMEOUT.
+  t.inject_stall = env_int("DCN_CORE_TEST_STALL", 0) == 1 ? 1 : 0;
   t.nTY = (t.Ho + TH - 1) / TH;
   t.nTX = (t.Wo + TW - 1) / TW;
   t.BH = box_extent(TH, t.stride, t.dil, halo);

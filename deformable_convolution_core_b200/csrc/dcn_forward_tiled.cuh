@@ -36,6 +36,8 @@ struct TiledParams {
   float sigma;
   int TH, TW, nTY, nTX, halo, BH, BW;
   int items;           // N * nTY * nTX * G
+  int inject_stall;    // test knob: 1 = never load the first item's box, so the
+                       // bounded waits expire and the error path runs
   int batches;         // warp batches per item: ceil(TH * TW / kTiledBatch)
   uint32_t box_bytes;  // BH * BW * Cg * sizeof(T)
   uint32_t box_stride; // box_bytes rounded up to 1024
@@ -286,6 +288,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         break;
       }
       const ItemCoord c = item_coord(t, item);
+      if (t.inject_stall && i == 0) continue;  // the first box never arrives
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(&full[b], t.box_bytes);
       tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg,

@@ -252,3 +252,31 @@ def test_full_size_workload_sampled(gen_mod, oracle_mod, name, path):
     assert_fwd(got, ref, xs, wl.dtype, name)
     # the whole output is finite and, for bf16, every value is a rounded fp32
     assert torch.isfinite(out).all()
+
+
+def test_bounded_wait_expiry_is_reported_and_recoverable():
+    """Failure detection without a GPU fault: with the test knob the first TMA
+    box of every CTA never arrives, the bounded mbarrier waits give up (about a
+    second), the kernel sets the device error word and returns;
+    dcn_core_sync_status reports DCN_ERR_TIMEOUT and clears the word, and the
+    next call works normally."""
+    p, x, off, mask = random_case(2, 23, 29, 3, 16, dtype="f32")
+    xd, od, md = to_dev(x, "f32"), to_dev(off, "f32"), to_dev(mask, "f32")
+    with forward_path("auto"):
+        ref = gpu_forward(p, xd, od, md)
+        dcn.dcn_core_sync_status()
+        old = os.environ.get("DCN_CORE_TEST_STALL")
+        os.environ["DCN_CORE_TEST_STALL"] = "1"
+        try:
+            gpu_forward(p, xd, od, md)
+            with pytest.raises(dcn.DcnError) as e:
+                dcn.dcn_core_sync_status()
+            assert e.value.status == dcn.DCN_ERR_TIMEOUT
+        finally:
+            if old is None:
+                os.environ.pop("DCN_CORE_TEST_STALL", None)
+            else:
+                os.environ["DCN_CORE_TEST_STALL"] = old
+        out = gpu_forward(p, xd, od, md)
+        dcn.dcn_core_sync_status()
+    assert torch.equal(out, ref)
