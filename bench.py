@@ -344,6 +344,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
         result["sweep"] = run_sweep(gen, peak)
         result["projection"] = run_projection(gen, peak)
+        result["block_core_path"] = run_block_core_path(gen)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, inputs, backward)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, inputs, backward)
@@ -457,6 +458,54 @@ def l1_ceiling_gsamples(wl, sm_mhz=1965.0, sms=148):
     """Samples/s (1e9) if every on-chip byte path delivered 128 B per clock
     per SM and a sample needed only its 2x2 footprint (4 * Cg * size bytes)."""
     return sms * 128.0 * sm_mhz * 1e6 / (4.0 * wl.Cg * wl.esize) / 1e9
+
+
+def run_block_core_path(gen, name="internimage_l_stage1_bf16_n64_96x96_c160", reps=20):
+    """The DCNv3 block around the core operator, bf16, three launches on one
+    stream: offset/mask projection (tensor cores) -> core forward -> output_proj
+    (tensor cores, C -> C).  Median per-launch CUDA-event times."""
+    import numpy as np
+    import torch
+    import deformable_convolution_core_b200 as dcn
+    wl = gen.WORKLOADS[name]
+    d = gen.make_inputs(wl)
+    pj = gen.make_projection_inputs(wl, wl.C)
+    p = dcn.problem_for(wl)
+    bf = torch.bfloat16
+    x = torch.from_numpy(d["x"]).cuda().to(bf)
+    q = torch.from_numpy(pj["query"]).cuda().to(bf)
+    w = torch.from_numpy(pj["weight"]).cuda().to(bf)
+    b = torch.from_numpy(pj["bias"]).cuda()
+    w_out = (torch.from_numpy(gen.normal(wl.seed, gen.TID_OUT_WEIGHT, (wl.C, wl.C), 0.0,
+                                         wl.C ** -0.5)).cuda().to(bf))
+    M = wl.N * wl.Ho * wl.Wo
+    off = torch.empty((M, wl.G * wl.KK * 2), dtype=bf, device="cuda")
+    msk = torch.empty((M, wl.G * wl.KK), dtype=bf, device="cuda")
+    core = torch.empty((M, wl.C), dtype=bf, device="cuda")
+    y = torch.empty((M, wl.C), dtype=bf, device="cuda")
+    s = torch.cuda.Stream()
+    stages = [lambda: dcn.dcn_core_offset_mask_projection(p, q, wl.C, w, b, off, msk, s),
+              lambda: dcn.dcn_core_forward(p, x, off, msk, core, s),
+              lambda: dcn.dcn_core_linear_bf16(core, M, wl.C, w_out, wl.C, None, y, "bf16", s)]
+    for _ in range(3):
+        for f in stages:
+            f()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+    for r in range(reps):
+        for i, f in enumerate(stages):
+            ev[r][i].record(s)
+            f()
+        ev[r][3].record(s)
+    torch.cuda.synchronize()
+    dcn.dcn_core_sync_status(s)
+    t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in ev])
+    med = np.median(t, axis=0)
+    return {"workload": name, "projection_ms": round(float(med[0]), 4),
+            "core_forward_ms": round(float(med[1]), 4),
+            "output_proj_ms": round(float(med[2]), 4),
+            "total_ms": round(float(np.median(t.sum(axis=1))), 4),
+            "Mpixels/s": round(M / (float(np.median(t.sum(axis=1))) * 1e-3) / 1e6, 1)}
 
 
 def run_sweep(gen, peak, reps=30, warmup=3):

@@ -26,6 +26,7 @@ _LIB_PATH = os.path.join(_HERE, "libdcngen.so")
 TID_X, TID_OFFSET, TID_MASK, TID_GRAD_OUT, TID_FAR_SELECT, TID_FAR_VALUE = 1, 2, 3, 4, 5, 6
 # inputs of the offset / mask projection: query features, weight, bias
 TID_QUERY, TID_WEIGHT, TID_BIAS = 7, 8, 9
+TID_OUT_WEIGHT = 10  # output_proj weight of the block's core path
 
 _lib = None
 
