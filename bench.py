@@ -314,12 +314,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (seeded counter-based generator)",
-        "config": {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
-                   "N": wl.N, "H": wl.H, "W": wl.W, "G": wl.G, "Cg": wl.Cg, "K": wl.K,
-                   "stride": wl.stride, "offset_scale": wl.offset_scale,
-                   "softmax": wl.softmax, "remove_center": wl.remove_center,
-                   "per_gpu_batch": wl.N,
-                   "parallelism": f"replicas x{world} (no collective)",
+        "config": {**workload_config(wl, backward, world),
                    "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB touched per step, "
                          "no flush between steps"},
         "gsamples_per_s": round(world * samples / (ms_per_step * 1e-3) / 1e9, 3),
@@ -607,6 +602,15 @@ def cpu_baseline(wl, inputs, backward, n_images=None):
                       "including the float64 widening of the inputs"}
 
 
+def workload_config(wl, backward, world):
+    """The `config` object of the JSON line: the workload and its shape."""
+    return {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
+            "N": wl.N, "H": wl.H, "W": wl.W, "G": wl.G, "Cg": wl.Cg, "K": wl.K,
+            "stride": wl.stride, "offset_scale": wl.offset_scale, "softmax": wl.softmax,
+            "remove_center": wl.remove_center, "per_gpu_batch": wl.N,
+            "parallelism": f"replicas x{world} (no collective)"}
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: rank 0 only, on host cores, each step a
     bounded sample (one image) of the workload."""
@@ -635,7 +639,7 @@ def run_reference(args, world, rank):
             "ms_per_step": round(1e3 * statistics.median(secs), 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded counter-based generator)",
-            "config": {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
+            "config": {**workload_config(wl, backward, world),
                        "sample": f"1 of {wl.N} images per step"},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"1 of {wl.N} images of {wl.name} per step"},
