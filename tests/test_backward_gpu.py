@@ -91,6 +91,10 @@ CASES = [
     (2, 19, 17, 5, 16, dict(softmax=0, remove_center=1)),
     (2, 15, 21, 4, 8, dict(remove_center=1, stride=2)),
     (2, 17, 19, 3, 16, dict(K=5, pad=2, remove_center=1)),
+    (1, 17, 19, 2, 16, dict(K=7, pad=3, remove_center=1, softmax=0)),
+    (2, 25, 23, 3, 16, dict(stride=2, dilation=2, pad=2)),
+    (2, 13, 14, 3, 32, dict(softmax=0)),
+    (1, 2, 40, 2, 16, dict()),
 ]
 
 
