@@ -45,7 +45,7 @@ def _load():
         dp = ctypes.POINTER(ctypes.c_double)
         i64p = ctypes.POINTER(ctypes.c_int64)
         ci, cd, i64 = ctypes.c_int, ctypes.c_double, ctypes.c_int64
-        shape = [ci] * 9 + [cd, ci, ci, ci]
+        shape = [ci] * 9 + [cd, ci, ci, ci, ci, ci, ci]
         lib.oracle_output_extent.argtypes = [ci] * 5
         lib.oracle_output_extent.restype = ci
         lib.oracle_forward.argtypes = [dp] * 4 + shape
@@ -76,8 +76,10 @@ def output_extent(n_in: int, K: int, stride: int, pad: int, dil: int) -> int:
     return int(_load().oracle_output_extent(n_in, K, stride, pad, dil))
 
 
-def output_hw(H, W, K, stride, pad, dil):
-    return output_extent(H, K, stride, pad, dil), output_extent(W, K, stride, pad, dil)
+def output_hw(H, W, K, stride, pad, dil, stride_w=None, pad_w=None, dil_w=None):
+    return (output_extent(H, K, stride, pad, dil),
+            output_extent(W, K, stride if stride_w is None else stride_w,
+                          pad if pad_w is None else pad_w, dil if dil_w is None else dil_w))
 
 
 def taps(K: int, remove_center=0) -> int:
@@ -86,21 +88,26 @@ def taps(K: int, remove_center=0) -> int:
     return K * K - (1 if remove_center else 0)
 
 
-def _shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd, remove_center):
+def _shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd, remove_center,
+                stride_w=None, pad_w=None, dil_w=None):
+    """Arguments of the C entry points: stride, pad and dil are the height
+    axis's; the width axis takes the *_w values, or the same ones when None."""
     return (int(N), int(H), int(W), int(G), int(Cg), int(K), int(stride), int(pad),
             int(dil), float(offset_scale), int(softmax), int(bool(fd)),
-            int(bool(remove_center)))
+            int(bool(remove_center)), int(stride if stride_w is None else stride_w),
+            int(pad if pad_w is None else pad_w), int(dil if dil_w is None else dil_w))
 
 
 def forward(x, offset, mask, *, G, K=3, stride=1, pad=1, dil=1, offset_scale=1.0,
-            softmax=1, fd=False, remove_center=0) -> np.ndarray:
+            softmax=1, fd=False, remove_center=0, stride_w=None, pad_w=None,
+            dil_w=None) -> np.ndarray:
     """Forward of the whole problem.  x: (N,H,W,G*Cg), offset: (N,Ho,Wo,G*T*2),
     mask: (N,Ho,Wo,G*T) with T = taps(K, remove_center).  Returns float64
     (N,Ho,Wo,G*Cg)."""
     x, offset, mask = _d(x), _d(offset), _d(mask)
     N, H, W, C = x.shape
     Cg = C // G
-    Ho, Wo = output_hw(H, W, K, stride, pad, dil)
+    Ho, Wo = output_hw(H, W, K, stride, pad, dil, stride_w, pad_w, dil_w)
     out = np.zeros((N, Ho, Wo, C), dtype=np.float64)
     if out.size == 0:
         return out
@@ -109,13 +116,15 @@ def forward(x, offset, mask, *, G, K=3, stride=1, pad=1, dil=1, offset_scale=1.0
     assert mask.shape == (N, Ho, Wo, G * T), mask.shape
     rc = _load().oracle_forward(_p(x), _p(offset), _p(mask), _p(out),
                                 *_shape_args(N, H, W, G, Cg, K, stride, pad, dil,
-                                             offset_scale, softmax, fd, remove_center))
+                                             offset_scale, softmax, fd, remove_center,
+                                             stride_w, pad_w, dil_w))
     assert rc == 0, rc
     return out
 
 
 def forward_units(x, offset, mask, units, *, G, K=3, stride=1, pad=1, dil=1,
-                  offset_scale=1.0, softmax=1, fd=False, remove_center=0) -> np.ndarray:
+                  offset_scale=1.0, softmax=1, fd=False, remove_center=0, stride_w=None,
+                  pad_w=None, dil_w=None) -> np.ndarray:
     """Forward outputs of selected units u = ((n*Ho+ho)*Wo+wo)*G+g only.
     Returns float64 (len(units), Cg)."""
     x, offset, mask = _d(x), _d(offset), _d(mask)
@@ -127,13 +136,14 @@ def forward_units(x, offset, mask, units, *, G, K=3, stride=1, pad=1, dil=1,
         _p(x), _p(offset), _p(mask), units.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
         units.size, _p(out),
         *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd,
-                     remove_center))
+                     remove_center, stride_w, pad_w, dil_w))
     assert rc == 0, rc
     return out
 
 
 def backward(x, offset, mask, grad_out, *, G, K=3, stride=1, pad=1, dil=1,
-             offset_scale=1.0, softmax=1, fd=False, remove_center=0):
+             offset_scale=1.0, softmax=1, fd=False, remove_center=0, stride_w=None, pad_w=None,
+             dil_w=None):
     """Returns float64 (grad_input, grad_offset, grad_mask); grad_mask is the
     gradient with respect to the logits when softmax=1."""
     x, offset, mask, grad_out = _d(x), _d(offset), _d(mask), _d(grad_out)
@@ -144,13 +154,15 @@ def backward(x, offset, mask, grad_out, *, G, K=3, stride=1, pad=1, dil=1,
     gm = np.zeros_like(mask)
     rc = _load().oracle_backward(_p(x), _p(offset), _p(mask), _p(grad_out), _p(gx), _p(goff),
                                  _p(gm), *_shape_args(N, H, W, G, Cg, K, stride, pad, dil,
-                                                      offset_scale, softmax, fd, remove_center))
+                                                      offset_scale, softmax, fd, remove_center,
+                                                      stride_w, pad_w, dil_w))
     assert rc == 0, rc
     return gx, goff, gm
 
 
 def backward_units(x, offset, mask, grad_out, units, *, G, K=3, stride=1, pad=1, dil=1,
-                   offset_scale=1.0, softmax=1, fd=False, remove_center=0):
+                   offset_scale=1.0, softmax=1, fd=False, remove_center=0, stride_w=None,
+                   pad_w=None, dil_w=None):
     """Offset and mask gradients of selected units.  Returns float64
     (goff (len, T*2), gmask (len, T)), T = taps(K, remove_center)."""
     x, offset, mask, grad_out = _d(x), _d(offset), _d(mask), _d(grad_out)
@@ -164,7 +176,7 @@ def backward_units(x, offset, mask, grad_out, units, *, G, K=3, stride=1, pad=1,
         _p(x), _p(offset), _p(mask), _p(grad_out),
         units.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), units.size, _p(goff), _p(gm),
         *_shape_args(N, H, W, G, Cg, K, stride, pad, dil, offset_scale, softmax, fd,
-                     remove_center))
+                     remove_center, stride_w, pad_w, dil_w))
     assert rc == 0, rc
     return goff, gm
 

@@ -27,7 +27,10 @@
  *    3x3 convolution" remark needs;
  *  - zero padding per corner; a sample contributes (and has a derivative)
  *    only when -1 <= Y < H and -1 <= X < W, which also drops NaN and inf;
- *  - the sampling grid is the usual convolution grid ho*s - p + a*d;
+ *  - the sampling grid is the usual convolution grid ho*s - p + a*d, with a
+ *    stride, padding and dilation per axis (the height ones apply to ho and
+ *    a, the width ones to wo and b; the pages' modules take one value for
+ *    both, which is the case stride_w = stride and so on);
  *  - offsets are stored as (dx, dy) pairs, taps row-major (k = a*K + b);
  *  - the softmax subtracts the per-group maximum before exponentiating;
  *  - location rounding: in "fp32-location" mode (fd = 0) each of
@@ -57,7 +60,9 @@
 #include <string.h>
 
 typedef struct {
-  int64_t N, H, W, G, Cg, K, stride, pad, dil, Ho, Wo;
+  int64_t N, H, W, G, Cg, K, Ho, Wo;
+  int64_t stride, pad, dil;        /* height axis */
+  int64_t stride_w, pad_w, dil_w;  /* width axis */
   int64_t T; /* taps per (pixel, group) */
   double sigma;
   int softmax, fd, remove_center;
@@ -72,12 +77,13 @@ int oracle_output_extent(int in, int K, int stride, int pad, int dil) {
 
 static prob_t make_prob(int N, int H, int W, int G, int Cg, int K, int stride,
                         int pad, int dil, double sigma, int softmax, int fd,
-                        int remove_center) {
+                        int remove_center, int stride_w, int pad_w, int dil_w) {
   prob_t p;
   p.N = N; p.H = H; p.W = W; p.G = G; p.Cg = Cg; p.K = K;
   p.stride = stride; p.pad = pad; p.dil = dil;
+  p.stride_w = stride_w; p.pad_w = pad_w; p.dil_w = dil_w;
   p.Ho = oracle_output_extent(H, K, stride, pad, dil);
-  p.Wo = oracle_output_extent(W, K, stride, pad, dil);
+  p.Wo = oracle_output_extent(W, K, stride_w, pad_w, dil_w);
   p.sigma = sigma; p.softmax = softmax; p.fd = fd;
   p.remove_center = remove_center != 0;
   p.T = (int64_t)K * K - p.remove_center;
@@ -124,7 +130,7 @@ static void mask_weights(const double* logits, int64_t KK, int softmax, double* 
 static void location(const prob_t* p, int64_t ho, int64_t wo, int64_t a, int64_t b,
                      double dx, double dy, double* Y, double* X) {
   int64_t base_y = ho * p->stride - p->pad + a * p->dil;
-  int64_t base_x = wo * p->stride - p->pad + b * p->dil;
+  int64_t base_x = wo * p->stride_w - p->pad_w + b * p->dil_w;
   if (p->fd) {
     *Y = (double)base_y + p->sigma * dy;
     *X = (double)base_x + p->sigma * dx;
@@ -191,8 +197,9 @@ static void forward_unit(const prob_t* p, const double* x, const double* off,
 int oracle_forward(const double* x, const double* offset, const double* mask,
                    double* out, int N, int H, int W, int G, int Cg, int K,
                    int stride, int pad, int dil, double sigma, int softmax, int fd,
-                   int remove_center) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+                   int remove_center, int stride_w, int pad_w, int dil_w) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center,
+                       stride_w, pad_w, dil_w);
   if (!usable(&p)) return -1;
   for (int64_t n = 0; n < p.N; ++n)
     for (int64_t ho = 0; ho < p.Ho; ++ho)
@@ -210,8 +217,10 @@ int oracle_forward(const double* x, const double* offset, const double* mask,
 int oracle_forward_units(const double* x, const double* offset, const double* mask,
                          const int64_t* units, int64_t n_units, double* out, int N,
                          int H, int W, int G, int Cg, int K, int stride, int pad,
-                         int dil, double sigma, int softmax, int fd, int remove_center) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+                         int dil, double sigma, int softmax, int fd, int remove_center,
+                         int stride_w, int pad_w, int dil_w) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center,
+                       stride_w, pad_w, dil_w);
   if (!usable(&p)) return -1;
   for (int64_t i = 0; i < n_units; ++i) {
     int64_t u = units[i];
@@ -304,8 +313,9 @@ int oracle_backward(const double* x, const double* offset, const double* mask,
                     const double* grad_out, double* grad_input, double* grad_offset,
                     double* grad_mask, int N, int H, int W, int G, int Cg, int K,
                     int stride, int pad, int dil, double sigma, int softmax, int fd,
-                    int remove_center) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+                    int remove_center, int stride_w, int pad_w, int dil_w) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center,
+                       stride_w, pad_w, dil_w);
   if (!usable(&p)) return -1;
   const int64_t KK = p.T;
   memset(grad_input, 0, sizeof(double) * (size_t)(p.N * p.H * p.W * p.G * p.Cg));
@@ -326,8 +336,10 @@ int oracle_backward_units(const double* x, const double* offset, const double* m
                           const double* grad_out, const int64_t* units, int64_t n_units,
                           double* goff, double* gmask, int N, int H, int W, int G,
                           int Cg, int K, int stride, int pad, int dil, double sigma,
-                          int softmax, int fd, int remove_center) {
-  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center);
+                          int softmax, int fd, int remove_center, int stride_w, int pad_w,
+                          int dil_w) {
+  prob_t p = make_prob(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, fd, remove_center,
+                       stride_w, pad_w, dil_w);
   if (!usable(&p)) return -1;
   const int64_t KK = p.T;
   for (int64_t i = 0; i < n_units; ++i) {

@@ -439,3 +439,70 @@ def test_linear_matches_explicit_sums(oracle_mod):
         for j in range(5):
             assert abs(y[idx + (j,)] - (b[j] + sum(x[idx + (c,)] * w[j, c] for c in range(4)))) <= 1e-14
     assert np.array_equal(oracle_mod.linear(x, np.eye(4)), x)
+
+
+# --- separate height / width stride, padding and dilation ---------------------------
+
+AXES = [dict(stride=1, stride_w=2, pad=1, pad_w=0, dil=1, dil_w=1),
+        dict(stride=2, stride_w=1, pad=2, pad_w=1, dil=2, dil_w=1),
+        dict(stride=1, stride_w=1, pad=0, pad_w=3, dil=1, dil_w=3)]
+
+
+@pytest.mark.parametrize("ax", AXES)
+def test_grid_sample_brute_force_separate_axes(oracle_mod, ax):
+    N, H, W, G, Cg, K = 2, 9, 10, 2, 3, 3
+    sigma = 2.0
+    Ho, Wo = oracle_mod.output_hw(H, W, K, ax["stride"], ax["pad"], ax["dil"],
+                                  ax["stride_w"], ax["pad_w"], ax["dil_w"])
+    # the size rule per axis
+    assert Ho == (H + 2 * ax["pad"] - ax["dil"] * (K - 1) - 1) // ax["stride"] + 1
+    assert Wo == (W + 2 * ax["pad_w"] - ax["dil_w"] * (K - 1) - 1) // ax["stride_w"] + 1
+    x = rand(N, H, W, G * Cg)
+    off = rand(N, Ho, Wo, G * K * K * 2, lo=-2.5, hi=2.5)
+    mask = rand(N, Ho, Wo, G * K * K, lo=-2, hi=2)
+    got = oracle_mod.forward(x, off, mask, G=G, K=K, offset_scale=sigma, softmax=1, fd=True, **ax)
+    xt = torch.from_numpy(x).reshape(N, H, W, G, Cg)
+    o = torch.from_numpy(off).reshape(N, Ho, Wo, G, K * K, 2)
+    m = torch.softmax(torch.from_numpy(mask).reshape(N, Ho, Wo, G, K * K), dim=-1)
+    ref = torch.zeros(N, Ho, Wo, G, Cg, dtype=torch.float64)
+    hh = torch.arange(Ho, dtype=torch.float64).view(Ho, 1)
+    ww = torch.arange(Wo, dtype=torch.float64).view(1, Wo)
+    for g in range(G):
+        img = xt[:, :, :, g, :].permute(0, 3, 1, 2)
+        for k in range(K * K):
+            a, b = divmod(k, K)
+            Y = hh * ax["stride"] - ax["pad"] + a * ax["dil"] + sigma * o[:, :, :, g, k, 1]
+            X = ww * ax["stride_w"] - ax["pad_w"] + b * ax["dil_w"] + sigma * o[:, :, :, g, k, 0]
+            grid = torch.stack([(2 * X + 1) / W - 1, (2 * Y + 1) / H - 1], dim=-1)
+            s = torch.nn.functional.grid_sample(img, grid, mode="bilinear", padding_mode="zeros",
+                                                align_corners=False)
+            ref[:, :, :, g, :] += m[:, :, :, g, k, None] * s.permute(0, 2, 3, 1)
+    np.testing.assert_allclose(got, ref.reshape(N, Ho, Wo, G * Cg).numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_finite_differences_separate_axes(oracle_mod):
+    ax = dict(stride=2, stride_w=1, pad=1, pad_w=2, dil=1, dil_w=2)
+    N, H, W, G, Cg, K, sigma = 1, 6, 5, 2, 3, 3, 2.0
+    Ho, Wo = oracle_mod.output_hw(H, W, K, ax["stride"], ax["pad"], ax["dil"],
+                                  ax["stride_w"], ax["pad_w"], ax["dil_w"])
+    x = rand(N, H, W, G * Cg)
+    off = kink_free_offsets(N, Ho, Wo, G, K * K, sigma)
+    m = rand(N, Ho, Wo, G * K * K, lo=-1.5, hi=1.5)
+    gout = rand(N, Ho, Wo, G * Cg)
+    kw = dict(G=G, K=K, offset_scale=sigma, softmax=1, fd=True, **ax)
+    gx, goff, gm = oracle_mod.backward(x, off, m, gout, **kw)
+
+    def L(xx, oo, mm):
+        return float((oracle_mod.forward(xx, oo, mm, **kw) * gout).sum())
+
+    h = 1e-4
+    for arr, grad, which in ((x, gx, 0), (off, goff, 1), (m, gm, 2)):
+        flat = arr.reshape(-1)
+        for i in RNG.choice(flat.size, size=min(flat.size, 40), replace=False):
+            args_p, args_q = [x, off, m], [x, off, m]
+            pp, qq = flat.copy(), flat.copy()
+            pp[i] += h
+            qq[i] -= h
+            args_p[which], args_q[which] = pp.reshape(arr.shape), qq.reshape(arr.shape)
+            fd = (L(*args_p) - L(*args_q)) / (2 * h)
+            assert abs(grad.reshape(-1)[i] - fd) <= 1e-7 * max(1.0, abs(fd))
