@@ -19,7 +19,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdcncore.so")
 
 # DCN_CORE_ABI_VERSION of include/dcn_core.h that DcnProblem mirrors.
-ABI_VERSION = 2
+ABI_VERSION = 3
 DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
 # Scratch the allocation-free backward owns per GPU (DCN_CORE_NOALLOC_SCRATCH_BYTES).
 DCN_CORE_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -55,19 +55,28 @@ class DcnProblem(ctypes.Structure):
                 ("G", ctypes.c_int), ("Cg", ctypes.c_int), ("K", ctypes.c_int),
                 ("stride", ctypes.c_int), ("pad", ctypes.c_int), ("dilation", ctypes.c_int),
                 ("offset_scale", ctypes.c_float), ("softmax", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("remove_center", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("remove_center", ctypes.c_int),
+                ("separate_axes", ctypes.c_int), ("stride_w", ctypes.c_int),
+                ("pad_w", ctypes.c_int), ("dilation_w", ctypes.c_int)]
 
     def __repr__(self):
         return "DcnProblem(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
 def make_problem(N, H, W, G, Cg, K=3, stride=1, pad=1, dilation=1, offset_scale=1.0,
-                 softmax=1, dtype="f32", remove_center=0) -> DcnProblem:
+                 softmax=1, dtype="f32", remove_center=0, stride_w=None, pad_w=None,
+                 dilation_w=None) -> DcnProblem:
+    """stride, pad and dilation apply to both axes unless a width value
+    (stride_w, pad_w, dilation_w) is given; then they are the height axis's."""
     if isinstance(dtype, str):
         dtype = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16, "bfloat16": DCN_BF16}[dtype]
+    separate = stride_w is not None or pad_w is not None or dilation_w is not None
+    sw = stride if stride_w is None else stride_w
+    pw = pad if pad_w is None else pad_w
+    dw = dilation if dilation_w is None else dilation_w
     return DcnProblem(int(N), int(H), int(W), int(G), int(Cg), int(K), int(stride), int(pad),
                       int(dilation), float(offset_scale), int(softmax), int(dtype),
-                      int(remove_center))
+                      int(remove_center), int(separate), int(sw), int(pw), int(dw))
 
 
 def problem_for(wl) -> DcnProblem:

@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
     const char* xg = xbytes + g_off * sizeof(T);
     const size_t upix = size_t(tc.n * t.Ho + u.ho) * t.Wo + u.wo;
     const size_t unit = upix * t.G + u.g;
-    const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride - t.pad;
+    const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride_w - t.pad_w;
 
     float go[CPL];
     Quad<T>::load(gobytes + (upix * t.C + size_t(u.g) * t.Cg + size_t(sub) * CPL) * sizeof(T), go);
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
     auto tap = [&](int k, int ka, int kb, float mk) -> float {
       const float2 d = St::pair(s_off[(row0 + k) * t.P1 + u.pix]);
       const float Y = tap_coord(by + ka * t.dil, t.sigma, d.y);
-      const float X = tap_coord(bx + kb * t.dil, t.sigma, d.x);
+      const float X = tap_coord(bx + kb * t.dil_w, t.sigma, d.x);
       const Footprint f = footprint(Y, X, t.H, t.W);
       float s = 0.f, gX = 0.f, gY = 0.f;
       if (f.in_support) {
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
           const float2 d = St::pair(s_off[(row0 + k) * t.P1 + u.pix]);
           const int q = tap_pos(KKS, k);  // window position of tap k
           const float Y = tap_coord(by + (q / K) * t.dil, t.sigma, d.y);
-          const float X = tap_coord(bx + (q % K) * t.dil, t.sigma, d.x);
+          const float X = tap_coord(bx + (q % K) * t.dil_w, t.sigma, d.x);
           f[j] = footprint(Y, X, t.H, t.W);
           const int base = f[j].y0 * int(rowE) + f[j].x0 * int(pixE);
           cofs[j][0] = base;

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(&full[b], t.box_bytes);
       tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg,
-                   c.wo0 * t.stride - t.pad - t.halo, c.ho0 * t.stride - t.pad - t.halo, c.n);
+                   c.wo0 * t.stride_w - t.pad_w - t.halo, c.ho0 * t.stride - t.pad - t.halo, c.n);
     }
     // Copies issued for items i-2 and i-1 may still be landing: wait for them
     // (bounded) before this thread, possibly the CTA's last, exits.
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const ItemCoord c = item_coord(t, item);
     const unsigned char* box_lane = bufs + size_t(b) * t.box_stride + sub * PB;
     const int Y0 = c.ho0 * t.stride - t.pad - t.halo;
-    const int X0 = c.wo0 * t.stride - t.pad - t.halo;
+    const int X0 = c.wo0 * t.stride_w - t.pad_w - t.halo;
     const size_t img = size_t(c.n) * t.H * t.W * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4;
     const char* xg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
     const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits);
@@ -298,7 +298,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         for (int k = 0; k < KK; ++k) {
           const int q = tap_pos(KK, k);
           const float Y = tap_coord(ho * t.stride - t.pad + (q / K) * t.dil, t.sigma, d[k].y);
-          const float X = tap_coord(wo * t.stride - t.pad + (q % K) * t.dil, t.sigma, d[k].x);
+          const float X =
+              tap_coord(wo * t.stride_w - t.pad_w + (q % K) * t.dil_w, t.sigma, d[k].x);
           const Footprint f = footprint(Y, X, t.H, t.W);
           const bool live = valid && f.in_support;
           // a sample that contributes nothing keeps code 0: box offset 0, no corner

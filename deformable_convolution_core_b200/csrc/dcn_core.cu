@@ -41,6 +41,11 @@ int esize(dcn_dtype d) { return d == DCN_BF16 ? 2 : 4; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Width-axis stride, padding and dilation: the height ones unless separate_axes.
+int stride_w(const dcn_problem* p) { return p->separate_axes ? p->stride_w : p->stride; }
+int pad_w(const dcn_problem* p) { return p->separate_axes ? p->pad_w : p->pad; }
+int dil_w(const dcn_problem* p) { return p->separate_axes ? p->dilation_w : p->dilation; }
+
 // Taps per (pixel, group): the K x K window, less its centre with remove_center.
 int taps(const dcn_problem* p) { return p->K * p->K - (p->remove_center ? 1 : 0); }
 
@@ -57,13 +62,15 @@ dcn_status check_problem(const dcn_problem* p, int64_t* Ho, int64_t* Wo) {
   if (p->N < 1 || p->H < 1 || p->W < 1 || p->G < 1 || p->Cg < 1) return DCN_ERR_INVALID_ARG;
   if (p->K < 1 || (p->K % 2) == 0) return DCN_ERR_INVALID_ARG;
   if (p->stride < 1 || p->pad < 0 || p->dilation < 1) return DCN_ERR_INVALID_ARG;
+  if (p->separate_axes != 0 && p->separate_axes != 1) return DCN_ERR_INVALID_ARG;
+  if (stride_w(p) < 1 || pad_w(p) < 0 || dil_w(p) < 1) return DCN_ERR_INVALID_ARG;
   if (p->softmax != 0 && p->softmax != 1) return DCN_ERR_INVALID_ARG;
   if (p->remove_center != 0 && p->remove_center != 1) return DCN_ERR_INVALID_ARG;
   if (p->remove_center && p->K < 3) return DCN_ERR_INVALID_ARG;  // no tap would be left
   if (p->dtype != DCN_F32 && p->dtype != DCN_BF16) return DCN_ERR_INVALID_ARG;
   if (!(p->offset_scale == p->offset_scale)) return DCN_ERR_INVALID_ARG;  // NaN
   const int64_t ho = out_extent(p->H, p->K, p->stride, p->pad, p->dilation);
-  const int64_t wo = out_extent(p->W, p->K, p->stride, p->pad, p->dilation);
+  const int64_t wo = out_extent(p->W, p->K, stride_w(p), pad_w(p), dil_w(p));
   if (ho < 1 || wo < 1) return DCN_ERR_INVALID_ARG;
   const int64_t C = int64_t(p->G) * p->Cg;
   const int64_t KK = taps(p);
@@ -74,7 +81,7 @@ dcn_status check_problem(const dcn_problem* p, int64_t* Ho, int64_t* Wo) {
   if (C > lim || n_in > lim || n_out > lim || n_off > lim) return DCN_ERR_INVALID_ARG;
   // Sampling coordinates are integers up to about H*stride + K*dilation in fp32.
   if (int64_t(p->H) * p->stride + int64_t(p->K) * p->dilation > (int64_t(1) << 22) ||
-      int64_t(p->W) * p->stride + int64_t(p->K) * p->dilation > (int64_t(1) << 22))
+      int64_t(p->W) * stride_w(p) + int64_t(p->K) * dil_w(p) > (int64_t(1) << 22))
     return DCN_ERR_UNSUPPORTED;
   *Ho = ho;
   *Wo = wo;
@@ -145,6 +152,7 @@ dcn_status make_plan(const dcn_problem* p, int64_t Ho, int64_t Wo, size_t entry_
   TileParams& t = plan->t;
   t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
   t.K = p->K; t.KK = taps(p); t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation;
+  t.stride_w = stride_w(p); t.pad_w = pad_w(p); t.dil_w = dil_w(p);
   t.kc = p->remove_center ? (p->K * p->K) / 2 : -1;
   t.Ho = int(Ho); t.Wo = int(Wo); t.sigma = p->offset_scale;
   size_t budget = kDefaultSmemBudget;
@@ -389,7 +397,7 @@ void choose_tiled_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, s
   for (int th = 1; th <= std::min(Ho, 64); ++th) {
     for (int tw = 1; tw <= std::min(Wo, 64); ++tw) {
       const int bh = box_extent(th, p->stride, p->dilation, halo);
-      int bw = box_extent(tw, p->stride, p->dilation, halo);
+      int bw = box_extent(tw, stride_w(p), dil_w(p), halo);
       bw = box_pitch(bw, cs);
       if (bh > 256 || bw > 256) continue;
       const size_t bytes = size_t(bh) * bw * cs;
@@ -488,6 +496,7 @@ dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   TiledParams& t = L->t;
   t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
   t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation; t.Ho = int(Ho); t.Wo = int(Wo);
+  t.stride_w = stride_w(p); t.pad_w = pad_w(p); t.dil_w = dil_w(p);
   t.sigma = p->offset_scale; t.halo = halo; t.TH = TH; t.TW = TW;
   // Test knob for the failure path: DCN_CORE_TEST_STALL=1 makes the first box
   // of every CTA never arrive; the bounded waits then give up and
@@ -496,7 +505,7 @@ dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   t.nTY = (t.Ho + TH - 1) / TH;
   t.nTX = (t.Wo + TW - 1) / TW;
   t.BH = box_extent(TH, t.stride, t.dil, halo);
-  t.BW = box_extent(TW, t.stride, t.dil, halo);
+  t.BW = box_extent(TW, t.stride_w, t.dil_w, halo);
   t.BW = box_pitch(t.BW, cs);
   if (t.BH > 256 || t.BW > 256) return DCN_ERR_UNSUPPORTED;
   t.box_bytes = uint32_t(size_t(t.BH) * t.BW * cs);
@@ -600,7 +609,7 @@ dcn_status dcn_core_output_hw(const dcn_problem* problem, int* Ho, int* Wo) {
   if (st != DCN_OK && st != DCN_ERR_UNSUPPORTED) return st;
   if (ho < 1 || wo < 1) {
     ho = out_extent(problem->H, problem->K, problem->stride, problem->pad, problem->dilation);
-    wo = out_extent(problem->W, problem->K, problem->stride, problem->pad, problem->dilation);
+    wo = out_extent(problem->W, problem->K, stride_w(problem), pad_w(problem), dil_w(problem));
   }
   *Ho = int(ho);
   *Wo = int(wo);

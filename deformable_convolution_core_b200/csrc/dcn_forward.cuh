@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(kThreads) dcn_forward_kernel(const FwdArgs a) 
     if (!u.valid) continue;
     const int row0 = u.g * KK;
     const char* xg = xbase + size_t(u.g) * t.Cg * S::kSize;
-    const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride - t.pad;
+    const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride_w - t.pad_w;
 
     float acc[CPL];
 #pragma unroll
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(kThreads) dcn_forward_kernel(const FwdArgs a) 
     auto tap = [&](int k, int ka, int kb, float mk) {
       const float2 d = St::pair(s_off[(row0 + k) * t.P1 + u.pix]);
       const float Y = tap_coord(by + ka * t.dil, t.sigma, d.y);
-      const float X = tap_coord(bx + kb * t.dil, t.sigma, d.x);
+      const float X = tap_coord(bx + kb * t.dil_w, t.sigma, d.x);
       const Footprint f = footprint(Y, X, t.H, t.W);
       if (!f.in_support) return;
       const float hy = 1.f - f.ly, hx = 1.f - f.lx;

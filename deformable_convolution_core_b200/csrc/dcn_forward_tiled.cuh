@@ -32,7 +32,8 @@ constexpr int kTiledBatch = 32;                       // units per warp batch
 constexpr int kTiledMaxTaps = 9;  // the tiled kernel serves 3x3 windows (9 or 8 taps)
 
 struct TiledParams {
-  int N, H, W, G, Cg, C, stride, pad, dil, Ho, Wo;
+  int N, H, W, G, Cg, C, stride, pad, dil, Ho, Wo;  // stride/pad/dil: height axis
+  int stride_w, pad_w, dil_w;                       // width axis
   float sigma;
   int TH, TW, nTY, nTX, halo, BH, BW;
   int items;           // N * nTY * nTX * G
@@ -292,7 +293,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive_expect_tx(&full[b], t.box_bytes);
       tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg,
-                   c.wo0 * t.stride - t.pad - t.halo, c.ho0 * t.stride - t.pad - t.halo, c.n);
+                   c.wo0 * t.stride_w - t.pad_w - t.halo, c.ho0 * t.stride - t.pad - t.halo, c.n);
     }
     // Copies issued for items i-2 and i-1 may still be landing: wait for them
     // (bounded) before this thread, possibly the CTA's last, exits.
@@ -383,7 +384,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const ItemCoord c = item_coord(t, item);
     const unsigned char* box = bufs + size_t(b) * t.box_stride;
     const int Y0 = c.ho0 * t.stride - t.pad - t.halo;
-    const int X0 = c.wo0 * t.stride - t.pad - t.halo;
+    const int X0 = c.wo0 * t.stride_w - t.pad_w - t.halo;
     const char* ximg = reinterpret_cast<const char*>(a.x) + size_t(c.n) * t.H * t.W * pixB +
                        size_t(c.g) * CS;
 
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         for (int k = 0; k < KK; ++k) {
           const int ka = tap_pos(KK, k) / K, kb = tap_pos(KK, k) % K;
           const float Y = tap_coord(ho * t.stride - t.pad + ka * t.dil, t.sigma, d[k].y);
-          const float X = tap_coord(wo * t.stride - t.pad + kb * t.dil, t.sigma, d[k].x);
+          const float X = tap_coord(wo * t.stride_w - t.pad_w + kb * t.dil_w, t.sigma, d[k].x);
           const Footprint f = footprint(Y, X, t.H, t.W);
           const bool live = valid && f.in_support;
           const int by = f.y0 - Y0, bx = f.x0 - X0;

@@ -16,7 +16,8 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
 struct TileParams {
-  int N, H, W, G, Cg, C, K, KK, stride, pad, dil, Ho, Wo;
+  int N, H, W, G, Cg, C, K, KK, stride, pad, dil, Ho, Wo;  // stride/pad/dil: height axis
+  int stride_w, pad_w, dil_w;                              // width axis
   int kc;       // window position (a*K + b) left out by remove_center, else -1
   float sigma;
   int TH, TW, nTY, nTX;

@@ -25,7 +25,8 @@
  *   offset  (N, Ho, Wo, G*KK*2)     ((n*Ho + ho)*Wo + wo)*G*KK*2 + (g*KK + k)*2 + {0: dx, 1: dy}
  *   mask    (N, Ho, Wo, G*KK)       ((n*Ho + ho)*Wo + wo)*G*KK + g*KK + k
  *   output  (N, Ho, Wo, C)          ((n*Ho + ho)*Wo + wo)*C + g*Cg + c
- *   Ho = floor((H + 2*pad - dilation*(K-1) - 1) / stride) + 1, Wo likewise.
+ *   Ho = floor((H + 2*pad - dilation*(K-1) - 1) / stride) + 1, Wo likewise
+ *   (with the width axis's values when separate_axes = 1).
  *
  * Ownership and execution: every pointer is owned by the caller.  Device
  * pointers must stay valid until the enqueued work has finished.  All work is
@@ -51,7 +52,7 @@
 extern "C" {
 #endif
 
-#define DCN_CORE_ABI_VERSION 2
+#define DCN_CORE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define DCN_API __attribute__((visibility("default")))
@@ -86,6 +87,13 @@ typedef enum {
  *   dtype        storage type of input, offset, mask and output
  *   remove_center  0: all K*K window positions are taps;  1: the centre
  *                position is left out (KK = K*K - 1 taps; needs K >= 3)
+ *   separate_axes  0: stride, pad and dilation apply to both axes (the
+ *                modules' single values); 1: they apply to the height axis
+ *                (ho and the tap row a) and stride_w, pad_w, dilation_w to
+ *                the width axis (wo and the tap column b)
+ *   stride_w >= 1, pad_w >= 0, dilation_w >= 1   (read when separate_axes = 1)
+ * With separate axes the grid is Y = ho*stride - pad + a*dilation + ...,
+ * X = wo*stride_w - pad_w + b*dilation_w + ..., and Wo uses the width values.
  */
 typedef struct {
   int N, H, W, G, Cg;
@@ -95,6 +103,8 @@ typedef struct {
   int softmax;
   dcn_dtype dtype;
   int remove_center;
+  int separate_axes;
+  int stride_w, pad_w, dilation_w;
 } dcn_problem;
 
 /* Output spatial size.  DCN_ERR_INVALID_ARG if the problem is invalid or the

@@ -67,4 +67,7 @@ def assert_bwd(got, ref, what="", dtype="f32"):
 def problem_kwargs(problem) -> dict:
     return dict(G=problem.G, K=problem.K, stride=problem.stride, pad=problem.pad,
                 dil=problem.dilation, offset_scale=problem.offset_scale, softmax=problem.softmax,
-                remove_center=problem.remove_center)
+                remove_center=problem.remove_center,
+                stride_w=problem.stride_w if problem.separate_axes else None,
+                pad_w=problem.pad_w if problem.separate_axes else None,
+                dil_w=problem.dilation_w if problem.separate_axes else None)

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 2
+    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 3
     for st in range(5):
         assert dcn.dcn_status_string(st)
     assert "unknown" in dcn.dcn_status_string(99)
@@ -47,6 +47,9 @@ def test_output_hw(lib):
     assert dcn.dcn_core_output_hw(dcn.make_problem(1, 7, 9, 1, 8, K=5, pad=0, dilation=1)) == (3, 5)
     with pytest.raises(dcn.DcnError):
         dcn.dcn_core_output_hw(dcn.make_problem(1, 2, 2, 1, 8, K=5, pad=0))
+    # separate axes: Ho from the height values, Wo from the width ones
+    assert dcn.dcn_core_output_hw(dcn.make_problem(1, 20, 21, 1, 8, stride=2, pad=1,
+                                                   stride_w=1, pad_w=0, dilation_w=2)) == (10, 17)
     # removing the centre tap leaves the output grid unchanged
     assert dcn.dcn_core_output_hw(dcn.make_problem(1, 7, 9, 1, 8, K=3, remove_center=1)) == (7, 9)
 
@@ -81,6 +84,10 @@ FAKE = 1 << 20  # an address that is 16- and 32-byte aligned; never dereferenced
     (dict(softmax=2), dcn.DCN_ERR_INVALID_ARG),
     (dict(remove_center=2), dcn.DCN_ERR_INVALID_ARG),
     (dict(remove_center=1, K=1, pad=0), dcn.DCN_ERR_INVALID_ARG),  # no tap left
+    (dict(stride_w=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(pad_w=-1), dcn.DCN_ERR_INVALID_ARG),
+    (dict(dilation_w=0), dcn.DCN_ERR_INVALID_ARG),
+    (dict(W=2, pad_w=0, dilation_w=2), dcn.DCN_ERR_INVALID_ARG),   # empty output along W
     (dict(dtype=7), dcn.DCN_ERR_INVALID_ARG),
     (dict(offset_scale=float("nan")), dcn.DCN_ERR_INVALID_ARG),
     (dict(H=2, W=2, K=5, pad=0), dcn.DCN_ERR_INVALID_ARG),     # empty output

@@ -56,7 +56,9 @@ def near_kink_taps(p, off):
     a, b = (k // K).reshape(1, 1, 1, 1, -1), (k % K).reshape(1, 1, 1, 1, -1)
     s = np.float32(p.offset_scale)
     Y = (ho * p.stride - p.pad + a * p.dilation).astype(np.float32) + s * o[..., 1]
-    X = (wo * p.stride - p.pad + b * p.dilation).astype(np.float32) + s * o[..., 0]
+    sw, pw, dw = ((p.stride_w, p.pad_w, p.dilation_w) if p.separate_axes
+                  else (p.stride, p.pad, p.dilation))
+    X = (wo * sw - pw + b * dw).astype(np.float32) + s * o[..., 0]
     fy, fx = Y - np.floor(Y), X - np.floor(X)
     near = (np.minimum(fy, 1 - fy) < 1e-6) | (np.minimum(fx, 1 - fx) < 1e-6)
     return int(near.sum())
@@ -95,6 +97,8 @@ CASES = [
     (2, 25, 23, 3, 16, dict(stride=2, dilation=2, pad=2)),
     (2, 13, 14, 3, 32, dict(softmax=0)),
     (1, 2, 40, 2, 16, dict()),
+    (2, 23, 29, 3, 16, dict(stride_w=2, pad_w=0)),
+    (2, 26, 21, 4, 16, dict(stride=2, dilation_w=2, pad_w=2, softmax=0)),
 ]
 
 
@@ -107,9 +111,11 @@ def test_backward_matches_oracle(oracle_mod, case, dtype, path):
     N, H, W, G, Cg, kw = case
     if dtype == "bf16" and Cg * 2 < 16:
         pytest.skip("bf16 needs Cg >= 8")
-    kw = {"K": 3, "stride": 1, "pad": 1, "dilation": 1, "softmax": 1, "remove_center": 0, **kw}
+    kw = {"K": 3, "stride": 1, "pad": 1, "dilation": 1, "softmax": 1, "remove_center": 0,
+          "stride_w": None, "pad_w": None, "dilation_w": None, **kw}
     p = dcn.make_problem(N, H, W, G, Cg, kw["K"], kw["stride"], kw["pad"], kw["dilation"],
-                         2.0, kw["softmax"], dtype, kw["remove_center"])
+                         2.0, kw["softmax"], dtype, kw["remove_center"], kw["stride_w"],
+                         kw["pad_w"], kw["dilation_w"])
     Ho, Wo = dcn.dcn_core_output_hw(p)
     KK = dcn.taps(p)
     x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)

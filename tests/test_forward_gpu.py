@@ -22,10 +22,11 @@ RNG = np.random.default_rng(2024)
 
 
 def random_case(N, H, W, G, Cg, K=3, stride=1, pad=None, dil=1, sigma=2.0, softmax=1,
-                dtype="f32", off_sd=1.5, off_lo=None, remove_center=0):
+                dtype="f32", off_sd=1.5, off_lo=None, remove_center=0, stride_w=None,
+                pad_w=None, dil_w=None):
     pad = (K // 2) * dil if pad is None else pad
     p = dcn.make_problem(N, H, W, G, Cg, K, stride, pad, dil, sigma, softmax, dtype,
-                         remove_center)
+                         remove_center, stride_w, pad_w, dil_w)
     Ho, Wo = dcn.dcn_core_output_hw(p)
     T = dcn.taps(p)
     x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
@@ -98,6 +99,10 @@ CASES = [
     (2, 13, 14, 3, 32, dict(dtype="f32", softmax=0, remove_center=1)),
     (2, 17, 19, 3, 16, dict(dtype="f32", K=5, remove_center=1)),
     (1, 17, 19, 2, 16, dict(dtype="bf16", K=7, softmax=0, dil=2, remove_center=1)),
+    # separate height / width stride, padding and dilation
+    (2, 23, 29, 3, 16, dict(dtype="f32", stride=1, stride_w=2, pad=1, pad_w=0)),
+    (2, 26, 21, 4, 16, dict(dtype="bf16", stride=2, stride_w=1, dil=1, dil_w=2, pad_w=2)),
+    (1, 19, 33, 3, 8, dict(dtype="f32", K=5, pad=2, pad_w=0, dil_w=2, remove_center=1)),
 ]
 
 
