@@ -16,11 +16,14 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdcncore.so")
+# DCN_CORE_LIBRARY selects another build of the library, e.g. the
+# bounds-checked libdcncore_checked.so.
+LIB_PATH = os.environ.get("DCN_CORE_LIBRARY") or os.path.join(_HERE, "libdcncore.so")
 
 # DCN_CORE_ABI_VERSION of include/dcn_core.h that DcnProblem mirrors.
 ABI_VERSION = 3
 DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
+DCN_ERR_OUT_OF_BOUNDS = 5  # only from the bounds-checked build
 # Scratch the allocation-free backward owns per GPU (DCN_CORE_NOALLOC_SCRATCH_BYTES).
 DCN_CORE_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 DCN_F32, DCN_BF16 = 0, 1
@@ -277,4 +280,4 @@ __all__ = ["DcnProblem", "DcnError", "make_problem", "problem_for", "taps", "loa
            "library_path", "EXPORTED_SYMBOLS", *EXPORTED_SYMBOLS, "ABI_VERSION",
            "DCN_CORE_NOALLOC_SCRATCH_BYTES",
            "DCN_OK", "DCN_ERR_INVALID_ARG", "DCN_ERR_UNSUPPORTED", "DCN_ERR_CUDA",
-           "DCN_ERR_TIMEOUT", "DCN_F32", "DCN_BF16"]
+           "DCN_ERR_TIMEOUT", "DCN_ERR_OUT_OF_BOUNDS", "DCN_F32", "DCN_BF16"]

@@ -17,6 +17,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libdcncore.so")
+# The bounds-checked build: every global access of the kernels is tested
+# against its tensor's extent first (a substitute for a memory checker).
+LIB_CHECKED = os.path.join(HERE, "libdcncore_checked.so")
 SOURCES = [os.path.join(CSRC, "dcn_core.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "dcn_core.h")]
@@ -35,26 +38,29 @@ def nvcc_command(out: str, extra: list[str] | None = None) -> list[str]:
             "-I", INCLUDE, "-o", out] + (extra or []) + SOURCES
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(d) > t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or needs_build():
-        tmp = LIB + ".tmp.%d" % os.getpid()
-        cmd = nvcc_command(tmp, ["-Xptxas", "-v"] if verbose else None)
-        res = subprocess.run(cmd, capture_output=True, text=True)
+def build(force: bool = False, verbose: bool = False, checked: bool = False) -> str:
+    """Build libdcncore.so (or, with checked=True, libdcncore_checked.so with
+    -DDCN_CHECK_BOUNDS) next to this file, if a source is newer."""
+    lib = LIB_CHECKED if checked else LIB
+    if force or needs_build(lib):
+        tmp = lib + ".tmp.%d" % os.getpid()
+        extra = (["-Xptxas", "-v"] if verbose else []) + (["-DDCN_CHECK_BOUNDS"] if checked else [])
+        res = subprocess.run(nvcc_command(tmp, extra), capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
         if verbose:
             sys.stderr.write(res.stderr)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                checked="--checked" in sys.argv))

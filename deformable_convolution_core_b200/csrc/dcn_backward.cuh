@@ -147,24 +147,28 @@ struct GxScatter;
 template <>
 struct GxScatter<false> {
   float* p;
-  __device__ __forceinline__ GxScatter(void* base, const unsigned int*, bool, int)
-      : p(static_cast<float*>(base)) {}
+  size_t n;  // accumulator elements (checked in the bounds-checked build)
+  __device__ __forceinline__ GxScatter(void* base, const unsigned int*, bool, int, size_t n_)
+      : p(static_cast<float*>(base)), n(n_) {}
   // accumulator[e .. e+3] += (lo, hi) if pred
   __device__ __forceinline__ void add(size_t e, float2 lo, float2 hi, bool pred) const {
+    if (pred && !in_range(e + 3, n)) pred = false;
     red_add_v4_pred(p + e, lo, hi, pred);
   }
 };
 template <>
 struct GxScatter<true> {
   unsigned long long* p;
+  size_t n;     // accumulator elements (checked in the bounds-checked build)
   float scale;  // 2^S, or 0 when the bounds are not finite
   __device__ __forceinline__ GxScatter(void* base, const unsigned int* hdr, bool softmax,
-                                       int cbits)
-      : p(static_cast<unsigned long long*>(base)) {
+                                       int cbits, size_t n_)
+      : p(static_cast<unsigned long long*>(base)), n(n_) {
     int S = 0;
     scale = det_exponent(hdr, softmax, cbits, &S) ? __int_as_float((S + 127) << 23) : 0.f;
   }
   __device__ __forceinline__ void add(size_t e, float2 lo, float2 hi, bool pred) const {
+    if (pred && !in_range(e + 3, n)) pred = false;
     // v * 2^S is exact (a power-of-two scaling below 2^62); the conversion rounds
     // it to the nearest integer.
     const long long a = __float2ll_rn(lo.x * scale), b = __float2ll_rn(lo.y * scale);
@@ -247,7 +251,10 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
   const size_t img_off = size_t(tc.n) * t.H * rowE + size_t(sub) * CPL;
   const char* xbytes = reinterpret_cast<const char*>(a.x);
   const char* gobytes = reinterpret_cast<const char*>(a.gout);
-  const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits);
+  const size_t n_img = size_t(t.N) * t.H * rowE;  // input (and accumulator) elements
+  const size_t n_out = size_t(t.N) * t.Ho * t.Wo * pixE;
+  const size_t n_taps = size_t(t.N) * t.Ho * t.Wo * t.G * KK;
+  const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits, n_img);
 
   for (int v0 = warp * UPW; v0 < units; v0 += kWarps * UPW) {
     const UnitCoord u = unit_coord(t, tc, v0 + lane / LANES);
@@ -260,7 +267,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
     const int by = u.ho * t.stride - t.pad, bx = u.wo * t.stride_w - t.pad_w;
 
     float go[CPL];
-    Quad<T>::load(gobytes + (upix * t.C + size_t(u.g) * t.Cg + size_t(sub) * CPL) * sizeof(T), go);
+    const size_t gi = upix * t.C + size_t(u.g) * t.Cg + size_t(sub) * CPL;
+    Quad<T>::load_pred(gobytes + gi * sizeof(T), in_range(gi + CPL - 1, n_out), go);
 
     // One tap: returns s_k (reduced over the unit's lanes) and writes the
     // offset gradient of the tap.
@@ -281,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float cv[CPL] = {0.f, 0.f, 0.f, 0.f};
-          if (cval[c]) Quad<T>::load(xg + cofs[c] * ptrdiff_t(sizeof(T)), cv);
+          if (cval[c] && in_range(size_t(ptrdiff_t(g_off) + cofs[c]) + CPL - 1, n_img))
+            Quad<T>::load(xg + cofs[c] * ptrdiff_t(sizeof(T)), cv);
           float dsum = 0.f;
 #pragma unroll
           for (int j = 0; j < CPL; ++j) dsum = fmaf(go[j], cv[j], dsum);
@@ -301,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
       }
       if (sub == 0) {
         const float sc = t.sigma * mk;
-        Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
+        if (in_range(unit * KK + k, n_taps))
+          Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
       }
       return s;
     };
@@ -342,7 +352,9 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
           cval[j][3] = f[j].v11;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
-            Quad<T>::load_pred(xg + ptrdiff_t(cofs[j][c]) * ptrdiff_t(sizeof(T)), cval[j][c],
+            Quad<T>::load_pred(xg + ptrdiff_t(cofs[j][c]) * ptrdiff_t(sizeof(T)),
+                               cval[j][c] && in_range(size_t(ptrdiff_t(g_off) + cofs[j][c]) +
+                                                          CPL - 1, n_img),
                                cv[j][c]);
         }
 #pragma unroll
@@ -373,7 +385,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
           }
           if (sub == 0) {
             const float sc = t.sigma * m[k];
-            Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
+            if (in_range(unit * KK + k, n_taps))
+              Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
           }
         }
       }
@@ -385,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
         }
 #pragma unroll
         for (int k = 0; k < KKS; ++k)
-          Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? m[k] * (s[k] - ms) : s[k]);
+          if (in_range(unit * KK + k, n_taps))
+            Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? m[k] * (s[k] - ms) : s[k]);
       }
     } else {
       // Runtime tap count: keep s_k in the tap's staged offset slot, which no
@@ -414,7 +428,8 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
         for (int k = 0; k < KK; ++k) {
           const float sk = s_at(k);
           const float mk = mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv);
-          Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? mk * (sk - ms) : sk);
+          if (in_range(unit * KK + k, n_taps))
+            Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? mk * (sk - ms) : sk);
         }
       }
     }

@@ -211,6 +211,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   };
 
   // Raw inputs of the next batch, prefetched in the staging layout.
+  const size_t n_taps = size_t(t.N) * t.Ho * t.Wo * t.G * KK;  // offset pairs, mask values
+  const size_t n_img = size_t(t.N) * t.H * t.W * t.C;           // input, accumulator elements
+  const size_t n_out = size_t(t.N) * t.Ho * t.Wo * t.C;
   Pair pf_pair[KK];
   One pf_one[KK];
   auto prefetch = [&](int beta) {
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
     for (int k = 0; k < KK; ++k) {
       const unsigned long long src = __shfl_sync(0xFFFFFFFFu, qv, st_unit[k]);
-      if (src != ~0ull) {
+      if (src != ~0ull && in_range(size_t(src) + st_tap[k], n_taps)) {
         pf_pair[k] = IO::ld_pair(a.off, size_t(src) + st_tap[k]);
         pf_one[k] = IO::ld_one(a.mask, size_t(src) + st_tap[k]);
       } else {
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const int X0 = c.wo0 * t.stride_w - t.pad_w - t.halo;
     const size_t img = size_t(c.n) * t.H * t.W * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4;
     const char* xg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
-    const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits);
+    const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits, n_img);
 
     for (; beta < (il + 1) * nb; beta += kTiledWarps) {
       // Staging: the prefetched inputs go to the unit slots.
@@ -342,7 +345,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         float go[4];
         Quad<T>::load_pred(reinterpret_cast<const char*>(a.gout) +
                                (pix * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4) * sizeof(T),
-                           uvalid, go);
+                           uvalid && in_range(pix * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4 + 3,
+                                              n_out),
+                           go);
         const float2 g01 = make_float2(go[0], go[1]), g23 = make_float2(go[2], go[3]);
         float sk[KK];
 #pragma unroll
@@ -369,7 +374,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
               const void* src =
                   far ? static_cast<const void*>(xg + ptrdiff_t(e) * ptrdiff_t(sizeof(T)))
                       : static_cast<const void*>(bp + (dy * t.BW + dx) * CS);
-              BwdPiece<T>::load(src, in, cv[cc]);
+              BwdPiece<T>::load(src,
+                                in && (!far || in_range(img + size_t(e) + 3, n_img)), cv[cc]);
             }
           } else {
             // every footprint is in the box: plain shared loads (corners outside
@@ -401,7 +407,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           sk[k] = sv;
           if (sub == 0 && uvalid) {
             const float sc = t.sigma * mk;
-            Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
+            if (in_range(unit * KK + k, n_taps))
+              Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
           }
         }
         if (sub == 0 && uvalid) {
@@ -413,7 +420,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           }
 #pragma unroll
           for (int k = 0; k < KK; ++k)
-            Quad<T>::store_one(a.gmask, unit * KK + k,
+            if (in_range(unit * KK + k, n_taps)) Quad<T>::store_one(a.gmask, unit * KK + k,
                                SOFTMAX ? ms_[k] * (sk[k] - msum) : sk[k]);
         }
       }

@@ -7,6 +7,43 @@
 
 namespace dcn {
 
+// Device error word, read and cleared by dcn_core_sync_status: bit 0 = a
+// bounded wait gave up, bit 1 = the bounds-checked build skipped an access
+// that would have left its tensor.
+constexpr unsigned int kErrTimeout = 1u, kErrOutOfBounds = 2u;
+__device__ unsigned int g_dcn_error_word = 0;
+
+// ---------------------------------------------------------------------------
+// Bounds-checked build (compiled with -DDCN_CHECK_BOUNDS), the substitute for
+// a memory checker: every global load, store and reduction of the kernels is
+// first tested against its tensor's extent, and an access that would leave it
+// is skipped and recorded in the error word.  Without the macro the tests
+// compile away.
+// ---------------------------------------------------------------------------
+#ifdef DCN_CHECK_BOUNDS
+constexpr bool kCheckBounds = true;
+#else
+constexpr bool kCheckBounds = false;
+#endif
+
+// Element i of a tensor of n elements?
+__device__ __forceinline__ bool in_range(size_t i, size_t n) {
+  if (!kCheckBounds) return true;
+  const bool ok = i < n;
+  if (!ok) atomicOr(&g_dcn_error_word, kErrOutOfBounds);
+  return ok;
+}
+
+// [p, p + nbytes) inside the tensor [base, base + bytes)?
+__device__ __forceinline__ bool in_tensor(const void* p, size_t nbytes, const void* base,
+                                          size_t bytes) {
+  if (!kCheckBounds) return true;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+  const bool ok = a >= b && a + nbytes <= b + bytes;
+  if (!ok) atomicOr(&g_dcn_error_word, kErrOutOfBounds);
+  return ok;
+}
+
 // ---------------------------------------------------------------------------
 // Division by a runtime-invariant divisor with one multiply-high and a shift
 // (Granlund and Montgomery, "Division by invariant integers using

@@ -21,11 +21,6 @@
 #include "dcn_projection.cuh"
 
 namespace dcn {
-
-// Device error word: set by a kernel whose bounded wait gave up; read and
-// cleared by dcn_core_sync_status.
-__device__ unsigned int g_dcn_error_word = 0;
-
 namespace {
 
 // Shared memory a CTA may use for its staged offsets and mask, by default.
@@ -715,7 +710,7 @@ dcn_status dcn_core_sync_status(cudaStream_t stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     cudaMemcpyToSymbol(g_dcn_error_word, &zero, sizeof(zero));
-    return DCN_ERR_TIMEOUT;
+    return (word & kErrOutOfBounds) ? DCN_ERR_OUT_OF_BOUNDS : DCN_ERR_TIMEOUT;
   }
   return DCN_OK;
 }
@@ -727,6 +722,8 @@ const char* dcn_status_string(dcn_status status) {
     case DCN_ERR_UNSUPPORTED: return "unsupported argument (alignment, channel width or dtype)";
     case DCN_ERR_CUDA: return "CUDA error";
     case DCN_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case DCN_ERR_OUT_OF_BOUNDS:
+      return "an access outside a tensor was skipped (bounds-checked build)";
     default: return "unknown status";
   }
 }

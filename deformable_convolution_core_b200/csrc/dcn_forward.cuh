@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kThreads) dcn_forward_kernel(const FwdArgs a) 
   const size_t rowB = size_t(t.W) * pixB;
   const char* xbase = reinterpret_cast<const char*>(a.x) +
                       size_t(tc.n) * t.H * rowB + size_t(sub) * CPL * S::kSize;
+  const size_t x_bytes = size_t(t.N) * t.H * rowB;                     // bounds-checked build
+  const size_t out_bytes = size_t(t.N) * t.Ho * t.Wo * t.C * S::kSize;  // bounds-checked build
 
   for (int v0 = warp * UPW; v0 < units; v0 += kWarps * UPW) {
     const UnitCoord u = unit_coord(t, tc, v0 + lane / LANES);
@@ -82,10 +84,10 @@ __global__ void __launch_bounds__(kThreads) dcn_forward_kernel(const FwdArgs a) 
       V c00, c01, c10, c11;
 #pragma unroll
       for (int i = 0; i < NW; ++i) c00.w[i] = c01.w[i] = c10.w[i] = c11.w[i] = 0u;
-      if (f.v00) ldg_nc(c00, p);
-      if (f.v01) ldg_nc(c01, p + pixB);
-      if (f.v10) ldg_nc(c10, p + rowB);
-      if (f.v11) ldg_nc(c11, p + rowB + pixB);
+      if (f.v00 && in_tensor(p, VB, a.x, x_bytes)) ldg_nc(c00, p);
+      if (f.v01 && in_tensor(p + pixB, VB, a.x, x_bytes)) ldg_nc(c01, p + pixB);
+      if (f.v10 && in_tensor(p + rowB, VB, a.x, x_bytes)) ldg_nc(c10, p + rowB);
+      if (f.v11 && in_tensor(p + rowB + pixB, VB, a.x, x_bytes)) ldg_nc(c11, p + rowB + pixB);
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
         float s = acc[j];
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) dcn_forward_kernel(const FwdArgs a) 
     char* op = reinterpret_cast<char*>(a.out) +
                ((size_t(tc.n * t.Ho + u.ho) * t.Wo + u.wo) * t.C + size_t(u.g) * t.Cg +
                 size_t(sub) * CPL) * S::kSize;
-    stg(op, o);
+    if (in_tensor(op, VB, a.out, out_bytes)) stg(op, o);
   }
 }
 

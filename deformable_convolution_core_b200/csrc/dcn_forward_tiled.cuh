@@ -342,6 +342,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   };
 
   // Raw inputs of the next batch, prefetched in the staging layout.
+  const size_t n_entries = size_t(t.N) * t.Ho * t.Wo * t.G * KK;  // offset pairs, mask values
+  const size_t x_bytes = size_t(t.N) * t.H * t.W * pixB;            // bounds-checked build
+  const size_t out_bytes = size_t(t.N) * t.Ho * t.Wo * pixB;
   Pair pf_pair[KK];
   One pf_one[KK];
   auto prefetch = [&](int beta) {
@@ -353,7 +356,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
     for (int k = 0; k < KK; ++k) {
       const unsigned long long src = __shfl_sync(0xFFFFFFFFu, qv, st_unit[k]);
-      if (src != ~0ull) {
+      if (src != ~0ull && in_range(size_t(src) + st_tap[k], n_entries)) {
         pf_pair[k] = IO::ld_pair(a.off, size_t(src) + st_tap[k]);
         pf_one[k] = IO::ld_one(a.mask, size_t(src) + st_tap[k]);
       } else {
@@ -477,7 +480,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         const char* gp = ximg + (size_t(in ? yc : 0) * t.W + (in ? xc : 0)) * pixB;
 #pragma unroll
         for (int j = 0; j < NP; ++j)
-          fv[j] = in ? ldg128(gp + Role::piece(j, q, dyc) * 16) : make_uint4(0u, 0u, 0u, 0u);
+          fv[j] = (in && in_tensor(gp + Role::piece(j, q, dyc) * 16, 16, a.x, x_bytes))
+                      ? ldg128(gp + Role::piece(j, q, dyc) * 16)
+                      : make_uint4(0u, 0u, 0u, 0u);
         if (!in) fw = 0.f;
       };
       auto far_first = [&](int u, uint4 (&fv)[NP], float& fw) {
@@ -569,10 +574,12 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           if (CS == 32) {
             const int ch = 8 * q + 4 * dxc + 2 * dyc;
             const uint32_t w = pack_bf16x2(h2[0], h2[1]);
-            asm volatile("st.global.b32 [%0], %1;" ::"l"(op + ch * 2), "r"(w) : "memory");
+            if (in_tensor(op + ch * 2, 4, a.out, out_bytes))
+              asm volatile("st.global.b32 [%0], %1;" ::"l"(op + ch * 2), "r"(w) : "memory");
           } else {
             const int ch = 4 * (q + 2 * dxc) + 2 * dyc;
-            asm volatile("st.global.v2.f32 [%0], {%1, %2};" ::"l"(op + ch * 4), "f"(h2[0]),
+            if (in_tensor(op + ch * 4, 8, a.out, out_bytes))
+              asm volatile("st.global.v2.f32 [%0], {%1, %2};" ::"l"(op + ch * 4), "f"(h2[0]),
                          "f"(h2[1])
                          : "memory");
           }

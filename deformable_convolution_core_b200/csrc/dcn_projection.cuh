@@ -280,17 +280,22 @@ __global__ void __launch_bounds__(kPjThreads, 1)
         const float b = (a.bias != nullptr && cin) ? a.bias[col] : 0.f;
         T* dst;
         size_t pitch;
+        const T* tensor;  // the output tensor of this column (bounds-checked build)
         if (col < a.n_off) {
           dst = static_cast<T*>(a.offset) + col;
           pitch = size_t(a.n_off);
+          tensor = static_cast<const T*>(a.offset);
         } else {
           dst = static_cast<T*>(a.mask) + (col - a.n_off);
           pitch = size_t(n_mask);
+          tensor = static_cast<const T*>(a.mask);
         }
+        const size_t tensor_bytes = size_t(a.M) * pitch * sizeof(T);
         dst += size_t(row0) * pitch;
 #pragma unroll 8
         for (int r = 0; r < 32; ++r) {
-          if (cin && r < rows) Storage<T>::store_float(dst, st[r * kPjEpiPitch + lane] + b);
+          if (cin && r < rows && in_tensor(dst, sizeof(T), tensor, tensor_bytes))
+            Storage<T>::store_float(dst, st[r * kPjEpiPitch + lane] + b);
           dst += pitch;
         }
         __syncwarp();

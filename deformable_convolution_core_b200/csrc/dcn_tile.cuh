@@ -122,8 +122,8 @@ __device__ __forceinline__ void stage_tile(const TileParams& t, const TileCoord&
     const int r = int(fdiv(uint32_t(pix), t.fd_TW));
     const int c = pix - r * t.TW;
     const int ho = tc.ho0 + r, wo = tc.wo0 + c;
-    if (ho < t.Ho && wo < t.Wo) {
-      const size_t q = (size_t(tc.n * t.Ho + ho) * t.Wo + wo) * GKK + j;
+    const size_t q = (size_t(tc.n * t.Ho + ho) * t.Wo + wo) * GKK + j;
+    if (ho < t.Ho && wo < t.Wo && in_range(q, size_t(t.N) * t.Ho * t.Wo * GKK)) {
       s_off[j * t.P1 + pix] = Staged<T>::load_pair(off, q);
       s_msk[j * t.P1 + pix] = Staged<T>::load_one(mask, q);
     }

@@ -65,7 +65,8 @@ typedef enum {
   DCN_ERR_INVALID_ARG = 1,
   DCN_ERR_UNSUPPORTED = 2,
   DCN_ERR_CUDA = 3,
-  DCN_ERR_TIMEOUT = 4
+  DCN_ERR_TIMEOUT = 4,
+  DCN_ERR_OUT_OF_BOUNDS = 5  /* only from a library built with -DDCN_CHECK_BOUNDS */
 } dcn_status;
 
 typedef enum {
@@ -271,8 +272,10 @@ DCN_API dcn_status dcn_core_linear_bf16(const void* input, int M, int K, const v
                                         dcn_dtype out_dtype, cudaStream_t stream);
 
 /* Synchronises `stream` and reports: DCN_ERR_CUDA if CUDA reports an error,
- * DCN_ERR_TIMEOUT if a kernel of this library gave up a bounded wait since
- * the last call (the device error word is then cleared), else DCN_OK. */
+ * DCN_ERR_OUT_OF_BOUNDS if the bounds-checked build (compiled with
+ * -DDCN_CHECK_BOUNDS) skipped an access outside a tensor, DCN_ERR_TIMEOUT if a
+ * kernel of this library gave up a bounded wait since the last call (the
+ * device error word is then cleared), else DCN_OK. */
 DCN_API dcn_status dcn_core_sync_status(cudaStream_t stream);
 
 /* Static description of a status code. */

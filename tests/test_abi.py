@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 3
-    for st in range(5):
+    for st in range(6):
         assert dcn.dcn_status_string(st)
     assert "unknown" in dcn.dcn_status_string(99)
 
