@@ -376,7 +376,12 @@ def run_e2e(step, inputs, args, barrier, world):
                 step.x.copy_(hx, non_blocking=True)
                 step.off.copy_(ho, non_blocking=True)
                 step.mask.copy_(hm, non_blocking=True)
-        if step.backward:
+        if step.backward and not step.deterministic:
+            # grad_out in and the three gradients out, chunked and overlapped
+            dcn.dcn_core_backward_host(step.p, step.x, step.off, step.mask, hg, hgx, hgo, hgm,
+                                       step.gout, step.gx, step.goff, step.gm, step.ws,
+                                       step.ws_bytes, step.sh)
+        elif step.backward:
             with torch.cuda.stream(s):
                 step.gout.copy_(hg, non_blocking=True)
             step.bwd()

@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("DCN_CORE_LIBRARY") or os.path.join(_HERE, "libdcncore.so")
 
 # DCN_CORE_ABI_VERSION of include/dcn_core.h that DcnProblem mirrors.
-ABI_VERSION = 3
+ABI_VERSION = 4
 DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
 DCN_ERR_OUT_OF_BOUNDS = 5  # only from the bounds-checked build
 # Scratch the allocation-free backward owns per GPU (DCN_CORE_NOALLOC_SCRATCH_BYTES).
@@ -35,6 +35,7 @@ EXPORTED_SYMBOLS = (
     "dcn_core_forward_host",
     "dcn_core_backward_workspace",
     "dcn_core_backward",
+    "dcn_core_backward_host",
     "dcn_core_backward_noalloc",
     "dcn_core_backward_deterministic_workspace",
     "dcn_core_backward_deterministic",
@@ -124,6 +125,8 @@ def load_library():
     lib.dcn_core_backward_workspace.restype = ctypes.c_size_t
     lib.dcn_core_backward.argtypes = [pp] + [vp] * 8 + [ctypes.c_size_t, vp]
     lib.dcn_core_backward.restype = st
+    lib.dcn_core_backward_host.argtypes = [pp] + [vp] * 12 + [ctypes.c_size_t, vp]
+    lib.dcn_core_backward_host.restype = st
     lib.dcn_core_backward_noalloc.argtypes = [pp] + [vp] * 8
     lib.dcn_core_backward_noalloc.restype = st
     lib.dcn_core_backward_deterministic_workspace.argtypes = [pp]
@@ -214,6 +217,18 @@ def dcn_core_backward(problem: DcnProblem, input, offset, mask, grad_out, grad_i
         ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
         _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _ptr(workspace),
         int(workspace_bytes), _stream(stream)), "dcn_core_backward")
+
+
+def dcn_core_backward_host(problem: DcnProblem, input, offset, mask, h_grad_out, h_grad_input,
+                           h_grad_offset, h_grad_mask, d_grad_out, d_grad_input, d_grad_offset,
+                           d_grad_mask, workspace=None, workspace_bytes=0, stream=None) -> None:
+    """Backward with grad_out and the three gradients on (pinned) host
+    buffers; input, offset and mask are the device tensors of the forward."""
+    _check(load_library().dcn_core_backward_host(
+        ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(h_grad_out),
+        _ptr(h_grad_input), _ptr(h_grad_offset), _ptr(h_grad_mask), _ptr(d_grad_out),
+        _ptr(d_grad_input), _ptr(d_grad_offset), _ptr(d_grad_mask), _ptr(workspace),
+        int(workspace_bytes), _stream(stream)), "dcn_core_backward_host")
 
 
 def dcn_core_backward_noalloc(problem: DcnProblem, input, offset, mask, grad_out, grad_input,

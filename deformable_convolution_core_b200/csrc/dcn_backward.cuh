@@ -58,6 +58,12 @@ struct Quad<float> {
   __device__ __forceinline__ static void store_pair(void* base, size_t i, float a, float b) {
     reinterpret_cast<float2*>(base)[i] = make_float2(a, b);
   }
+  // (a, b) to the pair at p if pred != 0, without a branch
+  __device__ __forceinline__ static void store_pair_pred(void* p, float a, float b, uint32_t pred) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n @q st.global.v2.f32 [%0], {%1, %2};\n}"
+                 ::"l"(p), "f"(a), "f"(b), "r"(pred)
+                 : "memory");
+  }
   __device__ __forceinline__ static void store_one(void* base, size_t i, float a) {
     reinterpret_cast<float*>(base)[i] = a;
   }
@@ -85,6 +91,11 @@ struct Quad<__nv_bfloat16> {
   }
   __device__ __forceinline__ static void store_pair(void* base, size_t i, float a, float b) {
     reinterpret_cast<uint32_t*>(base)[i] = pack_bf16x2(a, b);
+  }
+  __device__ __forceinline__ static void store_pair_pred(void* p, float a, float b, uint32_t pred) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q st.global.b32 [%0], %1;\n}"
+                 ::"l"(p), "r"(pack_bf16x2(a, b)), "r"(pred)
+                 : "memory");
   }
   __device__ __forceinline__ static void store_one(void* base, size_t i, float a) {
     reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(a);
@@ -146,6 +157,7 @@ template <bool DET>
 struct GxScatter;
 template <>
 struct GxScatter<false> {
+  using Acc = float;
   float* p;
   size_t n;  // accumulator elements (checked in the bounds-checked build)
   __device__ __forceinline__ GxScatter(void* base, const unsigned int*, bool, int, size_t n_)
@@ -155,9 +167,20 @@ struct GxScatter<false> {
     if (pred && !in_range(e + 3, n)) pred = false;
     red_add_v4_pred(p + e, lo, hi, pred);
   }
+  // the same at q = p + e, the address computed by the caller, if pred != 0
+  // (e is only read by the bounds-checked build)
+  __device__ __forceinline__ void add_at(float* q, size_t e, float2 lo, float2 hi,
+                                         uint32_t pred) const {
+    if (pred != 0u && !in_range(e + 3, n)) pred = 0u;
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
+                 " @q red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n}" ::"l"(q),
+                 "f"(lo.x), "f"(lo.y), "f"(hi.x), "f"(hi.y), "r"(pred)
+                 : "memory");
+  }
 };
 template <>
 struct GxScatter<true> {
+  using Acc = unsigned long long;
   unsigned long long* p;
   size_t n;     // accumulator elements (checked in the bounds-checked build)
   float scale;  // 2^S, or 0 when the bounds are not finite
@@ -179,6 +202,10 @@ struct GxScatter<true> {
         " @q red.global.add.u64 [%0+16], %3;\n @q red.global.add.u64 [%0+24], %4;\n}" ::"l"(p + e),
         "l"(a), "l"(b), "l"(c), "l"(d), "r"(int(pred))
         : "memory");
+  }
+  __device__ __forceinline__ void add_at(unsigned long long* q, size_t e, float2 lo, float2 hi,
+                                         uint32_t pred) const {
+    add(size_t(q - p), lo, hi, pred != 0u && in_range(e + 3, n));
   }
 };
 

@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   const unsigned umask = 0xFu << (ul * LU);
   const int pixE = t.C;            // elements between horizontally adjacent pixels
   const int rowE = t.W * t.C;      // ... vertically adjacent pixels
+  const int cofs[4] = {0, pixE, rowE, rowE + pixE};  // corner (dy, dx) from corner (0, 0)
   const int npx = t.TH * t.TW;
   const int nb = t.batches;
   // the staging element e = lane + 32 k (k < KK) belongs to unit e / KK, tap e % KK
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const size_t img = size_t(c.n) * t.H * t.W * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4;
     const char* xg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
     const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits, n_img);
+    typename GxScatter<DET>::Acc* const gx_item = gxs.p + img;
 
     for (; beta < (il + 1) * nb; beta += kTiledWarps) {
       // Staging: the prefetched inputs go to the unit slots.
@@ -342,6 +344,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         const bool uvalid = v < npx && uho < t.Ho && uwo < t.Wo;
         const size_t pix = size_t(c.n * t.Ho + uho) * t.Wo + uwo;
         const size_t unit = pix * t.G + c.g;
+        // grad_offset pairs of this unit, written by its first lane without a branch
+        char* const goff_u = reinterpret_cast<char*>(a.goff) + unit * KK * sizeof(Pair);
+        const uint32_t st_ok = (sub == 0 && uvalid) ? 1u : 0u;
         float go[4];
         Quad<T>::load_pred(reinterpret_cast<const char*>(a.gout) +
                                (pix * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4) * sizeof(T),
@@ -385,17 +390,17 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
               BoxPiece<T>::load(bp + ((cc >> 1) * t.BW + (cc & 1)) * CS, cv[cc]);
           }
           float dc[4];
+          auto* const p00 = gx_item + ce;  // accumulator at corner (y0, x0)
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
-            const int dy = cc >> 1, dx = cc & 1;
-            const bool in = ((code >> (24 + cc)) & 1u) != 0u;
-            const int e = ce + dy * rowE + dx * pixE;  // element offset of the corner
+            const uint32_t inb = code & (1u << (24 + cc));  // corner in the image
             float2 pd = __fmul2_rn(make_float2(cv[cc][0], cv[cc][1]), g01);
             pd = __ffma2_rn(make_float2(cv[cc][2], cv[cc][3]), g23, pd);
-            dc[cc] = in ? pd.x + pd.y : 0.f;
+            dc[cc] = inb ? pd.x + pd.y : 0.f;
             const float wv = mk * cw[cc];
             const float2 w2 = make_float2(wv, wv);
-            gxs.add(img + size_t(e), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23), in);
+            gxs.add_at(p00 + cofs[cc], kCheckBounds ? img + size_t(ce + cofs[cc]) : 0,
+                       __fmul2_rn(w2, g01), __fmul2_rn(w2, g23), inb);
           }
           // a sample that contributes nothing has no corner in the image: every dc is 0
           float sv = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];
@@ -405,11 +410,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           gX = unit_sum<LU>(gX, umask);
           gY = unit_sum<LU>(gY, umask);
           sk[k] = sv;
-          if (sub == 0 && uvalid) {
-            const float sc = t.sigma * mk;
-            if (in_range(unit * KK + k, n_taps))
-              Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
-          }
+          const float sc = t.sigma * mk;
+          Quad<T>::store_pair_pred(goff_u + k * sizeof(Pair), sc * gX, sc * gY,
+                                   (st_ok != 0u && in_range(unit * KK + k, n_taps)) ? 1u : 0u);
         }
         if (sub == 0 && uvalid) {
           const float* ms_ = reinterpret_cast<const float*>(sl + kBwdMaskAt);

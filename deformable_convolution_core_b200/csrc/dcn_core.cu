@@ -13,6 +13,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <numeric>
 
 #include "dcn_backward.cuh"
 #include "dcn_backward_tiled.cuh"
@@ -476,7 +477,7 @@ dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   const int e = esize(p->dtype);
   const int cs = p->Cg * e;
   const size_t slot_bytes = size_t(kTiledWarps) * kTiledBatch * kSlotBytes;
-  const size_t fixed = slot_bytes + 64;
+  const size_t fixed = slot_bytes + kTiledTailBytes;  // mbarriers, abort flag, zero area
   if (size_t(L->dev.smem_optin) <= fixed + 2048) return DCN_ERR_UNSUPPORTED;
   const size_t box_budget = (size_t(L->dev.smem_optin) - fixed) / 2 / 1024 * 1024;
   const int halo = env_int("DCN_CORE_HALO", 5);
@@ -590,6 +591,84 @@ dcn_status backward_launch(const dcn_problem* p, int64_t Ho, int64_t Wo, const P
   }
   return backward_dispatch(p, plan, a, det, stream);
 }
+// ---------------------------------------------------------------------------
+// Host entry points.  The batch is cut into chunks of whole images; chunk i's
+// host-to-device copies run on a library stream, its kernels on the caller's
+// stream and its device-to-host copies on a second library stream, so that
+// the two copy directions (separate copy engines) and the kernels overlap.
+// Events order the three streams and join the library streams back into the
+// caller's stream at the end.
+// ---------------------------------------------------------------------------
+constexpr int kHostChunks = 8;  // chunks per call, at most
+
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev[2 * kHostChunks + 2] = {};
+};
+
+// The pipe of the current device, created on first use.  The returned lock is
+// held while the caller enqueues: the events are re-recorded by the next call,
+// which is safe because a wait already enqueued refers to the record it saw.
+dcn_status host_pipe(HostPipe** out, std::unique_lock<std::mutex>* held) {
+  constexpr int kMaxDev = 64;
+  static HostPipe pipes[kMaxDev];
+  static bool ready[kMaxDev] = {};
+  static std::mutex lock;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DCN_ERR_CUDA;
+  *held = std::unique_lock<std::mutex>(lock);
+  if (!ready[dev]) {
+    HostPipe hp;
+    if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess)
+      return DCN_ERR_CUDA;
+    for (cudaEvent_t& e : hp.ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return DCN_ERR_CUDA;
+    pipes[dev] = hp;
+    ready[dev] = true;
+  }
+  *out = &pipes[dev];
+  return DCN_OK;
+}
+
+// Images per chunk: about N / kHostChunks, rounded up to a multiple that keeps
+// every tensor's chunk start 32-byte aligned (per_image: bytes of one image of
+// each tensor); one chunk when that multiple reaches N.
+struct ChunkPlan {
+  int64_t per = 1;
+  int chunks = 1;
+};
+ChunkPlan chunk_plan(int64_t N, std::initializer_list<size_t> per_image) {
+  int64_t q = 1;
+  for (size_t bytes : per_image) q = std::lcm<int64_t>(q, int64_t(32 / std::gcd(bytes, size_t(32))));
+  int64_t per = (N + kHostChunks - 1) / kHostChunks;
+  per = (per + q - 1) / q * q;
+  if (per >= N) per = N;
+  ChunkPlan cp;
+  cp.per = per;
+  cp.chunks = int((N + per - 1) / per);
+  return cp;
+}
+
+#define DCN_CU(call)                                   \
+  do {                                                 \
+    if ((call) != cudaSuccess) return DCN_ERR_CUDA;    \
+  } while (0)
+
+// Chunk offset helpers.
+inline const char* at(const void* p, size_t off) { return static_cast<const char*>(p) + off; }
+inline char* at(void* p, size_t off) { return static_cast<char*>(p) + off; }
+
+// Per-image byte counts of the problem's tensors.
+struct ImageBytes {
+  size_t x, off, msk, out;  // input (and grad_input), offset, mask, output (and grad_out)
+};
+ImageBytes image_bytes(const dcn_problem* p, int64_t Ho, int64_t Wo) {
+  const size_t e = size_t(esize(p->dtype));
+  const size_t C = size_t(p->G) * p->Cg, KK = size_t(taps(p)), px = size_t(Ho) * Wo;
+  return {size_t(p->H) * p->W * C * e, px * p->G * KK * 2 * e, px * p->G * KK * e, px * C * e};
+}
+
 }  // namespace
 }  // namespace dcn
 
@@ -642,20 +721,40 @@ dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input
   if (!h_input || !h_offset || !h_mask || !h_output) return DCN_ERR_INVALID_ARG;
   st = check_forward_pointers(problem, d_input, d_offset, d_mask, d_output);
   if (st != DCN_OK) return st;
-  const size_t e = size_t(esize(problem->dtype));
-  const size_t C = size_t(problem->G) * problem->Cg, KK = size_t(taps(problem));
-  const size_t b_in = size_t(problem->N) * problem->H * problem->W * C * e;
-  const size_t px = size_t(problem->N) * Ho * Wo;
-  const size_t b_off = px * problem->G * KK * 2 * e, b_msk = px * problem->G * KK * e;
-  const size_t b_out = px * C * e;
-  if (cudaMemcpyAsync(d_input, h_input, b_in, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(d_offset, h_offset, b_off, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
-      cudaMemcpyAsync(d_mask, h_mask, b_msk, cudaMemcpyHostToDevice, stream) != cudaSuccess)
-    return DCN_ERR_CUDA;
-  st = dcn_core_forward(problem, d_input, d_offset, d_mask, d_output, stream);
+  const ImageBytes ib = image_bytes(problem, Ho, Wo);
+  const ChunkPlan cp = chunk_plan(problem->N, {ib.x, ib.off, ib.msk, ib.out});
+  HostPipe* hp = nullptr;
+  std::unique_lock<std::mutex> held;
+  st = host_pipe(&hp, &held);
   if (st != DCN_OK) return st;
-  if (cudaMemcpyAsync(h_output, d_output, b_out, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
-    return DCN_ERR_CUDA;
+  cudaEvent_t* const ev = hp->ev;  // [0] start, [1 + i] chunk i in, [1 + C + i] chunk i out, [2C + 1] done
+  DCN_CU(cudaEventRecord(ev[0], stream));
+  DCN_CU(cudaStreamWaitEvent(hp->h2d, ev[0], 0));
+  DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[0], 0));
+  for (int i = 0; i < cp.chunks; ++i) {
+    const int64_t n0 = int64_t(i) * cp.per, n = std::min<int64_t>(cp.per, problem->N - n0);
+    const size_t ox = size_t(n0) * ib.x, oo = size_t(n0) * ib.off, om = size_t(n0) * ib.msk,
+                 oy = size_t(n0) * ib.out;
+    DCN_CU(cudaMemcpyAsync(at(d_input, ox), at(h_input, ox), size_t(n) * ib.x,
+                           cudaMemcpyHostToDevice, hp->h2d));
+    DCN_CU(cudaMemcpyAsync(at(d_offset, oo), at(h_offset, oo), size_t(n) * ib.off,
+                           cudaMemcpyHostToDevice, hp->h2d));
+    DCN_CU(cudaMemcpyAsync(at(d_mask, om), at(h_mask, om), size_t(n) * ib.msk,
+                           cudaMemcpyHostToDevice, hp->h2d));
+    DCN_CU(cudaEventRecord(ev[1 + i], hp->h2d));
+    DCN_CU(cudaStreamWaitEvent(stream, ev[1 + i], 0));
+    dcn_problem q = *problem;
+    q.N = int(n);
+    st = dcn_core_forward(&q, at(d_input, ox), at(d_offset, oo), at(d_mask, om), at(d_output, oy),
+                          stream);
+    if (st != DCN_OK) return st;
+    DCN_CU(cudaEventRecord(ev[1 + cp.chunks + i], stream));
+    DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[1 + cp.chunks + i], 0));
+    DCN_CU(cudaMemcpyAsync(at(h_output, oy), at(d_output, oy), size_t(n) * ib.out,
+                           cudaMemcpyDeviceToHost, hp->d2h));
+  }
+  DCN_CU(cudaEventRecord(ev[2 * cp.chunks + 1], hp->d2h));
+  DCN_CU(cudaStreamWaitEvent(stream, ev[2 * cp.chunks + 1], 0));
   return DCN_OK;
 }
 
@@ -699,6 +798,72 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
   dcn_round_to_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
                                                      static_cast<uint2*>(grad_input), n4);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+dcn_status dcn_core_backward_host(const dcn_problem* problem, const void* input,
+                                  const void* offset, const void* mask, const void* h_grad_out,
+                                  void* h_grad_input, void* h_grad_offset, void* h_grad_mask,
+                                  void* d_grad_out, void* d_grad_input, void* d_grad_offset,
+                                  void* d_grad_mask, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!h_grad_out || !h_grad_input || !h_grad_offset || !h_grad_mask || !input || !offset ||
+      !mask || !d_grad_out || !d_grad_input || !d_grad_offset || !d_grad_mask)
+    return DCN_ERR_INVALID_ARG;
+  // Everything dcn_core_backward checks, on the whole problem, before the
+  // first copy is enqueued (chunk starts keep the alignment).
+  const bool bf16 = problem->dtype == DCN_BF16;
+  if (bf16 && (!workspace || workspace_bytes < bf16_accumulator_bytes(problem)))
+    return DCN_ERR_INVALID_ARG;
+  if (!aligned(input, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
+      !aligned(d_grad_out, 16) || !aligned(d_grad_input, 16) || !aligned(d_grad_offset, 16) ||
+      !aligned(d_grad_mask, 16) || (bf16 && !aligned(workspace, 16)))
+    return DCN_ERR_UNSUPPORTED;
+  {
+    Plan plan;
+    st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
+                                         : staged_bytes_per_entry<float>(),
+                   &plan, true);
+    if (st != DCN_OK) return st;
+  }
+  const ImageBytes ib = image_bytes(problem, Ho, Wo);
+  const ChunkPlan cp = chunk_plan(problem->N, {ib.x, ib.off, ib.msk, ib.out});
+  HostPipe* hp = nullptr;
+  std::unique_lock<std::mutex> held;
+  st = host_pipe(&hp, &held);
+  if (st != DCN_OK) return st;
+  cudaEvent_t* const ev = hp->ev;
+  DCN_CU(cudaEventRecord(ev[0], stream));
+  DCN_CU(cudaStreamWaitEvent(hp->h2d, ev[0], 0));
+  DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[0], 0));
+  for (int i = 0; i < cp.chunks; ++i) {
+    const int64_t n0 = int64_t(i) * cp.per, n = std::min<int64_t>(cp.per, problem->N - n0);
+    const size_t ox = size_t(n0) * ib.x, oo = size_t(n0) * ib.off, om = size_t(n0) * ib.msk,
+                 oy = size_t(n0) * ib.out;
+    DCN_CU(cudaMemcpyAsync(at(d_grad_out, oy), at(h_grad_out, oy), size_t(n) * ib.out,
+                           cudaMemcpyHostToDevice, hp->h2d));
+    DCN_CU(cudaEventRecord(ev[1 + i], hp->h2d));
+    DCN_CU(cudaStreamWaitEvent(stream, ev[1 + i], 0));
+    dcn_problem q = *problem;
+    q.N = int(n);
+    st = dcn_core_backward(&q, at(input, ox), at(offset, oo), at(mask, om), at(d_grad_out, oy),
+                           at(d_grad_input, ox), at(d_grad_offset, oo), at(d_grad_mask, om),
+                           workspace, workspace_bytes, stream);
+    if (st != DCN_OK) return st;
+    DCN_CU(cudaEventRecord(ev[1 + cp.chunks + i], stream));
+    DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[1 + cp.chunks + i], 0));
+    DCN_CU(cudaMemcpyAsync(at(h_grad_input, ox), at(d_grad_input, ox), size_t(n) * ib.x,
+                           cudaMemcpyDeviceToHost, hp->d2h));
+    DCN_CU(cudaMemcpyAsync(at(h_grad_offset, oo), at(d_grad_offset, oo), size_t(n) * ib.off,
+                           cudaMemcpyDeviceToHost, hp->d2h));
+    DCN_CU(cudaMemcpyAsync(at(h_grad_mask, om), at(d_grad_mask, om), size_t(n) * ib.msk,
+                           cudaMemcpyDeviceToHost, hp->d2h));
+  }
+  DCN_CU(cudaEventRecord(ev[2 * cp.chunks + 1], hp->d2h));
+  DCN_CU(cudaStreamWaitEvent(stream, ev[2 * cp.chunks + 1], 0));
+  return DCN_OK;
 }
 
 dcn_status dcn_core_sync_status(cudaStream_t stream) {

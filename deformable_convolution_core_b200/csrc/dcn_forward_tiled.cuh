@@ -30,6 +30,12 @@ constexpr int kTiledWarps = 15;  // consumer warps: with the producer, 4 warps p
 constexpr int kTiledThreads = (kTiledWarps + 1) * 32;  // + one TMA producer warp
 constexpr int kTiledBatch = 32;                       // units per warp batch
 constexpr int kTiledMaxTaps = 9;  // the tiled kernel serves 3x3 windows (9 or 8 taps)
+// Shared memory after the unit slots: the full/empty mbarriers and the abort
+// flag (bytes 0-35), then at kTiledZeroAt a 128-byte area of zeros that the
+// forward's box reads of far or dead taps are pointed at.
+constexpr int kTiledZeroAt = 64;
+constexpr int kTiledZeroBytes = 128;
+constexpr int kTiledTailBytes = kTiledZeroAt + kTiledZeroBytes;
 
 struct TiledParams {
   int N, H, W, G, Cg, C, stride, pad, dil, Ho, Wo;  // stride/pad/dil: height axis
@@ -262,6 +268,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       reinterpret_cast<uint64_t*>(slots + size_t(kTiledWarps) * kTiledBatch * kSlotBytes);
   uint64_t* empty = full + 2;
   int* s_abort = reinterpret_cast<int*>(empty + 2);
+  unsigned char* zero = reinterpret_cast<unsigned char*>(full) + kTiledZeroAt;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -272,6 +279,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (tid < kTiledZeroBytes / 4) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
   __syncthreads();
   volatile int* abort_flag = s_abort;
 
@@ -386,6 +394,13 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     if (*abort_flag) break;
     const ItemCoord c = item_coord(t, item);
     const unsigned char* box = bufs + size_t(b) * t.box_stride;
+    // Phase B reads piece j of a tap at box + min(code, zlim) + cdelta[j]: a
+    // box tap's code (>= 0, below the box size) is kept, a far or dead tap's
+    // (negative, so above 2^31 unsigned) becomes zlim, which puts this lane's
+    // pieces at zero + 48 + (cdelta[j] - cdelta[0]), inside the zero area
+    // (pieces of one lane lie at most 32 bytes apart).  zlim exceeds every box
+    // offset because the zero area lies after both buffers and the slots.
+    const uint32_t zlim = uint32_t((zero + 48 - cdelta[0]) - box);
     const int Y0 = c.ho0 * t.stride - t.pad - t.halo;
     const int X0 = c.wo0 * t.stride_w - t.pad_w - t.halo;
     const char* ximg = reinterpret_cast<const char*>(a.x) + size_t(c.n) * t.H * t.W * pixB +
@@ -510,16 +525,11 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         for (int e = 0; e < NV / 2; ++e) acc[e] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          const int code = csl[k];
+          const uint32_t off = min(uint32_t(csl[k]), zlim);  // far or dead: the zero area
           const float w = wsl[4 * k];
           const float2 w2 = make_float2(w, w);
-          const bool inbox = code >= 0;
 #pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (inbox) val = lds128(box + code + cdelta[j]);
-            IO::fma16(acc + j * (EPC / 2), w2, val);
-          }
+          for (int j = 0; j < NP; ++j) IO::fma16(acc + j * (EPC / 2), w2, lds128(box + off + cdelta[j]));
         }
         // First far tap (fetched during the previous step), then any others.
 #pragma unroll

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define DCN_CORE_ABI_VERSION 3
+#define DCN_CORE_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define DCN_API __attribute__((visibility("default")))
@@ -126,16 +126,49 @@ DCN_API dcn_status dcn_core_forward(const dcn_problem* problem, const void* inpu
 
 /*
  * Forward on HOST buffers: copies input, offset and mask from the host to the
- * caller's device buffers, runs dcn_core_forward and copies the output back,
- * all enqueued on `stream` (one cudaMemcpyAsync per tensor).  Host buffers
- * should be pinned for the copies to be asynchronous; they must not be
- * touched until the stream has reached this point.  Device buffers follow the
- * rules of dcn_core_forward.
+ * caller's device buffers, runs dcn_core_forward and copies the output back.
+ * The batch is cut into at most 8 chunks of whole images (chunk starts kept
+ * 32-byte aligned in every tensor; one chunk when N is small or the sizes do
+ * not allow it).  Chunk i's host-to-device copies run on a library-owned
+ * stream, its forward on `stream`, its device-to-host copy on a second
+ * library-owned stream, so that both copy directions and the kernels overlap.
+ * Events order the three: the first copy waits for the work enqueued on
+ * `stream` before the call, and `stream` waits for the last copy before any
+ * work enqueued after it, so from the caller's side everything happens on
+ * `stream` (CUDA graph capture included).  The two streams and a set of
+ * events per device are created on first use and kept by the library;
+ * concurrent calls from several host threads are serialised while they
+ * enqueue.  Host buffers should be pinned for the copies to be asynchronous;
+ * they must not be touched until `stream` has reached this point.  Device
+ * buffers follow the rules of dcn_core_forward.  Arguments are validated
+ * before anything is enqueued; a CUDA error part-way (DCN_ERR_CUDA) may leave
+ * the chunks before it enqueued.
  */
 DCN_API dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input,
                                  const void* h_offset, const void* h_mask,
                                  void* h_output, void* d_input, void* d_offset,
                                  void* d_mask, void* d_output, cudaStream_t stream);
+
+/*
+ * Backward with the gradients on HOST buffers, for a forward whose input,
+ * offset and mask are still on the device (as dcn_core_forward_host leaves
+ * them): copies grad_out from the host into d_grad_out, runs dcn_core_backward
+ * and copies grad_input, grad_offset and grad_mask back into the host
+ * buffers.  Chunked and overlapped like dcn_core_forward_host (grad_out in on
+ * one library stream, the backward of each chunk on `stream`, the three
+ * gradients out on the other).  input, offset, mask, d_grad_out,
+ * d_grad_input, d_grad_offset and d_grad_mask: device buffers with the rules
+ * of dcn_core_backward; the bf16 workspace is sized for the whole problem
+ * (dcn_core_backward_workspace) and reused by every chunk.  Errors as for
+ * dcn_core_forward_host.
+ */
+DCN_API dcn_status dcn_core_backward_host(const dcn_problem* problem, const void* input,
+                                  const void* offset, const void* mask,
+                                  const void* h_grad_out, void* h_grad_input,
+                                  void* h_grad_offset, void* h_grad_mask, void* d_grad_out,
+                                  void* d_grad_input, void* d_grad_offset,
+                                  void* d_grad_mask, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
 
 /* Device workspace the backward needs, in bytes: 0 for fp32 storage; for
  * bf16 storage an fp32 accumulator for grad_input, N*H*W*G*Cg*4 bytes. */

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 3
+    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 4
     for st in range(6):
         assert dcn.dcn_status_string(st)
     assert "unknown" in dcn.dcn_status_string(99)
@@ -171,6 +171,29 @@ def test_forward_host_rejects_before_copy(lib):
     assert e.value.status == dcn.DCN_ERR_INVALID_ARG
     with pytest.raises(dcn.DcnError) as e:
         dcn.dcn_core_forward_host(p, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+
+
+def test_backward_host_rejects_before_copy(lib):
+    """Every argument error of the chunked host backward is found before the
+    first copy is enqueued (no CUDA call is reached here)."""
+    p = dcn.make_problem(**GOOD)
+    dev3 = [FAKE] * 3          # input, offset, mask (device)
+    host4 = [FAKE] * 4         # grad_out, grad_input, grad_offset, grad_mask (host)
+    dgrads = [FAKE] * 4        # the device staging buffers
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward_host(p, *dev3, 0, *host4[1:], *dgrads, None, 0, 0)
+    assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward_host(p, *dev3, *host4, FAKE + 4, *dgrads[1:], None, 0, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    pb = dcn.make_problem(**{**GOOD, "dtype": "bf16"})
+    with pytest.raises(dcn.DcnError) as e:  # bf16 needs the fp32 accumulator workspace
+        dcn.dcn_core_backward_host(pb, *dev3, *host4, *dgrads, None, 0, 0)
+    assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    pc = dcn.make_problem(**{**GOOD, "Cg": 12})
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward_host(pc, *dev3, *host4, *dgrads, None, 0, 0)
     assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
 
 

@@ -218,3 +218,40 @@ def test_full_size_backward_bf16(gen_mod, oracle_mod):
     d = gen_mod.make_inputs(wl)
     p = dcn.problem_for(wl)
     check(oracle_mod, p, d["x"], d["offset"], d["mask"], d["grad_out"], "bf16")
+
+
+@pytest.mark.parametrize("N,H,W,G,dtype", [(5, 21, 23, 4, "f32"), (11, 12, 13, 3, "f32"),
+                                           (9, 16, 16, 2, "bf16"), (3, 7, 5, 2, "bf16"),
+                                           (1, 14, 15, 3, "f32")])
+def test_backward_host_entry_point(oracle_mod, N, H, W, G, dtype):
+    """The chunked host backward: grad_offset and grad_mask have the bits of
+    the device backward on the whole batch (they do not depend on the order of
+    additions), grad_input agrees within the usual gate, and all three match
+    the oracle."""
+    Cg = 16
+    p = dcn.make_problem(N, H, W, G, Cg, offset_scale=2.0, dtype=dtype)
+    Ho, Wo = dcn.dcn_core_output_hw(p)
+    x = RNG.standard_normal((N, H, W, G * Cg)).astype(np.float32)
+    off = (1.5 * RNG.standard_normal((N, Ho, Wo, G * 18))).astype(np.float32)
+    mask = RNG.standard_normal((N, Ho, Wo, G * 9)).astype(np.float32)
+    gout = RNG.standard_normal((N, Ho, Wo, G * Cg)).astype(np.float32)
+    xd, od, md, gd = (to_dev(a, dtype) for a in (x, off, mask, gout))
+    hg = gd.cpu().pin_memory()
+    hgx, hgo, hgm = (torch.full(t.shape, float("nan"), dtype=t.dtype).pin_memory()
+                     for t in (xd, od, md))
+    dg, dgx, dgo, dgm = (torch.full_like(t, 3.0) for t in (gd, xd, od, md))
+    ws = dcn.dcn_core_backward_workspace(p)
+    wbuf = torch.empty(ws, dtype=torch.uint8, device="cuda") if ws else None
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    dcn.dcn_core_backward_host(p, xd, od, md, hg, hgx, hgo, hgm, dg, dgx, dgo, dgm, wbuf, ws,
+                               stream=s)
+    dcn.dcn_core_sync_status(s)
+    rgx, rgo, rgm = gpu_backward(p, xd, od, md, gd)
+    torch.cuda.synchronize()
+    assert torch.equal(hgo, rgo.cpu()) and torch.equal(hgm, rgm.cpu())
+    assert_bwd(f64(hgx), f64(rgx), "host vs device grad_input", dtype)
+    rx, roff, rm = oracle_mod.backward(f64(xd), f64(od), f64(md), f64(gd), **problem_kwargs(p))
+    assert_bwd(f64(hgx), rx, "grad_input", dtype)
+    assert_bwd(f64(hgo), roff, "grad_offset", dtype)
+    assert_bwd(f64(hgm), rm, "grad_mask", dtype)

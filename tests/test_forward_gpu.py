@@ -203,21 +203,64 @@ def test_forward_is_deterministic_and_stream_safe(oracle_mod):
     dcn.dcn_core_sync_status(s)
 
 
-def test_forward_host_entry_point():
-    p, x, off, mask = random_case(2, 21, 23, 4, 16, dtype="f32")
+# (N, H, W, G, Cg, dtype): image counts that cut into ragged chunks (5 -> 2+2+1,
+# 11 -> five of 2 and 1, 17 -> four of 4 and 1, 9 -> four of 2 and 1) and sizes
+# whose 32-byte chunk alignment forces one chunk (N=3 at 7x5 bf16: 1260-byte mask
+# images; N=6 at 11x9, Cg 8)
+HOST_CASES = [(2, 21, 23, 4, 16, "f32"), (5, 21, 23, 4, 16, "f32"), (11, 12, 13, 3, 16, "f32"),
+              (17, 9, 10, 2, 16, "bf16"), (9, 16, 16, 2, 16, "bf16"), (3, 7, 5, 2, 16, "bf16"),
+              (6, 11, 9, 3, 8, "f32"), (1, 30, 30, 2, 16, "f32")]
+
+
+@pytest.mark.parametrize("case", HOST_CASES, ids=[f"N{c[0]}_{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_{c[5]}"
+                                                  for c in HOST_CASES])
+def test_forward_host_entry_point(case):
+    """The chunked, overlapped host path writes the same bits as the device
+    forward on the whole batch, and orders itself after earlier work on the
+    stream (the device buffers are first filled with garbage there)."""
+    N, H, W, G, Cg, dtype = case
+    p, x, off, mask = random_case(N, H, W, G, Cg, dtype=dtype)
     Ho, Wo = dcn.dcn_core_output_hw(p)
-    hx = torch.from_numpy(x).pin_memory()
-    ho = torch.from_numpy(off).pin_memory()
-    hm = torch.from_numpy(mask).pin_memory()
-    hout = torch.empty((2, Ho, Wo, 64), dtype=torch.float32).pin_memory()
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    hx, ho, hm = (torch.from_numpy(a).to(tdt).pin_memory() for a in (x, off, mask))
+    hout = torch.full((N, Ho, Wo, G * Cg), float("nan"), dtype=tdt).pin_memory()
     dx, do, dm = (torch.empty_like(t, device="cuda") for t in (hx, ho, hm))
-    dout = torch.empty(hout.shape, dtype=torch.float32, device="cuda")
+    dout = torch.empty(hout.shape, dtype=tdt, device="cuda")
     s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for t in (dx, do, dm, dout):
+            t.fill_(7.0)
     dcn.dcn_core_forward_host(p, hx, ho, hm, hout, dx, do, dm, dout, stream=s)
     dcn.dcn_core_sync_status(s)
     ref = gpu_forward(p, hx.cuda(), ho.cuda(), hm.cuda())
     torch.cuda.synchronize()
     assert torch.equal(hout, ref.cpu())
+    assert torch.equal(dx.cpu(), hx) and torch.equal(dm.cpu(), hm)
+
+
+def test_forward_host_in_a_cuda_graph():
+    """The host path's library streams join the caller's stream, so the call
+    can be captured and replayed."""
+    p, x, off, mask = random_case(5, 21, 23, 4, 16, dtype="f32")
+    Ho, Wo = dcn.dcn_core_output_hw(p)
+    hx, ho, hm = (torch.from_numpy(a).pin_memory() for a in (x, off, mask))
+    hout = torch.zeros((5, Ho, Wo, 64), dtype=torch.float32).pin_memory()
+    dx, do, dm = (torch.empty_like(t, device="cuda") for t in (hx, ho, hm))
+    dout = torch.empty(hout.shape, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    dcn.dcn_core_forward_host(p, hx, ho, hm, hout, dx, do, dm, dout, stream=s)  # warm-up
+    s.synchronize()
+    hout.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        dcn.dcn_core_forward_host(p, hx, ho, hm, hout, dx, do, dm, dout,
+                                  stream=torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    ref = gpu_forward(p, hx.cuda(), ho.cuda(), hm.cuda())
+    torch.cuda.synchronize()
+    assert torch.equal(hout, ref.cpu())
+    del g
 
 
 # --- full-size workloads, sampled ----------------------------------------------------
