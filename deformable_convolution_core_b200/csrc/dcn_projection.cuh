@@ -266,9 +266,12 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       tc_fence_after();
       const int mt = tile / a.n_tiles, nt = tile - mt * a.n_tiles;
       const int row0 = mt * kPjBM + q * 32;
-      const int rows = a.M - row0;  // rows of this quarter inside the image batch
+      const int rows = min(a.M - row0, 32);  // rows of this quarter inside the image batch
 #pragma unroll 1
       for (int c = 2 * h; c < 2 * h + 2; ++c) {
+        // a block with no column below Nout (the padding of the last column
+        // tile) or no row inside the batch has nothing to store
+        if (nt * kPjBN + c * 32 >= a.Nout || rows <= 0) continue;
         float v[32];
         tmem_ld32(tmem_base + (uint32_t(q * 32) << 16) + uint32_t(acc * kPjBN + c * 32), v);
 #pragma unroll
@@ -293,8 +296,8 @@ __global__ void __launch_bounds__(kPjThreads, 1)
         const size_t tensor_bytes = size_t(a.M) * pitch * sizeof(T);
         dst += size_t(row0) * pitch;
 #pragma unroll 8
-        for (int r = 0; r < 32; ++r) {
-          if (cin && r < rows && in_tensor(dst, sizeof(T), tensor, tensor_bytes))
+        for (int r = 0; r < rows; ++r) {
+          if (cin && in_tensor(dst, sizeof(T), tensor, tensor_bytes))
             Storage<T>::store_float(dst, st[r * kPjEpiPitch + lane] + b);
           dst += pitch;
         }
