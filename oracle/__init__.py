@@ -214,6 +214,44 @@ def linear(x, weight, bias=None):
     return y.reshape(a.shape[:-1] + (w.shape[0],))
 
 
+def guide(x, dw_weight, dw_bias, ln_gamma, ln_beta, ln_eps, pixels=None):
+    """Guide features of the DCNv3 block's offset / mask branch (InternImage-L
+    DCNv3 explainer (wmrh.cn), section 二 step 1: the input passes a depthwise
+    convolution, LayerNorm and GELU before the linear layers of steps 2-3), in
+    float64:
+        conv[n, y, x, c] = dw_bias[c] + sum_{a, b < 3} dw_weight[a, b, c] * x[n, y+a-1, x+b-1, c]
+                           (zero outside the image: a 3x3 window, stride 1, padding 1)
+        z = (conv - mean_c conv) / sqrt(var_c conv + ln_eps) * ln_gamma + ln_beta
+            (mean and biased variance over the C channels of one pixel)
+        out = z * (1 + erf(z / sqrt(2))) / 2       (GELU, exact form)
+    x (N, H, W, C); dw_weight (3, 3, C); dw_bias, ln_gamma, ln_beta (C,).
+    Returns (N, H, W, C), or, with `pixels` (flat indices n*H*W + y*W + x),
+    the rows of those pixels only, (len(pixels), C)."""
+    import math
+    a = _d(x)
+    N, H, W, C = a.shape
+    w = _d(dw_weight).reshape(3, 3, C)
+    xp = np.zeros((N, H + 2, W + 2, C))
+    xp[:, 1:H + 1, 1:W + 1, :] = a
+    if pixels is None:
+        pix = np.arange(N * H * W)
+    else:
+        pix = np.asarray(pixels, dtype=np.int64)
+    n, rem = pix // (H * W), pix % (H * W)
+    y, xx = rem // W, rem % W
+    conv = np.tile(_d(dw_bias).reshape(1, C), (len(pix), 1))
+    for ta in range(3):
+        for tb in range(3):
+            # padded row y + ta is input row y + ta - 1
+            conv = conv + w[ta, tb][None, :] * xp[n, y + ta, xx + tb, :]
+    mean = conv.mean(axis=1, keepdims=True)
+    var = ((conv - mean) ** 2).mean(axis=1, keepdims=True)
+    z = (conv - mean) / np.sqrt(var + float(ln_eps)) * _d(ln_gamma)[None, :] + _d(ln_beta)[None, :]
+    erf = np.vectorize(math.erf, otypes=[np.float64])
+    out = z * (1.0 + erf(z / math.sqrt(2.0))) / 2.0
+    return out.reshape(N, H, W, C) if pixels is None else out
+
+
 def workload_kwargs(wl) -> dict:
     """Keyword arguments of forward()/backward() for a gen.Workload."""
     return dict(G=wl.G, K=wl.K, stride=wl.stride, pad=wl.pad, dil=wl.dilation,

@@ -441,6 +441,76 @@ def test_linear_matches_explicit_sums(oracle_mod):
     assert np.array_equal(oracle_mod.linear(x, np.eye(4)), x)
 
 
+# --- guide features: depthwise 3x3 + LayerNorm + GELU --------------------------------
+
+def guide_inputs(N, H, W, C):
+    return (rand(N, H, W, C), rand(3, 3, C), rand(C), rand(C, lo=0.5, hi=1.5), rand(C))
+
+
+@pytest.mark.parametrize("shape", [(2, 5, 7, 8), (1, 1, 1, 4), (1, 3, 9, 12), (2, 4, 4, 1)])
+def test_guide_matches_torch_library_ops(oracle_mod, shape):
+    """The oracle's loops against torch's own depthwise conv2d (groups = C),
+    layer_norm and exact GELU, all in float64 on the CPU."""
+    import torch.nn.functional as F
+    N, H, W, C = shape
+    x, w, b, g, be = guide_inputs(N, H, W, C)
+    eps = 1e-6
+    got = oracle_mod.guide(x, w, b, g, be, eps)
+    t = torch.from_numpy(x).permute(0, 3, 1, 2)                       # NCHW
+    wt = torch.from_numpy(w).permute(2, 0, 1).unsqueeze(1).contiguous()  # (C, 1, 3, 3)
+    conv = F.conv2d(t, wt, torch.from_numpy(b), stride=1, padding=1, groups=C)
+    z = F.layer_norm(conv.permute(0, 2, 3, 1), (C,), torch.from_numpy(g), torch.from_numpy(be), eps)
+    ref = F.gelu(z, approximate="none").numpy()
+    assert np.abs(got - ref).max() <= 1e-12
+    # the sampled form returns the same rows
+    pix = RNG.integers(0, N * H * W, size=5)
+    assert np.array_equal(oracle_mod.guide(x, w, b, g, be, eps, pixels=pix),
+                          got.reshape(-1, C)[pix])
+
+
+def test_guide_two_channel_closed_form(oracle_mod):
+    """Two channels with different values normalise to -1 and +1 (exactly, up
+    to eps), so with gamma = 1, beta = 0 the outputs are GELU(-1) = -Phi(-1)
+    and GELU(1) = Phi(1), Phi the standard normal CDF.  A centre-only kernel
+    passes the input through the convolution; the bias adds per channel."""
+    x = np.zeros((1, 3, 3, 2))
+    x[0, 1, 1] = [0.25, 2.0]
+    w = np.zeros((3, 3, 2))
+    w[1, 1] = 1.0
+    out = oracle_mod.guide(x, w, np.array([0.5, -0.5]), np.ones(2), np.zeros(2), 0.0)
+    # centre pixel: conv = (0.75, 1.5) -> z = (-1, 1)
+    assert abs(out[0, 1, 1, 0] - (-0.15865525393145707)) <= 1e-15
+    assert abs(out[0, 1, 1, 1] - 0.8413447460685429) <= 1e-15
+    # a corner pixel sees only the bias (0.5, -0.5) -> z = (1, -1)
+    assert abs(out[0, 0, 0, 0] - 0.8413447460685429) <= 1e-15
+    assert abs(out[0, 0, 0, 1] - (-0.15865525393145707)) <= 1e-15
+
+
+def test_guide_window_orientation(oracle_mod):
+    """Weight [a, b] multiplies input pixel (y + a - 1, x + b - 1): a one-hot
+    kernel shifts the image, and a shifted pixel beyond the border reads zero.
+    gamma = 0 would hide the convolution, so the check goes through a
+    constant-plus-channel-ramp input whose normalisation is known."""
+    N, H, W, C = 1, 4, 5, 2
+    base = RNG.uniform(1.0, 2.0, size=(N, H, W))
+    x = np.stack([base, base + 1.0], axis=-1)          # channel 1 = channel 0 + 1
+    for a in range(3):
+        for b in range(3):
+            w = np.zeros((3, 3, C))
+            w[a, b] = 1.0
+            # eps = 1e-30: the +-1 normalisation stays exact in float64, and a
+            # constant (all-zero) pixel normalises to 0 instead of 0/0
+            out = oracle_mod.guide(x, w, np.zeros(C), np.ones(C), np.zeros(C), 1e-30)
+            for y in range(H):
+                for xx in range(W):
+                    yy, xs = y + a - 1, xx + b - 1
+                    inside = 0 <= yy < H and 0 <= xs < W
+                    # inside: conv = (v, v + 1) -> z = (-1, 1); outside: conv = (0, 0) -> z = 0,
+                    # GELU(0) = 0
+                    exp = (-0.15865525393145707, 0.8413447460685429) if inside else (0.0, 0.0)
+                    assert np.allclose(out[0, y, xx], exp, atol=1e-15), (a, b, y, xx)
+
+
 # --- separate height / width stride, padding and dilation ---------------------------
 
 AXES = [dict(stride=1, stride_w=2, pad=1, pad_w=0, dil=1, dil_w=1),
