@@ -45,6 +45,10 @@ FALLBACK_BF16_TFLOPS = 1590.0
 PROJECTION_SWEEP = [("internimage_l_stage1_fp32_n32_96x96_c160", 160),
                     ("internimage_l_stage1_bf16_n64_96x96_c160", 160),
                     ("internimage_l_stage2_bf16_n64_48x48_c320", 320)]
+# guide features (depthwise 3x3 + LayerNorm + GELU) on the stage shapes
+GUIDE_SWEEP = ["internimage_l_stage1_fp32_n32_96x96_c160", "internimage_l_stage1_bf16_n64_96x96_c160",
+               "internimage_l_stage2_bf16_n64_48x48_c320", "internimage_l_stage3_bf16_n64_24x24_c640",
+               "internimage_l_stage4_bf16_n64_12x12_c1280"]
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -339,6 +343,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
         result["sweep"] = run_sweep(gen, peak)
         result["projection"] = run_projection(gen, peak)
+        result["guide"] = run_guide(gen, peak)
         result["block_core_path"] = run_block_core_path(gen)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, inputs, backward)
@@ -460,20 +465,61 @@ def l1_ceiling_gsamples(wl, sm_mhz=1965.0, sms=148):
     return sms * 128.0 * sm_mhz * 1e6 / (4.0 * wl.Cg * wl.esize) / 1e9
 
 
+def run_guide(gen, peak, launches=20):
+    """dcn_core_offset_mask_guide (depthwise 3x3 + LayerNorm + GELU, bf16 query
+    out) on the stage shapes: bytes = input read + query written (+ the 12 C
+    parameter floats)."""
+    import torch
+    import deformable_convolution_core_b200 as dcn
+    out = {}
+    for name in GUIDE_SWEEP:
+        wl = gen.WORKLOADS[name]
+        p = dcn.problem_for(wl)
+        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        x = torch.from_numpy(gen.make_inputs(wl)["x"]).cuda().to(tdt)
+        gp = {k: torch.from_numpy(v).cuda() for k, v in gen.make_guide_params(wl).items()}
+        q = torch.empty(x.shape, dtype=torch.bfloat16, device="cuda")
+        s = torch.cuda.Stream()
+
+        def call():
+            dcn.dcn_core_offset_mask_guide(p, x, gp["dw_weight"], gp["dw_bias"], gp["ln_gamma"],
+                                           gp["ln_beta"], 1e-6, q, s)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(launches):
+            call()
+        e1.record(s)
+        torch.cuda.synchronize()
+        dcn.dcn_core_sync_status(s)
+        ms = e0.elapsed_time(e1) / launches
+        nbytes = x.numel() * x.element_size() + q.numel() * 2 + 12 * wl.C * 4
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
+                     "MB": round(nbytes / 1e6, 1), "bound": "hbm"}
+        del x, q, gp
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_block_core_path(gen, name="internimage_l_stage1_bf16_n64_96x96_c160", reps=20):
-    """The DCNv3 block around the core operator, bf16, three launches on one
-    stream: offset/mask projection (tensor cores) -> core forward -> output_proj
-    (tensor cores, C -> C).  Median per-launch CUDA-event times."""
+    """The DCNv3 block around the core operator, bf16, four launches on one
+    stream: guide features (depthwise 3x3 + LayerNorm + GELU) -> offset/mask
+    projection (tensor cores) -> core forward -> output_proj (tensor cores,
+    C -> C).  Median per-launch CUDA-event times."""
     import numpy as np
     import torch
     import deformable_convolution_core_b200 as dcn
     wl = gen.WORKLOADS[name]
     d = gen.make_inputs(wl)
     pj = gen.make_projection_inputs(wl, wl.C)
+    gp = {k: torch.from_numpy(v).cuda() for k, v in gen.make_guide_params(wl).items()}
     p = dcn.problem_for(wl)
     bf = torch.bfloat16
     x = torch.from_numpy(d["x"]).cuda().to(bf)
-    q = torch.from_numpy(pj["query"]).cuda().to(bf)
+    q = torch.empty(x.shape, dtype=bf, device="cuda")  # the guide features
     w = torch.from_numpy(pj["weight"]).cuda().to(bf)
     b = torch.from_numpy(pj["bias"]).cuda()
     w_out = (torch.from_numpy(gen.normal(wl.seed, gen.TID_OUT_WEIGHT, (wl.C, wl.C), 0.0,
@@ -484,26 +530,30 @@ def run_block_core_path(gen, name="internimage_l_stage1_bf16_n64_96x96_c160", re
     core = torch.empty((M, wl.C), dtype=bf, device="cuda")
     y = torch.empty((M, wl.C), dtype=bf, device="cuda")
     s = torch.cuda.Stream()
-    stages = [lambda: dcn.dcn_core_offset_mask_projection(p, q, wl.C, w, b, off, msk, s),
+    stages = [lambda: dcn.dcn_core_offset_mask_guide(p, x, gp["dw_weight"], gp["dw_bias"],
+                                                     gp["ln_gamma"], gp["ln_beta"], 1e-6, q, s),
+              lambda: dcn.dcn_core_offset_mask_projection(p, q, wl.C, w, b, off, msk, s),
               lambda: dcn.dcn_core_forward(p, x, off, msk, core, s),
               lambda: dcn.dcn_core_linear_bf16(core, M, wl.C, w_out, wl.C, None, y, "bf16", s)]
     for _ in range(3):
         for f in stages:
             f()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+    k = len(stages)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(k + 1)] for _ in range(reps)]
     for r in range(reps):
         for i, f in enumerate(stages):
             ev[r][i].record(s)
             f()
-        ev[r][3].record(s)
+        ev[r][k].record(s)
     torch.cuda.synchronize()
     dcn.dcn_core_sync_status(s)
-    t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in ev])
+    t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(k)] for e in ev])
     med = np.median(t, axis=0)
-    return {"workload": name, "projection_ms": round(float(med[0]), 4),
-            "core_forward_ms": round(float(med[1]), 4),
-            "output_proj_ms": round(float(med[2]), 4),
+    return {"workload": name, "guide_ms": round(float(med[0]), 4),
+            "projection_ms": round(float(med[1]), 4),
+            "core_forward_ms": round(float(med[2]), 4),
+            "output_proj_ms": round(float(med[3]), 4),
             "total_ms": round(float(np.median(t.sum(axis=1))), 4),
             "Mpixels/s": round(M / (float(np.median(t.sum(axis=1))) * 1e-3) / 1e6, 1)}
 

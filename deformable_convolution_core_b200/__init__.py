@@ -39,6 +39,7 @@ EXPORTED_SYMBOLS = (
     "dcn_core_backward_noalloc",
     "dcn_core_backward_deterministic_workspace",
     "dcn_core_backward_deterministic",
+    "dcn_core_offset_mask_guide",
     "dcn_core_offset_mask_projection",
     "dcn_core_linear_bf16",
     "dcn_core_sync_status",
@@ -133,6 +134,8 @@ def load_library():
     lib.dcn_core_backward_deterministic_workspace.restype = ctypes.c_size_t
     lib.dcn_core_backward_deterministic.argtypes = [pp] + [vp] * 8 + [ctypes.c_size_t, vp]
     lib.dcn_core_backward_deterministic.restype = st
+    lib.dcn_core_offset_mask_guide.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp]
+    lib.dcn_core_offset_mask_guide.restype = st
     lib.dcn_core_offset_mask_projection.argtypes = [pp, vp, ctypes.c_int, vp, vp, vp, vp, vp]
     lib.dcn_core_offset_mask_projection.restype = st
     lib.dcn_core_linear_bf16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, vp, vp,
@@ -262,6 +265,15 @@ def dcn_core_backward_deterministic(problem: DcnProblem, input, offset, mask, gr
         ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
         _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _ptr(workspace),
         int(workspace_bytes), _stream(stream)), "dcn_core_backward_deterministic")
+
+
+def dcn_core_offset_mask_guide(problem: DcnProblem, input, dw_weight, dw_bias, ln_gamma,
+                               ln_beta, ln_eps: float, query, stream=None) -> None:
+    """Depthwise 3x3 + LayerNorm + GELU of the block's input into the bf16
+    query of the offset / mask projection (see include/dcn_core.h)."""
+    _check(load_library().dcn_core_offset_mask_guide(
+        ctypes.byref(problem), _ptr(input), _ptr(dw_weight), _ptr(dw_bias), _ptr(ln_gamma),
+        _ptr(ln_beta), float(ln_eps), _ptr(query), _stream(stream)), "dcn_core_offset_mask_guide")
 
 
 def dcn_core_offset_mask_projection(problem: DcnProblem, query, Cq: int, weight, bias, offset,

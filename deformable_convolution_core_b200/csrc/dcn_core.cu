@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -19,6 +20,7 @@
 #include "dcn_backward_tiled.cuh"
 #include "dcn_forward.cuh"
 #include "dcn_forward_tiled.cuh"
+#include "dcn_guide.cuh"
 #include "dcn_projection.cuh"
 
 namespace dcn {
@@ -1154,6 +1156,90 @@ extern "C" dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem
   return bf16_gemm(query, M, Cq, weight, int64_t(problem->G) * KK * 3,
                    int64_t(problem->G) * KK * 2, bias, offset, mask,
                    problem->dtype == DCN_BF16, stream);
+}
+
+namespace dcn {
+namespace {
+
+template <typename T, int LP>
+dcn_status guide_launch_lp(const GuideArgs& a, cudaStream_t stream) {
+  const unsigned grid = unsigned(int64_t(a.N) * a.tiles_y * a.tiles_x);
+  const unsigned block = kGuideWarps * 32;
+  const size_t smem = size_t(a.NJ) * block * sizeof(float4);  // at most 64 KB
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(dcn_guide_kernel<T, LP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(smem)) != cudaSuccess)
+    return DCN_ERR_CUDA;
+  dcn_guide_kernel<T, LP><<<grid, block, smem, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+template <typename T>
+dcn_status guide_launch(int LP, const GuideArgs& a, cudaStream_t stream) {
+  switch (LP) {
+    case 32: return guide_launch_lp<T, 32>(a, stream);
+    case 16: return guide_launch_lp<T, 16>(a, stream);
+    case 8: return guide_launch_lp<T, 8>(a, stream);
+    default: return guide_launch_lp<T, 4>(a, stream);
+  }
+}
+
+}  // namespace
+}  // namespace dcn
+
+extern "C" dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, const void* input,
+                                                 const float* dw_weight, const float* dw_bias,
+                                                 const float* ln_gamma, const float* ln_beta,
+                                                 float ln_eps, void* query, cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!input || !dw_weight || !query) return DCN_ERR_INVALID_ARG;
+  if (!std::isfinite(ln_eps) || ln_eps < 0.f) return DCN_ERR_INVALID_ARG;
+  const int C = problem->G * problem->Cg;
+  if (C % 4 != 0) return DCN_ERR_UNSUPPORTED;
+  const int Q = C / 4;
+  // lanes per pixel: the group size whose quads per lane fill the lanes best
+  // (ties to the larger group), at most kGuideMaxQuads quads per lane
+  int LP = 0, NJ = 0;
+  double best = -1.0;
+  for (int lp : {32, 16, 8, 4}) {
+    const int nj = (Q + lp - 1) / lp;
+    if (nj > kGuideMaxQuads) continue;
+    const double eff = double(Q) / double(lp * nj);
+    if (eff > best + 1e-9) {
+      best = eff;
+      LP = lp;
+      NJ = nj;
+    }
+  }
+  if (LP == 0) return DCN_ERR_UNSUPPORTED;
+  if (!aligned(input, 16) || !aligned(dw_weight, 16) || (dw_bias && !aligned(dw_bias, 16)) ||
+      (ln_gamma && !aligned(ln_gamma, 16)) || (ln_beta && !aligned(ln_beta, 16)) ||
+      !aligned(query, 8))
+    return DCN_ERR_UNSUPPORTED;
+  GuideArgs a;
+  a.x = input;
+  a.w = dw_weight;
+  a.bias = dw_bias;
+  a.gamma = ln_gamma;
+  a.beta = ln_beta;
+  a.eps = ln_eps;
+  a.out = static_cast<__nv_bfloat16*>(query);
+  a.N = problem->N;
+  a.H = problem->H;
+  a.W = problem->W;
+  a.C = C;
+  a.Q = Q;
+  a.NJ = NJ;
+  a.tiles_x = (problem->W + kGuideWarps * (32 / LP) - 1) / (kGuideWarps * (32 / LP));
+  a.tiles_y = (problem->H + kGuideRows - 1) / kGuideRows;
+  if (int64_t(a.N) * a.tiles_y * a.tiles_x > INT_MAX) return DCN_ERR_UNSUPPORTED;
+  const size_t elems = size_t(problem->N) * problem->H * problem->W * C;
+  a.x_bytes = elems * size_t(esize(problem->dtype));
+  a.out_bytes = elems * 2;
+  return problem->dtype == DCN_BF16 ? guide_launch<__nv_bfloat16>(LP, a, stream)
+                                    : guide_launch<float>(LP, a, stream);
 }
 
 extern "C" dcn_status dcn_core_linear_bf16(const void* input, int M, int K, const void* weight,

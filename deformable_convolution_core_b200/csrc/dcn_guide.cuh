@@ -1,0 +1,162 @@
+// Guide features of the offset / mask branch (sm_100a).
+//
+// Before its linear layers predict the offsets and the mask, the DCNv3 block
+// passes its input through a depthwise convolution, LayerNorm and GELU
+// (InternImage-L DCNv3 explainer (wmrh.cn), section 二 step 1: a light 3x3
+// look at the neighbourhood that guides where to sample).  One kernel does
+// all three per pixel and writes the bf16 query the projection GEMM reads:
+//   conv[c] = bias[c] + sum_{a, b < 3} w[a][b][c] * x[y + a - 1][x + b - 1][c]
+//             (zero outside the image; stride 1)
+//   z[c]    = (conv[c] - mean) / sqrt(var + eps) * gamma[c] + beta[c]
+//             (mean and biased variance over the pixel's C channels)
+//   out[c]  = z[c] * (1 + erf(z[c] / sqrt(2))) / 2, rounded to bf16 once.
+// Arithmetic is fp32 (two-pass variance).
+//
+// Layout of the work: a pixel's C channels are Q = C/4 quads, spread over a
+// group of LP lanes (quad sub + LP*j for lane sub, j < NJ), so a warp holds
+// 32/LP pixels of one row; LP is picked on the host so that the quads fill
+// the lanes (C = 160: 8 lanes x 5 quads, four pixels per warp).  A lane
+// convolves one quad at a time and parks the result in shared memory for the
+// two LayerNorm passes, so registers do not grow with C.  A CTA of
+// kGuideWarps warps covers adjacent columns and walks kGuideRows rows down:
+// consecutive windows of a lane group share six of their nine input pixels
+// and neighbouring groups share columns, so the input is read from DRAM
+// about once and re-read from L1.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "dcn_common.cuh"
+
+namespace dcn {
+
+constexpr int kGuideWarps = 8;
+constexpr int kGuideRows = 8;
+constexpr int kGuideMaxQuads = 16;  // quads per lane (NJ), at most
+
+struct GuideArgs {
+  const void* x;       // (N, H, W, C) of T
+  const float* w;      // (3, 3, C): w[(a * 3 + b) * C + c]
+  const float* bias;   // (C) or null
+  const float* gamma;  // (C) or null (1)
+  const float* beta;   // (C) or null (0)
+  float eps;
+  __nv_bfloat16* out;  // (N, H, W, C)
+  int N, H, W, C, Q, NJ;
+  int tiles_x, tiles_y;
+  size_t x_bytes, out_bytes;  // bounds-checked build
+};
+
+// Four consecutive channels of storage type T as floats (read-only path).
+template <typename T>
+__device__ __forceinline__ float4 guide_ld4(const T* p);
+template <>
+__device__ __forceinline__ float4 guide_ld4<float>(const float* p) {
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
+template <>
+__device__ __forceinline__ float4 guide_ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  return make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y),
+                     bf16hi_to_f32(u.y));
+}
+
+__device__ __forceinline__ float4 ld4_or(const float* p, bool ok, float dflt) {
+  return ok && p != nullptr ? __ldg(reinterpret_cast<const float4*>(p))
+                            : make_float4(dflt, dflt, dflt, dflt);
+}
+
+// Sum over the LP lanes of this lane's group (xor offsets below LP stay inside it).
+template <int LP>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = LP / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float gelu_erf(float z) {
+  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
+}
+
+template <typename T, int LP>
+__global__ void __launch_bounds__(kGuideWarps * 32) dcn_guide_kernel(const GuideArgs a) {
+  constexpr int PPW = 32 / LP;  // pixels per warp
+  constexpr int kThreads = kGuideWarps * 32;
+  // conv results of this thread's quads, [quad j][thread]: consecutive lanes
+  // touch consecutive 16-byte words, and each thread reads back only its own
+  extern __shared__ float4 conv_buf[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gi = lane / LP, sub = lane - gi * LP;
+  int t = blockIdx.x;
+  const int tx = t % a.tiles_x;
+  t /= a.tiles_x;
+  const int ty = t % a.tiles_y;
+  const int n = t / a.tiles_y;
+  const int col = (tx * kGuideWarps + warp) * PPW + gi;
+  const bool col_ok = col < a.W;
+  const T* xs = static_cast<const T*>(a.x);
+  const float inv_c = 1.0f / float(a.C);
+
+#pragma unroll 1
+  for (int i = 0; i < kGuideRows; ++i) {
+    const int y = ty * kGuideRows + i;
+    if (y >= a.H) break;  // the same for the whole CTA
+    // depthwise 3x3 convolution, one quad of channels at a time
+    float s = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < a.NJ; ++j) {
+      const int q = sub + LP * j;
+      const bool q_ok = col_ok && q < a.Q;
+      float4 acc = ld4_or(a.bias != nullptr ? a.bias + 4 * q : nullptr, q_ok, 0.f);
+#pragma unroll
+      for (int ta = 0; ta < 3; ++ta) {
+        const int yy = y + ta - 1;
+        if (yy < 0 || yy >= a.H) continue;  // the same for the whole CTA
+#pragma unroll
+        for (int tb = 0; tb < 3; ++tb) {
+          const int xx = col + tb - 1;
+          const T* px = xs + (size_t(n * a.H + yy) * a.W + xx) * a.C + 4 * q;
+          if (q_ok && xx >= 0 && xx < a.W && in_tensor(px, 4 * sizeof(T), a.x, a.x_bytes)) {
+            const float4 v = guide_ld4<T>(px);
+            const float4 wv = __ldg(reinterpret_cast<const float4*>(a.w + (ta * 3 + tb) * a.C + 4 * q));
+            acc.x = fmaf(wv.x, v.x, acc.x);
+            acc.y = fmaf(wv.y, v.y, acc.y);
+            acc.z = fmaf(wv.z, v.z, acc.z);
+            acc.w = fmaf(wv.w, v.w, acc.w);
+          }
+        }
+      }
+      s += (acc.x + acc.y) + (acc.z + acc.w);  // quads outside the channels hold 0
+      conv_buf[j * kThreads + tid] = acc;
+    }
+    // LayerNorm over the pixel's channels: the mean, then the mean squared deviation
+    const float mean = group_sum<LP>(s) * inv_c;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < a.NJ; ++j) {
+      if (sub + LP * j >= a.Q) break;
+      const float4 v = conv_buf[j * kThreads + tid];
+      const float d0 = v.x - mean, d1 = v.y - mean, d2 = v.z - mean, d3 = v.w - mean;
+      ss = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, ss))));
+    }
+    const float rstd = 1.0f / sqrtf(group_sum<LP>(ss) * inv_c + a.eps);
+    if (!col_ok) continue;
+    __nv_bfloat16* op = a.out + (size_t(n * a.H + y) * a.W + col) * a.C;
+#pragma unroll 1
+    for (int j = 0; j < a.NJ; ++j) {
+      const int q = sub + LP * j;
+      if (q >= a.Q) break;
+      const float4 v = conv_buf[j * kThreads + tid];
+      const float4 g = ld4_or(a.gamma != nullptr ? a.gamma + 4 * q : nullptr, true, 1.f);
+      const float4 b = ld4_or(a.beta != nullptr ? a.beta + 4 * q : nullptr, true, 0.f);
+      const float o0 = gelu_erf((v.x - mean) * rstd * g.x + b.x);
+      const float o1 = gelu_erf((v.y - mean) * rstd * g.y + b.y);
+      const float o2 = gelu_erf((v.z - mean) * rstd * g.z + b.z);
+      const float o3 = gelu_erf((v.w - mean) * rstd * g.w + b.w);
+      if (in_tensor(op + 4 * q, 8, a.out, a.out_bytes))
+        *reinterpret_cast<uint2*>(op + 4 * q) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+    }
+  }
+}
+
+}  // namespace dcn

@@ -27,6 +27,8 @@ TID_X, TID_OFFSET, TID_MASK, TID_GRAD_OUT, TID_FAR_SELECT, TID_FAR_VALUE = 1, 2,
 # inputs of the offset / mask projection: query features, weight, bias
 TID_QUERY, TID_WEIGHT, TID_BIAS = 7, 8, 9
 TID_OUT_WEIGHT = 10  # output_proj weight of the block's core path
+# parameters of the guide branch: depthwise weight and bias, LayerNorm gamma and beta
+TID_DW_WEIGHT, TID_DW_BIAS, TID_LN_GAMMA, TID_LN_BETA = 11, 12, 13, 14
 
 _lib = None
 
@@ -157,3 +159,15 @@ def make_projection_inputs(wl, Cq: int, seed=None) -> dict:
 
 __all__ = ["WORKLOADS", "Workload", "output_hw", "make_inputs", "make_projection_inputs", "uniform", "normal",
            "redraw_pairs", "raw_hash", "draw", "build"]
+
+
+def make_guide_params(wl, seed=None) -> dict:
+    """Host float32 parameters of the guide branch for a workload's C channels:
+    depthwise weight (3, 3, C) ~ N(0, 1/9), bias ~ N(0, 0.1^2), LayerNorm
+    gamma ~ N(1, 0.1^2) and beta ~ N(0, 0.1^2)."""
+    seed = wl.seed if seed is None else seed
+    C = wl.C
+    return {"dw_weight": normal(seed, TID_DW_WEIGHT, (3, 3, C), 0.0, 1.0 / 3.0),
+            "dw_bias": normal(seed, TID_DW_BIAS, (C,), 0.0, 0.1),
+            "ln_gamma": normal(seed, TID_LN_GAMMA, (C,), 1.0, 0.1),
+            "ln_beta": normal(seed, TID_LN_BETA, (C,), 0.0, 0.1)}

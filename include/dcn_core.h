@@ -289,6 +289,31 @@ DCN_API dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem, c
                                                    cudaStream_t stream);
 
 /*
+ * Guide features of the offset / mask branch (InternImage-L DCNv3 explainer
+ * (wmrh.cn), section 二 step 1: before the linear layers of the projection,
+ * the block's input passes a depthwise convolution, LayerNorm and GELU).  One
+ * pass per pixel, fp32 arithmetic:
+ *   conv[c] = dw_bias[c] + sum_{a,b<3} dw_weight[(a*3 + b)*C + c] * input[n, y+a-1, x+b-1, c]
+ *             (3x3 window, stride 1, zero padding 1: the output keeps H x W)
+ *   z[c]    = (conv[c] - mean) / sqrt(var + ln_eps) * ln_gamma[c] + ln_beta[c]
+ *             (mean and biased variance over the C = G*Cg channels of the pixel)
+ *   query[n, y, x, c] = z * (1 + erf(z / sqrt(2))) / 2   (GELU), rounded once to bf16
+ *   input      device, (N, H, W, C) of problem->dtype, 16-byte aligned
+ *   dw_weight  device, fp32, (3, 3, C); dw_bias, ln_gamma, ln_beta device fp32 (C),
+ *              each may be NULL (0, 1 and 0); all 16-byte aligned
+ *   query      device, bf16, (N, H, W, C), 8-byte aligned, written entirely; it is
+ *              the query of dcn_core_offset_mask_projection when Ho = H and Wo = W
+ * Only N, H, W, G, Cg and dtype of the problem are used (after the usual
+ * checks).  C must be a multiple of 4 and at most 2048, else
+ * DCN_ERR_UNSUPPORTED; ln_eps must be finite and >= 0, else
+ * DCN_ERR_INVALID_ARG.
+ */
+DCN_API dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, const void* input,
+                                              const float* dw_weight, const float* dw_bias,
+                                              const float* ln_gamma, const float* ln_beta,
+                                              float ln_eps, void* query, cudaStream_t stream);
+
+/*
  * The linear layers on either side of the core operator in the DCNv3 block
  * (InternImage-L DCNv3 explainer (wmrh.cn), section 二: input_proj before it,
  * output_proj after it), as one tensor-core GEMM with bf16 operands:

@@ -197,6 +197,25 @@ def test_backward_host_rejects_before_copy(lib):
     assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
 
 
+def test_guide_rejects_before_launch(lib):
+    p = dcn.make_problem(**GOOD)
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_offset_mask_guide(p, 0, FAKE, FAKE, FAKE, FAKE, 1e-6, FAKE, 0)
+    assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    for eps in (-1.0, float("nan"), float("inf")):
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_offset_mask_guide(p, FAKE, FAKE, None, None, None, eps, FAKE, 0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+    for bad in (dict(G=1, Cg=6), dict(G=3, Cg=688)):  # C not a multiple of 4; C above 2048
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_offset_mask_guide(dcn.make_problem(**{**GOOD, **bad}), FAKE, FAKE, None,
+                                           None, None, 1e-6, FAKE, 0)
+        assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    with pytest.raises(dcn.DcnError) as e:  # an unaligned weight
+        dcn.dcn_core_offset_mask_guide(p, FAKE, FAKE + 4, None, None, None, 1e-6, FAKE, 0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+
+
 def test_library_has_no_oracle_dependency():
     """The CUDA library and binding never reference the oracle."""
     pkg = os.path.join(ROOT, "deformable_convolution_core_b200")

@@ -1,0 +1,125 @@
+"""Guide features of the offset / mask branch (dcn_core_offset_mask_guide:
+depthwise 3x3, LayerNorm, GELU, bf16 out) against the oracle, element by
+element.
+
+Gate: the output is rounded once to bf16 (relative error at most 2^-9 of the
+value); the fp32 convolution, LayerNorm and erf before it add errors of order
+1e-6 on values of order one.  So |got - ref| <= 2^-8 |ref| + 2e-5.
+"""
+import numpy as np
+import pytest
+import torch
+
+import deformable_convolution_core_b200 as dcn
+from tests.dcn_testutil import f64, gpu_forward, problem_kwargs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+RNG = np.random.default_rng(53)
+
+
+def gate(got, ref):
+    return np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 2e-5
+
+
+def params(C, affine=True):
+    w = RNG.uniform(-0.5, 0.5, size=(3, 3, C)).astype(np.float32)
+    if not affine:
+        return w, None, None, None
+    b = RNG.uniform(-0.2, 0.2, size=C).astype(np.float32)
+    g = RNG.uniform(0.5, 1.5, size=C).astype(np.float32)
+    be = RNG.uniform(-0.3, 0.3, size=C).astype(np.float32)
+    return w, b, g, be
+
+
+def run_guide(p, x_dev, w, b, g, be, eps, stream=None):
+    dev = lambda a: None if a is None else torch.from_numpy(a).cuda()
+    q = torch.empty(x_dev.shape, dtype=torch.bfloat16, device="cuda")
+    dcn.dcn_core_offset_mask_guide(p, x_dev, dev(w), dev(b), dev(g), dev(be), eps, q, stream)
+    return q
+
+
+# (N, H, W, G, Cg, dtype): the lanes-per-pixel choices 8 x 5 quads (C=160), 16 x 1
+# (C=64), 16 x 5 (320), 32 x 10 (1280), 4 x 1 with three live quads (C=12),
+# 4 x 13 (C=196, ragged), 32 x 16 with 64 KB of shared memory (C=2048); ragged
+# column and row tiles; a one-pixel image
+CASES = [(2, 13, 11, 10, 16, "f32"), (1, 9, 37, 4, 16, "bf16"), (2, 5, 70, 20, 16, "bf16"),
+         (1, 3, 3, 80, 16, "f32"), (1, 1, 1, 2, 4, "f32"), (2, 17, 9, 3, 4, "f32"),
+         (1, 4, 5, 49, 4, "f32"), (1, 6, 7, 128, 16, "bf16"), (3, 10, 33, 12, 16, "bf16")]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"N{c[0]}_{c[1]}x{c[2]}_C{c[3] * c[4]}_{c[5]}"
+                                             for c in CASES])
+def test_guide_matches_oracle(oracle_mod, case):
+    N, H, W, G, Cg, dtype = case
+    C = G * Cg
+    p = dcn.make_problem(N, H, W, G, Cg, dtype=dtype)
+    x = RNG.standard_normal((N, H, W, C)).astype(np.float32)
+    xd = to_dev(x, dtype)
+    w, b, g, be = params(C)
+    q = run_guide(p, xd, w, b, g, be, 1e-6)
+    dcn.dcn_core_sync_status()
+    ref = oracle_mod.guide(f64(xd), w, b, g, be, 1e-6)
+    ok = gate(f64(q), ref)
+    assert ok.all(), f"{int((~ok).sum())} of {ok.size} outside the gate, max err {np.abs(f64(q) - ref).max():.3e}"
+
+
+def test_guide_without_affine_parameters(oracle_mod):
+    """NULL bias, gamma and beta read as 0, 1 and 0."""
+    N, H, W, G, Cg = 2, 8, 12, 4, 16
+    C = G * Cg
+    p = dcn.make_problem(N, H, W, G, Cg)
+    x = RNG.standard_normal((N, H, W, C)).astype(np.float32)
+    w = params(C, affine=False)[0]
+    q = run_guide(p, to_dev(x, "f32"), w, None, None, None, 1e-5)
+    dcn.dcn_core_sync_status()
+    ref = oracle_mod.guide(x, w, np.zeros(C), np.ones(C), np.zeros(C), 1e-5)
+    assert gate(f64(q), ref).all()
+
+
+def test_guide_at_stage1_size(oracle_mod):
+    """InternImage-L stage 1 in bf16 (N=64, 96x96, C=160): sampled pixels plus
+    every pixel of the image border of two images."""
+    N, H, W, G, Cg = 64, 96, 96, 10, 16
+    C = G * Cg
+    p = dcn.make_problem(N, H, W, G, Cg, dtype="bf16")
+    xd = torch.randn((N, H, W, C), device="cuda").to(torch.bfloat16)
+    w, b, g, be = params(C)
+    q = run_guide(p, xd, w, b, g, be, 1e-6)
+    dcn.dcn_core_sync_status()
+    border = [n * H * W + y * W + xx for n in (0, N - 1) for y in range(H) for xx in range(W)
+              if y in (0, H - 1) or xx in (0, W - 1)]
+    pix = np.unique(np.concatenate([RNG.integers(0, N * H * W, size=3000), np.array(border)]))
+    ref = oracle_mod.guide(f64(xd), w, b, g, be, 1e-6, pixels=pix)
+    got = f64(q).reshape(-1, C)[pix]
+    ok = gate(got, ref)
+    assert ok.all(), f"{int((~ok).sum())} outside the gate, max err {np.abs(got - ref).max():.3e}"
+
+
+def test_guide_projection_forward_chain(oracle_mod):
+    """The offset / mask branch end to end, bf16: guide -> projection (tensor
+    cores) -> core forward.  Each GPU stage is checked against the oracle fed
+    that stage's GPU inputs."""
+    N, H, W, G, Cg = 2, 20, 18, 4, 16
+    C = G * Cg
+    p = dcn.make_problem(N, H, W, G, Cg, offset_scale=2.0, dtype="bf16")
+    xd = to_dev(RNG.standard_normal((N, H, W, C)).astype(np.float32), "bf16")
+    w, b, g, be = params(C)
+    q = run_guide(p, xd, w, b, g, be, 1e-6)
+    pw = torch.from_numpy((RNG.standard_normal((G * 27, C)) / np.sqrt(C)).astype(np.float32))
+    pw = pw.to(torch.bfloat16).cuda()
+    pb = torch.from_numpy((0.1 * RNG.standard_normal(G * 27)).astype(np.float32)).cuda()
+    off = torch.empty((N, H, W, G * 18), dtype=torch.bfloat16, device="cuda")
+    msk = torch.empty((N, H, W, G * 9), dtype=torch.bfloat16, device="cuda")
+    dcn.dcn_core_offset_mask_projection(p, q, C, pw, pb, off, msk)
+    out = gpu_forward(p, xd, off, msk)
+    torch.cuda.synchronize()
+    dcn.dcn_core_sync_status()
+    ref_q = oracle_mod.guide(f64(xd), w, b, g, be, 1e-6)
+    assert gate(f64(q), ref_q).all()
+    ro, rm = oracle_mod.projection(f64(q), f64(pw), f64(pb), G=G)
+    tol = 4 * C * 2.0 ** -24 * 8 + 2.0 ** -8
+    assert np.abs(f64(off) - ro).max() <= tol * max(1.0, np.abs(ro).max())
+    assert np.abs(f64(msk) - rm).max() <= tol * max(1.0, np.abs(rm).max())
+    ref = oracle_mod.forward(f64(xd), f64(off), f64(msk), **problem_kwargs(p))
+    assert np.abs(f64(out) - ref).max() <= 1e-2 * np.abs(ref).max()
