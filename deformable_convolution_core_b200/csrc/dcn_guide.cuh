@@ -16,8 +16,10 @@
 // group of LP lanes (quad sub + LP*j for lane sub, j < NJ), so a warp holds
 // 32/LP pixels of one row; LP is picked on the host so that the quads fill
 // the lanes (C = 160: 8 lanes x 5 quads, four pixels per warp).  A lane
-// convolves one quad at a time and parks the result in shared memory for the
-// two LayerNorm passes, so registers do not grow with C.  A CTA of
+// convolves up to kGuideChunk of its quads at once in registers (one address
+// per tap) and parks the results in shared memory for the two LayerNorm
+// passes, so registers do not grow with C.  The weights and the affine
+// parameters are staged in shared memory once per CTA.  A CTA of
 // kGuideWarps warps covers adjacent columns and walks kGuideRows rows down:
 // consecutive windows of a lane group share six of their nine input pixels
 // and neighbouring groups share columns, so the input is read from DRAM
@@ -33,6 +35,7 @@ namespace dcn {
 constexpr int kGuideWarps = 8;
 constexpr int kGuideRows = 8;
 constexpr int kGuideMaxQuads = 16;  // quads per lane (NJ), at most
+constexpr int kGuideChunk = 5;      // quads per lane convolved together in registers
 
 struct GuideArgs {
   const void* x;       // (N, H, W, C) of T
@@ -78,14 +81,38 @@ __device__ __forceinline__ float gelu_erf(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
 }
 
+// Three CTAs per SM for groups of 8 or 16 lanes (more warps to cover the
+// load latency; measured 10% faster at C = 160); 32-lane groups are
+// left to the compiler (their spills at three cost more than the warps gain).
 template <typename T, int LP>
-__global__ void __launch_bounds__(kGuideWarps * 32) dcn_guide_kernel(const GuideArgs a) {
+__global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
+    dcn_guide_kernel(const GuideArgs a) {
   constexpr int PPW = 32 / LP;  // pixels per warp
   constexpr int kThreads = kGuideWarps * 32;
-  // conv results of this thread's quads, [quad j][thread]: consecutive lanes
-  // touch consecutive 16-byte words, and each thread reads back only its own
-  extern __shared__ float4 conv_buf[];
+  constexpr int CH = kGuideChunk;
+  // Shared memory: the 9 weight quads and the bias, gamma and beta quads of
+  // every channel (12 * Q float4, staged once per CTA), then the conv results
+  // of this thread's quads, [quad j][thread]: consecutive lanes touch
+  // consecutive 16-byte words, and each thread reads back only its own.
+  extern __shared__ float4 guide_smem[];
+  float4* const w_s = guide_smem;            // [(a * 3 + b) * Q + q]
+  float4* const bias_s = w_s + 9 * a.Q;      // [q]
+  float4* const gamma_s = bias_s + a.Q;
+  float4* const beta_s = gamma_s + a.Q;
+  float4* const conv_buf = beta_s + a.Q;     // [j * kThreads + tid]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 12 * a.Q; i += kThreads) {
+    float4 v;
+    if (i < 9 * a.Q) v = __ldg(reinterpret_cast<const float4*>(a.w) + i);
+    else {
+      const int r = (i - 9 * a.Q) / a.Q, q = i - 9 * a.Q - r * a.Q;
+      const float* src = r == 0 ? a.bias : (r == 1 ? a.gamma : a.beta);
+      v = ld4_or(src != nullptr ? src + 4 * q : nullptr, true, r == 1 ? 1.f : 0.f);
+    }
+    w_s[i] = v;
+  }
+  __syncthreads();
+
   const int gi = lane / LP, sub = lane - gi * LP;
   int t = blockIdx.x;
   const int tx = t % a.tiles_x;
@@ -95,39 +122,56 @@ __global__ void __launch_bounds__(kGuideWarps * 32) dcn_guide_kernel(const Guide
   const int col = (tx * kGuideWarps + warp) * PPW + gi;
   const bool col_ok = col < a.W;
   const T* xs = static_cast<const T*>(a.x);
+  const size_t rowE = size_t(a.W) * a.C;  // elements per image row
   const float inv_c = 1.0f / float(a.C);
 
 #pragma unroll 1
   for (int i = 0; i < kGuideRows; ++i) {
     const int y = ty * kGuideRows + i;
     if (y >= a.H) break;  // the same for the whole CTA
-    // depthwise 3x3 convolution, one quad of channels at a time
+    // depthwise 3x3 convolution, CH quads of this lane at a time in registers
     float s = 0.f;
 #pragma unroll 1
-    for (int j = 0; j < a.NJ; ++j) {
-      const int q = sub + LP * j;
-      const bool q_ok = col_ok && q < a.Q;
-      float4 acc = ld4_or(a.bias != nullptr ? a.bias + 4 * q : nullptr, q_ok, 0.f);
+    for (int j0 = 0; j0 < a.NJ; j0 += CH) {
+      float4 acc[CH];
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        const int q = sub + LP * (j0 + u);
+        acc[u] = (j0 + u < a.NJ && col_ok && q < a.Q) ? bias_s[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
       for (int ta = 0; ta < 3; ++ta) {
         const int yy = y + ta - 1;
         if (yy < 0 || yy >= a.H) continue;  // the same for the whole CTA
+        const T* row = xs + size_t(n * a.H + yy) * rowE;
 #pragma unroll
         for (int tb = 0; tb < 3; ++tb) {
           const int xx = col + tb - 1;
-          const T* px = xs + (size_t(n * a.H + yy) * a.W + xx) * a.C + 4 * q;
-          if (q_ok && xx >= 0 && xx < a.W && in_tensor(px, 4 * sizeof(T), a.x, a.x_bytes)) {
-            const float4 v = guide_ld4<T>(px);
-            const float4 wv = __ldg(reinterpret_cast<const float4*>(a.w + (ta * 3 + tb) * a.C + 4 * q));
-            acc.x = fmaf(wv.x, v.x, acc.x);
-            acc.y = fmaf(wv.y, v.y, acc.y);
-            acc.z = fmaf(wv.z, v.z, acc.z);
-            acc.w = fmaf(wv.w, v.w, acc.w);
+          if (!(col_ok && xx >= 0 && xx < a.W)) continue;
+          const T* px = row + xx * a.C + 4 * sub;
+          const float4* wq = w_s + (ta * 3 + tb) * a.Q + sub;
+#pragma unroll
+          for (int u = 0; u < CH; ++u) {
+            const int j = j0 + u;
+            if (j < a.NJ && sub + LP * j < a.Q &&
+                in_tensor(px + 4 * LP * j, 4 * sizeof(T), a.x, a.x_bytes)) {
+              const float4 v = guide_ld4<T>(px + 4 * LP * j);
+              const float4 wv = wq[LP * j];
+              acc[u].x = fmaf(wv.x, v.x, acc[u].x);
+              acc[u].y = fmaf(wv.y, v.y, acc[u].y);
+              acc[u].z = fmaf(wv.z, v.z, acc[u].z);
+              acc[u].w = fmaf(wv.w, v.w, acc[u].w);
+            }
           }
         }
       }
-      s += (acc.x + acc.y) + (acc.z + acc.w);  // quads outside the channels hold 0
-      conv_buf[j * kThreads + tid] = acc;
+#pragma unroll
+      for (int u = 0; u < CH; ++u) {
+        if (j0 + u < a.NJ) {
+          s += (acc[u].x + acc[u].y) + (acc[u].z + acc[u].w);  // quads outside C hold 0
+          conv_buf[(j0 + u) * kThreads + tid] = acc[u];
+        }
+      }
     }
     // LayerNorm over the pixel's channels: the mean, then the mean squared deviation
     const float mean = group_sum<LP>(s) * inv_c;
@@ -147,8 +191,7 @@ __global__ void __launch_bounds__(kGuideWarps * 32) dcn_guide_kernel(const Guide
       const int q = sub + LP * j;
       if (q >= a.Q) break;
       const float4 v = conv_buf[j * kThreads + tid];
-      const float4 g = ld4_or(a.gamma != nullptr ? a.gamma + 4 * q : nullptr, true, 1.f);
-      const float4 b = ld4_or(a.beta != nullptr ? a.beta + 4 * q : nullptr, true, 0.f);
+      const float4 g = gamma_s[q], b = beta_s[q];
       const float o0 = gelu_erf((v.x - mean) * rstd * g.x + b.x);
       const float o1 = gelu_erf((v.y - mean) * rstd * g.y + b.y);
       const float o2 = gelu_erf((v.z - mean) * rstd * g.z + b.z);
