@@ -1165,7 +1165,8 @@ template <typename T, int LP>
 dcn_status guide_launch_lp(const GuideArgs& a, cudaStream_t stream) {
   const unsigned grid = unsigned(int64_t(a.N) * a.tiles_y * a.tiles_x);
   const unsigned block = kGuideWarps * 32;
-  const size_t smem = size_t(a.NJ) * block * sizeof(float4);  // at most 64 KB
+  // parameters (12 quads per channel quad) and the conv results: at most 160 KB
+  const size_t smem = (size_t(12) * a.Q + size_t(a.NJ) * block) * sizeof(float4);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(dcn_guide_kernel<T, LP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(smem)) != cudaSuccess)

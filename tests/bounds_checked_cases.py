@@ -104,6 +104,22 @@ def main():
     assert np.abs(f64(off) - ro).max() <= 1e-4 * np.abs(ro).max()
     assert np.abs(f64(msk) - rm).max() <= 1e-4 * np.abs(rm).max()
     print("ok projection", flush=True)
+    # the guide features: ragged column and row tiles, a one-pixel image, bf16
+    # input, and C = 196 (lanes left idle in the last quad group)
+    for (N, H, W, G, Cg, dtype) in ((2, 11, 37, 4, 16, "f32"), (1, 1, 1, 2, 16, "bf16"),
+                                    (1, 9, 5, 49, 4, "f32")):
+        C = G * Cg
+        pg = mk(N, H, W, G, Cg, dtype=dtype)
+        xg = to_dev(RNG.standard_normal((N, H, W, C)).astype(np.float32), dtype)
+        prm = [RNG.uniform(-0.5, 0.5, size=s_).astype(np.float32) for s_ in ((3, 3, C), (C,))]
+        prm += [RNG.uniform(0.5, 1.5, size=C).astype(np.float32),
+                RNG.uniform(-0.3, 0.3, size=C).astype(np.float32)]
+        qg = torch.empty(xg.shape, dtype=torch.bfloat16, device="cuda")
+        dcn.dcn_core_offset_mask_guide(pg, xg, *(torch.from_numpy(a).cuda() for a in prm), 1e-6, qg)
+        dcn.dcn_core_sync_status()
+        rg = oracle.guide(f64(xg), *prm, 1e-6)
+        assert (np.abs(f64(qg) - rg) <= 2.0 ** -8 * np.abs(rg) + 2e-5).all(), f"guide {N}x{H}x{W}x{C}"
+    print("ok guide", flush=True)
     print("all cases passed")
 
 

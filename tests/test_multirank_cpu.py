@@ -62,3 +62,55 @@ def test_bench_reference_arm_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_module_resolves_every_name():
+    """Every name a function of bench.py reads at module level is defined
+    (the GPU-only legs of the benchmark cannot run here, so this catches a
+    helper lost in an edit before a GPU run does)."""
+    import ast
+    import builtins
+    import importlib.util
+
+    path = os.path.join(ROOT, "bench.py")
+    spec = importlib.util.spec_from_file_location("bench_static_check", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    tree = ast.parse(open(path).read())
+    missing = set()
+    # module-level functions and class methods; a nested function is checked as
+    # part of the function around it (its free names are that function's locals)
+    tops = [n for n in tree.body if isinstance(n, ast.FunctionDef)]
+    tops += [m for c in tree.body if isinstance(c, ast.ClassDef) for m in c.body
+             if isinstance(m, ast.FunctionDef)]
+    for fn in tops:
+        local = {a.arg for a in fn.args.args + fn.args.kwonlyargs}
+        if fn.args.vararg:
+            local.add(fn.args.vararg.arg)
+        for n in ast.walk(fn):
+            if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Store):
+                local.add(n.id)
+            elif isinstance(n, (ast.FunctionDef, ast.Lambda)) and n is not fn:
+                if isinstance(n, ast.FunctionDef):
+                    local.add(n.name)
+                local.update(a.arg for a in n.args.args)
+            elif isinstance(n, (ast.Import, ast.ImportFrom)):
+                local.update((a.asname or a.name).split(".")[0] for a in n.names)
+            elif isinstance(n, ast.comprehension):
+                for t in ast.walk(n.target):
+                    if isinstance(t, ast.Name):
+                        local.add(t.id)
+            elif isinstance(n, ast.ExceptHandler) and n.name:
+                local.add(n.name)
+            elif isinstance(n, (ast.With, ast.AsyncWith)):
+                for it in n.items:
+                    if it.optional_vars is not None:
+                        for t in ast.walk(it.optional_vars):
+                            if isinstance(t, ast.Name):
+                                local.add(t.id)
+        for n in ast.walk(fn):
+            if (isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load) and n.id not in local
+                    and not hasattr(mod, n.id) and not hasattr(builtins, n.id)):
+                missing.add((fn.name, n.id))
+    assert not missing, sorted(missing)
+
