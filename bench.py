@@ -72,19 +72,31 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
-    kernel sources are unchanged since it was taken (else None)."""
+# Sources of the kernels the bench step launches: every file under csrc/ except
+# those that only define kernels the step never runs.
+OTHER_KERNEL_SOURCES = ("dcn_guide.cuh", "dcn_projection.cuh")
+
+
+def step_kernel_sources_sha() -> str:
+    """First 16 hex digits of sha256 over the step kernels' sources (sorted)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-    if not os.path.exists(path):
-        return None
     csrc = os.path.join(ROOT, "deformable_convolution_core_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(csrc)):
+        if f in OTHER_KERNEL_SOURCES:
+            continue
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
-    sha = h.hexdigest()[:16]
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel sources are unchanged since it was taken (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = step_kernel_sources_sha()
     for line in open(path):
         parts = dict(p.split("=", 1) for p in line.split() if "=" in p)
         if parts.get("kernel") == kernel and parts.get("src_sha") == sha:
