@@ -32,10 +32,14 @@ METRIC = "DCNv3 core fwd/bwd GB/s and Gsamples/s on 1 B200; fraction of HBM peak
 DEFAULT_WORKLOAD = "internimage_l_stage1_fp32_n32_96x96_c160"
 SWEEP = ["internimage_l_stage1_bf16_n64_96x96_c160", "internimage_l_stage2_bf16_n64_48x48_c320",
          "internimage_l_stage3_bf16_n64_24x24_c640", "internimage_l_stage4_bf16_n64_12x12_c1280",
+         "internimage_l_stage1_fp16_n64_96x96_c160",
+         "internimage_l_stage1_k5_bf16_n16_96x96_c160", "internimage_l_stage1_k7_bf16_n16_96x96_c160",
+         "internimage_l_stage1_cg8_bf16_n64_96x96_c160", "internimage_l_stage1_cg32_bf16_n64_96x96_c160",
          "dcnv4_hires_bf16_n2_256x256_c192_s1", "dcnv4_hires_bf16_n2_256x256_c192_s2",
          "dcnv4_hires_bf16_n2_256x256_c192_s1_remove_center",
          "internimage_l_stage2_bwd_fp32_n32_48x48_c320",
-         "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
+         "internimage_l_stage2_bwd_bf16_n32_48x48_c320",
+         "internimage_l_stage2_bwd_fp16_n32_48x48_c320"]
 # The same backward workloads through dcn_core_backward_deterministic.
 DETERMINISTIC_SWEEP = ["internimage_l_stage2_bwd_fp32_n32_48x48_c320",
                        "internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
@@ -50,6 +54,8 @@ GUIDE_SWEEP = ["internimage_l_stage1_fp32_n32_96x96_c160", "internimage_l_stage1
                "internimage_l_stage2_bf16_n64_48x48_c320", "internimage_l_stage3_bf16_n64_24x24_c640",
                "internimage_l_stage4_bf16_n64_12x12_c1280"]
 L2_BYTES = 126 * 1024 * 1024
+# torch dtype of each storage type name
+TORCH_DTYPES = {"f32": "float32", "bf16": "bfloat16", "f16": "float16"}
 
 
 def bf16_peak():
@@ -196,7 +202,7 @@ class Step:
         self.wl = wl
         self.backward = backward
         self.deterministic = deterministic
-        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        tdt = getattr(torch, TORCH_DTYPES[wl.dtype])
         self.p = dcn.problem_for(wl)
         dev = torch.device("cuda")
         self.x = torch.from_numpy(inputs["x"]).to(dev).to(tdt)
@@ -290,7 +296,6 @@ def run_ours(args, world, rank, local):
     total_ms, fwd_ms, bwd_ms = timed(step, args.steps, args.warmup, barrier)
     time.sleep(0.25)
     clock_summary = clocks.summary()
-    clocks.stop()
     total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], "cuda")
     ms_per_step = total_ms / args.steps
 
@@ -339,8 +344,9 @@ def run_ours(args, world, rank, local):
                           "GB/s": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9, 1),
                           "Gsamples/s": round(wl.samples / (fwd_ms * 1e-3) / 1e9, 2),
                           "frac_of_hbm": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9 / peak, 4),
-                          "frac_of_l1_ceiling": round(wl.samples / (fwd_ms * 1e-3) / 1e9 /
-                                                      l1_ceiling_gsamples(wl), 4)},
+                          "frac_of_l1_ceiling": round(
+                              wl.samples / (fwd_ms * 1e-3) / 1e9 /
+                              l1_ceiling_gsamples(wl, clock_summary.get("sm_mhz")), 4)},
                       "backward": None if bwd_ms == 0 else {
                           "ms": round(bwd_ms, 4),
                           "GB/s": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
@@ -353,13 +359,25 @@ def run_ours(args, world, rank, local):
         "clocks": clock_summary,
     }
     if rank == 0 and world == 1 and not args.no_sweep and args.workload == DEFAULT_WORKLOAD:
-        result["sweep"] = run_sweep(gen, peak)
+        result["sweep"] = run_sweep(gen, peak, clocks)
         result["projection"] = run_projection(gen, peak)
         result["guide"] = run_guide(gen, peak)
         result["block_core_path"] = run_block_core_path(gen)
+    clocks.stop()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, inputs, backward)
         result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(wl, inputs, backward)
+    if "sweep" in result:
+        # last on the line, so that a truncated tail still shows it: the
+        # InternImage-L stage forwards (bf16, N=64) against the HBM roofline
+        # and the on-chip ceiling
+        result["stage_forward_fractions"] = {
+            name.split("_bf16")[0].replace("internimage_l_", ""): {
+                "frac_of_hbm": result["sweep"][name]["frac_of_hbm"],
+                "frac_of_l1_ceiling": result["sweep"][name]["frac_of_l1_ceiling"],
+                "ms": result["sweep"][name]["ms"]}
+            for name in SWEEP if name.startswith("internimage_l_stage") and "_bf16_" in name
+            and "_bwd_" not in name}
     del step
     return result
 
@@ -456,7 +474,7 @@ def run_projection(gen, peak, launches=20):
         wl = gen.WORKLOADS[name]
         d = gen.make_projection_inputs(wl, cq)
         p = dcn.problem_for(wl)
-        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        tdt = getattr(torch, TORCH_DTYPES[wl.dtype])
         q = torch.from_numpy(d["query"]).cuda().to(torch.bfloat16)
         w = torch.from_numpy(d["weight"]).cuda().to(torch.bfloat16)
         b = torch.from_numpy(d["bias"]).cuda()
@@ -490,10 +508,16 @@ def run_projection(gen, peak, launches=20):
     return out
 
 
-def l1_ceiling_gsamples(wl, sm_mhz=1965.0, sms=148):
+NOMINAL_SM_MHZ = 1965.0
+
+
+def l1_ceiling_gsamples(wl, sm_mhz=None, sms=148):
     """Samples/s (1e9) if every on-chip byte path delivered 128 B per clock
-    per SM and a sample needed only its 2x2 footprint (4 * Cg * size bytes)."""
-    return sms * 128.0 * sm_mhz * 1e6 / (4.0 * wl.Cg * wl.esize) / 1e9
+    per SM and a sample needed only its 2x2 footprint (4 * Cg * size bytes),
+    at the SM clock sampled while the passes ran (the nominal maximum when no
+    sample was taken)."""
+    mhz = sm_mhz if sm_mhz else NOMINAL_SM_MHZ
+    return sms * 128.0 * mhz * 1e6 / (4.0 * wl.Cg * wl.esize) / 1e9
 
 
 def run_guide(gen, peak, launches=20):
@@ -506,7 +530,7 @@ def run_guide(gen, peak, launches=20):
     for name in GUIDE_SWEEP:
         wl = gen.WORKLOADS[name]
         p = dcn.problem_for(wl)
-        tdt = torch.float32 if wl.dtype == "f32" else torch.bfloat16
+        tdt = getattr(torch, TORCH_DTYPES[wl.dtype])
         x = torch.from_numpy(gen.make_inputs(wl)["x"]).cuda().to(tdt)
         gp = {k: torch.from_numpy(v).cuda() for k, v in gen.make_guide_params(wl).items()}
         q = torch.empty(x.shape, dtype=torch.bfloat16, device="cuda")
@@ -589,14 +613,18 @@ def run_block_core_path(gen, name="internimage_l_stage1_bf16_n64_96x96_c160", re
             "Mpixels/s": round(M / (float(np.median(t.sum(axis=1))) * 1e-3) / 1e6, 1)}
 
 
-def run_sweep(gen, peak, reps=30, warmup=3):
+def run_sweep(gen, peak, clocks=None, reps=30, warmup=3):
     """The other workloads' passes, one launch at a time: L2 is flushed (a
     2 x L2 buffer is written) before every timed launch, and the median and
-    the 10th / 90th percentiles of the per-launch CUDA-event times are kept."""
+    the 10th / 90th percentiles of the per-launch CUDA-event times are kept.
+    The on-chip ceiling of each row uses the median SM clock sampled while
+    the sweep ran."""
     import numpy as np
     import torch
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
     out = {}
+    if clocks is not None:
+        clocks.begin_region()
     runs = [(name, False) for name in SWEEP] + [(name, True) for name in DETERMINISTIC_SWEEP]
     for name, det in runs:
         wl = gen.WORKLOADS[name]
@@ -629,12 +657,17 @@ def run_sweep(gen, peak, reps=30, warmup=3):
                     "ms_p10": round(float(np.percentile(ms_all, 10)), 4),
                     "ms_p90": round(float(np.percentile(ms_all, 90)), 4),
                     "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peak, 4),
-                    "Gsamples/s": round(gsps, 2),
-                    "frac_of_l1_ceiling": round(gsps / l1_ceiling_gsamples(wl), 4),
-                    "MB": round(b / 1e6, 1), "l2": "flushed before every launch"}
+                    "Gsamples/s": round(gsps, 2), "frac_of_l1_ceiling": None,
+                    "MB": round(b / 1e6, 1), "l2": "flushed before every launch",
+                    "_wl": wl}
         del step
         torch.cuda.empty_cache()
     del flush
+    sm_mhz = clocks.summary().get("sm_mhz") if clocks is not None else None
+    for row in out.values():
+        row["frac_of_l1_ceiling"] = round(row["Gsamples/s"] / l1_ceiling_gsamples(row.pop("_wl"),
+                                                                                 sm_mhz), 4)
+    out["l1_ceiling_sm_mhz"] = sm_mhz if sm_mhz else f"nominal {NOMINAL_SM_MHZ}"
     return out
 
 

@@ -21,12 +21,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("DCN_CORE_LIBRARY") or os.path.join(_HERE, "libdcncore.so")
 
 # DCN_CORE_ABI_VERSION of include/dcn_core.h that DcnProblem mirrors.
-ABI_VERSION = 4
+ABI_VERSION = 5
 DCN_OK, DCN_ERR_INVALID_ARG, DCN_ERR_UNSUPPORTED, DCN_ERR_CUDA, DCN_ERR_TIMEOUT = 0, 1, 2, 3, 4
 DCN_ERR_OUT_OF_BOUNDS = 5  # only from the bounds-checked build
 # Scratch the allocation-free backward owns per GPU (DCN_CORE_NOALLOC_SCRATCH_BYTES).
 DCN_CORE_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
-DCN_F32, DCN_BF16 = 0, 1
+DCN_F32, DCN_BF16, DCN_F16 = 0, 1, 2
+# storage-type names accepted wherever a dtype is given as a string
+DTYPES = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16, "bfloat16": DCN_BF16,
+          "f16": DCN_F16, "float16": DCN_F16}
 
 # Every entry point of include/dcn_core.h.
 EXPORTED_SYMBOLS = (
@@ -74,7 +77,7 @@ def make_problem(N, H, W, G, Cg, K=3, stride=1, pad=1, dilation=1, offset_scale=
     """stride, pad and dilation apply to both axes unless a width value
     (stride_w, pad_w, dilation_w) is given; then they are the height axis's."""
     if isinstance(dtype, str):
-        dtype = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16, "bfloat16": DCN_BF16}[dtype]
+        dtype = DTYPES[dtype]
     separate = stride_w is not None or pad_w is not None or dilation_w is not None
     sw = stride if stride_w is None else stride_w
     pw = pad if pad_w is None else pad_w
@@ -237,16 +240,16 @@ def dcn_core_backward_host(problem: DcnProblem, input, offset, mask, h_grad_out,
 def dcn_core_backward_noalloc(problem: DcnProblem, input, offset, mask, grad_out, grad_input,
                               grad_offset, grad_mask, stream=None) -> None:
     """Backward without a workspace, for callers that cannot allocate device
-    memory (see include/dcn_core.h).  For bf16 storage the fp32 grad_input
+    memory (see include/dcn_core.h).  For bf16 or fp16 storage the fp32 grad_input
     accumulator must fit the library's fixed DCN_CORE_NOALLOC_SCRATCH_BYTES
     array; calls that may overlap on the GPU must be serialised."""
     status = load_library().dcn_core_backward_noalloc(
         ctypes.byref(problem), _ptr(input), _ptr(offset), _ptr(mask), _ptr(grad_out),
         _ptr(grad_input), _ptr(grad_offset), _ptr(grad_mask), _stream(stream))
-    if status == DCN_ERR_UNSUPPORTED and problem.dtype == DCN_BF16:
+    if status == DCN_ERR_UNSUPPORTED and problem.dtype != DCN_F32:
         need = problem.N * problem.H * problem.W * problem.G * problem.Cg * 4
         if need > DCN_CORE_NOALLOC_SCRATCH_BYTES:
-            raise DcnError(status, f"dcn_core_backward_noalloc: the bf16 accumulator needs {need} "
+            raise DcnError(status, f"dcn_core_backward_noalloc: the fp32 accumulator of 2-byte storage needs {need} "
                                    f"bytes, more than the {DCN_CORE_NOALLOC_SCRATCH_BYTES} bytes "
                                    "of scratch this entry point owns")
     _check(status, "dcn_core_backward_noalloc")
@@ -292,8 +295,7 @@ def dcn_core_linear_bf16(input, M: int, K: int, weight, Nout: int, bias, output,
     """output (M, Nout) = input (M, K) @ weight (Nout, K).T + bias on the tensor
     cores; bf16 operands, fp32 accumulation, output in out_dtype."""
     if isinstance(out_dtype, str):
-        out_dtype = {"f32": DCN_F32, "float32": DCN_F32, "bf16": DCN_BF16,
-                     "bfloat16": DCN_BF16}[out_dtype]
+        out_dtype = DTYPES[out_dtype]
     _check(load_library().dcn_core_linear_bf16(
         _ptr(input), int(M), int(K), _ptr(weight), int(Nout), _ptr(bias), _ptr(output),
         int(out_dtype), _stream(stream)), "dcn_core_linear_bf16")
@@ -307,4 +309,5 @@ __all__ = ["DcnProblem", "DcnError", "make_problem", "problem_for", "taps", "loa
            "library_path", "EXPORTED_SYMBOLS", *EXPORTED_SYMBOLS, "ABI_VERSION",
            "DCN_CORE_NOALLOC_SCRATCH_BYTES",
            "DCN_OK", "DCN_ERR_INVALID_ARG", "DCN_ERR_UNSUPPORTED", "DCN_ERR_CUDA",
-           "DCN_ERR_TIMEOUT", "DCN_ERR_OUT_OF_BOUNDS", "DCN_F32", "DCN_BF16"]
+           "DCN_ERR_TIMEOUT", "DCN_ERR_OUT_OF_BOUNDS", "DCN_F32", "DCN_BF16", "DCN_F16",
+           "DTYPES"]

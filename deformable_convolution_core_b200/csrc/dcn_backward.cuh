@@ -16,6 +16,8 @@
 // so each corner is loaded once and reduced immediately.
 #pragma once
 
+#include <type_traits>
+
 #include "dcn_tile.cuh"
 
 namespace dcn {
@@ -101,14 +103,52 @@ struct Quad<__nv_bfloat16> {
     reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(a);
   }
 };
+template <>
+struct Quad<__half> {
+  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
+    uint32_t w0, w1;
+    asm("ld.global.nc.v2.b32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "l"(p));
+    v[0] = f16lo_to_f32(w0);
+    v[1] = f16hi_to_f32(w0);
+    v[2] = f16lo_to_f32(w1);
+    v[3] = f16hi_to_f32(w1);
+  }
+  __device__ __forceinline__ static void load_pred(const void* p, bool pred, float (&v)[4]) {
+    uint32_t w0, w1;
+    asm("{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n mov.b32 %0, 0;\n mov.b32 %1, 0;\n"
+        " @q ld.global.nc.v2.b32 {%0, %1}, [%2];\n}"
+        : "=r"(w0), "=r"(w1)
+        : "l"(p), "r"(int(pred)));
+    v[0] = f16lo_to_f32(w0);
+    v[1] = f16hi_to_f32(w0);
+    v[2] = f16lo_to_f32(w1);
+    v[3] = f16hi_to_f32(w1);
+  }
+  __device__ __forceinline__ static void store_pair(void* base, size_t i, float a, float b) {
+    reinterpret_cast<uint32_t*>(base)[i] = pack_f16x2(a, b);
+  }
+  __device__ __forceinline__ static void store_pair_pred(void* p, float a, float b, uint32_t pred) {
+    asm volatile("{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n @q st.global.b32 [%0], %1;\n}"
+                 ::"l"(p), "r"(pack_f16x2(a, b)), "r"(pred)
+                 : "memory");
+  }
+  __device__ __forceinline__ static void store_one(void* base, size_t i, float a) {
+    reinterpret_cast<__half*>(base)[i] = __float2half_rn(a);
+  }
+};
 
-// fp32 accumulator -> bf16 grad_input, rounded to nearest even once.
-__global__ void dcn_round_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out,
+// fp32 accumulator -> grad_input of a 2-byte storage type (bf16 or fp16),
+// rounded to nearest even once.
+template <typename T>
+__global__ void dcn_round_to_half_kernel(const float4* __restrict__ in, uint2* __restrict__ out,
                                          size_t n4) {
   for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += size_t(gridDim.x) * blockDim.x) {
     const float4 v = __ldg(in + i);
-    out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    if constexpr (sizeof(T) == 2 && std::is_same<T, __half>::value)
+      out[i] = make_uint2(pack_f16x2(v.x, v.y), pack_f16x2(v.z, v.w));
+    else
+      out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
   }
 }
 
@@ -207,6 +247,21 @@ struct GxScatter<true> {
                                          uint32_t pred) const {
     add(size_t(q - p), lo, hi, pred != 0u && in_range(e + 3, n));
   }
+  // accumulator[q + 4i] += v[i], i < 4, if pred: the channels c, c+4, c+8,
+  // c+12 of a 16-channel group, so that the four lanes c = 0..3 of a unit
+  // write one 32-byte sector per instruction (e: q's element, checked build)
+  __device__ __forceinline__ void add4_strided(unsigned long long* q, size_t e, float2 lo,
+                                               float2 hi, uint32_t pred) const {
+    if (pred != 0u && !in_range(e + 12, n)) pred = 0u;
+    const long long a = __float2ll_rn(lo.x * scale), b = __float2ll_rn(lo.y * scale);
+    const long long c = __float2ll_rn(hi.x * scale), d = __float2ll_rn(hi.y * scale);
+    asm volatile(
+        "{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
+        " @q red.global.add.u64 [%0], %1;\n @q red.global.add.u64 [%0+32], %2;\n"
+        " @q red.global.add.u64 [%0+64], %3;\n @q red.global.add.u64 [%0+96], %4;\n}" ::"l"(q),
+        "l"(a), "l"(b), "l"(c), "l"(d), "r"(pred)
+        : "memory");
+  }
 };
 
 // max |v| over n values, as float bits, into *out (atomicMax; *out starts at 0).
@@ -239,6 +294,73 @@ __global__ void dcn_fixed_to_grad_kernel(const long long* __restrict__ acc, T* _
     const float f = ok ? float(double(acc[i]) * inv) : __int_as_float(0x7fc00000);
     Storage<T>::store_float(out + i, f);
   }
+}
+
+// ---------------------------------------------------------------------------
+// The per-tap arithmetic of the backward, shared by both kernels so that
+// grad_offset and grad_mask have the same bits whatever the kernel, tile or
+// lane mapping (every operation is an explicitly rounded intrinsic: no
+// contraction choice is left to the compiler).  With 16 channels per group the
+// corner dot product d_c = <g, x_c> is summed in one canonical order: four
+// channel quarters q, each (x0 g0 + x2 g2) + (x1 g1 + x3 g3) as two packed
+// pairs, then (d_q0 + d_q1) + (d_q2 + d_q3).  Pairwise sums are exact under
+// swapping their operands, so a lane that meets the quarters in the order
+// q ^ r (any r) gets the same bits.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float quarter_dot(float2 x01, float2 x23, float2 g01, float2 g23) {
+  const float2 pd = __ffma2_rn(x23, g23, __fmul2_rn(x01, g01));
+  return __fadd_rn(pd.x, pd.y);
+}
+
+struct TapGrads {
+  float s;   // <g, v_k> = sum_c b_c d_c
+  float gx;  // <g, dv/dX>
+  float gy;  // <g, dv/dY>
+};
+
+// Bilinear weights b00, b01, b10, b11 of fractional parts (ly, lx).
+__device__ __forceinline__ void bilinear_weights(float ly, float lx, float (&b)[4]) {
+  const float hy = __fsub_rn(1.f, ly), hx = __fsub_rn(1.f, lx);
+  b[0] = __fmul_rn(hy, hx);
+  b[1] = __fmul_rn(hy, lx);
+  b[2] = __fmul_rn(ly, hx);
+  b[3] = __fmul_rn(ly, lx);
+}
+
+__device__ __forceinline__ TapGrads tap_grads(const float (&d)[4], float ly, float lx) {
+  const float hy = __fsub_rn(1.f, ly), hx = __fsub_rn(1.f, lx);
+  float b[4];
+  bilinear_weights(ly, lx, b);
+  TapGrads r;
+  r.s = __fmaf_rn(b[3], d[3], __fmaf_rn(b[2], d[2], __fmaf_rn(b[1], d[1], __fmul_rn(b[0], d[0]))));
+  r.gx = __fmaf_rn(ly, __fsub_rn(d[3], d[2]), __fmul_rn(hy, __fsub_rn(d[1], d[0])));
+  r.gy = __fmaf_rn(lx, __fsub_rn(d[3], d[1]), __fmul_rn(hx, __fsub_rn(d[2], d[0])));
+  return r;
+}
+
+// grad logit_k (softmax: m_k (s_k - sum_j m_j s_j)) or grad mask_k (raw: s_k).
+template <bool SOFTMAX, int KK>
+__device__ __forceinline__ float mask_grad_sum(const float (&m)[KK], const float (&s)[KK]) {
+  float ms = 0.f;
+  if (SOFTMAX) {
+#pragma unroll
+    for (int k = 0; k < KK; ++k) ms = __fmaf_rn(m[k], s[k], ms);
+  }
+  return ms;
+}
+template <bool SOFTMAX>
+__device__ __forceinline__ float mask_grad(float m, float s, float ms) {
+  return SOFTMAX ? __fmul_rn(m, __fsub_rn(s, ms)) : s;
+}
+
+// Sum of a corner dot product over the unit's lanes (one channel quarter per
+// lane), lowest lane bit first: (d_q0 + d_q1) + (d_q2 + d_q3) for four lanes,
+// the canonical order above.
+template <int LANES>
+__device__ __forceinline__ float quarters_sum(float v, unsigned mask) {
+#pragma unroll
+  for (int o = 1; o < LANES; o <<= 1) v = __fadd_rn(v, __shfl_xor_sync(mask, v, o));
+  return v;
 }
 
 template <int LANES>
@@ -304,43 +426,42 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
       const float Y = tap_coord(by + ka * t.dil, t.sigma, d.y);
       const float X = tap_coord(bx + kb * t.dil_w, t.sigma, d.x);
       const Footprint f = footprint(Y, X, t.H, t.W);
-      float s = 0.f, gX = 0.f, gY = 0.f;
+      // (lanes of one unit share the footprint, so the branch is unit-uniform)
+      float dc[4] = {0.f, 0.f, 0.f, 0.f};
+      float ly = 0.f, lx = 0.f;
       if (f.in_support) {
-        const float hy = 1.f - f.ly, hx = 1.f - f.lx;
+        ly = f.ly;
+        lx = f.lx;
         const ptrdiff_t base = ptrdiff_t(f.y0) * ptrdiff_t(rowE) + ptrdiff_t(f.x0) * ptrdiff_t(pixE);
         const ptrdiff_t cofs[4] = {base, base + ptrdiff_t(pixE), base + ptrdiff_t(rowE),
                                    base + ptrdiff_t(rowE + pixE)};
         const bool cval[4] = {f.v00, f.v01, f.v10, f.v11};
-        const float cw[4] = {hy * hx, hy * f.lx, f.ly * hx, f.ly * f.lx};
-        float dc[4];
+        float cw[4];
+        bilinear_weights(ly, lx, cw);
+        const float2 g01 = make_float2(go[0], go[1]), g23 = make_float2(go[2], go[3]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float cv[CPL] = {0.f, 0.f, 0.f, 0.f};
           if (cval[c] && in_range(size_t(ptrdiff_t(g_off) + cofs[c]) + CPL - 1, n_img))
             Quad<T>::load(xg + cofs[c] * ptrdiff_t(sizeof(T)), cv);
-          float dsum = 0.f;
-#pragma unroll
-          for (int j = 0; j < CPL; ++j) dsum = fmaf(go[j], cv[j], dsum);
-          dc[c] = dsum;
-          const float wv = mk * cw[c];
-          gxs.add(size_t(ptrdiff_t(g_off) + cofs[c]), make_float2(wv * go[0], wv * go[1]),
-                  make_float2(wv * go[2], wv * go[3]), cval[c]);
+          dc[c] = quarter_dot(make_float2(cv[0], cv[1]), make_float2(cv[2], cv[3]), g01, g23);
+          const float wv = __fmul_rn(mk, cw[c]);
+          const float2 w2 = make_float2(wv, wv);
+          gxs.add(size_t(ptrdiff_t(g_off) + cofs[c]), __fmul2_rn(w2, g01), __fmul2_rn(w2, g23),
+                  cval[c]);
         }
-        s = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];
-        gX = hy * (dc[1] - dc[0]) + f.ly * (dc[3] - dc[2]);
-        gY = hx * (dc[2] - dc[0]) + f.lx * (dc[3] - dc[1]);
       }
       if (LANES > 1) {
-        s = unit_sum<LANES>(s, umask);
-        gX = unit_sum<LANES>(gX, umask);
-        gY = unit_sum<LANES>(gY, umask);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dc[c] = quarters_sum<LANES>(dc[c], umask);
       }
+      const TapGrads tg = tap_grads(dc, ly, lx);
       if (sub == 0) {
-        const float sc = t.sigma * mk;
+        const float sc = __fmul_rn(t.sigma, mk);
         if (in_range(unit * KK + k, n_taps))
-          Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
+          Quad<T>::store_pair(a.goff, unit * KK + k, __fmul_rn(sc, tg.gx), __fmul_rn(sc, tg.gy));
       }
-      return s;
+      return tg.s;
     };
 
     if constexpr (KKS > 0) {
@@ -387,46 +508,38 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
 #pragma unroll
         for (int j = 0; j < GRP; ++j) {
           const int k = k0 + j;
-          const float hy = 1.f - f[j].ly, hx = 1.f - f[j].lx;
-          const float cw[4] = {hy * hx, hy * f[j].lx, f[j].ly * hx, f[j].ly * f[j].lx};
+          float cw[4];
+          bilinear_weights(f[j].ly, f[j].lx, cw);
           float dc[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            // <g, x[corner]> over the lane's four channels, as two packed pairs
-            float2 pd = __fmul2_rn(make_float2(cv[j][c][0], cv[j][c][1]), g01);
-            pd = __ffma2_rn(make_float2(cv[j][c][2], cv[j][c][3]), g23, pd);
-            dc[c] = pd.x + pd.y;
-            const float wv = m[k] * cw[c];
+            // <g, x[corner]>: the lane's quarter, then the sum over the unit's
+            // quarters in the canonical order (butterfly xor 1, then xor 2)
+            dc[c] = quarter_dot(make_float2(cv[j][c][0], cv[j][c][1]),
+                                make_float2(cv[j][c][2], cv[j][c][3]), g01, g23);
+            if (LANES > 1) dc[c] = quarters_sum<LANES>(dc[c], umask);
+            const float wv = __fmul_rn(m[k], cw[c]);
             const float2 w2 = make_float2(wv, wv);
             gxs.add(size_t(ptrdiff_t(g_off) + cofs[j][c]), __fmul2_rn(w2, g01),
                     __fmul2_rn(w2, g23), cval[j][c]);
           }
           // out-of-support samples have no valid corner: every dc is 0
-          s[k] = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];
-          float gX = hy * (dc[1] - dc[0]) + f[j].ly * (dc[3] - dc[2]);
-          float gY = hx * (dc[2] - dc[0]) + f[j].lx * (dc[3] - dc[1]);
-          if (LANES > 1) {
-            s[k] = unit_sum<LANES>(s[k], umask);
-            gX = unit_sum<LANES>(gX, umask);
-            gY = unit_sum<LANES>(gY, umask);
-          }
+          const TapGrads tg = tap_grads(dc, f[j].ly, f[j].lx);
+          s[k] = tg.s;
           if (sub == 0) {
-            const float sc = t.sigma * m[k];
+            const float sc = __fmul_rn(t.sigma, m[k]);
             if (in_range(unit * KK + k, n_taps))
-              Quad<T>::store_pair(a.goff, unit * KK + k, sc * gX, sc * gY);
+              Quad<T>::store_pair(a.goff, unit * KK + k, __fmul_rn(sc, tg.gx),
+                                  __fmul_rn(sc, tg.gy));
           }
         }
       }
       if (sub == 0) {
-        float ms = 0.f;
-        if (SOFTMAX) {
-#pragma unroll
-          for (int k = 0; k < KKS; ++k) ms = fmaf(m[k], s[k], ms);
-        }
+        const float ms = mask_grad_sum<SOFTMAX>(m, s);
 #pragma unroll
         for (int k = 0; k < KKS; ++k)
           if (in_range(unit * KK + k, n_taps))
-            Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? m[k] * (s[k] - ms) : s[k]);
+            Quad<T>::store_one(a.gmask, unit * KK + k, mask_grad<SOFTMAX>(m[k], s[k], ms));
       }
     } else {
       // Runtime tap count: keep s_k in the tap's staged offset slot, which no
@@ -450,13 +563,13 @@ __global__ void __launch_bounds__(kThreads, 2) dcn_backward_kernel(const BwdArgs
         float ms = 0.f;
         if (SOFTMAX)
           for (int k = 0; k < KK; ++k)
-            ms = fmaf(mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv),
-                      s_at(k), ms);
+            ms = __fmaf_rn(mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv),
+                           s_at(k), ms);
         for (int k = 0; k < KK; ++k) {
           const float sk = s_at(k);
           const float mk = mask_weight_at<T, SOFTMAX>(s_msk, row0 + k, t.P1, u.pix, mx, inv);
           if (in_range(unit * KK + k, n_taps))
-            Quad<T>::store_one(a.gmask, unit * KK + k, SOFTMAX ? mk * (sk - ms) : sk);
+            Quad<T>::store_one(a.gmask, unit * KK + k, mask_grad<SOFTMAX>(mk, sk, ms));
         }
       }
     }

@@ -4,25 +4,25 @@
 // (wmrh.cn), section 二 steps 2-4, differentiated; the DCNv3 extension build
 // guide (trdm.cn), section 2.1, names the backward device code this
 // replaces): per unit (pixel, group) and tap k, with d_c = <g, x[corner c]>
-// over the group's channels and g the unit's upstream gradient,
-//   s_k = sum_c w_c d_c,  grad (dx, dy)_k = offset_scale * m_k * (<g, dv/dX>, <g, dv/dY>),
+// over the group's 16 channels and g the unit's upstream gradient,
+//   s_k = sum_c b_c d_c,  grad (dx, dy)_k = offset_scale * m_k * (<g, dv/dX>, <g, dv/dY>),
+//   <g, dv/dX> = hy (d01 - d00) + ly (d11 - d10),  <g, dv/dY> = hx (d10 - d00) + lx (d11 - d01),
 //   grad logit_k = m_k (s_k - sum_j m_j s_j)  (raw mask: s_k),
-//   grad x[corner c] += m_k w_c g            (float4 reductions).
+//   grad x[corner c] += m_k b_c g            (16-byte vector reductions),
+// b_c the bilinear weights.
 //
-// What changes is where the corners come from.  The direct kernel gathers
-// them through L1 and L2 next to its grad_input reductions; both compete for
-// the same L1 wavefronts and L2 bandwidth.  Here the work items, the TMA box,
-// the producer warp and the bounded mbarrier protocol are those of
-// dcn_forward_tiled_kernel: a persistent CTA walks (image, output tile,
-// group) items and reads the footprints from the group's input box in shared
-// memory.  Phase A (one lane per unit) computes the softmax and, per tap, a
-// record: where corner (y0, x0) sits in the box (or that the corners must be
-// read from global memory), its element offset in the image for the
-// reductions, which corners lie in the image, and the fractional parts.
-// Phase B gives each unit four lanes of four channels: a lane loads its piece
-// of each corner, forms its partial dot products and issues its float4
-// reduction, so one warp instruction still covers a unit's whole 64-byte
-// corner chunk of grad_input.
+// The work items, boxes, zero band, staging and phase A follow
+// dcn_forward_tiled_kernel (clamped boxes, nbuf in flight, structures of
+// arrays).  Phase A stores per tap {ly, lx, m_k, box offset | in-image bits}
+// and the image offset of corner (y0, x0).  Phase B gives each unit four
+// lanes, one per bilinear corner: a lane reads its corner's 16 channels from
+// the box (conflict-free, as in the forward) with the unit's upstream gradient
+// loaded in the same piece order, so d_c is one in-lane dot product; three
+// shuffles bring the four d_c to the unit's first lane, which forms s_k and the
+// offset gradient.  Every lane then scatters its four channels of m_k b_c g
+// into each corner, so one warp instruction covers a corner's whole 64-byte
+// chunk of eight units.  A far tap (footprint outside the box) reads its
+// corner from global memory instead.
 #pragma once
 
 #include "dcn_backward.cuh"
@@ -44,76 +44,114 @@ struct TiledBwdArgs {
   TiledParams t;
 };
 
-// Unit slot of the backward (kSlotBytes, 8-byte aligned): tap k's record at 16*k holds
-// {code, element offset of corner (y0, x0) in the image, lx, ly}; the mask
-// weights m_k follow at kBwdMaskAt.  code bit 31: the corners are read from
-// global memory; bits 24-27: corners (0,0), (0,1), (1,0), (1,1) lie in the
-// image (all clear for a sample that contributes nothing); bits 0-23: byte
-// offset of corner (y0, x0) in the box.
-constexpr int kBwdMaskAt = kTiledMaxTaps * 16;
-static_assert(kBwdMaskAt + kTiledMaxTaps * 4 <= kSlotBytes, "backward slot layout");
-constexpr uint32_t kBwdFar = 0x80000000u;
+// Per-warp region of the backward: R[9][32] float4 {ly, lx, m, box offset |
+// in-image bits << 24} (bit 24 + c: corner c = (dy, dx) = (c >> 1, c & 1) lies
+// in the image; all clear for a tap that contributes nothing), CE[9][32] (element offset of corner (y0, x0) from the
+// image's group base), FM[32] (far taps), PIX[32] (output pixel, ~0 outside).
+// The same size as the forward's region; the staged inputs alias it.
+constexpr int kBwdRegR = 0;
+constexpr int kBwdRegCe = kTiledMaxTaps * kTiledBatch * 16;
+constexpr int kBwdRegFm = kBwdRegCe + kTiledMaxTaps * kTiledBatch * 4;
+constexpr int kBwdRegPix = kBwdRegFm + kTiledBatch * 4;
+static_assert(kBwdRegPix + kTiledBatch * 4 == kFwdRegion, "backward region = forward region");
+constexpr uint32_t kBwdOffMask = 0xFFFFFFu;  // box offset bits of R.w (in-image bits above)
 
-// A lane's four channels of one corner through a generic address (the box in
-// shared memory or the input in global memory); zeros unless `pred`, and a
-// false predicate issues no access.
+// Four channels of the upstream gradient (fp32) from storage type T.
 template <typename T>
-struct BwdPiece;
+struct BwdIO;
 template <>
-struct BwdPiece<float> {
-  __device__ __forceinline__ static void load(const void* p, bool pred, float (&v)[4]) {
-    asm volatile(
-        "{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
-        " mov.b32 %0, 0;\n mov.b32 %1, 0;\n mov.b32 %2, 0;\n mov.b32 %3, 0;\n"
-        " @q ld.v4.f32 {%0, %1, %2, %3}, [%4];\n}"
-        : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-        : "l"(p), "r"(int(pred))
-        : "memory");
-  }
-};
-// The same four channels from the box in shared memory (always in bounds).
-template <typename T>
-struct BoxPiece;
-template <>
-struct BoxPiece<float> {
-  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-                 : "r"(smem_addr(p)));
+struct BwdIO<float> {
+  // 16 bytes = 4 channels; zeros unless pred
+  __device__ __forceinline__ static void quad(const char* p, bool pred, float2& lo, float2& hi) {
+    float v[4];
+    Quad<float>::load_pred(p, pred, v);
+    lo = make_float2(v[0], v[1]);
+    hi = make_float2(v[2], v[3]);
   }
 };
 template <>
-struct BoxPiece<__nv_bfloat16> {
-  __device__ __forceinline__ static void load(const void* p, float (&v)[4]) {
-    uint32_t w0, w1;
-    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(smem_addr(p)));
-    v[0] = bf16lo_to_f32(w0);
-    v[1] = bf16hi_to_f32(w0);
-    v[2] = bf16lo_to_f32(w1);
-    v[3] = bf16hi_to_f32(w1);
-  }
-};
-template <>
-struct BwdPiece<__nv_bfloat16> {
-  __device__ __forceinline__ static void load(const void* p, bool pred, float (&v)[4]) {
-    uint32_t w0, w1;
-    asm volatile(
-        "{\n .reg .pred q;\n setp.ne.b32 q, %3, 0;\n mov.b32 %0, 0;\n mov.b32 %1, 0;\n"
-        " @q ld.v2.b32 {%0, %1}, [%2];\n}"
-        : "=r"(w0), "=r"(w1)
-        : "l"(p), "r"(int(pred))
-        : "memory");
-    v[0] = bf16lo_to_f32(w0);
-    v[1] = bf16hi_to_f32(w0);
-    v[2] = bf16lo_to_f32(w1);
-    v[3] = bf16hi_to_f32(w1);
+struct BwdIO<__nv_bfloat16> {
+  __device__ __forceinline__ static void quad(const char* p, bool pred, float2& lo, float2& hi) {
+    float v[4];
+    Quad<__nv_bfloat16>::load_pred(p, pred, v);
+    lo = make_float2(v[0], v[1]);
+    hi = make_float2(v[2], v[3]);
   }
 };
 
-// KKS: 9 (the 3x3 window) or 8 (the window without its centre).  CS = the
-// group's bytes per pixel = 16 channels.  DET: exact fixed-point accumulation
-// of grad_input (GxScatter).
-template <typename T, int CS, int KKS, bool SOFTMAX, bool DET>
+template <>
+struct BwdIO<__half> {
+  __device__ __forceinline__ static void quad(const char* p, bool pred, float2& lo, float2& hi) {
+    float v[4];
+    Quad<__half>::load_pred(p, pred, v);
+    lo = make_float2(v[0], v[1]);
+    hi = make_float2(v[2], v[3]);
+  }
+};
+
+// Dot product of a 16-byte piece (storage type T) with the matching gradient
+// channels, in the canonical order of quarter_dot: the sum of the piece's
+// quarters (one for fp32, two for 2-byte types, added pairwise).
+template <typename T>
+__device__ __forceinline__ float piece_dot(const uint4& v, const float2* g);
+template <>
+__device__ __forceinline__ float piece_dot<float>(const uint4& v, const float2* g) {
+  return quarter_dot(make_float2(__uint_as_float(v.x), __uint_as_float(v.y)),
+                     make_float2(__uint_as_float(v.z), __uint_as_float(v.w)), g[0], g[1]);
+}
+template <>
+__device__ __forceinline__ float piece_dot<__nv_bfloat16>(const uint4& v, const float2* g) {
+  const float q0 = quarter_dot(make_float2(bf16lo_to_f32(v.x), bf16hi_to_f32(v.x)),
+                               make_float2(bf16lo_to_f32(v.y), bf16hi_to_f32(v.y)), g[0], g[1]);
+  const float q1 = quarter_dot(make_float2(bf16lo_to_f32(v.z), bf16hi_to_f32(v.z)),
+                               make_float2(bf16lo_to_f32(v.w), bf16hi_to_f32(v.w)), g[2], g[3]);
+  return __fadd_rn(q0, q1);
+}
+
+template <>
+__device__ __forceinline__ float piece_dot<__half>(const uint4& v, const float2* g) {
+  const float q0 = quarter_dot(f16x2_to_f32x2(v.x), f16x2_to_f32x2(v.y), g[0], g[1]);
+  const float q1 = quarter_dot(f16x2_to_f32x2(v.z), f16x2_to_f32x2(v.w), g[2], g[3]);
+  return __fadd_rn(q0, q1);
+}
+
+// Sum of a lane's pieces in the canonical order: (p0 + p1) for two pieces,
+// (p0 + p1) + (p2 + p3) for four; the lane's slot order (piece j ^ rot) only
+// swaps the operands of these pairwise sums.
+template <int NP>
+__device__ __forceinline__ float pieces_sum(const float (&p)[NP]) {
+  if constexpr (NP == 2) return __fadd_rn(p[0], p[1]);
+  else return __fadd_rn(__fadd_rn(p[0], p[1]), __fadd_rn(p[2], p[3]));
+}
+
+// 16 bytes of storage type T (a piece of the upstream gradient) -> fp32 pairs.
+template <typename T>
+__device__ __forceinline__ void piece_widen(const uint4& v, float2* g);
+template <>
+__device__ __forceinline__ void piece_widen<float>(const uint4& v, float2* g) {
+  g[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+  g[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+template <>
+__device__ __forceinline__ void piece_widen<__nv_bfloat16>(const uint4& v, float2* g) {
+  g[0] = make_float2(bf16lo_to_f32(v.x), bf16hi_to_f32(v.x));
+  g[1] = make_float2(bf16lo_to_f32(v.y), bf16hi_to_f32(v.y));
+  g[2] = make_float2(bf16lo_to_f32(v.z), bf16hi_to_f32(v.z));
+  g[3] = make_float2(bf16lo_to_f32(v.w), bf16hi_to_f32(v.w));
+}
+
+template <>
+__device__ __forceinline__ void piece_widen<__half>(const uint4& v, float2* g) {
+  g[0] = f16x2_to_f32x2(v.x);
+  g[1] = f16x2_to_f32x2(v.y);
+  g[2] = f16x2_to_f32x2(v.z);
+  g[3] = f16x2_to_f32x2(v.w);
+}
+
+// KKS: 9 (the 3x3 window) or 8 (the window without its centre).  DET: exact
+// fixed-point accumulation of grad_input (GxScatter).  FAR: some footprint can
+// leave the box.
+template <typename T, int KKS, bool SOFTMAX, bool DET, bool FAR>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     dcn_backward_tiled_kernel(const __grid_constant__ CUtensorMap xmap, const TiledBwdArgs a) {
   using IO = TiledIO<T>;
@@ -121,72 +159,83 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   using One = typename IO::One;
   constexpr int KK = KKS, K = tap_side(KKS);
   static_assert(K == 3 && KK <= kTiledMaxTaps, "the tiled kernel serves 3x3 tap sets");
-  static_assert(CS == 16 * int(sizeof(T)), "16 channels per group");
-  constexpr int LU = 4;          // phase-B lanes per unit, four channels each
-  constexpr int UPW = 32 / LU;   // units per phase-B step
-  constexpr int PB = 4 * int(sizeof(T));  // bytes of a lane's piece of one corner
-  static_assert(KK * sizeof(Pair) <= kLogitAt && kLogitAt + KK * sizeof(One) <= kSlotBytes,
-                "staged inputs fit in a slot");
+  constexpr int CS = 16 * int(sizeof(T));  // bytes of one pixel of the group
+  constexpr int NP = CS / 16;              // 16-byte pieces per corner
+  constexpr int GP = 8 / NP;               // gradient pairs per piece
 
   const TiledParams& t = a.t;
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* bufs = smem;
-  unsigned char* slots = smem + 2 * size_t(t.box_stride);
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(slots + size_t(kTiledWarps) * kTiledBatch * kSlotBytes);
-  uint64_t* empty = full + 2;
-  int* s_abort = reinterpret_cast<int*>(empty + 2);
+  const int nbuf = t.nbuf;
+  unsigned char* const bufs = smem;
+  unsigned char* const zero = smem + size_t(nbuf) * t.box_stride;
+  unsigned char* const regions = zero + zero_band_bytes(t.BW, CS);
+  uint64_t* const full = reinterpret_cast<uint64_t*>(regions + size_t(kTiledWarps) * kFwdRegion);
+  uint64_t* const empty = full + kTiledMaxBufs;
+  int* const s_abort = reinterpret_cast<int*>(empty + kTiledMaxBufs);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(&empty[0], kTiledWarps);
-    mbar_init(&empty[1], kTiledWarps);
+    for (int i = 0; i < nbuf; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kTiledWarps);
+    }
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int i = tid; i < zero_band_bytes(t.BW, CS) / 16; i += kTiledThreads)
+    reinterpret_cast<uint4*>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   volatile int* abort_flag = s_abort;
 
-  // ---- producer warp: one TMA box per item, two buffers in flight ----
+  // ---- producer warp: one TMA box per item, nbuf buffers in flight ----
   if (warp == kTiledWarps) {
     if (lane != 0) return;
-    int i = 0;
+    int i = 0, b = 0;
+    uint32_t ph = 0;
     for (;; ++i) {
       const int item = int(blockIdx.x) + i * int(gridDim.x);
       if (item >= t.items || *abort_flag) break;
-      const int b = i & 1;
-      if (i >= 2 && !mbar_wait_bounded(&empty[b], ((i >> 1) - 1) & 1)) {
-        atomicOr(a.error_word, 1u);
+      if (i >= nbuf && !mbar_wait_bounded(&empty[b], ph ^ 1u)) {
+        atomicOr(a.error_word, kErrTimeout);
         *abort_flag = 1;
         break;
       }
       const ItemCoord c = item_coord(t, item);
-      if (t.inject_stall && i == 0) continue;  // the first box never arrives
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&full[b], t.box_bytes);
-      tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg,
-                   c.wo0 * t.stride_w - t.pad_w - t.halo, c.ho0 * t.stride - t.pad - t.halo, c.n);
+      if (!(t.inject_stall && i == 0)) {  // test knob: the first box never arrives
+        const int Y0 = box_origin(c.ho0 * t.stride - t.pad - t.halo, t.BH, t.H, t.clamp_box);
+        const int X0 = box_origin(c.wo0 * t.stride_w - t.pad_w - t.halo, t.BW, t.W, t.clamp_box);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&full[b], t.box_bytes);
+        tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg, X0, Y0, c.n);
+      }
+      if (++b == nbuf) {
+        b = 0;
+        ph ^= 1u;
+      }
     }
-    // Copies issued for items i-2 and i-1 may still be landing: wait for them
-    // (bounded) before this thread, possibly the CTA's last, exits.
-    for (int j = i - 2; j < i; ++j)
-      if (j >= 0) (void)mbar_wait_bounded(&full[j & 1], (j >> 1) & 1);
+    for (int j = i - nbuf < 0 ? 0 : i - nbuf; j < i; ++j)
+      if (!(t.inject_stall && j == 0))
+        (void)mbar_wait_bounded(&full[j % nbuf], uint32_t(j / nbuf) & 1u);
     return;
   }
 
   // ---- consumer warps ----
-  unsigned char* myslots = slots + size_t(warp) * kTiledBatch * kSlotBytes;
-  const int ul = lane / LU;  // phase B: unit of this lane within a step
-  const int sub = lane - ul * LU;
-  const unsigned umask = 0xFu << (ul * LU);
-  const int pixE = t.C;            // elements between horizontally adjacent pixels
-  const int rowE = t.W * t.C;      // ... vertically adjacent pixels
-  const int cofs[4] = {0, pixE, rowE, rowE + pixE};  // corner (dy, dx) from corner (0, 0)
+  unsigned char* const reg = regions + size_t(warp) * kFwdRegion;
+  const uint32_t reg_a = smem_addr(reg);
+  const uint32_t zero_a = smem_addr(zero);
+  const int u8 = lane >> 2, r = lane & 3, dy = r >> 1, dx = r & 1, rho = u8 & 1;
+  const int rot = NP == 2 ? rho : 2 * dy + rho;  // piece j ^ rot in read j (as the forward)
+  const uint32_t corner_b = uint32_t((dy * t.BW + dx) * CS + 16 * rot);
+  const int ulead = lane & ~3;  // the unit's first lane
   const int npx = t.TH * t.TW;
   const int nb = t.batches;
-  // the staging element e = lane + 32 k (k < KK) belongs to unit e / KK, tap e % KK
+  const float Hf = float(t.H), Wf = float(t.W);
+  const int pixE = t.C, rowE = t.W * t.C;  // element steps to the next pixel / row
+  const int cofs_r = dy * rowE + dx * pixE;  // this lane's corner from corner (y0, x0)
+  const size_t n_img = size_t(t.N) * t.H * t.W * t.C;  // accumulator elements
+  const size_t x_bytes = n_img * sizeof(T);
+  const size_t n_out = size_t(t.N) * t.Ho * t.Wo * t.C;
+  const size_t n_taps = size_t(t.N) * t.Ho * t.Wo * t.G * KK;
   int st_unit[KK], st_tap[KK];
 #pragma unroll
   for (int k = 0; k < KK; ++k) {
@@ -194,45 +243,32 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     st_tap[k] = (lane + 32 * k) - st_unit[k] * KK;
   }
 
-  // Batch beta of this CTA (over all its items) -> this lane's unit.
-  auto batch_unit = [&](int beta, bool& valid, int& ho, int& wo, size_t& qbase) {
+  auto batch_unit = [&](int beta, int& ho, int& wo, uint32_t& q) {
     const int il = beta / nb;
     const int v = (beta - il * nb) * kTiledBatch + lane;
-    const int item = int(blockIdx.x) + il * int(gridDim.x);
-    valid = false;
-    ho = wo = 0;
-    qbase = 0;
-    if (item >= t.items) return;
-    const ItemCoord c = item_coord(t, item);
+    const ItemCoord c = item_coord(t, int(blockIdx.x) + il * int(gridDim.x));
     const int rr = int(fdiv(uint32_t(v), t.fd_TW));
     ho = c.ho0 + rr;
     wo = c.wo0 + (v - rr * t.TW);
-    valid = (v < npx) && (ho < t.Ho) && (wo < t.Wo);
-    qbase = ((size_t(c.n * t.Ho + ho) * t.Wo + wo) * t.G + c.g) * KK;
+    const bool valid = (v < npx) && (ho < t.Ho) && (wo < t.Wo);
+    q = valid ? (uint32_t((c.n * t.Ho + ho) * t.Wo + wo) * uint32_t(t.G) + uint32_t(c.g)) *
+                    uint32_t(KK)
+              : ~0u;
+    return c;
   };
 
-  // Raw inputs of the next batch, prefetched in the staging layout.
-  const size_t n_taps = size_t(t.N) * t.Ho * t.Wo * t.G * KK;  // offset pairs, mask values
-  const size_t n_img = size_t(t.N) * t.H * t.W * t.C;           // input, accumulator elements
-  const size_t n_out = size_t(t.N) * t.Ho * t.Wo * t.C;
   Pair pf_pair[KK];
   One pf_one[KK];
   auto prefetch = [&](int beta) {
-    bool valid;
     int ho, wo;
-    size_t qbase;
-    batch_unit(beta, valid, ho, wo, qbase);
-    const unsigned long long qv = valid ? (unsigned long long)qbase : ~0ull;
+    uint32_t q;
+    batch_unit(beta, ho, wo, q);
 #pragma unroll
     for (int k = 0; k < KK; ++k) {
-      const unsigned long long src = __shfl_sync(0xFFFFFFFFu, qv, st_unit[k]);
-      if (src != ~0ull && in_range(size_t(src) + st_tap[k], n_taps)) {
-        pf_pair[k] = IO::ld_pair(a.off, size_t(src) + st_tap[k]);
-        pf_one[k] = IO::ld_one(a.mask, size_t(src) + st_tap[k]);
-      } else {
-        pf_pair[k] = Pair();
-        pf_one[k] = One();
-      }
+      const uint32_t src = __shfl_sync(0xFFFFFFFFu, q, st_unit[k]);
+      const bool ok = src != ~0u && in_range(size_t(src) + st_tap[k], n_taps);
+      pf_pair[k] = ok ? IO::ld_pair(a.off, size_t(src) + st_tap[k]) : Pair();
+      pf_one[k] = ok ? IO::ld_one(a.mask, size_t(src) + st_tap[k]) : One();
     }
   };
 
@@ -242,47 +278,54 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   int beta = warp;
   if (beta < total_batches) prefetch(beta);
 
+  int b = 0;
+  uint32_t ph = 0;
   for (int il = 0; il < n_items_cta; ++il) {
-    const int b = il & 1;
-    const int item = int(blockIdx.x) + il * int(gridDim.x);
-    // Every consumer warp observes every item's box (see the forward kernel).
-    if (!mbar_wait_bounded(&full[b], (il >> 1) & 1)) {
-      atomicOr(a.error_word, 1u);
+    if (!mbar_wait_bounded_sleep(&full[b], ph)) {
+      atomicOr(a.error_word, kErrTimeout);
       *abort_flag = 1;
     }
     if (*abort_flag) break;
-    const ItemCoord c = item_coord(t, item);
-    const unsigned char* box_lane = bufs + size_t(b) * t.box_stride + sub * PB;
-    const int Y0 = c.ho0 * t.stride - t.pad - t.halo;
-    const int X0 = c.wo0 * t.stride_w - t.pad_w - t.halo;
-    const size_t img = size_t(c.n) * t.H * t.W * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4;
-    const char* xg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
+    const ItemCoord c = item_coord(t, int(blockIdx.x) + il * int(gridDim.x));
+    const uint32_t box_a = smem_addr(bufs + size_t(b) * t.box_stride);
+    const uint32_t lane_base = box_a + corner_b;
+    const uint32_t zoff = zero_a - box_a;
+    const int Y0 = box_origin(c.ho0 * t.stride - t.pad - t.halo, t.BH, t.H, t.clamp_box);
+    const int X0 = box_origin(c.wo0 * t.stride_w - t.pad_w - t.halo, t.BW, t.W, t.clamp_box);
+    // element offset of the item's image and group: the base of CE
+    const size_t img = size_t(c.n) * t.H * t.W * t.C + size_t(c.g) * t.Cg;
+    const char* const ximg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
     const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits, n_img);
-    typename GxScatter<DET>::Acc* const gx_item = gxs.p + img;
+    // this lane's first accumulator channel of corner (y0, x0) at CE = 0
+    typename GxScatter<DET>::Acc* const gx_lane = gxs.p + img + (DET ? r : 4 * r);
 
     for (; beta < (il + 1) * nb; beta += kTiledWarps) {
-      // Staging: the prefetched inputs go to the unit slots.
 #pragma unroll
       for (int k = 0; k < KK; ++k) {
-        unsigned char* sl = myslots + st_unit[k] * kSlotBytes;
-        reinterpret_cast<Pair*>(sl)[st_tap[k]] = pf_pair[k];
-        reinterpret_cast<One*>(sl + kLogitAt)[st_tap[k]] = pf_one[k];
+        const int e = lane + 32 * k;
+        if (sizeof(T) == 4)
+          reinterpret_cast<Pair*>(reg)[e] = pf_pair[k];
+        else
+          reinterpret_cast<uint32_t*>(reg)[e] = *reinterpret_cast<const uint32_t*>(&pf_pair[k]);
+        reinterpret_cast<float*>(reg + kFwdStageMask)[e] = IO::one(pf_one[k]);
       }
-      bool valid;
       int ho, wo;
-      size_t qbase;
-      batch_unit(beta, valid, ho, wo, qbase);
+      uint32_t q;
+      batch_unit(beta, ho, wo, q);
+      const bool valid = q != ~0u;
       __syncwarp();
 
       // Phase A: this lane's unit -> mask weights and the tap records.
       {
-        unsigned char* sl = myslots + lane * kSlotBytes;
         float2 d[KK];
         float m[KK];
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          d[k] = IO::pair(reinterpret_cast<const Pair*>(sl)[k]);
-          m[k] = IO::one(reinterpret_cast<const One*>(sl + kLogitAt)[k]);
+          const int e = lane * KK + k;
+          d[k] = sizeof(T) == 4
+                     ? IO::pair(reinterpret_cast<const Pair*>(reg)[e])
+                     : IO::pair(*reinterpret_cast<const Pair*>(reg + 4 * e));
+          m[k] = reinterpret_cast<const float*>(reg + kFwdStageMask)[e];
         }
         if (SOFTMAX) {
           float mx = m[0];
@@ -298,141 +341,156 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
           for (int k = 0; k < KK; ++k) m[k] *= inv;
         }
-        __syncwarp();  // every lane has read its staged inputs
+        __syncwarp();
+        const int yb = ho * t.stride - t.pad, xb = wo * t.stride_w - t.pad_w;
+        uint32_t fm = 0u;
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          const int q = tap_pos(KK, k);
-          const float Y = tap_coord(ho * t.stride - t.pad + (q / K) * t.dil, t.sigma, d[k].y);
-          const float X =
-              tap_coord(wo * t.stride_w - t.pad_w + (q % K) * t.dil_w, t.sigma, d[k].x);
-          const Footprint f = footprint(Y, X, t.H, t.W);
-          const bool live = valid && f.in_support;
-          // a sample that contributes nothing keeps code 0: box offset 0, no corner
-          uint32_t code = 0;
-          int ce = 0;
-          if (live) {
-            code = (uint32_t(f.v00) | uint32_t(f.v01) << 1 | uint32_t(f.v10) << 2 |
-                    uint32_t(f.v11) << 3)
-                   << 24;
-            const int by = f.y0 - Y0, bx = f.x0 - X0;
-            if (by >= 0 && by + 1 < t.BH && bx >= 0 && bx + 1 < t.BW)
-              code |= uint32_t((by * t.BW + bx) * CS);
-            else
-              code |= kBwdFar;
-            ce = f.y0 * rowE + f.x0 * pixE;
-          }
-          // slots are 8-byte aligned (184-byte stride): two 8-byte stores
-          reinterpret_cast<uint2*>(sl + 16 * k)[0] = make_uint2(code, uint32_t(ce));
-          reinterpret_cast<uint2*>(sl + 16 * k)[1] =
-              make_uint2(__float_as_uint(f.lx), __float_as_uint(f.ly));
-          reinterpret_cast<float*>(sl + kBwdMaskAt)[k] = m[k];
+          const int ka = tap_pos(KK, k) / K, kb = tap_pos(KK, k) % K;
+          const float Y = tap_coord(yb + ka * t.dil, t.sigma, d[k].y);
+          const float X = tap_coord(xb + kb * t.dil_w, t.sigma, d[k].x);
+          const float fy = floorf(Y), fx = floorf(X);
+          const int y0 = __float2int_rd(Y), x0 = __float2int_rd(X);
+          const int by = y0 - Y0, bx = x0 - X0;
+          const bool inbox = unsigned(by) < unsigned(t.BH - 1) && unsigned(bx) < unsigned(t.BW - 1);
+          // -1 <= Y < H and -1 <= X < W (NaN fails): the sample has a corner in the image
+          const bool live = valid && (Y >= -1.0f) && (Y < Hf) && (X >= -1.0f) && (X < Wf);
+          const bool box_tap = live && inbox;
+          const bool far = FAR && live && !inbox;
+          const uint32_t inb = live ? (uint32_t(y0 >= 0 && x0 >= 0) |
+                                       uint32_t(y0 >= 0 && x0 + 1 < t.W) << 1 |
+                                       uint32_t(y0 + 1 < t.H && x0 >= 0) << 2 |
+                                       uint32_t(y0 + 1 < t.H && x0 + 1 < t.W) << 3)
+                                    : 0u;
+          const uint32_t off = box_tap ? uint32_t((by * t.BW + bx) * CS) : zoff;
+          reinterpret_cast<float4*>(reg + kBwdRegR)[k * kTiledBatch + lane] =
+              make_float4(live ? Y - fy : 0.f, live ? X - fx : 0.f, m[k],
+                          __uint_as_float(off | (inb << 24)));
+          reinterpret_cast<int*>(reg + kBwdRegCe)[k * kTiledBatch + lane] =
+              live ? y0 * rowE + x0 * pixE : 0;
+          fm |= far ? (1u << k) : 0u;
         }
+        reinterpret_cast<uint32_t*>(reg + kBwdRegFm)[lane] = fm;
+        reinterpret_cast<uint32_t*>(reg + kBwdRegPix)[lane] =
+            valid ? uint32_t((c.n * t.Ho + ho) * t.Wo + wo) : ~0u;
       }
       __syncwarp();
-      // The next batch's inputs are loaded while this one is processed.
       if (beta + kTiledWarps < total_batches) prefetch(beta + kTiledWarps);
 
-      // Phase B: UPW units per step, LU lanes of four channels each.
-      const int v0 = (beta - il * nb) * kTiledBatch;
+      // Phase B: 8 units per step, one lane per corner.
 #pragma unroll 1
-      for (int s = 0; s < kTiledBatch / UPW; ++s) {
-        const int u = s * UPW + ul;
-        const unsigned char* sl = myslots + u * kSlotBytes;
-        const int v = v0 + u;
-        const int rr = int(fdiv(uint32_t(v), t.fd_TW));
-        const int uho = c.ho0 + rr, uwo = c.wo0 + (v - rr * t.TW);
-        const bool uvalid = v < npx && uho < t.Ho && uwo < t.Wo;
-        const size_t pix = size_t(c.n * t.Ho + uho) * t.Wo + uwo;
-        const size_t unit = pix * t.G + c.g;
-        // grad_offset pairs of this unit, written by its first lane without a branch
-        char* const goff_u = reinterpret_cast<char*>(a.goff) + unit * KK * sizeof(Pair);
-        const uint32_t st_ok = (sub == 0 && uvalid) ? 1u : 0u;
-        float go[4];
-        Quad<T>::load_pred(reinterpret_cast<const char*>(a.gout) +
-                               (pix * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4) * sizeof(T),
-                           uvalid && in_range(pix * t.C + size_t(c.g) * t.Cg + size_t(sub) * 4 + 3,
-                                              n_out),
-                           go);
-        const float2 g01 = make_float2(go[0], go[1]), g23 = make_float2(go[2], go[3]);
+      for (int s = 0; s < kTiledBatch / 8; ++s) {
+        const int u = s * 8 + u8;
+        uint32_t pix, fm;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(pix) : "r"(reg_a + kBwdRegPix + 4u * u));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(fm) : "r"(reg_a + kBwdRegFm + 4u * u));
+        const bool uvalid = pix != ~0u;
+        const size_t ob = size_t(uvalid ? pix : 0u) * t.C + size_t(c.g) * t.Cg;  // output element
+        // upstream gradient: all 16 channels in this lane's piece order, and this
+        // lane's four scatter channels
+        const char* const gp = reinterpret_cast<const char*>(a.gout) + ob * sizeof(T);
+        const bool gok = uvalid && in_range(ob + 15, n_out);
+        float2 gs[8];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) piece_widen<T>(ldg128_pred(gp + 16 * (j ^ rot), gok), gs + j * GP);
+        // scatter channels of this lane: 4r .. 4r+3 (fp32 vector reductions), or
+        // r, r+4, r+8, r+12 (fixed point: one 32-byte sector per instruction)
+        float2 gr_lo, gr_hi;
+        if (DET) {
+          float v[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = gok ? Storage<T>::to_float(reinterpret_cast<const T*>(gp)[r + 4 * i]) : 0.f;
+          gr_lo = make_float2(v[0], v[1]);
+          gr_hi = make_float2(v[2], v[3]);
+        } else {
+          BwdIO<T>::quad(gp + 4 * r * sizeof(T), gok, gr_lo, gr_hi);
+        }
+        char* const goff_u = reinterpret_cast<char*>(a.goff) +
+                             (size_t(uvalid ? pix : 0u) * t.G + c.g) * KK * sizeof(Pair);
+        const uint32_t lead_ok = (r == 0 && uvalid) ? 1u : 0u;
+        const uint32_t ra = reg_a + kBwdRegR + uint32_t(u) * 16u;
+        const uint32_t ca = reg_a + kBwdRegCe + uint32_t(u) * 4u;
         float sk[KK];
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          const uint2 r0 = reinterpret_cast<const uint2*>(sl + 16 * k)[0];
-          const uint2 r1 = reinterpret_cast<const uint2*>(sl + 16 * k)[1];
-          const float mk = reinterpret_cast<const float*>(sl + kBwdMaskAt)[k];
-          const uint32_t code = r0.x;
-          const int ce = int(r0.y);
-          const float lx = __uint_as_float(r1.x), ly = __uint_as_float(r1.y);
-          const bool far = (code & kBwdFar) != 0u;
-          const unsigned char* bp = box_lane + (code & 0xFFFFFFu);
-          const float hy = 1.f - ly, hx = 1.f - lx;
-          const float cw[4] = {hy * hx, hy * lx, ly * hx, ly * lx};
-          float cv[4][4];
-          if (__any_sync(0xFFFFFFFFu, far)) {
-            // some footprint of this step lies outside the box: box or global
-            // memory per lane through a generic address, predicated per corner
+          const uint4 rw = lds128_a(ra + k * kTiledBatch * 16);
+          int ce;
+          asm volatile("ld.shared.s32 %0, [%1];" : "=r"(ce) : "r"(ca + k * kTiledBatch * 4));
+          const float lx = __uint_as_float(rw.y), ly = __uint_as_float(rw.x);
+          const float m = __uint_as_float(rw.z);
+          const uint32_t inb = rw.w >> 24;
+          const uint32_t a0 = lane_base + (rw.w & kBwdOffMask);
+          float pp[NP];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              const int dy = cc >> 1, dx = cc & 1;
-              const bool in = ((code >> (24 + cc)) & 1u) != 0u;
-              const int e = ce + dy * rowE + dx * pixE;
-              const void* src =
-                  far ? static_cast<const void*>(xg + ptrdiff_t(e) * ptrdiff_t(sizeof(T)))
-                      : static_cast<const void*>(bp + (dy * t.BW + dx) * CS);
-              BwdPiece<T>::load(src,
-                                in && (!far || in_range(img + size_t(e) + 3, n_img)), cv[cc]);
+          for (int j = 0; j < NP; ++j) pp[j] = piece_dot<T>(lds128_a(a0 ^ uint32_t(16 * j)), gs + j * GP);
+          if (FAR && __any_sync(0xFFFFFFFFu, (fm >> k) & 1u)) {
+            if ((fm >> k) & 1u) {
+              // this corner from global memory (zero outside the image)
+              const bool in = (inb >> r) & 1u;
+              const char* xp = ximg + ptrdiff_t(ce + cofs_r) * ptrdiff_t(sizeof(T));
+#pragma unroll
+              for (int j = 0; j < NP; ++j) {
+                const char* q = xp + 16 * (j ^ rot);
+                pp[j] = piece_dot<T>(ldg128_pred(q, in && in_tensor(q, 16, a.x, x_bytes)),
+                                     gs + j * GP);
+              }
             }
-          } else {
-            // every footprint is in the box: plain shared loads (corners outside
-            // the image read the box's zero fill, and dc is masked below anyway)
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              BoxPiece<T>::load(bp + ((cc >> 1) * t.BW + (cc & 1)) * CS, cv[cc]);
           }
-          float dc[4];
-          auto* const p00 = gx_item + ce;  // accumulator at corner (y0, x0)
+          const float dc = pieces_sum<NP>(pp);
+          // corner products d00, d01, d10, d11 at the unit's first lane
+          const float d0 = __shfl_sync(0xFFFFFFFFu, dc, ulead);
+          const float d1 = __shfl_sync(0xFFFFFFFFu, dc, ulead + 1);
+          const float d2 = __shfl_sync(0xFFFFFFFFu, dc, ulead + 2);
+          const float d3 = __shfl_sync(0xFFFFFFFFu, dc, ulead + 3);
+          const float dd[4] = {d0, d1, d2, d3};
+          const TapGrads tg = tap_grads(dd, ly, lx);
+          sk[k] = tg.s;
+          const float sm = __fmul_rn(t.sigma, m);
+          Quad<T>::store_pair_pred(goff_u + k * sizeof(Pair), __fmul_rn(sm, tg.gx),
+                                   __fmul_rn(sm, tg.gy),
+                                   (lead_ok != 0u && in_range((size_t(pix) * t.G + c.g) * KK + k,
+                                                              n_taps))
+                                       ? 1u
+                                       : 0u);
+          // grad_input: this lane's four channels of m b_c g into each corner
+          float bw[4];
+          bilinear_weights(ly, lx, bw);
+          const float wc[4] = {__fmul_rn(m, bw[0]), __fmul_rn(m, bw[1]), __fmul_rn(m, bw[2]),
+                               __fmul_rn(m, bw[3])};
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
-            const uint32_t inb = code & (1u << (24 + cc));  // corner in the image
-            float2 pd = __fmul2_rn(make_float2(cv[cc][0], cv[cc][1]), g01);
-            pd = __ffma2_rn(make_float2(cv[cc][2], cv[cc][3]), g23, pd);
-            dc[cc] = inb ? pd.x + pd.y : 0.f;
-            const float wv = mk * cw[cc];
-            const float2 w2 = make_float2(wv, wv);
-            gxs.add_at(p00 + cofs[cc], kCheckBounds ? img + size_t(ce + cofs[cc]) : 0,
-                       __fmul2_rn(w2, g01), __fmul2_rn(w2, g23), inb);
+            const int e = ce + (cc >> 1) * rowE + (cc & 1) * pixE;
+            const float2 w2 = make_float2(wc[cc], wc[cc]);
+            if constexpr (DET)
+              gxs.add4_strided(gx_lane + e,
+                               kCheckBounds ? img + size_t(r) + size_t(ptrdiff_t(e)) : 0,
+                               __fmul2_rn(w2, gr_lo), __fmul2_rn(w2, gr_hi), (inb >> cc) & 1u);
+            else
+              gxs.add_at(gx_lane + e,
+                         kCheckBounds ? img + size_t(4 * r) + size_t(ptrdiff_t(e)) : 0,
+                         __fmul2_rn(w2, gr_lo), __fmul2_rn(w2, gr_hi), (inb >> cc) & 1u);
           }
-          // a sample that contributes nothing has no corner in the image: every dc is 0
-          float sv = cw[0] * dc[0] + cw[1] * dc[1] + cw[2] * dc[2] + cw[3] * dc[3];
-          float gX = hy * (dc[1] - dc[0]) + ly * (dc[3] - dc[2]);
-          float gY = hx * (dc[2] - dc[0]) + lx * (dc[3] - dc[1]);
-          sv = unit_sum<LU>(sv, umask);
-          gX = unit_sum<LU>(gX, umask);
-          gY = unit_sum<LU>(gY, umask);
-          sk[k] = sv;
-          const float sc = t.sigma * mk;
-          Quad<T>::store_pair_pred(goff_u + k * sizeof(Pair), sc * gX, sc * gY,
-                                   (st_ok != 0u && in_range(unit * KK + k, n_taps)) ? 1u : 0u);
         }
-        if (sub == 0 && uvalid) {
-          const float* ms_ = reinterpret_cast<const float*>(sl + kBwdMaskAt);
-          float msum = 0.f;
-          if (SOFTMAX) {
-#pragma unroll
-            for (int k = 0; k < KK; ++k) msum = fmaf(ms_[k], sk[k], msum);
-          }
+        if (lead_ok) {
+          const size_t q0 = (size_t(pix) * t.G + c.g) * KK;
+          float mk[KK];  // the mask weights, read back from the records
 #pragma unroll
           for (int k = 0; k < KK; ++k)
-            if (in_range(unit * KK + k, n_taps)) Quad<T>::store_one(a.gmask, unit * KK + k,
-                               SOFTMAX ? ms_[k] * (sk[k] - msum) : sk[k]);
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(mk[k]) : "r"(ra + k * kTiledBatch * 16 + 8));
+          const float msum = mask_grad_sum<SOFTMAX>(mk, sk);
+#pragma unroll
+          for (int k = 0; k < KK; ++k)
+            if (in_range(q0 + k, n_taps))
+              Quad<T>::store_one(a.gmask, q0 + k, mask_grad<SOFTMAX>(mk[k], sk[k], msum));
         }
       }
-      __syncwarp();  // slots are rewritten by the next batch
+      __syncwarp();
     }
     __syncwarp();
-    if (lane == 0) {
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&empty[b]))
-                   : "memory");
+    if (lane == 0) mbar_arrive(&empty[b]);
+    if (++b == nbuf) {
+      b = 0;
+      ph ^= 1u;
     }
   }
 }

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace dcn {
@@ -88,6 +89,23 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// fp16 storage: widened to fp32 exactly (every fp16 value is an fp32 value);
+// fp32 -> fp16 rounds to nearest even (overflow to +-inf, as the conversion
+// defines).
+__device__ __forceinline__ float f16lo_to_f32(uint32_t w) {
+  return __low2float(*reinterpret_cast<const __half2*>(&w));
+}
+__device__ __forceinline__ float f16hi_to_f32(uint32_t w) {
+  return __high2float(*reinterpret_cast<const __half2*>(&w));
+}
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);  // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 // Read-only gathers of 16 or 32 bytes through the non-coherent path.
 template <int BYTES>
 struct Vec;
@@ -141,6 +159,25 @@ struct Storage<float> {
   __device__ __forceinline__ static void pack(uint32_t (&w)[N], const float* acc) {
 #pragma unroll
     for (int j = 0; j < N; ++j) w[j] = __float_as_uint(acc[j]);
+  }
+};
+
+template <>
+struct Storage<__half> {
+  static constexpr int kSize = 2;
+  __device__ __forceinline__ static float to_float(__half v) { return __half2float(v); }
+  // round to nearest even
+  __device__ __forceinline__ static void store_float(__half* p, float v) {
+    *p = __float2half_rn(v);
+  }
+  template <int N>
+  __device__ __forceinline__ static float chan(const uint32_t (&w)[N], int j) {
+    return (j & 1) ? f16hi_to_f32(w[j >> 1]) : f16lo_to_f32(w[j >> 1]);
+  }
+  template <int N>
+  __device__ __forceinline__ static void pack(uint32_t (&w)[N], const float* acc) {
+#pragma unroll
+    for (int j = 0; j < N; ++j) w[j] = pack_f16x2(acc[2 * j], acc[2 * j + 1]);
   }
 };
 

@@ -35,7 +35,17 @@ int64_t out_extent(int in, int K, int stride, int pad, int dil) {
   return span / stride + 1;
 }
 
-int esize(dcn_dtype d) { return d == DCN_BF16 ? 2 : 4; }
+int esize(dcn_dtype d) { return d == DCN_F32 ? 4 : 2; }
+
+// Calls f with a value of the storage type of d (fp32, bf16 or fp16).
+template <typename F>
+auto with_storage(dcn_dtype d, F&& f) {
+  switch (d) {
+    case DCN_BF16: return f(__nv_bfloat16());
+    case DCN_F16: return f(__half());
+    default: return f(float());
+  }
+}
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -65,7 +75,8 @@ dcn_status check_problem(const dcn_problem* p, int64_t* Ho, int64_t* Wo) {
   if (p->softmax != 0 && p->softmax != 1) return DCN_ERR_INVALID_ARG;
   if (p->remove_center != 0 && p->remove_center != 1) return DCN_ERR_INVALID_ARG;
   if (p->remove_center && p->K < 3) return DCN_ERR_INVALID_ARG;  // no tap would be left
-  if (p->dtype != DCN_F32 && p->dtype != DCN_BF16) return DCN_ERR_INVALID_ARG;
+  if (p->dtype != DCN_F32 && p->dtype != DCN_BF16 && p->dtype != DCN_F16)
+    return DCN_ERR_INVALID_ARG;
   if (!(p->offset_scale == p->offset_scale)) return DCN_ERR_INVALID_ARG;  // NaN
   const int64_t ho = out_extent(p->H, p->K, p->stride, p->pad, p->dilation);
   const int64_t wo = out_extent(p->W, p->K, stride_w(p), pad_w(p), dil_w(p));
@@ -264,6 +275,7 @@ bool backward_lane_map(const dcn_problem* p, LaneMap* lm) {
     case 8: *lm = {4, 2}; return true;
     case 16: *lm = {4, 4}; return true;
     case 32: *lm = {4, 8}; return true;
+    case 64: *lm = {4, 16}; return true;
     default: return false;
   }
 }
@@ -276,6 +288,7 @@ dcn_status backward_dispatch_t(const dcn_problem* p, const Plan& plan, const Bwd
     case 2: return backward_dispatch_kk<T, 2, DET>(p, plan, args, stream);
     case 4: return backward_dispatch_kk<T, 4, DET>(p, plan, args, stream);
     case 8: return backward_dispatch_kk<T, 8, DET>(p, plan, args, stream);
+    case 16: return backward_dispatch_kk<T, 16, DET>(p, plan, args, stream);
     default: return DCN_ERR_UNSUPPORTED;
   }
 }
@@ -283,14 +296,14 @@ dcn_status backward_dispatch_t(const dcn_problem* p, const Plan& plan, const Bwd
 // det: the accumulator is 64-bit fixed point (the deterministic backward).
 dcn_status backward_dispatch(const dcn_problem* p, const Plan& plan, const BwdArgs& args,
                              bool det, cudaStream_t stream) {
-  if (det)
-    return p->dtype == DCN_BF16 ? backward_dispatch_t<__nv_bfloat16, true>(p, plan, args, stream)
-                                : backward_dispatch_t<float, true>(p, plan, args, stream);
-  return p->dtype == DCN_BF16 ? backward_dispatch_t<__nv_bfloat16, false>(p, plan, args, stream)
-                              : backward_dispatch_t<float, false>(p, plan, args, stream);
+  return with_storage(p->dtype, [&](auto tag) {
+    using T = decltype(tag);
+    return det ? backward_dispatch_t<T, true>(p, plan, args, stream)
+               : backward_dispatch_t<T, false>(p, plan, args, stream);
+  });
 }
 
-// Bytes of the fp32 grad_input accumulator that bf16 storage needs.
+// Bytes of the fp32 grad_input accumulator that 2-byte storage (bf16, fp16) needs.
 size_t bf16_accumulator_bytes(const dcn_problem* p) {
   return size_t(p->N) * p->H * p->W * p->G * p->Cg * sizeof(float);
 }
@@ -325,6 +338,36 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// Unique id of the current CUDA context (cuCtxGetId; 0 if it cannot be
+// read).  The per-device state the library keeps (the error word's address,
+// the host entry points' streams and events, the allocation-free backward's
+// array address) is tagged with it: after cudaDeviceReset the device has a
+// new context and the state is created again instead of being reused.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = []() -> PFN_cuCtxGetCurrent_v4000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  }();
+  static PFN_cuCtxGetId_v12000 get_id = []() -> PFN_cuCtxGetId_v12000 {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  }();
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&c) != CUDA_SUCCESS || c == nullptr ||
+      get_id(c, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 struct DeviceInfo {
   int sms = 0;
   int smem_optin = 0;
@@ -337,11 +380,13 @@ dcn_status device_info(DeviceInfo* out) {
   constexpr int kMaxDev = 64;
   static DeviceInfo cache[kMaxDev];
   static bool ready[kMaxDev] = {};
+  static unsigned long long ctx[kMaxDev] = {};  // context the entry was made in
   static std::mutex lock;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DCN_ERR_CUDA;
   std::lock_guard<std::mutex> guard(lock);
-  if (!ready[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!ready[dev] || ctx[dev] != id) {
     DeviceInfo d;
     void* ew = nullptr;
     if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
@@ -351,6 +396,7 @@ dcn_status device_info(DeviceInfo* out) {
       return DCN_ERR_CUDA;
     d.error_word = static_cast<unsigned int*>(ew);
     cache[dev] = d;
+    ctx[dev] = id;
     ready[dev] = true;
   }
   *out = cache[dev];
@@ -386,38 +432,6 @@ int box_extent(int tile, int stride, int dil, int halo) {
   return (tile - 1) * stride + 2 * dil + 2 + 2 * halo;
 }
 
-// Pick the output tile: largest useful area under the shared-memory budget,
-// penalising ragged-edge waste, idle lanes and the halo the box carries.
-void choose_tiled_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, size_t box_budget,
-                       int* TH_out, int* TW_out) {
-  double best = 1e300;
-  int bth = 1, btw = 1;
-  for (int th = 1; th <= std::min(Ho, 64); ++th) {
-    for (int tw = 1; tw <= std::min(Wo, 64); ++tw) {
-      const int bh = box_extent(th, p->stride, p->dilation, halo);
-      int bw = box_extent(tw, stride_w(p), dil_w(p), halo);
-      bw = box_pitch(bw, cs);
-      if (bh > 256 || bw > 256) continue;
-      const size_t bytes = size_t(bh) * bw * cs;
-      if (bytes > box_budget) continue;
-      const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * p->G;
-      const int px = th * tw;
-      const int64_t batches = (px + kTiledBatch - 1) / kTiledBatch;
-      const double per_item = double(batches) * kTiledBatch * taps(p)  // unit-samples
-                              + 0.05 * double(bytes) / 32.0            // box fill
-                              + 300.0;                                 // item overhead
-      const double cost = double(items) * per_item;
-      if (cost < best) {
-        best = cost;
-        bth = th;
-        btw = tw;
-      }
-    }
-  }
-  *TH_out = bth;
-  *TW_out = btw;
-}
-
 // Launch a persistent tiled kernel: as many CTAs as fit on the GPU at once,
 // never more than there are items.
 template <typename Kernel, typename Args>
@@ -436,92 +450,54 @@ dcn_status launch_persistent(Kernel k, const CUtensorMap& map, const Args& args,
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
 }
 
-template <typename T, int CS>
+template <typename T, bool FAR>
+dcn_status forward_tiled_dispatch_far(const dcn_problem* p, const CUtensorMap& map,
+                                      const TiledArgs& args, size_t smem, int sms,
+                                      cudaStream_t stream) {
+  if (p->remove_center)
+    return p->softmax
+               ? launch_persistent(dcn_forward_tiled_kernel<T, 8, true, FAR>, map, args, smem, sms, stream)
+               : launch_persistent(dcn_forward_tiled_kernel<T, 8, false, FAR>, map, args, smem, sms, stream);
+  return p->softmax
+             ? launch_persistent(dcn_forward_tiled_kernel<T, 9, true, FAR>, map, args, smem, sms, stream)
+             : launch_persistent(dcn_forward_tiled_kernel<T, 9, false, FAR>, map, args, smem, sms, stream);
+}
+
+template <typename T>
 dcn_status forward_tiled_dispatch(const dcn_problem* p, const CUtensorMap& map,
-                                  const TiledArgs& args, size_t smem, int sms,
+                                  const TiledArgs& args, bool far, size_t smem, int sms,
                                   cudaStream_t stream) {
-  if (p->remove_center)
-    return p->softmax
-               ? launch_persistent(dcn_forward_tiled_kernel<T, CS, 8, true>, map, args, smem, sms, stream)
-               : launch_persistent(dcn_forward_tiled_kernel<T, CS, 8, false>, map, args, smem, sms, stream);
-  return p->softmax
-             ? launch_persistent(dcn_forward_tiled_kernel<T, CS, 9, true>, map, args, smem, sms, stream)
-             : launch_persistent(dcn_forward_tiled_kernel<T, CS, 9, false>, map, args, smem, sms, stream);
+  return far ? forward_tiled_dispatch_far<T, true>(p, map, args, smem, sms, stream)
+             : forward_tiled_dispatch_far<T, false>(p, map, args, smem, sms, stream);
 }
 
-template <typename T, int CS, bool DET>
+template <typename T, bool DET, bool FAR>
+dcn_status backward_tiled_dispatch_far(const dcn_problem* p, const CUtensorMap& map,
+                                       const TiledBwdArgs& args, size_t smem, int sms,
+                                       cudaStream_t stream) {
+  if (p->remove_center)
+    return p->softmax
+               ? launch_persistent(dcn_backward_tiled_kernel<T, 8, true, DET, FAR>, map, args, smem, sms, stream)
+               : launch_persistent(dcn_backward_tiled_kernel<T, 8, false, DET, FAR>, map, args, smem, sms, stream);
+  return p->softmax
+             ? launch_persistent(dcn_backward_tiled_kernel<T, 9, true, DET, FAR>, map, args, smem, sms, stream)
+             : launch_persistent(dcn_backward_tiled_kernel<T, 9, false, DET, FAR>, map, args, smem, sms, stream);
+}
+
+template <typename T, bool DET>
 dcn_status backward_tiled_dispatch(const dcn_problem* p, const CUtensorMap& map,
-                                   const TiledBwdArgs& args, size_t smem, int sms,
+                                   const TiledBwdArgs& args, bool far, size_t smem, int sms,
                                    cudaStream_t stream) {
-  if (p->remove_center)
-    return p->softmax
-               ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, true, DET>, map, args, smem, sms, stream)
-               : launch_persistent(dcn_backward_tiled_kernel<T, CS, 8, false, DET>, map, args, smem, sms, stream);
-  return p->softmax
-             ? launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, true, DET>, map, args, smem, sms, stream)
-             : launch_persistent(dcn_backward_tiled_kernel<T, CS, 9, false, DET>, map, args, smem, sms, stream);
+  return far ? backward_tiled_dispatch_far<T, DET, true>(p, map, args, smem, sms, stream)
+             : backward_tiled_dispatch_far<T, DET, false>(p, map, args, smem, sms, stream);
 }
 
-// Everything a tiled launch needs: the tile and box geometry, the shared
-// memory size and the input's tensor map.  `tile_env` names the variable that
-// may force the tile ("THxTW", for tuning sweeps).
-struct TiledLaunch {
-  TiledParams t;
-  CUtensorMap map;
-  size_t smem;
-  DeviceInfo dev;
-};
-
-dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
-                         const char* tile_env, TiledLaunch* L) {
-  dcn_status st = device_info(&L->dev);
-  if (st != DCN_OK) return st;
+// Input tensor map viewed as (C, W, H, N), innermost first; one box is
+// (Cg, BW, BH, 1) starting at (g*Cg, X0, Y0, n).  Outside the tensor the box
+// is zero filled, which is exactly the operator's zero padding.
+dcn_status encode_input_map(const dcn_problem* p, const TiledParams& t, const void* x,
+                            CUtensorMap* map) {
   const int e = esize(p->dtype);
-  const int cs = p->Cg * e;
-  const size_t slot_bytes = size_t(kTiledWarps) * kTiledBatch * kSlotBytes;
-  const size_t fixed = slot_bytes + kTiledTailBytes;  // mbarriers, abort flag, zero area
-  if (size_t(L->dev.smem_optin) <= fixed + 2048) return DCN_ERR_UNSUPPORTED;
-  const size_t box_budget = (size_t(L->dev.smem_optin) - fixed) / 2 / 1024 * 1024;
-  const int halo = env_int("DCN_CORE_HALO", 5);
-  int TH = 0, TW = 0;
-  if (const char* s = std::getenv(tile_env)) {
-    if (std::sscanf(s, "%dx%d", &TH, &TW) != 2 || TH < 1 || TW < 1) TH = TW = 0;
-  }
-  if (TH == 0) choose_tiled_tile(p, int(Ho), int(Wo), cs, halo, box_budget, &TH, &TW);
-  TH = std::min<int>(TH, int(Ho));
-  TW = std::min<int>(TW, int(Wo));
-
-  TiledParams& t = L->t;
-  t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
-  t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation; t.Ho = int(Ho); t.Wo = int(Wo);
-  t.stride_w = stride_w(p); t.pad_w = pad_w(p); t.dil_w = dil_w(p);
-  t.sigma = p->offset_scale; t.halo = halo; t.TH = TH; t.TW = TW;
-  // Test knob for the failure path: DCN_CORE_TEST_STALL=1 makes the first box
-  // of every CTA never arrive; the bounded waits then give up and
-  // dcn_core_sync_status reports DCN_ERR_TIMEOUT.
-  t.inject_stall = env_int("DCN_CORE_TEST_STALL", 0) == 1 ? 1 : 0;
-  t.nTY = (t.Ho + TH - 1) / TH;
-  t.nTX = (t.Wo + TW - 1) / TW;
-  t.BH = box_extent(TH, t.stride, t.dil, halo);
-  t.BW = box_extent(TW, t.stride_w, t.dil_w, halo);
-  t.BW = box_pitch(t.BW, cs);
-  if (t.BH > 256 || t.BW > 256) return DCN_ERR_UNSUPPORTED;
-  t.box_bytes = uint32_t(size_t(t.BH) * t.BW * cs);
-  t.box_stride = (t.box_bytes + 1023u) / 1024u * 1024u;
-  const int64_t items = int64_t(t.N) * t.nTY * t.nTX * t.G;
-  if (items > INT_MAX) return DCN_ERR_UNSUPPORTED;
-  t.items = int(items);
-  t.batches = (TH * TW + kTiledBatch - 1) / kTiledBatch;
-  t.fd_G = make_fastdiv(uint32_t(t.G));
-  t.fd_nTX = make_fastdiv(uint32_t(t.nTX));
-  t.fd_tiles = make_fastdiv(uint32_t(t.nTY * t.nTX));
-  t.fd_TW = make_fastdiv(uint32_t(TW));
-  L->smem = 2 * size_t(t.box_stride) + fixed;
-  if (L->smem > size_t(L->dev.smem_optin)) return DCN_ERR_UNSUPPORTED;
-
-  // Tensor map of the input viewed as (C, W, H, N), innermost first; one box
-  // is (Cg, BW, BH, 1) starting at (g*Cg, X0, Y0, n).  Outside the tensor the
-  // box is zero filled, which is exactly the operator's zero padding.
   const cuuint64_t dims[4] = {cuuint64_t(t.C), cuuint64_t(t.W), cuuint64_t(t.H),
                               cuuint64_t(t.N)};
   const cuuint64_t strides[3] = {cuuint64_t(t.C) * e, cuuint64_t(t.W) * t.C * e,
@@ -529,26 +505,141 @@ dcn_status tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const voi
   const cuuint32_t box[4] = {cuuint32_t(t.Cg), cuuint32_t(t.BW), cuuint32_t(t.BH), 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUresult cr = tensor_map_encoder()(
-      &L->map,
-      p->dtype == DCN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+      map,
+      p->dtype == DCN_BF16  ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+      : p->dtype == DCN_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
       4, const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
       CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return cr == CUDA_SUCCESS ? DCN_OK : DCN_ERR_UNSUPPORTED;
 }
 
+// Forward tile choice.  The box of a tile is clamped to the image and its
+// zero ring, so a tile near the border gets more halo inside and a small
+// image's box covers it all (no far taps).  Cost, in lane-samples: every
+// batch of 32 units costs its taps whether its lanes are used or not; an item
+// costs a fixed overhead and its box fill; where footprints can leave the
+// box, taps near the tile's edges go to global memory at several times the
+// cost.  Boxes must leave room for at least two in flight.
+struct FwdTile {
+  int TH = 0, TW = 0, BH = 0, BW = 0, nbuf = 0;
+  uint32_t box_bytes = 0, box_stride = 0;
+  bool far = true;
+};
+
+int clamp_extent(int box, int extent) { return std::min(box, extent + 2); }
+
+bool fwd_tile_geometry(const dcn_problem* p, int TH, int TW, int cs, int halo, size_t optin,
+                       FwdTile* f) {
+  f->TH = TH;
+  f->TW = TW;
+  f->BH = clamp_extent(box_extent(TH, p->stride, p->dilation, halo), p->H);
+  f->BW = box_pitch(clamp_extent(box_extent(TW, stride_w(p), dil_w(p), halo), p->W), cs);
+  if (f->BH > 256 || f->BW > 256) return false;
+  f->box_bytes = uint32_t(size_t(f->BH) * f->BW * cs);
+  f->box_stride = (f->box_bytes + 1023u) / 1024u * 1024u;
+  const size_t fixed = fwd_tiled_smem(0, 0, f->BW, cs);
+  if (optin <= fixed) return false;
+  f->nbuf = int(std::min<size_t>(kTiledMaxBufs, (optin - fixed) / f->box_stride));
+  if (f->nbuf < 2) return false;
+  f->far = !(f->BH >= p->H + 2 && f->BW >= p->W + 2);
+  return true;
+}
+
+void choose_fwd_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, size_t optin,
+                     FwdTile* out) {
+  double best = 1e300;
+  for (int th = 1; th <= std::min(Ho, 64); ++th) {
+    for (int tw = 1; tw <= std::min(Wo, 64); ++tw) {
+      FwdTile f;
+      if (!fwd_tile_geometry(p, th, tw, cs, halo, optin, &f)) continue;
+      const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * p->N * p->G;
+      const int px = th * tw;
+      const double lane_samples = double((px + kTiledBatch - 1) / kTiledBatch) * kTiledBatch *
+                                  taps(p);
+      const double far_frac = f.far ? 0.3 * (1.0 / th + 1.0 / tw) : 0.0;
+      const double per_item = lane_samples * (1.0 + 10.0 * far_frac) +
+                              0.02 * double(f.box_bytes) / cs + 400.0 + (f.nbuf < 3 ? 200.0 : 0.0);
+      const double cost = double(items) * per_item;
+      if (cost < best) {
+        best = cost;
+        *out = f;
+      }
+    }
+  }
+}
+
+struct BoxLaunch {
+  TiledParams t;
+  CUtensorMap map;
+  size_t smem;
+  DeviceInfo dev;
+  bool far;
+};
+
+dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
+                             const char* tile_env, BoxLaunch* L) {
+  dcn_status st = device_info(&L->dev);
+  if (st != DCN_OK) return st;
+  const int cs = p->Cg * esize(p->dtype);
+  const int halo = std::max(0, env_int("DCN_CORE_HALO", 5));
+  const size_t optin = size_t(L->dev.smem_optin);
+  FwdTile f;
+  int TH = 0, TW = 0;
+  if (const char* s = std::getenv(tile_env)) {  // "THxTW", for tuning sweeps
+    if (std::sscanf(s, "%dx%d", &TH, &TW) != 2 || TH < 1 || TW < 1) TH = TW = 0;
+  }
+  if (TH > 0) {
+    if (!fwd_tile_geometry(p, std::min<int>(TH, int(Ho)), std::min<int>(TW, int(Wo)), cs, halo,
+                           optin, &f))
+      return DCN_ERR_UNSUPPORTED;
+  } else {
+    choose_fwd_tile(p, int(Ho), int(Wo), cs, halo, optin, &f);
+    if (f.nbuf == 0) return DCN_ERR_UNSUPPORTED;
+  }
+  if (const int nb = env_int("DCN_CORE_TILED_BUFS", 0); nb >= 2 && nb < f.nbuf) f.nbuf = nb;
+
+  TiledParams& t = L->t;
+  t.N = p->N; t.H = p->H; t.W = p->W; t.G = p->G; t.Cg = p->Cg; t.C = p->G * p->Cg;
+  t.stride = p->stride; t.pad = p->pad; t.dil = p->dilation; t.Ho = int(Ho); t.Wo = int(Wo);
+  t.stride_w = stride_w(p); t.pad_w = pad_w(p); t.dil_w = dil_w(p);
+  t.sigma = p->offset_scale; t.halo = halo; t.TH = f.TH; t.TW = f.TW;
+  t.inject_stall = env_int("DCN_CORE_TEST_STALL", 0) == 1 ? 1 : 0;
+  t.nTY = (t.Ho + t.TH - 1) / t.TH;
+  t.nTX = (t.Wo + t.TW - 1) / t.TW;
+  t.BH = f.BH;
+  t.BW = f.BW;
+  t.clamp_box = 1;
+  t.nbuf = f.nbuf;
+  t.box_bytes = f.box_bytes;
+  t.box_stride = f.box_stride;
+  const int64_t items = int64_t(t.N) * t.nTY * t.nTX * t.G;
+  if (items > INT_MAX) return DCN_ERR_UNSUPPORTED;
+  t.items = int(items);
+  t.batches = (t.TH * t.TW + kTiledBatch - 1) / kTiledBatch;
+  t.fd_G = make_fastdiv(uint32_t(t.G));
+  t.fd_nTX = make_fastdiv(uint32_t(t.nTX));
+  t.fd_tiles = make_fastdiv(uint32_t(t.nTY * t.nTX));
+  t.fd_TW = make_fastdiv(uint32_t(t.TW));
+  L->far = f.far;
+  L->smem = fwd_tiled_smem(t.nbuf, t.box_stride, t.BW, cs);
+  if (L->smem > optin) return DCN_ERR_UNSUPPORTED;
+  return encode_input_map(p, t, x, &L->map);
+}
+
 dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
                          const void* off, const void* mask, void* out, cudaStream_t stream) {
-  TiledLaunch L;
-  dcn_status st = tiled_prepare(p, Ho, Wo, x, "DCN_CORE_TILED_TILE", &L);
+  BoxLaunch L;
+  dcn_status st = box_tiled_prepare(p, Ho, Wo, x, "DCN_CORE_TILED_TILE", &L);
   if (st != DCN_OK) return st;
   TiledArgs args;
   args.t = L.t;
   args.x = x; args.off = off; args.mask = mask; args.out = out;
   args.error_word = L.dev.error_word;
-  if (p->dtype == DCN_BF16)
-    return forward_tiled_dispatch<__nv_bfloat16, 32>(p, L.map, args, L.smem, L.dev.sms, stream);
-  return forward_tiled_dispatch<float, 64>(p, L.map, args, L.smem, L.dev.sms, stream);
+  return with_storage(p->dtype, [&](auto tag) {
+    return forward_tiled_dispatch<decltype(tag)>(p, L.map, args, L.far, L.smem, L.dev.sms, stream);
+  });
 }
 
 // The tiled backward applies where the tiled forward does (3x3 tap sets,
@@ -564,8 +655,8 @@ bool backward_tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
 // Launch the tiled backward on the zero-filled accumulator a.gx.
 dcn_status backward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const BwdArgs& a,
                           bool det, cudaStream_t stream) {
-  TiledLaunch L;
-  dcn_status st = tiled_prepare(p, Ho, Wo, a.x, "DCN_CORE_BWD_TILED_TILE", &L);
+  BoxLaunch L;
+  dcn_status st = box_tiled_prepare(p, Ho, Wo, a.x, "DCN_CORE_BWD_TILED_TILE", &L);
   if (st != DCN_OK) return st;
   TiledBwdArgs args;
   args.t = L.t;
@@ -574,13 +665,11 @@ dcn_status backward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const Bw
   args.det_hdr = a.det_hdr; args.det_cbits = a.det_cbits;
   args.error_word = L.dev.error_word;
   const int sms = L.dev.sms;
-  if (det)
-    return p->dtype == DCN_BF16
-               ? backward_tiled_dispatch<__nv_bfloat16, 32, true>(p, L.map, args, L.smem, sms, stream)
-               : backward_tiled_dispatch<float, 64, true>(p, L.map, args, L.smem, sms, stream);
-  return p->dtype == DCN_BF16
-             ? backward_tiled_dispatch<__nv_bfloat16, 32, false>(p, L.map, args, L.smem, sms, stream)
-             : backward_tiled_dispatch<float, 64, false>(p, L.map, args, L.smem, sms, stream);
+  return with_storage(p->dtype, [&](auto tag) {
+    using T = decltype(tag);
+    return det ? backward_tiled_dispatch<T, true>(p, L.map, args, L.far, L.smem, sms, stream)
+               : backward_tiled_dispatch<T, false>(p, L.map, args, L.far, L.smem, sms, stream);
+  });
 }
 
 // The backward's kernel launch on a zero-filled accumulator: the tiled kernel
@@ -605,8 +694,23 @@ constexpr int kHostChunks = 8;  // chunks per call, at most
 
 struct HostPipe {
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t ev[2 * kHostChunks + 2] = {};
+  // [0] start, [1 + i] chunk i in, [1 + C + i] chunk i out, [2C + 1] and
+  // [2C + 2] the joins of the device-to-host and host-to-device streams
+  cudaEvent_t ev[2 * kHostChunks + 3] = {};
 };
+
+// Joins both library streams back into the caller's stream.  Runs on every
+// exit after the fork, so that an error part-way leaves no copy outside the
+// caller's stream order (and a stream capture no unjoined fork).
+dcn_status join_host_pipe(HostPipe* hp, int chunks, cudaStream_t stream, dcn_status st) {
+  cudaEvent_t* const ev = hp->ev;
+  const bool ok = cudaEventRecord(ev[2 * chunks + 1], hp->d2h) == cudaSuccess &&
+                  cudaStreamWaitEvent(stream, ev[2 * chunks + 1], 0) == cudaSuccess &&
+                  cudaEventRecord(ev[2 * chunks + 2], hp->h2d) == cudaSuccess &&
+                  cudaStreamWaitEvent(stream, ev[2 * chunks + 2], 0) == cudaSuccess;
+  if (st != DCN_OK) return st;
+  return ok ? DCN_OK : DCN_ERR_CUDA;
+}
 
 // The pipe of the current device, created on first use.  The returned lock is
 // held while the caller enqueues: the events are re-recorded by the next call,
@@ -615,11 +719,13 @@ dcn_status host_pipe(HostPipe** out, std::unique_lock<std::mutex>* held) {
   constexpr int kMaxDev = 64;
   static HostPipe pipes[kMaxDev];
   static bool ready[kMaxDev] = {};
+  static unsigned long long ctx[kMaxDev] = {};  // context the pipe was made in
   static std::mutex lock;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DCN_ERR_CUDA;
   *held = std::unique_lock<std::mutex>(lock);
-  if (!ready[dev]) {
+  const unsigned long long id = current_context_id();
+  if (!ready[dev] || ctx[dev] != id) {
     HostPipe hp;
     if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess)
@@ -627,6 +733,7 @@ dcn_status host_pipe(HostPipe** out, std::unique_lock<std::mutex>* held) {
     for (cudaEvent_t& e : hp.ev)
       if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return DCN_ERR_CUDA;
     pipes[dev] = hp;
+    ctx[dev] = id;
     ready[dev] = true;
   }
   *out = &pipes[dev];
@@ -704,13 +811,15 @@ dcn_status dcn_core_forward(const dcn_problem* problem, const void* input, const
     if (st != DCN_ERR_UNSUPPORTED) return st;
   }
   Plan plan;
-  const size_t entry = problem->dtype == DCN_BF16 ? staged_bytes_per_entry<__nv_bfloat16>()
-                                                  : staged_bytes_per_entry<float>();
+  const size_t entry = with_storage(problem->dtype, [](auto tag) {
+    return size_t(staged_bytes_per_entry<decltype(tag)>());
+  });
   st = make_plan(problem, Ho, Wo, entry, &plan);
   if (st != DCN_OK) return st;
   FwdArgs args{input, offset, mask, output, plan.t};
-  return problem->dtype == DCN_BF16 ? forward_dispatch<__nv_bfloat16>(problem, plan, args, stream)
-                                    : forward_dispatch<float>(problem, plan, args, stream);
+  return with_storage(problem->dtype, [&](auto tag) {
+    return forward_dispatch<decltype(tag)>(problem, plan, args, stream);
+  });
 }
 
 dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input,
@@ -729,41 +838,43 @@ dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input
   std::unique_lock<std::mutex> held;
   st = host_pipe(&hp, &held);
   if (st != DCN_OK) return st;
-  cudaEvent_t* const ev = hp->ev;  // [0] start, [1 + i] chunk i in, [1 + C + i] chunk i out, [2C + 1] done
+  cudaEvent_t* const ev = hp->ev;
   DCN_CU(cudaEventRecord(ev[0], stream));
-  DCN_CU(cudaStreamWaitEvent(hp->h2d, ev[0], 0));
-  DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[0], 0));
-  for (int i = 0; i < cp.chunks; ++i) {
-    const int64_t n0 = int64_t(i) * cp.per, n = std::min<int64_t>(cp.per, problem->N - n0);
-    const size_t ox = size_t(n0) * ib.x, oo = size_t(n0) * ib.off, om = size_t(n0) * ib.msk,
-                 oy = size_t(n0) * ib.out;
-    DCN_CU(cudaMemcpyAsync(at(d_input, ox), at(h_input, ox), size_t(n) * ib.x,
-                           cudaMemcpyHostToDevice, hp->h2d));
-    DCN_CU(cudaMemcpyAsync(at(d_offset, oo), at(h_offset, oo), size_t(n) * ib.off,
-                           cudaMemcpyHostToDevice, hp->h2d));
-    DCN_CU(cudaMemcpyAsync(at(d_mask, om), at(h_mask, om), size_t(n) * ib.msk,
-                           cudaMemcpyHostToDevice, hp->h2d));
-    DCN_CU(cudaEventRecord(ev[1 + i], hp->h2d));
-    DCN_CU(cudaStreamWaitEvent(stream, ev[1 + i], 0));
-    dcn_problem q = *problem;
-    q.N = int(n);
-    st = dcn_core_forward(&q, at(d_input, ox), at(d_offset, oo), at(d_mask, om), at(d_output, oy),
-                          stream);
-    if (st != DCN_OK) return st;
-    DCN_CU(cudaEventRecord(ev[1 + cp.chunks + i], stream));
-    DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[1 + cp.chunks + i], 0));
-    DCN_CU(cudaMemcpyAsync(at(h_output, oy), at(d_output, oy), size_t(n) * ib.out,
-                           cudaMemcpyDeviceToHost, hp->d2h));
-  }
-  DCN_CU(cudaEventRecord(ev[2 * cp.chunks + 1], hp->d2h));
-  DCN_CU(cudaStreamWaitEvent(stream, ev[2 * cp.chunks + 1], 0));
-  return DCN_OK;
+  auto chunks = [&]() -> dcn_status {
+    DCN_CU(cudaStreamWaitEvent(hp->h2d, ev[0], 0));
+    DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[0], 0));
+    for (int i = 0; i < cp.chunks; ++i) {
+      const int64_t n0 = int64_t(i) * cp.per, n = std::min<int64_t>(cp.per, problem->N - n0);
+      const size_t ox = size_t(n0) * ib.x, oo = size_t(n0) * ib.off, om = size_t(n0) * ib.msk,
+                   oy = size_t(n0) * ib.out;
+      DCN_CU(cudaMemcpyAsync(at(d_input, ox), at(h_input, ox), size_t(n) * ib.x,
+                             cudaMemcpyHostToDevice, hp->h2d));
+      DCN_CU(cudaMemcpyAsync(at(d_offset, oo), at(h_offset, oo), size_t(n) * ib.off,
+                             cudaMemcpyHostToDevice, hp->h2d));
+      DCN_CU(cudaMemcpyAsync(at(d_mask, om), at(h_mask, om), size_t(n) * ib.msk,
+                             cudaMemcpyHostToDevice, hp->h2d));
+      DCN_CU(cudaEventRecord(ev[1 + i], hp->h2d));
+      DCN_CU(cudaStreamWaitEvent(stream, ev[1 + i], 0));
+      dcn_problem q = *problem;
+      q.N = int(n);
+      const dcn_status cs = dcn_core_forward(&q, at(d_input, ox), at(d_offset, oo),
+                                             at(d_mask, om), at(d_output, oy), stream);
+      if (cs != DCN_OK) return cs;
+      DCN_CU(cudaEventRecord(ev[1 + cp.chunks + i], stream));
+      DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[1 + cp.chunks + i], 0));
+      DCN_CU(cudaMemcpyAsync(at(h_output, oy), at(d_output, oy), size_t(n) * ib.out,
+                             cudaMemcpyDeviceToHost, hp->d2h));
+    }
+    return DCN_OK;
+  };
+  return join_host_pipe(hp, cp.chunks, stream, chunks());
 }
+
 
 size_t dcn_core_backward_workspace(const dcn_problem* problem) {
   int64_t Ho, Wo;
   if (check_problem(problem, &Ho, &Wo) != DCN_OK) return 0;
-  return problem->dtype == DCN_BF16 ? bf16_accumulator_bytes(problem) : 0;
+  return problem->dtype != DCN_F32 ? bf16_accumulator_bytes(problem) : 0;
 }
 
 dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, const void* offset,
@@ -775,7 +886,7 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
   if (st != DCN_OK) return st;
   if (!input || !offset || !mask || !grad_out || !grad_input || !grad_offset || !grad_mask)
     return DCN_ERR_INVALID_ARG;
-  const bool bf16 = problem->dtype == DCN_BF16;
+  const bool bf16 = problem->dtype != DCN_F32;  // 2-byte storage: fp32 accumulator
   const size_t acc_bytes = bf16_accumulator_bytes(problem);
   if (bf16 && (!workspace || workspace_bytes < acc_bytes)) return DCN_ERR_INVALID_ARG;
   if (!aligned(input, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
@@ -783,8 +894,9 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
       !aligned(grad_mask, 16) || (bf16 && !aligned(workspace, 16)))
     return DCN_ERR_UNSUPPORTED;
   Plan plan;
-  st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
-                                       : staged_bytes_per_entry<float>(),
+  st = make_plan(problem, Ho, Wo, with_storage(problem->dtype, [](auto tag) {
+                   return staged_bytes_per_entry<decltype(tag)>();
+                 }),
                  &plan, true);
   if (st != DCN_OK) return st;
   float* acc = bf16 ? static_cast<float*>(workspace) : static_cast<float*>(grad_input);
@@ -797,8 +909,12 @@ dcn_status dcn_core_backward(const dcn_problem* problem, const void* input, cons
   DeviceInfo dev;
   if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
   const unsigned grid = unsigned(std::min<size_t>((n4 + 255) / 256, size_t(dev.sms) * 8));
-  dcn_round_to_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const float4*>(workspace),
-                                                     static_cast<uint2*>(grad_input), n4);
+  if (problem->dtype == DCN_F16)
+    dcn_round_to_half_kernel<__half><<<grid, 256, 0, stream>>>(
+        static_cast<const float4*>(workspace), static_cast<uint2*>(grad_input), n4);
+  else
+    dcn_round_to_half_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const float4*>(workspace), static_cast<uint2*>(grad_input), n4);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
 }
 
@@ -816,7 +932,7 @@ dcn_status dcn_core_backward_host(const dcn_problem* problem, const void* input,
     return DCN_ERR_INVALID_ARG;
   // Everything dcn_core_backward checks, on the whole problem, before the
   // first copy is enqueued (chunk starts keep the alignment).
-  const bool bf16 = problem->dtype == DCN_BF16;
+  const bool bf16 = problem->dtype != DCN_F32;  // 2-byte storage: fp32 accumulator
   if (bf16 && (!workspace || workspace_bytes < bf16_accumulator_bytes(problem)))
     return DCN_ERR_INVALID_ARG;
   if (!aligned(input, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
@@ -825,8 +941,9 @@ dcn_status dcn_core_backward_host(const dcn_problem* problem, const void* input,
     return DCN_ERR_UNSUPPORTED;
   {
     Plan plan;
-    st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
-                                         : staged_bytes_per_entry<float>(),
+    st = make_plan(problem, Ho, Wo, with_storage(problem->dtype, [](auto tag) {
+                     return staged_bytes_per_entry<decltype(tag)>();
+                   }),
                    &plan, true);
     if (st != DCN_OK) return st;
   }
@@ -838,34 +955,36 @@ dcn_status dcn_core_backward_host(const dcn_problem* problem, const void* input,
   if (st != DCN_OK) return st;
   cudaEvent_t* const ev = hp->ev;
   DCN_CU(cudaEventRecord(ev[0], stream));
-  DCN_CU(cudaStreamWaitEvent(hp->h2d, ev[0], 0));
-  DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[0], 0));
-  for (int i = 0; i < cp.chunks; ++i) {
-    const int64_t n0 = int64_t(i) * cp.per, n = std::min<int64_t>(cp.per, problem->N - n0);
-    const size_t ox = size_t(n0) * ib.x, oo = size_t(n0) * ib.off, om = size_t(n0) * ib.msk,
-                 oy = size_t(n0) * ib.out;
-    DCN_CU(cudaMemcpyAsync(at(d_grad_out, oy), at(h_grad_out, oy), size_t(n) * ib.out,
-                           cudaMemcpyHostToDevice, hp->h2d));
-    DCN_CU(cudaEventRecord(ev[1 + i], hp->h2d));
-    DCN_CU(cudaStreamWaitEvent(stream, ev[1 + i], 0));
-    dcn_problem q = *problem;
-    q.N = int(n);
-    st = dcn_core_backward(&q, at(input, ox), at(offset, oo), at(mask, om), at(d_grad_out, oy),
-                           at(d_grad_input, ox), at(d_grad_offset, oo), at(d_grad_mask, om),
-                           workspace, workspace_bytes, stream);
-    if (st != DCN_OK) return st;
-    DCN_CU(cudaEventRecord(ev[1 + cp.chunks + i], stream));
-    DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[1 + cp.chunks + i], 0));
-    DCN_CU(cudaMemcpyAsync(at(h_grad_input, ox), at(d_grad_input, ox), size_t(n) * ib.x,
-                           cudaMemcpyDeviceToHost, hp->d2h));
-    DCN_CU(cudaMemcpyAsync(at(h_grad_offset, oo), at(d_grad_offset, oo), size_t(n) * ib.off,
-                           cudaMemcpyDeviceToHost, hp->d2h));
-    DCN_CU(cudaMemcpyAsync(at(h_grad_mask, om), at(d_grad_mask, om), size_t(n) * ib.msk,
-                           cudaMemcpyDeviceToHost, hp->d2h));
-  }
-  DCN_CU(cudaEventRecord(ev[2 * cp.chunks + 1], hp->d2h));
-  DCN_CU(cudaStreamWaitEvent(stream, ev[2 * cp.chunks + 1], 0));
-  return DCN_OK;
+  auto chunks = [&]() -> dcn_status {
+    DCN_CU(cudaStreamWaitEvent(hp->h2d, ev[0], 0));
+    DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[0], 0));
+    for (int i = 0; i < cp.chunks; ++i) {
+      const int64_t n0 = int64_t(i) * cp.per, n = std::min<int64_t>(cp.per, problem->N - n0);
+      const size_t ox = size_t(n0) * ib.x, oo = size_t(n0) * ib.off, om = size_t(n0) * ib.msk,
+                   oy = size_t(n0) * ib.out;
+      DCN_CU(cudaMemcpyAsync(at(d_grad_out, oy), at(h_grad_out, oy), size_t(n) * ib.out,
+                             cudaMemcpyHostToDevice, hp->h2d));
+      DCN_CU(cudaEventRecord(ev[1 + i], hp->h2d));
+      DCN_CU(cudaStreamWaitEvent(stream, ev[1 + i], 0));
+      dcn_problem q = *problem;
+      q.N = int(n);
+      const dcn_status cs = dcn_core_backward(
+          &q, at(input, ox), at(offset, oo), at(mask, om), at(d_grad_out, oy),
+          at(d_grad_input, ox), at(d_grad_offset, oo), at(d_grad_mask, om), workspace,
+          workspace_bytes, stream);
+      if (cs != DCN_OK) return cs;
+      DCN_CU(cudaEventRecord(ev[1 + cp.chunks + i], stream));
+      DCN_CU(cudaStreamWaitEvent(hp->d2h, ev[1 + cp.chunks + i], 0));
+      DCN_CU(cudaMemcpyAsync(at(h_grad_input, ox), at(d_grad_input, ox), size_t(n) * ib.x,
+                             cudaMemcpyDeviceToHost, hp->d2h));
+      DCN_CU(cudaMemcpyAsync(at(h_grad_offset, oo), at(d_grad_offset, oo), size_t(n) * ib.off,
+                             cudaMemcpyDeviceToHost, hp->d2h));
+      DCN_CU(cudaMemcpyAsync(at(h_grad_mask, om), at(d_grad_mask, om), size_t(n) * ib.msk,
+                             cudaMemcpyDeviceToHost, hp->d2h));
+    }
+    return DCN_OK;
+  };
+  return join_host_pipe(hp, cp.chunks, stream, chunks());
 }
 
 dcn_status dcn_core_sync_status(cudaStream_t stream) {
@@ -915,19 +1034,22 @@ static __device__ __align__(256) float
 constexpr int kNoallocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[kNoallocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoallocMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
+// per device and context (with that device current) and cached.
 dcn_status noalloc_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices)
     return DCN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
+  const unsigned long long id = current_context_id();
+  if (g_noalloc_addr[dev] == nullptr || g_noalloc_ctx[dev] != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return DCN_ERR_CUDA;
     g_noalloc_addr[dev] = p;
+    g_noalloc_ctx[dev] = id;
   }
   *out = g_noalloc_addr[dev];
   return DCN_OK;
@@ -950,12 +1072,13 @@ extern "C" dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, cons
       !aligned(grad_out, 16) || !aligned(grad_input, 16) || !aligned(grad_offset, 16) ||
       !aligned(grad_mask, 16))
     return DCN_ERR_UNSUPPORTED;
-  const bool bf16 = problem->dtype == DCN_BF16;
+  const bool bf16 = problem->dtype != DCN_F32;  // 2-byte storage: fp32 accumulator
   const size_t acc_bytes = bf16_accumulator_bytes(problem);  // fp32 grad_input size
   if (bf16 && acc_bytes > size_t(DCN_CORE_NOALLOC_SCRATCH_BYTES)) return DCN_ERR_UNSUPPORTED;
   Plan plan;
-  st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
-                                       : staged_bytes_per_entry<float>(),
+  st = make_plan(problem, Ho, Wo, with_storage(problem->dtype, [](auto tag) {
+                   return staged_bytes_per_entry<decltype(tag)>();
+                 }),
                  &plan, true);
   if (st != DCN_OK) return st;
   float* acc = static_cast<float*>(grad_input);
@@ -974,8 +1097,12 @@ extern "C" dcn_status dcn_core_backward_noalloc(const dcn_problem* problem, cons
   DeviceInfo dev;
   if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
   const unsigned grid = unsigned(std::min<size_t>((n4 + 255) / 256, size_t(dev.sms) * 8));
-  dcn_round_to_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
-                                                     static_cast<uint2*>(grad_input), n4);
+  if (problem->dtype == DCN_F16)
+    dcn_round_to_half_kernel<__half><<<grid, 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(acc), static_cast<uint2*>(grad_input), n4);
+  else
+    dcn_round_to_half_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(acc), static_cast<uint2*>(grad_input), n4);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
 }
 
@@ -1051,20 +1178,20 @@ extern "C" dcn_status dcn_core_backward_deterministic(
       !aligned(grad_out, 16) || !aligned(grad_input, 16) || !aligned(grad_offset, 16) ||
       !aligned(grad_mask, 16) || !aligned(workspace, 256))
     return DCN_ERR_UNSUPPORTED;
-  const bool bf16 = problem->dtype == DCN_BF16;
   Plan plan;
-  st = make_plan(problem, Ho, Wo, bf16 ? staged_bytes_per_entry<__nv_bfloat16>()
-                                       : staged_bytes_per_entry<float>(),
+  st = make_plan(problem, Ho, Wo, with_storage(problem->dtype, [](auto tag) {
+                   return staged_bytes_per_entry<decltype(tag)>();
+                 }),
                  &plan, true);
   if (st != DCN_OK) return st;
   DeviceInfo dev;
   if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
   if (cudaMemsetAsync(workspace, 0, ws_bytes, stream) != cudaSuccess) return DCN_ERR_CUDA;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  return bf16 ? det_passes<__nv_bfloat16>(problem, Ho, Wo, plan, input, offset, mask, grad_out,
-                                          grad_input, grad_offset, grad_mask, ws, dev.sms, stream)
-              : det_passes<float>(problem, Ho, Wo, plan, input, offset, mask, grad_out,
-                                  grad_input, grad_offset, grad_mask, ws, dev.sms, stream);
+  return with_storage(problem->dtype, [&](auto tag) {
+    return det_passes<decltype(tag)>(problem, Ho, Wo, plan, input, offset, mask, grad_out,
+                                     grad_input, grad_offset, grad_mask, ws, dev.sms, stream);
+  });
 }
 
 // ---------------------------------------------------------------------------
@@ -1107,7 +1234,7 @@ namespace {
 // out0[m, j] (j < n_split) / out1[m, j - n_split] (j >= n_split) =
 //     sum_c a[m, c] * w[j, c] + bias[j]  on the tensor cores.
 dcn_status bf16_gemm(const void* a, int64_t M, int K, const void* w, int64_t nout,
-                     int64_t n_split, const float* bias, void* out0, void* out1, bool bf16_out,
+                     int64_t n_split, const float* bias, void* out0, void* out1, dcn_dtype out_dtype,
                      cudaStream_t stream) {
   if (K % 8 != 0) return DCN_ERR_UNSUPPORTED;  // TMA rows must be 16-byte multiples
   if (!aligned(a, 16) || !aligned(w, 16) || !aligned(out0, 16) || !aligned(out1, 16) ||
@@ -1135,8 +1262,9 @@ dcn_status bf16_gemm(const void* a, int64_t M, int K, const void* w, int64_t nou
   dcn_status st;
   if ((st = bf16_kmajor_map(&amap, a, uint64_t(K), uint64_t(M))) != DCN_OK) return st;
   if ((st = bf16_kmajor_map(&wmap, w, uint64_t(K), uint64_t(nout))) != DCN_OK) return st;
-  return bf16_out ? launch_projection<__nv_bfloat16>(amap, wmap, args, dev.sms, stream)
-                  : launch_projection<float>(amap, wmap, args, dev.sms, stream);
+  return with_storage(out_dtype, [&](auto tag) {
+    return launch_projection<decltype(tag)>(amap, wmap, args, dev.sms, stream);
+  });
 }
 
 }  // namespace
@@ -1155,24 +1283,34 @@ extern "C" dcn_status dcn_core_offset_mask_projection(const dcn_problem* problem
   const int64_t KK = taps(problem);
   return bf16_gemm(query, M, Cq, weight, int64_t(problem->G) * KK * 3,
                    int64_t(problem->G) * KK * 2, bias, offset, mask,
-                   problem->dtype == DCN_BF16, stream);
+                   problem->dtype, stream);
 }
 
 namespace dcn {
 namespace {
 
-template <typename T, int LP>
-dcn_status guide_launch_lp(const GuideArgs& a, cudaStream_t stream) {
+template <typename T, int LP, int NJS>
+dcn_status guide_launch_nj(const GuideArgs& a, cudaStream_t stream) {
   const unsigned grid = unsigned(int64_t(a.N) * a.tiles_y * a.tiles_x);
   const unsigned block = kGuideWarps * 32;
   // parameters (12 quads per channel quad) and the conv results: at most 160 KB
   const size_t smem = (size_t(12) * a.Q + size_t(a.NJ) * block) * sizeof(float4);
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(dcn_guide_kernel<T, LP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(smem)) != cudaSuccess)
+      cudaFuncSetAttribute(dcn_guide_kernel<T, LP, NJS>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return DCN_ERR_CUDA;
-  dcn_guide_kernel<T, LP><<<grid, block, smem, stream>>>(a);
+  dcn_guide_kernel<T, LP, NJS><<<grid, block, smem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+// The compile-time quad count where the quads fill the lane groups exactly
+// (C = 160, 320, 640: 5 quads per lane; C = 1280: 10), else the general kernel.
+template <typename T, int LP>
+dcn_status guide_launch_lp(const GuideArgs& a, cudaStream_t stream) {
+  if (a.Q == LP * a.NJ && a.NJ == 5) return guide_launch_nj<T, LP, 5>(a, stream);
+  if constexpr (LP == 32)
+    if (a.Q == LP * a.NJ && a.NJ == 10) return guide_launch_nj<T, LP, 10>(a, stream);
+  return guide_launch_nj<T, LP, 0>(a, stream);
 }
 
 template <typename T>
@@ -1239,15 +1377,16 @@ extern "C" dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, con
   const size_t elems = size_t(problem->N) * problem->H * problem->W * C;
   a.x_bytes = elems * size_t(esize(problem->dtype));
   a.out_bytes = elems * 2;
-  return problem->dtype == DCN_BF16 ? guide_launch<__nv_bfloat16>(LP, a, stream)
-                                    : guide_launch<float>(LP, a, stream);
+  return with_storage(problem->dtype, [&](auto tag) {
+    return guide_launch<decltype(tag)>(LP, a, stream);
+  });
 }
 
 extern "C" dcn_status dcn_core_linear_bf16(const void* input, int M, int K, const void* weight,
                                            int Nout, const float* bias, void* output,
                                            dcn_dtype out_dtype, cudaStream_t stream) {
   if (!input || !weight || !output || M < 1 || K < 1 || Nout < 1) return DCN_ERR_INVALID_ARG;
-  if (out_dtype != DCN_F32 && out_dtype != DCN_BF16) return DCN_ERR_INVALID_ARG;
-  return bf16_gemm(input, M, K, weight, Nout, Nout, bias, output, output, out_dtype == DCN_BF16,
-                   stream);
+  if (out_dtype != DCN_F32 && out_dtype != DCN_BF16 && out_dtype != DCN_F16)
+    return DCN_ERR_INVALID_ARG;
+  return bf16_gemm(input, M, K, weight, Nout, Nout, bias, output, output, out_dtype, stream);
 }

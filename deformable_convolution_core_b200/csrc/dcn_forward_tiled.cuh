@@ -6,50 +6,36 @@
 // wavefront per distinct 128-byte line touched, i.e. one per corner whatever
 // its size, so a direct-gather kernel is capped near four L1 cycles per
 // sample.  Here a persistent CTA walks work items (image n, output tile,
-// group g); for each item one TMA tensor copy brings the group's Cg channels
-// of the input box the tile can reach (tile + kernel extent + halo, zero
-// filled outside the image) into shared memory, double-buffered on two
-// mbarriers.  The four corners of one sample are then two 2-pixel row chunks
-// of the box; 4*Cg*sizeof(T)/16 lanes each read one 16-byte piece, and with
-// the box row pitch chosen so that the two rows fall into complementary bank
-// halves the whole footprint is one conflict-free shared-memory wavefront
-// per 128 bytes.  Samples whose corners lie outside the box (large offsets)
-// read those corners from global memory instead; the result is the same.
+// group g); for each item one TMA tensor copy brings the group's 16 channels
+// of the input box the tile can reach into shared memory, with up to eight
+// boxes in flight on full/empty mbarriers.
 //
-// Every mbarrier wait is bounded; on expiry the kernel sets the device error
-// word, waits (bounded) for its own copies in flight and returns.
+// Per warp batch of 32 units (pixel, group):
+//   staging  the batch's offsets and mask, loaded coalesced one batch ahead,
+//            are written to the warp's region in their global order (element
+//            e = 9u + k at word e: conflict-free both ways, 9 being odd);
+//   phase A  one lane per unit: softmax over the taps, then per tap its four
+//            corner weights and the byte offset of corner (y0, x0) in the box,
+//            stored as structures of arrays W[k][u], OFF[k][u];
+//   phase B  four lanes per unit, one per bilinear corner, each holding all
+//            16 channels of its corner, 8 units per step.  A lane reads its
+//            corner as two (bf16) or four (fp32) 16-byte pieces; the units of
+//            a quarter-warp read complementary pieces (unit parity rho), so
+//            every footprint read is one conflict-free wavefront per 128
+//            bytes whatever the offsets.  A reduce-scatter over the four
+//            corner lanes ends with four channels per lane, stored directly.
+// A tap whose footprint lies in the box reads it there.  A tap that
+// contributes nothing gets weight 0 and reads a band of zeros (exact even for
+// non-finite inputs).  A tap whose footprint leaves the box ("far") also reads
+// the zeros in the box pass; its record then carries the weights' factors and
+// the corner's coordinates, and a second pass reads its corners from global
+// memory.  With the box covering the whole image and its zero ring (small
+// images) there are no far taps.
 #pragma once
 
-#include <cuda.h>
-
-#include "dcn_common.cuh"
+#include "dcn_tma.cuh"
 
 namespace dcn {
-
-constexpr int kTiledWarps = 15;  // consumer warps: with the producer, 4 warps per SM sub-partition
-constexpr int kTiledThreads = (kTiledWarps + 1) * 32;  // + one TMA producer warp
-constexpr int kTiledBatch = 32;                       // units per warp batch
-constexpr int kTiledMaxTaps = 9;  // the tiled kernel serves 3x3 windows (9 or 8 taps)
-// Shared memory after the unit slots: the full/empty mbarriers and the abort
-// flag (bytes 0-35), then at kTiledZeroAt a 128-byte area of zeros that the
-// forward's box reads of far or dead taps are pointed at.
-constexpr int kTiledZeroAt = 64;
-constexpr int kTiledZeroBytes = 128;
-constexpr int kTiledTailBytes = kTiledZeroAt + kTiledZeroBytes;
-
-struct TiledParams {
-  int N, H, W, G, Cg, C, stride, pad, dil, Ho, Wo;  // stride/pad/dil: height axis
-  int stride_w, pad_w, dil_w;                       // width axis
-  float sigma;
-  int TH, TW, nTY, nTX, halo, BH, BW;
-  int items;           // N * nTY * nTX * G
-  int inject_stall;    // test knob: 1 = never load the first item's box, so the
-                       // bounded waits expire and the error path runs
-  int batches;         // warp batches per item: ceil(TH * TW / kTiledBatch)
-  uint32_t box_bytes;  // BH * BW * Cg * sizeof(T)
-  uint32_t box_stride; // box_bytes rounded up to 1024
-  FastDiv fd_G, fd_nTX, fd_tiles, fd_TW;
-};
 
 struct TiledArgs {
   const void* x;
@@ -60,270 +46,127 @@ struct TiledArgs {
   TiledParams t;
 };
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+// Per-warp region of the forward: W[9][32] float4, OFF[9][32], FM[32] (far
+// taps of each unit, bit k = tap k), OUT[32] (element offset of the unit's
+// output channels, or ~0 for a unit outside the output).  The staged inputs
+// of a batch alias it: they are read into registers before the records are
+// written.
+constexpr int kFwdRegW = 0;
+constexpr int kFwdRegOff = kTiledMaxTaps * kTiledBatch * 16;
+constexpr int kFwdRegFm = kFwdRegOff + kTiledMaxTaps * kTiledBatch * 4;
+constexpr int kFwdRegOut = kFwdRegFm + kTiledBatch * 4;
+constexpr int kFwdRegion = kFwdRegOut + kTiledBatch * 4;  // 6016 bytes
+static_assert(kFwdRegion % 128 == 0, "warp regions stay 128-byte aligned");
+// Staged offsets and mask: element e of the batch (unit e / KK, tap e % KK):
+// the offset pair at 4e (bf16) or 8e (fp32), the mask value (as fp32) after them.
+constexpr int kFwdStageMask = kTiledMaxTaps * kTiledBatch * 8;
+static_assert(kFwdStageMask + kTiledMaxTaps * kTiledBatch * 4 <= kFwdRegion, "staging fits");
+// After the regions: full[8], empty[8] mbarriers and the abort flag.
+constexpr int kFwdTailBytes = 256;
+// Far-tap record: y0 + 1 and x0 + 1 packed into 14 bits each; as fp32 bits the
+// word is a finite number (below 2^28, sign clear), so the box pass may
+// multiply it by the zero band.
+constexpr int kFarShift = 14;
+
+// Zero band: (BW + 2) pixels of zeros; a dead or far tap's offset points at
+// it, so that every corner lane (row pitch BW) lands on zeros.
+__host__ __device__ constexpr int zero_band_bytes(int BW, int cs) {
+  return ((BW + 2) * cs + 127) / 128 * 128;
 }
 
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-               : "memory");
+// Shared-memory bytes of the forward kernel.
+__host__ __device__ constexpr size_t fwd_tiled_smem(int nbuf, uint32_t box_stride, int BW, int cs) {
+  return size_t(nbuf) * box_stride + size_t(zero_band_bytes(BW, cs)) +
+         size_t(kTiledWarps) * kFwdRegion + kFwdTailBytes;
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded wait for the phase with the given parity: gives up after 2^22
-// polls or one second, whichever comes first.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 0; i < (1u << 22); ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u && global_ns() - t0 > 1000000000ull) return false;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                             int c0, int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
-      "r"(smem_addr(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(const void* p) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(smem_addr(p)));
-  return v;
-}
-
-__device__ __forceinline__ uint4 ldg128(const void* p) {
-  uint4 v;
-  asm("ld.global.nc.v4.b32 {%0,%1,%2,%3}, [%4];"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p));
-  return v;
-}
-
-// Item -> (n, ho0, wo0, g); g is the fastest index, so consecutive items of a
-// CTA reuse one input neighbourhood (different channels) and one run of
-// offset/mask rows.
-struct ItemCoord {
-  int n, ho0, wo0, g;
-};
-
-__device__ __forceinline__ ItemCoord item_coord(const TiledParams& t, int item) {
-  ItemCoord c;
-  const uint32_t tile = fdiv(uint32_t(item), t.fd_G);
-  c.g = item - int(tile) * t.G;
-  const uint32_t n = fdiv(tile, t.fd_tiles);
-  const uint32_t rem = tile - n * uint32_t(t.nTY * t.nTX);
-  const uint32_t ty = fdiv(rem, t.fd_nTX);
-  c.n = int(n);
-  c.ho0 = int(ty) * t.TH;
-  c.wo0 = int(rem - ty * uint32_t(t.nTX)) * t.TW;
-  return c;
-}
-
-template <typename T>
-struct TiledIO;
-template <>
-struct TiledIO<float> {
-  static constexpr int kEpc = 4;  // channels per 16-byte piece
-  using Pair = float2;
-  using One = float;
-  __device__ __forceinline__ static Pair ld_pair(const void* base, size_t i) {
-    return __ldg(reinterpret_cast<const float2*>(base) + i);
-  }
-  __device__ __forceinline__ static One ld_one(const void* base, size_t i) {
-    return __ldg(reinterpret_cast<const float*>(base) + i);
-  }
-  __device__ __forceinline__ static float2 pair(Pair p) { return p; }
-  __device__ __forceinline__ static float one(One v) { return v; }
-  // acc += w * (the piece's 4 channels), as two packed fp32x2 FMAs.
-  __device__ __forceinline__ static void fma16(float2* acc, float2 w, const uint4& v) {
-    acc[0] = __ffma2_rn(make_float2(__uint_as_float(v.x), __uint_as_float(v.y)), w, acc[0]);
-    acc[1] = __ffma2_rn(make_float2(__uint_as_float(v.z), __uint_as_float(v.w)), w, acc[1]);
-  }
-  __device__ __forceinline__ static uint4 pack(const float (&acc)[4]) {
-    return make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
-                      __float_as_uint(acc[3]));
-  }
-};
-template <>
-struct TiledIO<__nv_bfloat16> {
-  static constexpr int kEpc = 8;
-  using Pair = uint32_t;
-  using One = unsigned short;
-  __device__ __forceinline__ static Pair ld_pair(const void* base, size_t i) {
-    return __ldg(reinterpret_cast<const unsigned int*>(base) + i);
-  }
-  __device__ __forceinline__ static One ld_one(const void* base, size_t i) {
-    return __ldg(reinterpret_cast<const unsigned short*>(base) + i);
-  }
-  __device__ __forceinline__ static float2 pair(Pair p) {
-    return make_float2(bf16lo_to_f32(p), bf16hi_to_f32(p));
-  }
-  __device__ __forceinline__ static float one(One v) { return __uint_as_float(uint32_t(v) << 16); }
-  // acc += w * (the piece's 8 channels, widened), as four packed fp32x2 FMAs.
-  __device__ __forceinline__ static void fma16(float2* acc, float2 w, const uint4& v) {
-    acc[0] = __ffma2_rn(make_float2(bf16lo_to_f32(v.x), bf16hi_to_f32(v.x)), w, acc[0]);
-    acc[1] = __ffma2_rn(make_float2(bf16lo_to_f32(v.y), bf16hi_to_f32(v.y)), w, acc[1]);
-    acc[2] = __ffma2_rn(make_float2(bf16lo_to_f32(v.z), bf16hi_to_f32(v.z)), w, acc[2]);
-    acc[3] = __ffma2_rn(make_float2(bf16lo_to_f32(v.w), bf16hi_to_f32(v.w)), w, acc[3]);
-  }
-  __device__ __forceinline__ static uint4 pack(const float (&acc)[8]) {
-    return make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                      pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-  }
-};
-
-// Tap records, written by the unit's owner lane in phase A and read by the
-// unit's eight lanes in phase B.  A unit slot holds w[9][4] (the tap's four
-// corner weights, mask weight folded in) followed by code[9], of which the
-// 8-tap set (remove_center) uses the first eight.  code >= 0 is
-// the byte offset in the box of corner (y0, x0) when the whole 2x2 footprint
-// lies in the box; otherwise code = INT_MIN | (y0 + 1) << 15 | (x0 + 1), and
-// the corners are read from global memory ((y0, x0) = (32766, 32766) marks a
-// sample that contributes nothing).
-constexpr int kFarCell = 32766;
-__device__ __forceinline__ int far_code(int y0, int x0) {
-  return int(0x80000000u | (uint32_t(y0 + 1) << 15) | uint32_t(x0 + 1));
-}
-// 184 bytes: w[9][4] (144) then code[9] (36), padded to a multiple of 8 so
-// that staged fp32 offset pairs (8-byte float2) stay aligned in every slot;
-// 46 words per slot also keeps both the 32-lane phase-A reads and the
-// four-unit phase-B reads free of bank conflicts.
-constexpr int kSlotBytes = 184;
-constexpr int kCodeAt = kTiledMaxTaps * 16;
-constexpr int kLogitAt = 80;               // staged mask values (before the records)
-constexpr int kFarMaskAt = kCodeAt + kTiledMaxTaps * 4;  // 180: bit k = tap k is read from global
-static_assert(kSlotBytes % 8 == 0 && kFarMaskAt + 4 <= kSlotBytes, "slot layout");
-
-// Phase-B lane roles: 8 lanes per unit, lane li = (corner r = li >> 1, q = li & 1).
-// A 32-byte group (bf16 x 16) is one 16-byte piece per lane: piece q.  A
-// 64-byte group (fp32 x 16) is two pieces per lane; in read j a lane takes
-// piece (2j + q + 2*dy) & 3, so the eight lanes of a unit touch eight
-// different bank quads when the box row pitch is even.
-template <int CS>
-struct LaneRole {
-  static constexpr int kPieces = CS / 32;  // pieces per lane: 1 or 2
-  __device__ __forceinline__ static int piece(int j, int q, int dyc) {
-    return CS == 32 ? q : ((2 * j + q + 2 * dyc) & 3);
-  }
-};
-
-// KKS: 9 (the 3x3 window) or 8 (the window without its centre).
-template <typename T, int CS, int KKS, bool SOFTMAX>
+// KKS: 9 (the 3x3 window) or 8 (the window without its centre).  FAR: some
+// footprint can leave the box (the box does not cover the whole image).
+template <typename T, int KKS, bool SOFTMAX, bool FAR>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     dcn_forward_tiled_kernel(const __grid_constant__ CUtensorMap xmap, const TiledArgs a) {
   using IO = TiledIO<T>;
   using Pair = typename IO::Pair;
   using One = typename IO::One;
-  using Role = LaneRole<CS>;
   constexpr int KK = KKS, K = tap_side(KKS);
   static_assert(K == 3 && KK <= kTiledMaxTaps, "the tiled kernel serves 3x3 tap sets");
-  constexpr int LU = 8;            // phase-B lanes per unit
-  constexpr int UPW = 32 / LU;     // units per phase-B step
-  constexpr int NP = Role::kPieces;
-  constexpr int EPC = IO::kEpc;    // channels per piece
-  static_assert(CS == 32 || CS == 64, "the tiled kernel serves 32- or 64-byte groups");
-  static_assert(KK * sizeof(Pair) <= kLogitAt && kLogitAt + KK * sizeof(One) <= kSlotBytes,
-                "staged inputs fit in a slot");
+  constexpr int CS = 16 * int(sizeof(T));  // bytes of one pixel of the group
+  constexpr int NP = CS / 16;              // 16-byte pieces per corner: 2 (bf16) or 4 (fp32)
 
   const TiledParams& t = a.t;
   extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* bufs = smem;
-  unsigned char* slots = smem + 2 * size_t(t.box_stride);
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(slots + size_t(kTiledWarps) * kTiledBatch * kSlotBytes);
-  uint64_t* empty = full + 2;
-  int* s_abort = reinterpret_cast<int*>(empty + 2);
-  unsigned char* zero = reinterpret_cast<unsigned char*>(full) + kTiledZeroAt;
+  const int nbuf = t.nbuf;
+  unsigned char* const bufs = smem;
+  unsigned char* const zero = smem + size_t(nbuf) * t.box_stride;
+  unsigned char* const regions = zero + zero_band_bytes(t.BW, CS);
+  uint64_t* const full = reinterpret_cast<uint64_t*>(regions + size_t(kTiledWarps) * kFwdRegion);
+  uint64_t* const empty = full + kTiledMaxBufs;
+  int* const s_abort = reinterpret_cast<int*>(empty + kTiledMaxBufs);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(&empty[0], kTiledWarps);
-    mbar_init(&empty[1], kTiledWarps);
+    for (int i = 0; i < nbuf; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kTiledWarps);
+    }
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (tid < kTiledZeroBytes / 4) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
+  for (int i = tid; i < zero_band_bytes(t.BW, CS) / 16; i += kTiledThreads)
+    reinterpret_cast<uint4*>(zero)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
   volatile int* abort_flag = s_abort;
 
-  // ---- producer warp: one TMA box per item, two buffers in flight ----
+  // ---- producer warp: one TMA box per item, nbuf buffers in flight ----
   if (warp == kTiledWarps) {
     if (lane != 0) return;
-    int i = 0;
+    int i = 0, b = 0;
+    uint32_t ph = 0;  // parity of this round over the buffers
     for (;; ++i) {
       const int item = int(blockIdx.x) + i * int(gridDim.x);
       if (item >= t.items || *abort_flag) break;
-      const int b = i & 1;
-      if (i >= 2 && !mbar_wait_bounded(&empty[b], ((i >> 1) - 1) & 1)) {
-        atomicOr(a.error_word, 1u);
+      if (i >= nbuf && !mbar_wait_bounded(&empty[b], ph ^ 1u)) {
+        atomicOr(a.error_word, kErrTimeout);
         *abort_flag = 1;
         break;
       }
       const ItemCoord c = item_coord(t, item);
-      if (t.inject_stall && i == 0) continue;  // the first box never arrives
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&full[b], t.box_bytes);
-      tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg,
-                   c.wo0 * t.stride_w - t.pad_w - t.halo, c.ho0 * t.stride - t.pad - t.halo, c.n);
+      if (!(t.inject_stall && i == 0)) {  // test knob: the first box never arrives
+        const int Y0 = box_origin(c.ho0 * t.stride - t.pad - t.halo, t.BH, t.H, t.clamp_box);
+        const int X0 = box_origin(c.wo0 * t.stride_w - t.pad_w - t.halo, t.BW, t.W, t.clamp_box);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&full[b], t.box_bytes);
+        tma_load_box(bufs + size_t(b) * t.box_stride, &xmap, &full[b], c.g * t.Cg, X0, Y0, c.n);
+      }
+      if (++b == nbuf) {
+        b = 0;
+        ph ^= 1u;
+      }
     }
-    // Copies issued for items i-2 and i-1 may still be landing: wait for them
+    // Copies issued for the last items may still be landing: wait for them
     // (bounded) before this thread, possibly the CTA's last, exits.
-    for (int j = i - 2; j < i; ++j)
-      if (j >= 0) (void)mbar_wait_bounded(&full[j & 1], (j >> 1) & 1);
+    for (int j = i - nbuf < 0 ? 0 : i - nbuf; j < i; ++j)
+      if (!(t.inject_stall && j == 0))
+        (void)mbar_wait_bounded(&full[j % nbuf], uint32_t(j / nbuf) & 1u);
     return;
   }
 
   // ---- consumer warps ----
-  unsigned char* myslots = slots + size_t(warp) * kTiledBatch * kSlotBytes;
-  const int ul = lane / LU;         // phase B: unit of this lane within a step
-  const int li = lane - ul * LU;
-  const int r = li >> 1, q = li & 1;
-  const int dyc = r >> 1, dxc = r & 1;
-  const unsigned umask = 0xFFu << (ul * LU);
-  int cdelta[NP];
-#pragma unroll
-  for (int j = 0; j < NP; ++j)
-    cdelta[j] = (dyc * t.BW + dxc) * CS + Role::piece(j, q, dyc) * 16;
-  const size_t pixB = size_t(t.C) * sizeof(T);
+  unsigned char* const reg = regions + size_t(warp) * kFwdRegion;
+  const uint32_t reg_a = smem_addr(reg);
+  const uint32_t zero_a = smem_addr(zero);
+  // phase-B roles: unit u8 of the step, corner r = (dy, dx), unit parity rho
+  const int u8 = lane >> 2, r = lane & 3, dy = r >> 1, dx = r & 1, rho = u8 & 1;
+  // piece rotation: bf16 lanes read pieces rho, 1 - rho; fp32 lanes read piece
+  // j ^ rot in their j-th read, rot = 2 dy + rho
+  const int rot = NP == 2 ? rho : 2 * dy + rho;
+  const uint32_t corner_b = uint32_t((dy * t.BW + dx) * CS + 16 * rot);
   const int npx = t.TH * t.TW;
   const int nb = t.batches;
+  const float Hf = float(t.H), Wf = float(t.W);
+  const size_t pixB = size_t(t.C) * sizeof(T);
+  const size_t x_bytes = size_t(t.N) * t.H * t.W * pixB;  // bounds-checked build
+  const size_t out_bytes = size_t(t.N) * t.Ho * t.Wo * pixB;
   // the staging element e = lane + 32 k (k < KK) belongs to unit e / KK, tap e % KK
   int st_unit[KK], st_tap[KK];
 #pragma unroll
@@ -332,45 +175,35 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     st_tap[k] = (lane + 32 * k) - st_unit[k] * KK;
   }
 
-  // Batch beta of this CTA (over all its items) -> this lane's unit.
-  auto batch_unit = [&](int beta, bool& valid, int& ho, int& wo, size_t& qbase) {
+  // Unit of this lane in batch beta (over all the CTA's items): element offset
+  // of its first offset pair / mask value, or ~0 outside the output.
+  auto batch_unit = [&](int beta, int& ho, int& wo, uint32_t& q) {
     const int il = beta / nb;
     const int v = (beta - il * nb) * kTiledBatch + lane;
-    const int item = int(blockIdx.x) + il * int(gridDim.x);
-    valid = false;
-    ho = wo = 0;
-    qbase = 0;
-    if (item >= t.items) return;
-    const ItemCoord c = item_coord(t, item);
+    const ItemCoord c = item_coord(t, int(blockIdx.x) + il * int(gridDim.x));
     const int rr = int(fdiv(uint32_t(v), t.fd_TW));
     ho = c.ho0 + rr;
     wo = c.wo0 + (v - rr * t.TW);
-    valid = (v < npx) && (ho < t.Ho) && (wo < t.Wo);
-    qbase = ((size_t(c.n * t.Ho + ho) * t.Wo + wo) * t.G + c.g) * KK;
+    const bool valid = (v < npx) && (ho < t.Ho) && (wo < t.Wo);
+    q = valid ? (uint32_t((c.n * t.Ho + ho) * t.Wo + wo) * uint32_t(t.G) + uint32_t(c.g)) *
+                    uint32_t(KK)
+              : ~0u;
+    return c;
   };
 
-  // Raw inputs of the next batch, prefetched in the staging layout.
   const size_t n_entries = size_t(t.N) * t.Ho * t.Wo * t.G * KK;  // offset pairs, mask values
-  const size_t x_bytes = size_t(t.N) * t.H * t.W * pixB;            // bounds-checked build
-  const size_t out_bytes = size_t(t.N) * t.Ho * t.Wo * pixB;
   Pair pf_pair[KK];
   One pf_one[KK];
   auto prefetch = [&](int beta) {
-    bool valid;
     int ho, wo;
-    size_t qbase;
-    batch_unit(beta, valid, ho, wo, qbase);
-    const unsigned long long qv = valid ? (unsigned long long)qbase : ~0ull;
+    uint32_t q;
+    batch_unit(beta, ho, wo, q);
 #pragma unroll
     for (int k = 0; k < KK; ++k) {
-      const unsigned long long src = __shfl_sync(0xFFFFFFFFu, qv, st_unit[k]);
-      if (src != ~0ull && in_range(size_t(src) + st_tap[k], n_entries)) {
-        pf_pair[k] = IO::ld_pair(a.off, size_t(src) + st_tap[k]);
-        pf_one[k] = IO::ld_one(a.mask, size_t(src) + st_tap[k]);
-      } else {
-        pf_pair[k] = Pair();
-        pf_one[k] = One();
-      }
+      const uint32_t src = __shfl_sync(0xFFFFFFFFu, q, st_unit[k]);
+      const bool ok = src != ~0u && in_range(size_t(src) + st_tap[k], n_entries);
+      pf_pair[k] = ok ? IO::ld_pair(a.off, size_t(src) + st_tap[k]) : Pair();
+      pf_one[k] = ok ? IO::ld_one(a.mask, size_t(src) + st_tap[k]) : One();
     }
   };
 
@@ -380,56 +213,58 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   int beta = warp;
   if (beta < total_batches) prefetch(beta);
 
+  int b = 0;
+  uint32_t ph = 0;
   for (int il = 0; il < n_items_cta; ++il) {
-    const int b = il & 1;
-    const int item = int(blockIdx.x) + il * int(gridDim.x);
     // Every consumer warp observes every item's box, even one in which it has
-    // no batch: that keeps each warp within one item of the producer, so the
-    // parity it waits for is never ambiguous and it arrives on `empty` exactly
-    // once per phase.
-    if (!mbar_wait_bounded(&full[b], (il >> 1) & 1)) {
-      atomicOr(a.error_word, 1u);
+    // no batch: that keeps each warp within nbuf - 1 items of the slowest, so
+    // the parity it waits for is never ambiguous and it arrives on `empty`
+    // exactly once per phase.
+    if (!mbar_wait_bounded_sleep(&full[b], ph)) {
+      atomicOr(a.error_word, kErrTimeout);
       *abort_flag = 1;
     }
     if (*abort_flag) break;
+    const int item = int(blockIdx.x) + il * int(gridDim.x);
     const ItemCoord c = item_coord(t, item);
-    const unsigned char* box = bufs + size_t(b) * t.box_stride;
-    // Phase B reads piece j of a tap at box + min(code, zlim) + cdelta[j]: a
-    // box tap's code (>= 0, below the box size) is kept, a far or dead tap's
-    // (negative, so above 2^31 unsigned) becomes zlim, which puts this lane's
-    // pieces at zero + 48 + (cdelta[j] - cdelta[0]), inside the zero area
-    // (pieces of one lane lie at most 32 bytes apart).  zlim exceeds every box
-    // offset because the zero area lies after both buffers and the slots.
-    const uint32_t zlim = uint32_t((zero + 48 - cdelta[0]) - box);
-    const int Y0 = c.ho0 * t.stride - t.pad - t.halo;
-    const int X0 = c.wo0 * t.stride_w - t.pad_w - t.halo;
-    const char* ximg = reinterpret_cast<const char*>(a.x) + size_t(c.n) * t.H * t.W * pixB +
-                       size_t(c.g) * CS;
+    const unsigned char* const box = bufs + size_t(b) * t.box_stride;
+    const uint32_t box_a = smem_addr(box);
+    const uint32_t lane_base = box_a + corner_b;
+    const uint32_t zoff = zero_a - box_a;  // box-relative offset of the zero band
+    const int Y0 = box_origin(c.ho0 * t.stride - t.pad - t.halo, t.BH, t.H, t.clamp_box);
+    const int X0 = box_origin(c.wo0 * t.stride_w - t.pad_w - t.halo, t.BW, t.W, t.clamp_box);
+    const char* const ximg = reinterpret_cast<const char*>(a.x) +
+                             size_t(c.n) * t.H * t.W * pixB + size_t(c.g) * CS;
 
     for (; beta < (il + 1) * nb; beta += kTiledWarps) {
-      // Staging: the prefetched inputs go to the unit slots.
+      // Staging: the prefetched inputs go to the region in their global order.
 #pragma unroll
       for (int k = 0; k < KK; ++k) {
-        unsigned char* sl = myslots + st_unit[k] * kSlotBytes;
-        reinterpret_cast<Pair*>(sl)[st_tap[k]] = pf_pair[k];
-        reinterpret_cast<One*>(sl + kLogitAt)[st_tap[k]] = pf_one[k];
+        const int e = lane + 32 * k;
+        if (sizeof(T) == 4)
+          reinterpret_cast<Pair*>(reg)[e] = pf_pair[k];
+        else
+          reinterpret_cast<uint32_t*>(reg)[e] = *reinterpret_cast<const uint32_t*>(&pf_pair[k]);
+        reinterpret_cast<float*>(reg + kFwdStageMask)[e] = IO::one(pf_one[k]);
       }
-      bool valid;
       int ho, wo;
-      size_t qbase;
-      batch_unit(beta, valid, ho, wo, qbase);
+      uint32_t q;
+      batch_unit(beta, ho, wo, q);
+      const bool valid = q != ~0u;
       __syncwarp();
 
-      // Phase A: this lane's unit -> softmax, then per tap the footprint code
-      // and the four corner weights.
+      // Phase A: this lane's unit -> softmax, then per tap the corner weights
+      // and the box offset of corner (y0, x0).
       {
-        unsigned char* sl = myslots + lane * kSlotBytes;
         float2 d[KK];
         float m[KK];
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          d[k] = IO::pair(reinterpret_cast<const Pair*>(sl)[k]);
-          m[k] = IO::one(reinterpret_cast<const One*>(sl + kLogitAt)[k]);
+          const int e = lane * KK + k;
+          d[k] = sizeof(T) == 4
+                     ? IO::pair(reinterpret_cast<const Pair*>(reg)[e])
+                     : IO::pair(*reinterpret_cast<const Pair*>(reg + 4 * e));
+          m[k] = reinterpret_cast<const float*>(reg + kFwdStageMask)[e];
         }
         if (SOFTMAX) {
           float mx = m[0];
@@ -445,165 +280,198 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
           for (int k = 0; k < KK; ++k) m[k] *= inv;
         }
-        __syncwarp();  // every lane has read its staged inputs
-        float* wsl = reinterpret_cast<float*>(sl);
-        int* csl = reinterpret_cast<int*>(sl + kCodeAt);
-        unsigned farmask = 0u;
+        __syncwarp();  // every lane has read its staged inputs: the records overwrite them
+        const int yb = ho * t.stride - t.pad, xb = wo * t.stride_w - t.pad_w;
+        uint32_t fm = 0u;
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
           const int ka = tap_pos(KK, k) / K, kb = tap_pos(KK, k) % K;
-          const float Y = tap_coord(ho * t.stride - t.pad + ka * t.dil, t.sigma, d[k].y);
-          const float X = tap_coord(wo * t.stride_w - t.pad_w + kb * t.dil_w, t.sigma, d[k].x);
-          const Footprint f = footprint(Y, X, t.H, t.W);
-          const bool live = valid && f.in_support;
-          const int by = f.y0 - Y0, bx = f.x0 - X0;
-          int code;
-          if (!live) code = far_code(kFarCell, kFarCell);
-          else if (by >= 0 && by + 1 < t.BH && bx >= 0 && bx + 1 < t.BW)
-            code = (by * t.BW + bx) * CS;
-          else {
-            code = far_code(f.y0, f.x0);
-            farmask |= 1u << k;
-          }
-          const float mk = live ? m[k] : 0.f;
-          const float hy = 1.f - f.ly, hx = 1.f - f.lx;
-          wsl[4 * k + 0] = hy * hx * mk;
-          wsl[4 * k + 1] = hy * f.lx * mk;
-          wsl[4 * k + 2] = f.ly * hx * mk;
-          wsl[4 * k + 3] = f.ly * f.lx * mk;
-          csl[k] = code;
+          const float Y = tap_coord(yb + ka * t.dil, t.sigma, d[k].y);
+          const float X = tap_coord(xb + kb * t.dil_w, t.sigma, d[k].x);
+          const float fy = floorf(Y), fx = floorf(X);
+          const int y0 = __float2int_rd(Y), x0 = __float2int_rd(X);  // NaN -> 0, inf saturates
+          const float ly = Y - fy, lx = X - fx;
+          const int by = y0 - Y0, bx = x0 - X0;
+          const bool inbox = unsigned(by) < unsigned(t.BH - 1) && unsigned(bx) < unsigned(t.BW - 1);
+          const bool box_tap = valid && inbox && (Y == Y) && (X == X);
+          const bool far = FAR && !box_tap && valid && (Y >= -1.0f) && (Y < Hf) &&
+                           (X >= -1.0f) && (X < Wf);
+          const float hy = 1.f - ly, hx = 1.f - lx;
+          const float wy0 = hy * m[k], wy1 = ly * m[k];
+          float4 w;
+          if (box_tap)
+            w = make_float4(wy0 * hx, wy0 * lx, wy1 * hx, wy1 * lx);
+          else if (far)
+            w = make_float4(wy0, wy1, lx,
+                            __uint_as_float((uint32_t(y0 + 1) << kFarShift) | uint32_t(x0 + 1)));
+          else
+            w = make_float4(0.f, 0.f, 0.f, 0.f);
+          reinterpret_cast<float4*>(reg + kFwdRegW)[k * kTiledBatch + lane] = w;
+          reinterpret_cast<uint32_t*>(reg + kFwdRegOff)[k * kTiledBatch + lane] =
+              box_tap ? uint32_t((by * t.BW + bx) * CS) : zoff;
+          fm |= far ? (1u << k) : 0u;
         }
-        *reinterpret_cast<unsigned*>(sl + kFarMaskAt) = farmask;
+        reinterpret_cast<uint32_t*>(reg + kFwdRegFm)[lane] = fm;
+        reinterpret_cast<uint32_t*>(reg + kFwdRegOut)[lane] =
+            valid ? uint32_t(((c.n * t.Ho + ho) * t.Wo + wo) * t.C + c.g * t.Cg) : ~0u;
       }
       __syncwarp();
       // The next batch's inputs are loaded while this one is gathered.
       if (beta + kTiledWarps < total_batches) prefetch(beta + kTiledWarps);
 
-      // Phase B: UPW units per step, eight lanes each.  Box taps are
-      // branch-free (predicated shared-memory reads); a unit's taps whose
-      // footprint leaves the box ("far" taps) read global memory: the first
-      // one of each unit is fetched a step ahead, any further ones in a
-      // warp-uniform loop.
-      const int v0 = (beta - il * nb) * kTiledBatch;
-      // Global read of this lane's corner piece(s) for tap k of the unit in slot sl.
-      auto far_fetch = [&](const unsigned char* sl, int k, uint4 (&fv)[NP], float& fw) {
-        const int code = reinterpret_cast<const int*>(sl + kCodeAt)[k];
-        fw = reinterpret_cast<const float*>(sl)[4 * k + r];
-        const int yc = ((code >> 15) & 0x7FFF) - 1 + dyc;
-        const int xc = (code & 0x7FFF) - 1 + dxc;
+      // Far taps: this lane's corner of tap k of unit u from global memory
+      // (zeros outside the image) and its weight.
+      auto far_fetch = [&](int u, int k, uint4 (&fv)[NP], float& fw) {
+        const uint4 rw = lds128_a(reg_a + kFwdRegW + uint32_t(k * kTiledBatch + u) * 16u);
+        const uint32_t pk = rw.w;
+        const int yc = int(pk >> kFarShift) - 1 + dy;
+        const int xc = int(pk & ((1u << kFarShift) - 1u)) - 1 + dx;
         const bool in = unsigned(yc) < unsigned(t.H) && unsigned(xc) < unsigned(t.W);
+        const float lx = __uint_as_float(rw.z);
+        fw = in ? __uint_as_float(dy ? rw.y : rw.x) * (dx ? lx : 1.f - lx) : 0.f;
         const char* gp = ximg + (size_t(in ? yc : 0) * t.W + (in ? xc : 0)) * pixB;
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          fv[j] = (in && in_tensor(gp + Role::piece(j, q, dyc) * 16, 16, a.x, x_bytes))
-                      ? ldg128(gp + Role::piece(j, q, dyc) * 16)
-                      : make_uint4(0u, 0u, 0u, 0u);
-        if (!in) fw = 0.f;
+        for (int j = 0; j < NP; ++j) {
+          const char* pp = gp + 16 * (j ^ rot);
+          fv[j] = ldg128_pred(pp, in && in_tensor(pp, 16, a.x, x_bytes));
+        }
       };
-      auto far_first = [&](int u, uint4 (&fv)[NP], float& fw) {
-        const unsigned char* sl = myslots + u * kSlotBytes;
-        const unsigned fm = *reinterpret_cast<const unsigned*>(sl + kFarMaskAt);
+      // The first far tap of unit u, fetched one step before it is used; fm
+      // returns the unit's other far taps.
+      auto far_first = [&](int u, uint4 (&fv)[NP], float& fw, uint32_t& fm) {
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(fm) : "r"(reg_a + kFwdRegFm + 4u * u));
         fw = 0.f;
 #pragma unroll
         for (int j = 0; j < NP; ++j) fv[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (fm) far_fetch(sl, __ffs(fm) - 1, fv, fw);
+        if (fm != 0u) {
+          far_fetch(u, __ffs(fm) - 1, fv, fw);
+          fm &= fm - 1u;
+        }
       };
+      // (2-byte storage only: for fp32 the two prefetched pieces sets would cost
+      // more registers than the rare far taps of fp32 workloads gain)
+      constexpr bool kAhead = FAR && NP == 2;
       uint4 fv_cur[NP], fv_nxt[NP];
-      float fw_cur, fw_nxt;
-      far_first(ul, fv_cur, fw_cur);
+      float fw_cur = 0.f, fw_nxt = 0.f;
+      uint32_t fm_cur = 0u, fm_nxt = 0u;
+      if (kAhead) far_first(u8, fv_cur, fw_cur, fm_cur);
+
+      // Phase B: 8 units per step, one lane per corner.
 #pragma unroll 1
-      for (int s = 0; s < kTiledBatch / UPW; ++s) {
-        const int u = s * UPW + ul;
-        const unsigned char* sl = myslots + u * kSlotBytes;
-        const float* wsl = reinterpret_cast<const float*>(sl) + r;
-        const int* csl = reinterpret_cast<const int*>(sl + kCodeAt);
-        if (s + 1 < kTiledBatch / UPW) far_first(u + UPW, fv_nxt, fw_nxt);
-        constexpr int NV = NP * EPC;  // 8 values per lane, as 4 packed pairs
-        static_assert(NV == 8, "eight accumulated values per lane");
-        float2 acc[NV / 2];
+      for (int s = 0; s < kTiledBatch / 8; ++s) {
+        const int u = s * 8 + u8;
+        if (kAhead && s + 1 < kTiledBatch / 8) far_first(u + 8, fv_nxt, fw_nxt, fm_nxt);
+        float2 acc[8];
 #pragma unroll
-        for (int e = 0; e < NV / 2; ++e) acc[e] = make_float2(0.f, 0.f);
+        for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
+        const uint32_t wa = reg_a + kFwdRegW + uint32_t(u) * 16u + uint32_t(r) * 4u;
+        const uint32_t oa = reg_a + kFwdRegOff + uint32_t(u) * 4u;
 #pragma unroll
         for (int k = 0; k < KK; ++k) {
-          const uint32_t off = min(uint32_t(csl[k]), zlim);  // far or dead: the zero area
-          const float w = wsl[4 * k];
+          float w;
+          uint32_t off;
+          asm volatile("ld.shared.f32 %0, [%1];" : "=f"(w) : "r"(wa + k * kTiledBatch * 16));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(off) : "r"(oa + k * kTiledBatch * 4));
           const float2 w2 = make_float2(w, w);
+          const uint32_t a0 = lane_base + off;
 #pragma unroll
-          for (int j = 0; j < NP; ++j) IO::fma16(acc + j * (EPC / 2), w2, lds128(box + off + cdelta[j]));
+          for (int j = 0; j < NP; ++j)
+            IO::fma16(acc + j * (8 / NP), w2, lds128_a(a0 ^ uint32_t(16 * j)));
         }
-        // First far tap (fetched during the previous step), then any others.
+        if (FAR) {
+          // The unit's first far tap (fetched during the previous step), then
+          // any others in a warp-uniform loop.
+          uint32_t fm = fm_cur;
+          if (kAhead) {
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          IO::fma16(acc + j * (EPC / 2), make_float2(fw_cur, fw_cur), fv_cur[j]);
-        unsigned more = *reinterpret_cast<const unsigned*>(sl + kFarMaskAt);
-        more &= more - 1u;
-        while (__any_sync(0xFFFFFFFFu, more != 0u)) {
-          if (more) {
-            uint4 fv[NP];
-            float fw;
-            far_fetch(sl, __ffs(more) - 1, fv, fw);
-#pragma unroll
-            for (int j = 0; j < NP; ++j) IO::fma16(acc + j * (EPC / 2), make_float2(fw, fw), fv[j]);
-            more &= more - 1u;
-          }
-        }
-        // Lanes with dy = 1 hold their pieces in the other order (fp32 only).
-        if (NP == 2 && dyc) {
-#pragma unroll
-          for (int e = 0; e < EPC / 2; ++e) {
-            const float2 tmp = acc[e];
-            acc[e] = acc[EPC / 2 + e];
-            acc[EPC / 2 + e] = tmp;
-          }
-        }
-        // Reduce-scatter over the four corner lanes of each piece: the dx pair
-        // splits the 8 values in halves, the dy pair splits those again, so each
-        // lane ends with 2 summed values: value index 4*dxc + 2*dyc + {0, 1}.
-        float h4[4], h2[2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float lo = (i & 1) ? acc[i >> 1].y : acc[i >> 1].x;           // value i
-          const float hi = (i & 1) ? acc[2 + (i >> 1)].y : acc[2 + (i >> 1)].x;  // value 4 + i
-          const float keep = dxc ? hi : lo;
-          const float send = dxc ? lo : hi;
-          h4[i] = keep + __shfl_xor_sync(umask, send, 2);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float keep = dyc ? h4[2 + i] : h4[i];
-          const float send = dyc ? h4[i] : h4[2 + i];
-          h2[i] = keep + __shfl_xor_sync(umask, send, 4);
-        }
-        const int v = v0 + u;
-        const int rr = int(fdiv(uint32_t(v), t.fd_TW));
-        const int uho = c.ho0 + rr, uwo = c.wo0 + (v - rr * t.TW);
-        if (v < npx && uho < t.Ho && uwo < t.Wo) {
-          const size_t pix = size_t(c.n * t.Ho + uho) * t.Wo + uwo;
-          char* op = reinterpret_cast<char*>(a.out) + (pix * t.C + size_t(c.g) * t.Cg) * sizeof(T);
-          // channel of h2[0]: piece p, element 2*dyc (+ 4*dxc for bf16's 8-wide pieces)
-          if (CS == 32) {
-            const int ch = 8 * q + 4 * dxc + 2 * dyc;
-            const uint32_t w = pack_bf16x2(h2[0], h2[1]);
-            if (in_tensor(op + ch * 2, 4, a.out, out_bytes))
-              asm volatile("st.global.b32 [%0], %1;" ::"l"(op + ch * 2), "r"(w) : "memory");
+            for (int j = 0; j < NP; ++j)
+              IO::fma16(acc + j * (8 / NP), make_float2(fw_cur, fw_cur), fv_cur[j]);
           } else {
-            const int ch = 4 * (q + 2 * dxc) + 2 * dyc;
-            if (in_tensor(op + ch * 4, 8, a.out, out_bytes))
-              asm volatile("st.global.v2.f32 [%0], {%1, %2};" ::"l"(op + ch * 4), "f"(h2[0]),
-                         "f"(h2[1])
-                         : "memory");
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(fm) : "r"(reg_a + kFwdRegFm + 4u * u));
+          }
+          while (__any_sync(0xFFFFFFFFu, fm != 0u)) {
+            if (fm != 0u) {
+              uint4 fv[NP];
+              float fw;
+              far_fetch(u, __ffs(fm) - 1, fv, fw);
+#pragma unroll
+              for (int j = 0; j < NP; ++j)
+                IO::fma16(acc + j * (8 / NP), make_float2(fw, fw), fv[j]);
+              fm &= fm - 1u;
+            }
+          }
+          if (kAhead) {
+#pragma unroll
+            for (int j = 0; j < NP; ++j) fv_cur[j] = fv_nxt[j];
+            fw_cur = fw_nxt;
+            fm_cur = fm_nxt;
           }
         }
+        // Reduce-scatter over the unit's four corner lanes, then store.
+        uint32_t ob;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ob) : "r"(reg_a + kFwdRegOut + 4u * u));
+        if constexpr (NP == 2) {
+          // acc[0..3]: piece rho (channels 8 rho ..), acc[4..7]: piece 1 - rho.
+          // dx partner: keep piece rho ^ dx, then dy partner: keep half dy of it.
+          float2 k4[4];
 #pragma unroll
-        for (int j = 0; j < NP; ++j) fv_cur[j] = fv_nxt[j];
-        fw_cur = fw_nxt;
+          for (int i = 0; i < 4; ++i) {
+            const float2 keep = dx ? acc[4 + i] : acc[i];
+            const float2 send = dx ? acc[i] : acc[4 + i];
+            k4[i].x = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, 1);
+            k4[i].y = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, 1);
+          }
+          float2 k2[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float2 keep = dy ? k4[2 + i] : k4[i];
+            const float2 send = dy ? k4[i] : k4[2 + i];
+            k2[i].x = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, 2);
+            k2[i].y = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, 2);
+          }
+          if (ob != ~0u) {
+            char* op = reinterpret_cast<char*>(a.out) +
+                       (size_t(ob) + size_t(8 * (rho ^ dx) + 4 * dy)) * sizeof(T);
+            if (in_tensor(op, 8, a.out, out_bytes))
+              asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(op),
+                           "r"(pack2<T>(k2[0].x, k2[0].y)), "r"(pack2<T>(k2[1].x, k2[1].y))
+                           : "memory");
+          }
+        } else {
+          // slot j = acc[2j, 2j+1] holds piece j ^ rot, rot = 2 dy + rho.  The dy
+          // partner's rot differs in bit 1: both keep slots 0, 1 and add the
+          // partner's slots 2, 3 (the same pieces).  Then the dx partner (same
+          // rot) splits slots 0 and 1.
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[i].x += __shfl_xor_sync(0xFFFFFFFFu, acc[4 + i].x, 2);
+            acc[i].y += __shfl_xor_sync(0xFFFFFFFFu, acc[4 + i].y, 2);
+          }
+          float2 k2[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float2 keep = dx ? acc[2 + i] : acc[i];
+            const float2 send = dx ? acc[i] : acc[2 + i];
+            k2[i].x = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, 1);
+            k2[i].y = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, 1);
+          }
+          if (ob != ~0u) {
+            char* op = reinterpret_cast<char*>(a.out) +
+                       (size_t(ob) + size_t(4 * (dx ^ rot))) * sizeof(T);
+            if (in_tensor(op, 16, a.out, out_bytes))
+              asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(op), "f"(k2[0].x),
+                           "f"(k2[0].y), "f"(k2[1].x), "f"(k2[1].y)
+                           : "memory");
+          }
+        }
       }
-      __syncwarp();  // slots are rewritten by the next batch
+      __syncwarp();  // the region is rewritten by the next batch
     }
     __syncwarp();
-    if (lane == 0) {
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(&empty[b]))
-                   : "memory");
+    if (lane == 0) mbar_arrive(&empty[b]);
+    if (++b == nbuf) {
+      b = 0;
+      ph ^= 1u;
     }
   }
 }

@@ -63,6 +63,12 @@ __device__ __forceinline__ float4 guide_ld4<__nv_bfloat16>(const __nv_bfloat16* 
   return make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y),
                      bf16hi_to_f32(u.y));
 }
+template <>
+__device__ __forceinline__ float4 guide_ld4<__half>(const __half* p) {
+  const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = f16x2_to_f32x2(u.x), b = f16x2_to_f32x2(u.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
 
 __device__ __forceinline__ float4 ld4_or(const float* p, bool ok, float dflt) {
   return ok && p != nullptr ? __ldg(reinterpret_cast<const float4*>(p))
@@ -84,12 +90,17 @@ __device__ __forceinline__ float gelu_erf(float z) {
 // Three CTAs per SM for groups of 8 or 16 lanes (more warps to cover the
 // load latency; measured 10% faster at C = 160); 32-lane groups are
 // left to the compiler (their spills at three cost more than the warps gain).
-template <typename T, int LP>
+// NJS > 0: the quads fill the lane groups exactly (Q = LP * NJS, the channel
+// widths of the InternImage stages), so the quad count is a compile-time
+// constant and no quad needs a bounds predicate; NJS = 0: any C.
+template <typename T, int LP, int NJS>
 __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
     dcn_guide_kernel(const GuideArgs a) {
   constexpr int PPW = 32 / LP;  // pixels per warp
   constexpr int kThreads = kGuideWarps * 32;
   constexpr int CH = kGuideChunk;
+  constexpr bool FULL = NJS > 0;
+  const int NJ = FULL ? NJS : a.NJ;
   // Shared memory: the 9 weight quads and the bias, gamma and beta quads of
   // every channel (12 * Q float4, staged once per CTA), then the conv results
   // of this thread's quads, [quad j][thread]: consecutive lanes touch
@@ -131,13 +142,17 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
     if (y >= a.H) break;  // the same for the whole CTA
     // depthwise 3x3 convolution, CH quads of this lane at a time in registers
     float s = 0.f;
-#pragma unroll 1
-    for (int j0 = 0; j0 < a.NJ; j0 += CH) {
-      float4 acc[CH];
+#pragma unroll(FULL ? 4 : 1)
+    for (int j0 = 0; j0 < NJ; j0 += CH) {
+      float2 acc[2 * CH];  // quad u: channels (x, y) in acc[2u], (z, w) in acc[2u + 1]
 #pragma unroll
       for (int u = 0; u < CH; ++u) {
         const int q = sub + LP * (j0 + u);
-        acc[u] = (j0 + u < a.NJ && col_ok && q < a.Q) ? bias_s[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 b = ((FULL || (j0 + u < NJ && q < a.Q)) && col_ok)
+                             ? bias_s[FULL && CH > NJS ? (u < NJS ? q : sub) : q]
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[2 * u] = make_float2(b.x, b.y);
+        acc[2 * u + 1] = make_float2(b.z, b.w);
       }
 #pragma unroll
       for (int ta = 0; ta < 3; ++ta) {
@@ -153,32 +168,32 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
 #pragma unroll
           for (int u = 0; u < CH; ++u) {
             const int j = j0 + u;
-            if (j < a.NJ && sub + LP * j < a.Q &&
+            if ((FULL ? j < NJS : (j < NJ && sub + LP * j < a.Q)) &&
                 in_tensor(px + 4 * LP * j, 4 * sizeof(T), a.x, a.x_bytes)) {
               const float4 v = guide_ld4<T>(px + 4 * LP * j);
               const float4 wv = wq[LP * j];
-              acc[u].x = fmaf(wv.x, v.x, acc[u].x);
-              acc[u].y = fmaf(wv.y, v.y, acc[u].y);
-              acc[u].z = fmaf(wv.z, v.z, acc[u].z);
-              acc[u].w = fmaf(wv.w, v.w, acc[u].w);
+              acc[2 * u] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(v.x, v.y), acc[2 * u]);
+              acc[2 * u + 1] =
+                  __ffma2_rn(make_float2(wv.z, wv.w), make_float2(v.z, v.w), acc[2 * u + 1]);
             }
           }
         }
       }
 #pragma unroll
       for (int u = 0; u < CH; ++u) {
-        if (j0 + u < a.NJ) {
-          s += (acc[u].x + acc[u].y) + (acc[u].z + acc[u].w);  // quads outside C hold 0
-          conv_buf[(j0 + u) * kThreads + tid] = acc[u];
+        if (j0 + u < NJ) {
+          const float2 lo = acc[2 * u], hi = acc[2 * u + 1];
+          s += (lo.x + lo.y) + (hi.x + hi.y);  // quads outside C hold 0
+          conv_buf[(j0 + u) * kThreads + tid] = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
       }
     }
     // LayerNorm over the pixel's channels: the mean, then the mean squared deviation
     const float mean = group_sum<LP>(s) * inv_c;
     float ss = 0.f;
-#pragma unroll 1
-    for (int j = 0; j < a.NJ; ++j) {
-      if (sub + LP * j >= a.Q) break;
+#pragma unroll(FULL ? 16 : 1)
+    for (int j = 0; j < NJ; ++j) {
+      if (!FULL && sub + LP * j >= a.Q) break;
       const float4 v = conv_buf[j * kThreads + tid];
       const float d0 = v.x - mean, d1 = v.y - mean, d2 = v.z - mean, d3 = v.w - mean;
       ss = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, ss))));
@@ -186,10 +201,10 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
     const float rstd = 1.0f / sqrtf(group_sum<LP>(ss) * inv_c + a.eps);
     if (!col_ok) continue;
     __nv_bfloat16* op = a.out + (size_t(n * a.H + y) * a.W + col) * a.C;
-#pragma unroll 1
-    for (int j = 0; j < a.NJ; ++j) {
+#pragma unroll(FULL ? 16 : 1)
+    for (int j = 0; j < NJ; ++j) {
       const int q = sub + LP * j;
-      if (q >= a.Q) break;
+      if (!FULL && q >= a.Q) break;
       const float4 v = conv_buf[j * kThreads + tid];
       const float4 g = gamma_s[q], b = beta_s[q];
       const float o0 = gelu_erf((v.x - mean) * rstd * g.x + b.x);

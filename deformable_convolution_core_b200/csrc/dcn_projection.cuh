@@ -26,7 +26,7 @@
 
 #include <cuda.h>
 
-#include "dcn_forward_tiled.cuh"
+#include "dcn_tma.cuh"
 
 namespace dcn {
 
@@ -127,10 +127,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
       : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // T: storage type of the offset and mask outputs (fp32 or bf16).

@@ -61,6 +61,22 @@ struct Staged<__nv_bfloat16> {
   }
 };
 
+template <>
+struct Staged<__half> {
+  using Pair = uint32_t;
+  using One = unsigned short;
+  __device__ __forceinline__ static float2 pair(const Pair& p) { return f16x2_to_f32x2(p); }
+  __device__ __forceinline__ static float one(const One& v) {
+    return __half2float(__ushort_as_half(v));
+  }
+  __device__ __forceinline__ static Pair load_pair(const void* base, size_t i) {
+    return __ldg(reinterpret_cast<const unsigned int*>(base) + i);
+  }
+  __device__ __forceinline__ static One load_one(const void* base, size_t i) {
+    return __ldg(reinterpret_cast<const unsigned short*>(base) + i);
+  }
+};
+
 template <typename T>
 __host__ __device__ constexpr int staged_bytes_per_entry() {
   return int(sizeof(typename Staged<T>::Pair) + sizeof(typename Staged<T>::One));

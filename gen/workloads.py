@@ -30,7 +30,7 @@ class Workload:
     dilation: int
     offset_scale: float
     softmax: int             # 1: mask holds logits (DCNv3); 0: mask used as-is (DCNv4)
-    dtype: str               # "f32" or "bf16" storage; arithmetic is fp32 either way
+    dtype: str               # "f32", "bf16" or "f16" storage; arithmetic is fp32 always
     Ho: int
     Wo: int
     x_dist: tuple = ("normal", 0.0, 1.0)
@@ -131,6 +131,35 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     # The same backward with bf16 storage (fp32 arithmetic, grad_input accumulated in fp32).
     _wl(name="internimage_l_stage2_bwd_bf16_n32_48x48_c320", cfg=5, N=32, H=48, W=48, G=20,
         dtype="bf16", Ho=48, Wo=48, backward=True, **_STAGE),
+    # Other tap sets and channel widths on the stage-1 bf16 shape (the direct
+    # kernels): 5x5 and 7x7 windows, 8 and 32 channels per group.
+    _wl(name="internimage_l_stage1_k5_bf16_n16_96x96_c160", cfg=6, N=16, H=96, W=96, G=10,
+        Cg=16, K=5, stride=1, pad=2, dilation=1, offset_scale=2.0, softmax=1, dtype="bf16",
+        Ho=96, Wo=96),
+    _wl(name="internimage_l_stage1_k7_bf16_n16_96x96_c160", cfg=6, N=16, H=96, W=96, G=10,
+        Cg=16, K=7, stride=1, pad=3, dilation=1, offset_scale=2.0, softmax=1, dtype="bf16",
+        Ho=96, Wo=96),
+    _wl(name="internimage_l_stage1_cg8_bf16_n64_96x96_c160", cfg=6, N=64, H=96, W=96, G=20,
+        Cg=8, K=3, stride=1, pad=1, dilation=1, offset_scale=2.0, softmax=1, dtype="bf16",
+        Ho=96, Wo=96),
+    _wl(name="internimage_l_stage1_cg32_bf16_n64_96x96_c160", cfg=6, N=64, H=96, W=96, G=5,
+        Cg=32, K=3, stride=1, pad=1, dilation=1, offset_scale=2.0, softmax=1, dtype="bf16",
+        Ho=96, Wo=96),
+    # fp16 storage (the autocast type the pages train and serve with), fp32
+    # arithmetic: the tiny case, the four stage shapes and the stage-2 backward.
+    _wl(name="tiny_fp16_n1_14x14_c64", cfg=1, N=1, H=14, W=14, G=4, Cg=16, K=3, stride=1,
+        pad=1, dilation=1, offset_scale=1.0, softmax=1, dtype="f16", Ho=14, Wo=14,
+        offset_dist=("uniform", -2.0, 2.0)),
+    _wl(name="internimage_l_stage1_fp16_n64_96x96_c160", cfg=3, N=64, H=96, W=96, G=10,
+        dtype="f16", Ho=96, Wo=96, far=(0.1, -8.0, 8.0), tags=("sweep",), **_STAGE),
+    _wl(name="internimage_l_stage2_fp16_n64_48x48_c320", cfg=3, N=64, H=48, W=48, G=20,
+        dtype="f16", Ho=48, Wo=48, far=(0.1, -8.0, 8.0), **_STAGE),
+    _wl(name="internimage_l_stage3_fp16_n64_24x24_c640", cfg=3, N=64, H=24, W=24, G=40,
+        dtype="f16", Ho=24, Wo=24, far=(0.1, -8.0, 8.0), **_STAGE),
+    _wl(name="internimage_l_stage4_fp16_n64_12x12_c1280", cfg=3, N=64, H=12, W=12, G=80,
+        dtype="f16", Ho=12, Wo=12, far=(0.1, -8.0, 8.0), **_STAGE),
+    _wl(name="internimage_l_stage2_bwd_fp16_n32_48x48_c320", cfg=5, N=32, H=48, W=48, G=20,
+        dtype="f16", Ho=48, Wo=48, backward=True, **_STAGE),
 ]}
 
 

@@ -16,8 +16,8 @@
  * window's centre position (K/2, K/2) is not sampled: the KK = K*K - 1 taps
  * are the other positions in row-major order, tap k at position k for
  * k < (K*K)/2 and at k + 1 after it.  Arithmetic is fp32 for both storage
- * types; bf16 values are widened exactly on load and the output is rounded to
- * nearest-even once.
+ * types; bf16 and fp16 values are widened exactly on load and the output is
+ * rounded to nearest-even once.
  *
  * Layouts (all tensors dense, row-major, element indices; C = G*Cg, KK = taps
  * = K*K, or K*K - 1 with remove_center):
@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define DCN_CORE_ABI_VERSION 4
+#define DCN_CORE_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define DCN_API __attribute__((visibility("default")))
@@ -71,7 +71,8 @@ typedef enum {
 
 typedef enum {
   DCN_F32 = 0,   /* fp32 storage                                    */
-  DCN_BF16 = 1   /* bf16 storage, fp32 arithmetic                   */
+  DCN_BF16 = 1,  /* bf16 storage, fp32 arithmetic                   */
+  DCN_F16 = 2    /* fp16 storage, fp32 arithmetic (ABI version 5)   */
 } dcn_dtype;
 
 /*
@@ -108,8 +109,12 @@ typedef struct {
   int stride_w, pad_w, dilation_w;
 } dcn_problem;
 
-/* Output spatial size.  DCN_ERR_INVALID_ARG if the problem is invalid or the
- * output would be empty. */
+/* Output spatial size, the convolution rule
+ *     Ho = floor((H + 2*pad - dilation*(K-1) - 1) / stride) + 1   (Wo likewise),
+ * which keeps the input's size at 3x3 / stride 1 / pad 1 as the DCNv3
+ * extension build guide (trdm.cn), section 2.3, checks.  Ho and Wo: host
+ * pointers, written on success.  DCN_ERR_INVALID_ARG if the problem is invalid
+ * or the output would be empty; nothing else is touched. */
 DCN_API dcn_status dcn_core_output_hw(const dcn_problem* problem, int* Ho, int* Wo);
 
 /*
@@ -118,7 +123,7 @@ DCN_API dcn_status dcn_core_output_hw(const dcn_problem* problem, int* Ho, int* 
  * written entirely.  All four must be 16-byte aligned and must not overlap
  * the output.  Supported channel widths: Cg*sizeof(dtype) a multiple of 16
  * bytes and at most 128 bytes: Cg in {4, 8, 16, 32} for fp32, {8, 16, 32,
- * 64} for bf16; other widths return DCN_ERR_UNSUPPORTED.
+ * 64} for bf16 and fp16; other widths return DCN_ERR_UNSUPPORTED.
  */
 DCN_API dcn_status dcn_core_forward(const dcn_problem* problem, const void* input,
                             const void* offset, const void* mask, void* output,
@@ -136,13 +141,15 @@ DCN_API dcn_status dcn_core_forward(const dcn_problem* problem, const void* inpu
  * `stream` before the call, and `stream` waits for the last copy before any
  * work enqueued after it, so from the caller's side everything happens on
  * `stream` (CUDA graph capture included).  The two streams and a set of
- * events per device are created on first use and kept by the library;
- * concurrent calls from several host threads are serialised while they
- * enqueue.  Host buffers should be pinned for the copies to be asynchronous;
- * they must not be touched until `stream` has reached this point.  Device
- * buffers follow the rules of dcn_core_forward.  Arguments are validated
- * before anything is enqueued; a CUDA error part-way (DCN_ERR_CUDA) may leave
- * the chunks before it enqueued.
+ * events per device are created on first use and kept by the library (and
+ * created again for a new context after cudaDeviceReset); concurrent calls
+ * from several host threads are serialised while they enqueue.  Host buffers
+ * should be pinned for the copies to be asynchronous; they must not be
+ * touched until `stream` has reached this point.  Device buffers follow the
+ * rules of dcn_core_forward.  Arguments are validated before anything is
+ * enqueued; an error part-way (DCN_ERR_CUDA, or a chunk's own error) may
+ * leave the chunks before it enqueued, and the library streams are joined
+ * back into `stream` on that path too, so no copy runs outside its order.
  */
 DCN_API dcn_status dcn_core_forward_host(const dcn_problem* problem, const void* h_input,
                                  const void* h_offset, const void* h_mask,
@@ -158,7 +165,7 @@ DCN_API dcn_status dcn_core_forward_host(const dcn_problem* problem, const void*
  * one library stream, the backward of each chunk on `stream`, the three
  * gradients out on the other).  input, offset, mask, d_grad_out,
  * d_grad_input, d_grad_offset and d_grad_mask: device buffers with the rules
- * of dcn_core_backward; the bf16 workspace is sized for the whole problem
+ * of dcn_core_backward; the 2-byte storage workspace is sized for the whole problem
  * (dcn_core_backward_workspace) and reused by every chunk.  Errors as for
  * dcn_core_forward_host.
  */
@@ -170,12 +177,19 @@ DCN_API dcn_status dcn_core_backward_host(const dcn_problem* problem, const void
                                   void* d_grad_mask, void* workspace,
                                   size_t workspace_bytes, cudaStream_t stream);
 
-/* Device workspace the backward needs, in bytes: 0 for fp32 storage; for
- * bf16 storage an fp32 accumulator for grad_input, N*H*W*G*Cg*4 bytes. */
+/* Device workspace the backward needs, in bytes (the backward of the DCNv3
+ * extension build guide (trdm.cn), section 2.1): 0 for fp32 storage; for
+ * bf16 or fp16 storage an fp32 accumulator for grad_input, N*H*W*G*Cg*4 bytes.
+ * Returns 0 for an invalid problem.  The caller allocates and owns it. */
 DCN_API size_t dcn_core_backward_workspace(const dcn_problem* problem);
 
 /*
- * Backward (gradients of the forward above).  grad_out: (N, Ho, Wo, C).
+ * Backward: the gradients of the forward above with respect to its input,
+ * offsets and mask, i.e. the backward device code of the DCNv3 extension
+ * build guide (trdm.cn), section 2.1, obtained by differentiating the
+ * sampling and weighted sum of the InternImage-L DCNv3 explainer (wmrh.cn),
+ * section 二 steps 2-4 (bilinear weights, softmax over the taps).  All
+ * pointers are device pointers owned by the caller.  grad_out: (N, Ho, Wo, C).
  *   grad_input  (N, H, W, C)   OVERWRITTEN: zero-filled on the stream, then
  *               accumulated by a vectorised atomic scatter (the order of
  *               the additions, hence the last bits, may differ between runs)
@@ -184,11 +198,11 @@ DCN_API size_t dcn_core_backward_workspace(const dcn_problem* problem);
  *               gradient with respect to the logits
  * The gradient with respect to an offset at an integer sample coordinate is
  * the one-sided derivative that floor() selects.  All gradients are computed
- * in fp32.  With bf16 storage the input gradient is accumulated in the
- * caller's workspace (dcn_core_backward_workspace bytes, 16-byte aligned,
- * contents on entry irrelevant) and rounded to bf16 once at the end; grad
- * offset and grad mask are rounded once.  Cg must be 4, 8, 16 or 32; all
- * pointers 16-byte aligned.  workspace may be NULL when the workspace size
+ * in fp32.  With bf16 or fp16 storage the input gradient is accumulated in
+ * the caller's workspace (dcn_core_backward_workspace bytes, 16-byte aligned,
+ * contents on entry irrelevant) and rounded to the storage type once at the
+ * end (nearest even); grad offset and grad mask are rounded once.  Cg must
+ * be 4, 8, 16, 32 or 64; all pointers 16-byte aligned.  workspace may be NULL when the workspace size
  * is 0; a missing or short workspace returns DCN_ERR_INVALID_ARG.
  */
 DCN_API dcn_status dcn_core_backward(const dcn_problem* problem, const void* input,
@@ -209,13 +223,14 @@ DCN_API dcn_status dcn_core_backward(const dcn_problem* problem, const void* inp
  * code that may not call cudaMalloc because it synchronises the device.
  *
  * Arguments and results are those of dcn_core_backward without the
- * workspace.  fp32 storage needs no scratch.  For bf16 storage the fp32
- * grad_input accumulator (N*H*W*G*Cg*4 bytes) lives in a fixed array inside
- * the library of DCN_CORE_NOALLOC_SCRATCH_BYTES; every GPU that loads the
- * library holds that array until the process exits, and a bf16 problem whose
+ * workspace.  fp32 storage needs no scratch.  For bf16 or fp16 storage the
+ * fp32 grad_input accumulator (N*H*W*G*Cg*4 bytes) lives in a fixed array
+ * inside the library of DCN_CORE_NOALLOC_SCRATCH_BYTES; every GPU that loads
+ * the library holds that array until the process exits, and a problem whose
  * accumulator is larger returns DCN_ERR_UNSUPPORTED without enqueuing work.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current): make that first call before any stream
+ * device and context, with that device current; after cudaDeviceReset the
+ * next call looks it up again): make that first call before any stream
  * capture.  Every call shares the one array and each call clears it on its
  * stream before use; calls whose work can overlap on the GPU (other streams,
  * other host threads on the same device) race on it and must be serialised
@@ -240,18 +255,18 @@ DCN_API size_t dcn_core_backward_deterministic_workspace(const dcn_problem* prob
  *
  * Arguments and results are those of dcn_core_backward; the workspace
  * (dcn_core_backward_deterministic_workspace bytes, 256-byte aligned, contents
- * on entry irrelevant) replaces the bf16 accumulator.  grad_offset and
+ * on entry irrelevant) replaces the 2-byte storage accumulator.  grad_offset and
  * grad_mask are computed exactly as by dcn_core_backward.  grad_input is
  * accumulated exactly in 64-bit fixed point: every fp32 contribution
  * m_k * w_corner * grad_out[c] is rounded to an integer multiple of 2^-S and
  * the integers are summed, so the order of the additions does not matter; the
- * sum is then rounded once to fp32 (and to nearest-even bf16 for bf16
+ * sum is then rounded once to fp32 (and to nearest-even bf16 or fp16 for 2-byte
  * storage).  S is chosen on the device from max|grad_out| (and max|mask| for
  * a raw mask) so that no sum can overflow: 2^-S is about 2^-62 times
  * (max|grad_out| * max|mask weight| * Ho*Wo*KK), far below fp32 resolution
  * for every element except those many orders of magnitude smaller than the
  * largest.  A non-finite grad_out (or raw mask) makes every grad_input
- * element NaN.  Cg must be 4, 8, 16 or 32; all pointers 16-byte aligned.
+ * element NaN.  Cg must be 4, 8, 16, 32 or 64; all pointers 16-byte aligned.
  * Slower than dcn_core_backward: the 64-bit reductions are scalar.
  */
 DCN_API dcn_status dcn_core_backward_deterministic(const dcn_problem* problem, const void* input,
@@ -321,7 +336,7 @@ DCN_API dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, const 
  *   input   device, bf16, (M, K) row-major; K >= 8 and a multiple of 8
  *   weight  device, bf16, (Nout, K) row-major (a linear layer's weight)
  *   bias    device, fp32, (Nout), or NULL
- *   output  device, (M, Nout) in out_dtype (fp32 or bf16), written entirely
+ *   output  device, (M, Nout) in out_dtype (fp32, bf16 or fp16), written entirely
  * Same arithmetic, alignment rules and errors as
  * dcn_core_offset_mask_projection (M*K and M*Nout below 2^31).
  */

@@ -1,7 +1,7 @@
 """Helpers shared by the GPU tests: device copies of the generator's arrays,
 exact widening back to float64, and the parity measures with their
 tolerances (forward fp32: 1e-5 * max|x|; bf16 storage: 1e-2 * max|ref|;
-backward fp32: 1e-4 * max|ref| per gradient)."""
+fp16 storage: 1e-3 * max|ref|; backward fp32: 1e-4 * max|ref| per gradient)."""
 from __future__ import annotations
 
 import numpy as np
@@ -13,8 +13,12 @@ FWD_F32_TOL = 1e-5     # max |gpu - ref| <= FWD_F32_TOL * max|x|
 FWD_BF16_TOL = 1e-2    # max |gpu - ref| <= FWD_BF16_TOL * max|ref|
 BWD_F32_TOL = 1e-4     # max |gpu - ref| <= BWD_F32_TOL * max|ref|, per gradient
 BWD_BF16_TOL = 1e-2    # bf16 storage: each gradient rounded to bf16 once; same gate as the forward
+# fp16 storage: one rounding to fp16 is at most 2^-11 relative; the gate allows
+# twice that, normalised by max|ref| like the bf16 gate (forward and backward).
+FWD_F16_TOL = 1e-3
+BWD_F16_TOL = 1e-3
 
-TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 
 
 def to_dev(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
@@ -49,7 +53,8 @@ def fwd_error(got: np.ndarray, ref: np.ndarray, x: np.ndarray, dtype: str):
     err = float(np.abs(got - ref).max()) if got.size else 0.0
     if dtype == "f32":
         return err, FWD_F32_TOL * max(float(np.abs(x).max()), 1e-30)
-    return err, FWD_BF16_TOL * max(float(np.abs(ref).max()), 1e-30)
+    tol = FWD_F16_TOL if dtype == "f16" else FWD_BF16_TOL
+    return err, tol * max(float(np.abs(ref).max()), 1e-30)
 
 
 def assert_fwd(got, ref, x, dtype, what=""):
@@ -59,7 +64,7 @@ def assert_fwd(got, ref, x, dtype, what=""):
 
 def assert_bwd(got, ref, what="", dtype="f32"):
     err = float(np.abs(got - ref).max()) if got.size else 0.0
-    tol = BWD_F32_TOL if dtype == "f32" else BWD_BF16_TOL
+    tol = {"f32": BWD_F32_TOL, "f16": BWD_F16_TOL}.get(dtype, BWD_BF16_TOL)
     bound = tol * max(float(np.abs(ref).max()), 1e-30)
     assert err <= bound, f"{what}: backward max error {err:.3e} > {bound:.3e}"
 

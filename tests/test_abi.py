@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 4
+    assert dcn.dcn_core_abi_version() == dcn.ABI_VERSION == 5
     for st in range(6):
         assert dcn.dcn_status_string(st)
     assert "unknown" in dcn.dcn_status_string(99)
@@ -89,6 +89,7 @@ FAKE = 1 << 20  # an address that is 16- and 32-byte aligned; never dereferenced
     (dict(dilation_w=0), dcn.DCN_ERR_INVALID_ARG),
     (dict(W=2, pad_w=0, dilation_w=2), dcn.DCN_ERR_INVALID_ARG),   # empty output along W
     (dict(dtype=7), dcn.DCN_ERR_INVALID_ARG),
+    (dict(dtype=3), dcn.DCN_ERR_INVALID_ARG),
     (dict(offset_scale=float("nan")), dcn.DCN_ERR_INVALID_ARG),
     (dict(H=2, W=2, K=5, pad=0), dcn.DCN_ERR_INVALID_ARG),     # empty output
     (dict(N=1 << 16, H=1 << 8, W=1 << 8, G=16, Cg=16), dcn.DCN_ERR_INVALID_ARG),  # >= 2^31 elements
@@ -137,6 +138,33 @@ def test_backward_rejects_before_launch(lib):
     with pytest.raises(dcn.DcnError) as e:
         dcn.dcn_core_backward(pc, *ptrs, None, 0, 0)
     assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+
+
+def test_noalloc_backward_rejects_before_launch(lib):
+    p = dcn.make_problem(**GOOD)
+    ptrs = [FAKE] * 7
+    for i in range(7):
+        bad = list(ptrs)
+        bad[i] = 0
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_backward_noalloc(p, *bad, stream=0)
+        assert e.value.status == dcn.DCN_ERR_INVALID_ARG
+        bad[i] = FAKE + 8          # every pointer must be 16-byte aligned
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_backward_noalloc(p, *bad, stream=0)
+        assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+    pc = dcn.make_problem(**{**GOOD, "Cg": 12})
+    with pytest.raises(dcn.DcnError) as e:
+        dcn.dcn_core_backward_noalloc(pc, *ptrs, stream=0)
+    assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
+
+
+def test_noalloc_scratch_size_matches_header():
+    """The binding's DCN_CORE_NOALLOC_SCRATCH_BYTES is the header's #define."""
+    text = open(os.path.join(ROOT, "include", "dcn_core.h")).read()
+    expr = re.search(r"#define\s+DCN_CORE_NOALLOC_SCRATCH_BYTES\s+\((.*?)\)\s*$", text, re.M).group(1)
+    assert re.fullmatch(r"[0-9u*\s]+", expr), expr
+    assert eval(expr.replace("u", "")) == dcn.DCN_CORE_NOALLOC_SCRATCH_BYTES
 
 
 def test_deterministic_backward_rejects_before_launch(lib):

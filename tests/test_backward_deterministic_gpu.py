@@ -70,7 +70,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("case", CASES, ids=["_".join(f"{k}{v}" for k, v in c.items())
                                              for c in CASES])
 def test_deterministic_backward_matches_oracle(oracle_mod, case, dtype):
@@ -89,12 +89,12 @@ def test_deterministic_backward_matches_oracle(oracle_mod, case, dtype):
     assert torch.equal(goff, ref[1]) and torch.equal(gm, ref[2])
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_deterministic_backward_is_bitwise_reproducible(gen_mod, dtype):
     """Reruns, another stream, other tile shapes and the direct kernel all
     give the same grad_input bits: the fixed-point sum does not depend on the
     order of the additions."""
-    wl = WORKLOADS[f"internimage_l_stage2_bwd_{'fp32' if dtype == 'f32' else 'bf16'}_n32_48x48_c320"]
+    wl = WORKLOADS[f"internimage_l_stage2_bwd_{ {'f32': 'fp32', 'bf16': 'bf16', 'f16': 'fp16'}[dtype]}_n32_48x48_c320"]
     d = gen_mod.make_inputs(wl, n_images=6)
     p = dcn.make_problem(6, wl.H, wl.W, wl.G, wl.Cg, offset_scale=wl.offset_scale, dtype=dtype)
     args = [to_dev(d[k], dtype) for k in ("x", "offset", "mask", "grad_out")]

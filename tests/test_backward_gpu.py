@@ -99,11 +99,13 @@ CASES = [
     (1, 2, 40, 2, 16, dict()),
     (2, 23, 29, 3, 16, dict(stride_w=2, pad_w=0)),
     (2, 26, 21, 4, 16, dict(stride=2, dilation_w=2, pad_w=2, softmax=0)),
+    (2, 11, 13, 2, 64, dict()),                  # 16 lanes per unit
+    (1, 9, 10, 3, 64, dict(softmax=0, stride=2)),
 ]
 
 
 @pytest.mark.parametrize("path", ["auto", "direct"])
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("case", CASES, ids=[f"{c[0]}x{c[1]}x{c[2]}_G{c[3]}_Cg{c[4]}_" +
                                              "_".join(f"{k}{v}" for k, v in c[5].items())
                                              for c in CASES])
@@ -213,16 +215,19 @@ def test_backward_rerun_differs_only_by_rounding(gen_mod):
     assert torch.allclose(a[0], b[0], rtol=0, atol=1e-5 * float(a[0].abs().max()))
 
 
-def test_full_size_backward_bf16(gen_mod, oracle_mod):
-    wl = WORKLOADS["internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_full_size_backward_half(gen_mod, oracle_mod, dtype):
+    """The stage-2 backward with 2-byte storage, every element against the
+    oracle fed the same rounded inputs."""
+    wl = WORKLOADS[f"internimage_l_stage2_bwd_{'bf16' if dtype == 'bf16' else 'fp16'}_n32_48x48_c320"]
     d = gen_mod.make_inputs(wl)
     p = dcn.problem_for(wl)
-    check(oracle_mod, p, d["x"], d["offset"], d["mask"], d["grad_out"], "bf16")
+    check(oracle_mod, p, d["x"], d["offset"], d["mask"], d["grad_out"], dtype)
 
 
 @pytest.mark.parametrize("N,H,W,G,dtype", [(5, 21, 23, 4, "f32"), (11, 12, 13, 3, "f32"),
                                            (9, 16, 16, 2, "bf16"), (3, 7, 5, 2, "bf16"),
-                                           (1, 14, 15, 3, "f32")])
+                                           (1, 14, 15, 3, "f32"), (6, 10, 9, 2, "f16")])
 def test_backward_host_entry_point(oracle_mod, N, H, W, G, dtype):
     """The chunked host backward: grad_offset and grad_mask have the bits of
     the device backward on the whole batch (they do not depend on the order of

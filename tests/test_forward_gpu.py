@@ -99,6 +99,14 @@ CASES = [
     (2, 13, 14, 3, 32, dict(dtype="f32", softmax=0, remove_center=1)),
     (2, 17, 19, 3, 16, dict(dtype="f32", K=5, remove_center=1)),
     (1, 17, 19, 2, 16, dict(dtype="bf16", K=7, softmax=0, dil=2, remove_center=1)),
+    # fp16 storage: the tiled kernel (3x3, 16 channels) and the direct one
+    (2, 23, 29, 3, 16, dict(dtype="f16")),
+    (1, 33, 17, 10, 16, dict(dtype="f16", softmax=0)),
+    (2, 15, 21, 4, 8, dict(dtype="f16")),        # 16-byte units, fp16
+    (2, 13, 14, 3, 32, dict(dtype="f16")),       # 64-byte units, fp16
+    (2, 25, 27, 3, 16, dict(dtype="f16", stride=2, softmax=0)),
+    (2, 23, 29, 3, 16, dict(dtype="f16", remove_center=1)),
+    (1, 17, 19, 2, 16, dict(dtype="f16", K=5)),
     # separate height / width stride, padding and dilation
     (2, 23, 29, 3, 16, dict(dtype="f32", stride=1, stride_w=2, pad=1, pad_w=0)),
     (2, 26, 21, 4, 16, dict(dtype="bf16", stride=2, stride_w=1, dil=1, dil_w=2, pad_w=2)),
@@ -125,7 +133,7 @@ def test_tiled_kernel_tile_and_halo_settings(oracle_mod, halo, tile):
     old = {k: os.environ.get(k) for k in ("DCN_CORE_HALO", "DCN_CORE_TILED_TILE")}
     os.environ["DCN_CORE_HALO"], os.environ["DCN_CORE_TILED_TILE"] = halo, tile
     try:
-        for dtype in ("f32", "bf16"):
+        for dtype in ("f32", "bf16", "f16"):
             p, x, off, mask = random_case(2, 37, 41, 3, 16, dtype=dtype, off_sd=3.0)
             check_full(oracle_mod, p, x, off, mask, dtype)
             p, x, off, mask = random_case(1, 40, 36, 2, 16, dtype=dtype, stride=2, softmax=0)
