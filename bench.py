@@ -605,12 +605,36 @@ def run_block_core_path(gen, name="internimage_l_stage1_bf16_n64_96x96_c160", re
     dcn.dcn_core_sync_status(s)
     t = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(k)] for e in ev])
     med = np.median(t, axis=0)
+    # the same branch with guide and projection in one kernel (the query stays on chip)
+    fused = lambda: dcn.dcn_core_offset_mask_guide_projection(
+        p, x, gp["dw_weight"], gp["dw_bias"], gp["ln_gamma"], gp["ln_beta"], 1e-6, w, b, off,
+        msk, s)
+    fstages = [fused] + stages[2:]
+    for _ in range(3):
+        for f in fstages:
+            f()
+    torch.cuda.synchronize()
+    fk = len(fstages)
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(fk + 1)] for _ in range(reps)]
+    for r in range(reps):
+        for i, f in enumerate(fstages):
+            fev[r][i].record(s)
+            f()
+        fev[r][fk].record(s)
+    torch.cuda.synchronize()
+    dcn.dcn_core_sync_status(s)
+    ft = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(fk)] for e in fev])
+    fmed = np.median(ft, axis=0)
+    total, ftotal = float(np.median(t.sum(axis=1))), float(np.median(ft.sum(axis=1)))
     return {"workload": name, "guide_ms": round(float(med[0]), 4),
             "projection_ms": round(float(med[1]), 4),
             "core_forward_ms": round(float(med[2]), 4),
             "output_proj_ms": round(float(med[3]), 4),
-            "total_ms": round(float(np.median(t.sum(axis=1))), 4),
-            "Mpixels/s": round(M / (float(np.median(t.sum(axis=1))) * 1e-3) / 1e6, 1)}
+            "total_ms": round(total, 4),
+            "Mpixels/s": round(M / (total * 1e-3) / 1e6, 1),
+            "fused_guide_projection_ms": round(float(fmed[0]), 4),
+            "fused_total_ms": round(ftotal, 4),
+            "fused_Mpixels/s": round(M / (ftotal * 1e-3) / 1e6, 1)}
 
 
 def run_sweep(gen, peak, clocks=None, reps=30, warmup=3):

@@ -45,6 +45,7 @@ EXPORTED_SYMBOLS = (
     "dcn_core_offset_mask_guide",
     "dcn_core_offset_mask_projection",
     "dcn_core_linear_bf16",
+    "dcn_core_offset_mask_guide_projection",
     "dcn_core_sync_status",
     "dcn_status_string",
     "dcn_core_abi_version",
@@ -141,6 +142,9 @@ def load_library():
     lib.dcn_core_offset_mask_guide.restype = st
     lib.dcn_core_offset_mask_projection.argtypes = [pp, vp, ctypes.c_int, vp, vp, vp, vp, vp]
     lib.dcn_core_offset_mask_projection.restype = st
+    lib.dcn_core_offset_mask_guide_projection.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_float,
+                                                          vp, vp, vp, vp, vp]
+    lib.dcn_core_offset_mask_guide_projection.restype = st
     lib.dcn_core_linear_bf16.argtypes = [vp, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, vp, vp,
                                          ctypes.c_int, vp]
     lib.dcn_core_linear_bf16.restype = st
@@ -288,6 +292,18 @@ def dcn_core_offset_mask_projection(problem: DcnProblem, query, Cq: int, weight,
     _check(load_library().dcn_core_offset_mask_projection(
         ctypes.byref(problem), _ptr(query), int(Cq), _ptr(weight), _ptr(bias), _ptr(offset),
         _ptr(mask), _stream(stream)), "dcn_core_offset_mask_projection")
+
+
+def dcn_core_offset_mask_guide_projection(problem: DcnProblem, input, dw_weight, dw_bias,
+                                          ln_gamma, ln_beta, ln_eps: float, weight, bias, offset,
+                                          mask, stream=None) -> None:
+    """Guide features and offset / mask projection in one kernel (the query
+    stays on chip; see include/dcn_core.h): the result of
+    dcn_core_offset_mask_guide followed by dcn_core_offset_mask_projection."""
+    _check(load_library().dcn_core_offset_mask_guide_projection(
+        ctypes.byref(problem), _ptr(input), _ptr(dw_weight), _ptr(dw_bias), _ptr(ln_gamma),
+        _ptr(ln_beta), float(ln_eps), _ptr(weight), _ptr(bias), _ptr(offset), _ptr(mask),
+        _stream(stream)), "dcn_core_offset_mask_guide_projection")
 
 
 def dcn_core_linear_bf16(input, M: int, K: int, weight, Nout: int, bias, output,

@@ -61,6 +61,19 @@ def build(force: bool = False, verbose: bool = False, checked: bool = False) -> 
     return lib
 
 
+def build_all(force: bool = False) -> list[str]:
+    """Build the library and its bounds-checked twin side by side (two nvcc
+    processes; each is one translation unit)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    with ThreadPoolExecutor(2) as ex:
+        jobs = [ex.submit(build, force, False, c) for c in (False, True)]
+        return [j.result() for j in jobs]
+
+
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
-                checked="--checked" in sys.argv))
+    if "--all" in sys.argv:
+        print(build_all(force="--force" in sys.argv))
+    else:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                    checked="--checked" in sys.argv))

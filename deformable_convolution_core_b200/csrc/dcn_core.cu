@@ -21,6 +21,7 @@
 #include "dcn_forward.cuh"
 #include "dcn_forward_tiled.cuh"
 #include "dcn_guide.cuh"
+#include "dcn_guide_projection.cuh"
 #include "dcn_projection.cuh"
 
 namespace dcn {
@@ -1379,6 +1380,93 @@ extern "C" dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, con
   a.out_bytes = elems * 2;
   return with_storage(problem->dtype, [&](auto tag) {
     return guide_launch<decltype(tag)>(LP, a, stream);
+  });
+}
+
+namespace dcn {
+namespace {
+
+template <typename T, typename TO, int LP>
+dcn_status guide_projection_launch(const CUtensorMap& wmap, const GuideProjArgs& a, int sms,
+                                   cudaStream_t stream) {
+  auto k = dcn_guide_projection_kernel<T, TO, LP, 5>;
+  const size_t smem = guide_proj_smem(a.nA, a.KB, a.Q);
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return DCN_ERR_CUDA;
+  k<<<unsigned(std::min(a.m_tiles, sms)), kGpThreads, smem, stream>>>(wmap, a);
+  return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace dcn
+
+extern "C" dcn_status dcn_core_offset_mask_guide_projection(
+    const dcn_problem* problem, const void* input, const float* dw_weight, const float* dw_bias,
+    const float* ln_gamma, const float* ln_beta, float ln_eps, const void* weight,
+    const float* bias, void* offset, void* mask, cudaStream_t stream) {
+  int64_t Ho, Wo;
+  dcn_status st = check_problem(problem, &Ho, &Wo);
+  if (st != DCN_OK) return st;
+  if (!input || !dw_weight || !weight || !offset || !mask) return DCN_ERR_INVALID_ARG;
+  if (!(ln_eps >= 0.f) || !std::isfinite(ln_eps)) return DCN_ERR_INVALID_ARG;
+  // the guide features keep the input's H x W: the projection's pixel grid must be it
+  if (Ho != problem->H || Wo != problem->W) return DCN_ERR_UNSUPPORTED;
+  const int C = problem->G * problem->Cg;
+  // five channel quads per lane in groups of 8 or 16 lanes: C = 160 or 320.  At
+  // C = 640 one 128-pixel A tile is 160 KB, and with the weight ring, the
+  // guide parameters and the epilogue buffer the block would need 289 KB of
+  // shared memory: those widths take the two calls.
+  int LP = 0;
+  for (int lp : {8, 16})
+    if (C == 4 * lp * 5) LP = lp;
+  if (LP == 0) return DCN_ERR_UNSUPPORTED;
+  if (!aligned(input, 16) || !aligned(dw_weight, 16) || (dw_bias && !aligned(dw_bias, 16)) ||
+      (ln_gamma && !aligned(ln_gamma, 16)) || (ln_beta && !aligned(ln_beta, 16)) ||
+      !aligned(weight, 16) || !aligned(offset, 16) || !aligned(mask, 16) ||
+      (bias && !aligned(bias, 4)))
+    return DCN_ERR_UNSUPPORTED;
+  if (tensor_map_encoder() == nullptr) return DCN_ERR_UNSUPPORTED;
+  DeviceInfo dev;
+  if (device_info(&dev) != DCN_OK) return DCN_ERR_CUDA;
+  const int64_t KK = taps(problem);
+  GuideProjArgs a;
+  a.x = input;
+  a.w = dw_weight;
+  a.bias = dw_bias;
+  a.gamma = ln_gamma;
+  a.beta = ln_beta;
+  a.eps = ln_eps;
+  a.pbias = bias;
+  a.offset = offset;
+  a.mask = mask;
+  a.error_word = dev.error_word;
+  a.N = problem->N;
+  a.H = problem->H;
+  a.W = problem->W;
+  a.C = C;
+  a.Q = C / 4;
+  const int64_t M = int64_t(problem->N) * problem->H * problem->W;
+  const int64_t nout = int64_t(problem->G) * KK * 3;
+  if (M * nout > INT_MAX) return DCN_ERR_INVALID_ARG;
+  a.M = int(M);
+  a.Nout = int(nout);
+  a.n_off = int(int64_t(problem->G) * KK * 2);
+  a.KB = (C + kPjBK - 1) / kPjBK;
+  a.m_tiles = int((M + kPjBM - 1) / kPjBM);
+  a.n_tiles = int((nout + kPjBN - 1) / kPjBN);
+  a.nA = guide_proj_smem(2, a.KB, a.Q) <= size_t(dev.smem_optin) ? 2 : 1;
+  if (guide_proj_smem(a.nA, a.KB, a.Q) > size_t(dev.smem_optin)) return DCN_ERR_UNSUPPORTED;
+  a.x_bytes = size_t(M) * C * size_t(esize(problem->dtype));
+  a.fd_W = make_fastdiv(uint32_t(problem->W));
+  a.fd_H = make_fastdiv(uint32_t(problem->H));
+  CUtensorMap wmap;
+  if ((st = bf16_kmajor_map(&wmap, weight, uint64_t(C), uint64_t(nout))) != DCN_OK) return st;
+  // input and output storage types follow the problem's
+  return with_storage(problem->dtype, [&](auto tag) {
+    using T = decltype(tag);
+    return LP == 8 ? guide_projection_launch<T, T, 8>(wmap, a, dev.sms, stream)
+                   : guide_projection_launch<T, T, 16>(wmap, a, dev.sms, stream);
   });
 }
 

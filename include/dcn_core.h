@@ -329,6 +329,31 @@ DCN_API dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, const 
                                               float ln_eps, void* query, cudaStream_t stream);
 
 /*
+ * The whole offset / mask branch of the DCNv3 block in one kernel: the guide
+ * features of dcn_core_offset_mask_guide computed straight into the operand
+ * of the projection of dcn_core_offset_mask_projection (InternImage-L DCNv3
+ * explainer (wmrh.cn), section 二 steps 1-3), so the bf16 query never goes to
+ * device memory.  The result is that of the two calls in a row (query =
+ * guide features, Cq = C = G*Cg): the same arithmetic, the same bf16 rounding
+ * of the query, the same tensor-core products.
+ *   input, dw_weight, dw_bias, ln_gamma, ln_beta, ln_eps: as for
+ *              dcn_core_offset_mask_guide (input of problem->dtype)
+ *   weight     device, bf16, (G*KK*3, C) row-major; bias device fp32 (G*KK*3) or NULL
+ *   offset, mask  device, (N, H, W, G*KK*2) and (N, H, W, G*KK) of problem->dtype,
+ *              written entirely
+ * The guide keeps the input's size, so the problem's output size must be
+ * H x W (stride 1, "same" padding), else DCN_ERR_UNSUPPORTED.  C must be 160
+ * or 320 (the InternImage-L stage-1 and stage-2 widths; a 128-pixel operand
+ * tile of a wider query does not fit in shared memory beside the weight
+ * ring), else DCN_ERR_UNSUPPORTED; alignment rules of the two calls it
+ * replaces.
+ */
+DCN_API dcn_status dcn_core_offset_mask_guide_projection(
+    const dcn_problem* problem, const void* input, const float* dw_weight, const float* dw_bias,
+    const float* ln_gamma, const float* ln_beta, float ln_eps, const void* weight,
+    const float* bias, void* offset, void* mask, cudaStream_t stream);
+
+/*
  * The linear layers on either side of the core operator in the DCNv3 block
  * (InternImage-L DCNv3 explainer (wmrh.cn), section 二: input_proj before it,
  * output_proj after it), as one tensor-core GEMM with bf16 operands:

@@ -123,3 +123,84 @@ def test_guide_projection_forward_chain(oracle_mod):
     assert np.abs(f64(msk) - rm).max() <= tol * max(1.0, np.abs(rm).max())
     ref = oracle_mod.forward(f64(xd), f64(off), f64(msk), **problem_kwargs(p))
     assert np.abs(f64(out) - ref).max() <= 1e-2 * np.abs(ref).max()
+
+
+def fused_inputs(N, H, W, G, dtype, affine=True):
+    C = G * 16
+    p = dcn.make_problem(N, H, W, G, 16, offset_scale=2.0, dtype=dtype)
+    xd = to_dev(RNG.standard_normal((N, H, W, C)).astype(np.float32), dtype)
+    w, b, g, be = params(C, affine)
+    pw = torch.from_numpy((RNG.standard_normal((G * 27, C)) / np.sqrt(C)).astype(np.float32))
+    pw = pw.to(torch.bfloat16).cuda()
+    pb = torch.from_numpy((0.1 * RNG.standard_normal(G * 27)).astype(np.float32)).cuda()
+    return p, xd, (w, b, g, be), pw, pb
+
+
+def projection_outputs(p, dtype):
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[dtype]
+    off = torch.empty((p.N, p.H, p.W, p.G * 18), dtype=tdt, device="cuda")
+    msk = torch.empty((p.N, p.H, p.W, p.G * 9), dtype=tdt, device="cuda")
+    return off, msk
+
+
+# (N, H, W, G, dtype): C = 160 (8 lanes x 5 quads, two A tiles in flight) and
+# 320 (16 lanes, one A tile); a last 128-pixel tile that is partly outside the
+# batch; a batch smaller than one tile; fp32, bf16 and fp16 inputs and outputs
+FUSED = [(2, 12, 13, 10, "bf16"), (3, 9, 11, 10, "f32"), (1, 20, 17, 20, "bf16"),
+         (2, 7, 9, 20, "f32"), (2, 11, 10, 10, "f16"), (1, 1, 3, 10, "bf16")]
+
+
+@pytest.mark.parametrize("case", FUSED, ids=[f"N{c[0]}_{c[1]}x{c[2]}_C{c[3] * 16}_{c[4]}"
+                                             for c in FUSED])
+def test_fused_guide_projection_equals_the_two_calls(oracle_mod, case):
+    """dcn_core_offset_mask_guide_projection gives, bit for bit, the offsets
+    and mask of the guide followed by the projection (the same arithmetic, the
+    same bf16 query, the same tensor-core products), and both match the oracle."""
+    N, H, W, G, dtype = case
+    C = G * 16
+    p, xd, (w, b, g, be), pw, pb = fused_inputs(N, H, W, G, dtype)
+    q = run_guide(p, xd, w, b, g, be, 1e-6)
+    off1, msk1 = projection_outputs(p, dtype)
+    dcn.dcn_core_offset_mask_projection(p, q, C, pw, pb, off1, msk1)
+    off2, msk2 = projection_outputs(p, dtype)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    dcn.dcn_core_offset_mask_guide_projection(p, xd, dev(w), dev(b), dev(g), dev(be), 1e-6, pw,
+                                              pb, off2, msk2)
+    torch.cuda.synchronize()
+    dcn.dcn_core_sync_status()
+    assert torch.equal(off1, off2) and torch.equal(msk1, msk2)
+    ref_q = oracle_mod.guide(f64(xd), w, b, g, be, 1e-6)
+    assert gate(f64(q), ref_q).all()
+    ro, rm = oracle_mod.projection(f64(q), f64(pw), f64(pb.cpu()), G=G)
+    tol = 4 * C * 2.0 ** -24 * 8 + (2.0 ** -8 if dtype != "f32" else 0.0)
+    assert np.abs(f64(off2) - ro).max() <= tol * max(1.0, np.abs(ro).max())
+    assert np.abs(f64(msk2) - rm).max() <= tol * max(1.0, np.abs(rm).max())
+
+
+def test_fused_guide_projection_at_stage1_size():
+    """InternImage-L stage 1, bf16 (N=64, 96x96, C=160): the fused branch equals
+    the two calls bit for bit over the whole batch."""
+    N, H, W, G = 64, 96, 96, 10
+    p, xd, (w, b, g, be), pw, pb = fused_inputs(N, H, W, G, "bf16")
+    dev = lambda a: torch.from_numpy(a).cuda()
+    q = run_guide(p, xd, w, b, g, be, 1e-6)
+    off1, msk1 = projection_outputs(p, "bf16")
+    dcn.dcn_core_offset_mask_projection(p, q, G * 16, pw, pb, off1, msk1)
+    off2, msk2 = projection_outputs(p, "bf16")
+    dcn.dcn_core_offset_mask_guide_projection(p, xd, dev(w), dev(b), dev(g), dev(be), 1e-6, pw,
+                                              pb, off2, msk2)
+    torch.cuda.synchronize()
+    dcn.dcn_core_sync_status()
+    assert torch.equal(off1, off2) and torch.equal(msk1, msk2)
+
+
+def test_fused_guide_projection_rejects_before_launch():
+    """Shapes the fused kernel does not serve are refused on the host."""
+    fake = 1 << 20
+    for p in (dcn.make_problem(1, 8, 8, 4, 16, dtype="bf16"),           # C = 64
+              dcn.make_problem(1, 8, 8, 40, 16, dtype="bf16"),          # C = 640
+              dcn.make_problem(1, 8, 8, 10, 16, stride=2, dtype="bf16")):  # output 4 x 4
+        with pytest.raises(dcn.DcnError) as e:
+            dcn.dcn_core_offset_mask_guide_projection(p, fake, fake, None, None, None, 1e-6,
+                                                      fake, None, fake, fake, stream=0)
+        assert e.value.status == dcn.DCN_ERR_UNSUPPORTED
