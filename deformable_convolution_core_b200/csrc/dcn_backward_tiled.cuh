@@ -115,6 +115,41 @@ __device__ __forceinline__ float piece_dot<__half>(const uint4& v, const float2*
   return __fadd_rn(q0, q1);
 }
 
+// 2-byte storage: a corner channel and its upstream-gradient channel are both
+// 16-bit values, so their product is exact in fp32.  sm_100a's mixed-precision
+// FMA (16-bit multiplicands, fp32 addend and result, one rounding) therefore
+// gives quarter_dot's bits on the raw words, without widening either operand.
+// The first product of each pair is formed with a -0 addend, which leaves
+// every product unchanged, including the sign of a zero.
+template <typename T>
+__device__ __forceinline__ float quarter_dot16(uint32_t x01, uint32_t x23, uint32_t g01,
+                                               uint32_t g23);
+#define DCN_QUARTER_DOT16(TYPE, SUFFIX)                                                       \
+  template <>                                                                                 \
+  __device__ __forceinline__ float quarter_dot16<TYPE>(uint32_t x01, uint32_t x23,           \
+                                                       uint32_t g01, uint32_t g23) {         \
+    float p0, p1;                                                                             \
+    asm("{\n .reg .b16 a0, a1, a2, a3, b0, b1, b2, b3;\n .reg .f32 t0, t1;\n"                  \
+        " mov.b32 {a0, a1}, %2;\n mov.b32 {a2, a3}, %3;\n"                                     \
+        " mov.b32 {b0, b1}, %4;\n mov.b32 {b2, b3}, %5;\n"                                     \
+        " fma.rn.f32." SUFFIX " t0, a0, b0, 0f80000000;\n"                                      \
+        " fma.rn.f32." SUFFIX " t1, a1, b1, 0f80000000;\n"                                      \
+        " fma.rn.f32." SUFFIX " %0, a2, b2, t0;\n"                                              \
+        " fma.rn.f32." SUFFIX " %1, a3, b3, t1;\n}"                                             \
+        : "=f"(p0), "=f"(p1)                                                                  \
+        : "r"(x01), "r"(x23), "r"(g01), "r"(g23));                                            \
+    return __fadd_rn(p0, p1);                                                                 \
+  }
+DCN_QUARTER_DOT16(__nv_bfloat16, "bf16")
+DCN_QUARTER_DOT16(__half, "f16")
+#undef DCN_QUARTER_DOT16
+
+// piece_dot of a 2-byte piece with the raw gradient piece g (same channels).
+template <typename T>
+__device__ __forceinline__ float piece_dot16(const uint4& v, const uint4& g) {
+  return __fadd_rn(quarter_dot16<T>(v.x, v.y, g.x, g.y), quarter_dot16<T>(v.z, v.w, g.z, g.w));
+}
+
 // Sum of a lane's pieces in the canonical order: (p0 + p1) for two pieces,
 // (p0 + p1) + (p2 + p3) for four; the lane's slot order (piece j ^ rot) only
 // swaps the operands of these pairwise sums.
@@ -195,7 +230,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     for (;; ++i) {
       const int item = int(blockIdx.x) + i * int(gridDim.x);
       if (item >= t.items || *abort_flag) break;
-      if (i >= nbuf && !mbar_wait_bounded(&empty[b], ph ^ 1u)) {
+      if (i >= nbuf && !mbar_wait_bounded_sleep(&empty[b], ph ^ 1u)) {
         atomicOr(a.error_word, kErrTimeout);
         *abort_flag = 1;
         break;
@@ -390,9 +425,19 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         // lane's four scatter channels
         const char* const gp = reinterpret_cast<const char*>(a.gout) + ob * sizeof(T);
         const bool gok = uvalid && in_range(ob + 15, n_out);
-        float2 gs[8];
+        // (fp32: as pairs; 2-byte types: the raw words, see quarter_dot16)
+        float2 gs[NP == 4 ? 8 : 1];
+        uint4 gw[NP == 2 ? 2 : 1];
 #pragma unroll
-        for (int j = 0; j < NP; ++j) piece_widen<T>(ldg128_pred(gp + 16 * (j ^ rot), gok), gs + j * GP);
+        for (int j = 0; j < NP; ++j) {
+          const uint4 gv = ldg128_pred(gp + 16 * (j ^ rot), gok);
+          if constexpr (NP == 4) piece_widen<T>(gv, gs + j * GP);
+          else gw[j] = gv;
+        }
+        auto pdot = [&](const uint4& v, int j) {
+          if constexpr (NP == 4) return piece_dot<T>(v, gs + j * GP);
+          else return piece_dot16<T>(v, gw[j]);
+        };
         // scatter channels of this lane: 4r .. 4r+3 (fp32 vector reductions), or
         // r, r+4, r+8, r+12 (fixed point: one 32-byte sector per instruction)
         float2 gr_lo, gr_hi;
@@ -422,7 +467,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           const uint32_t a0 = lane_base + (rw.w & kBwdOffMask);
           float pp[NP];
 #pragma unroll
-          for (int j = 0; j < NP; ++j) pp[j] = piece_dot<T>(lds128_a(a0 ^ uint32_t(16 * j)), gs + j * GP);
+          for (int j = 0; j < NP; ++j) pp[j] = pdot(lds128_a(a0 ^ uint32_t(16 * j)), j);
           if (FAR && __any_sync(0xFFFFFFFFu, (fm >> k) & 1u)) {
             if ((fm >> k) & 1u) {
               // this corner from global memory (zero outside the image)
@@ -431,8 +476,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
               for (int j = 0; j < NP; ++j) {
                 const char* q = xp + 16 * (j ^ rot);
-                pp[j] = piece_dot<T>(ldg128_pred(q, in && in_tensor(q, 16, a.x, x_bytes)),
-                                     gs + j * GP);
+                pp[j] = pdot(ldg128_pred(q, in && in_tensor(q, 16, a.x, x_bytes)), j);
               }
             }
           }

@@ -1374,6 +1374,7 @@ extern "C" dcn_status dcn_core_offset_mask_guide(const dcn_problem* problem, con
   a.NJ = NJ;
   a.tiles_x = (problem->W + kGuideWarps * (32 / LP) - 1) / (kGuideWarps * (32 / LP));
   a.tiles_y = (problem->H + kGuideRows - 1) / kGuideRows;
+  a.rows = (problem->H + a.tiles_y - 1) / a.tiles_y;  // e.g. 6 + 6 rows at H = 12, not 8 + 4
   if (int64_t(a.N) * a.tiles_y * a.tiles_x > INT_MAX) return DCN_ERR_UNSUPPORTED;
   const size_t elems = size_t(problem->N) * problem->H * problem->W * C;
   a.x_bytes = elems * size_t(esize(problem->dtype));

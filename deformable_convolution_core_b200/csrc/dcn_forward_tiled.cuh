@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     for (;; ++i) {
       const int item = int(blockIdx.x) + i * int(gridDim.x);
       if (item >= t.items || *abort_flag) break;
-      if (i >= nbuf && !mbar_wait_bounded(&empty[b], ph ^ 1u)) {
+      if (i >= nbuf && !mbar_wait_bounded_sleep(&empty[b], ph ^ 1u)) {
         atomicOr(a.error_word, kErrTimeout);
         *abort_flag = 1;
         break;

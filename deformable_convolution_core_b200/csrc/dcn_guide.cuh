@@ -20,7 +20,8 @@
 // per tap) and parks the results in shared memory for the two LayerNorm
 // passes, so registers do not grow with C.  The weights and the affine
 // parameters are staged in shared memory once per CTA.  A CTA of
-// kGuideWarps warps covers adjacent columns and walks kGuideRows rows down:
+// kGuideWarps warps covers adjacent columns and walks up to kGuideRows rows
+// down (the image's rows split evenly over the row tiles):
 // consecutive windows of a lane group share six of their nine input pixels
 // and neighbouring groups share columns, so the input is read from DRAM
 // about once and re-read from L1.
@@ -47,6 +48,7 @@ struct GuideArgs {
   __nv_bfloat16* out;  // (N, H, W, C)
   int N, H, W, C, Q, NJ;
   int tiles_x, tiles_y;
+  int rows;  // rows a CTA walks: ceil(H / tiles_y), at most kGuideRows
   size_t x_bytes, out_bytes;  // bounds-checked build
 };
 
@@ -112,15 +114,28 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
   float4* const beta_s = gamma_s + a.Q;
   float4* const conv_buf = beta_s + a.Q;     // [j * kThreads + tid]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < 12 * a.Q; i += kThreads) {
-    float4 v;
-    if (i < 9 * a.Q) v = __ldg(reinterpret_cast<const float4*>(a.w) + i);
-    else {
-      const int r = (i - 9 * a.Q) / a.Q, q = i - 9 * a.Q - r * a.Q;
-      const float* src = r == 0 ? a.bias : (r == 1 ? a.gamma : a.beta);
-      v = ld4_or(src != nullptr ? src + 4 * q : nullptr, true, r == 1 ? 1.f : 0.f);
+  // Several loads in flight per thread (at C = 1280 a thread stages 15 quads;
+  // at the narrow widths, under the 3-CTA register cap, two at a time).
+  constexpr int IF = LP <= 16 ? 2 : 4;
+  for (int i0 = tid; i0 < 12 * a.Q; i0 += IF * kThreads) {
+    float4 v[IF];
+#pragma unroll
+    for (int u = 0; u < IF; ++u) {
+      const int i = i0 + u * kThreads;
+      if (i >= 12 * a.Q) break;
+      if (i < 9 * a.Q) v[u] = __ldg(reinterpret_cast<const float4*>(a.w) + i);
+      else {
+        const int r = (i - 9 * a.Q) / a.Q, q = i - 9 * a.Q - r * a.Q;
+        const float* src = r == 0 ? a.bias : (r == 1 ? a.gamma : a.beta);
+        v[u] = ld4_or(src != nullptr ? src + 4 * q : nullptr, true, r == 1 ? 1.f : 0.f);
+      }
     }
-    w_s[i] = v;
+#pragma unroll
+    for (int u = 0; u < IF; ++u) {
+      const int i = i0 + u * kThreads;
+      if (i >= 12 * a.Q) break;
+      w_s[i] = v[u];
+    }
   }
   __syncthreads();
 
@@ -137,8 +152,11 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
   const float inv_c = 1.0f / float(a.C);
 
 #pragma unroll 1
-  for (int i = 0; i < kGuideRows; ++i) {
-    const int y = ty * kGuideRows + i;
+  // (the narrow widths, under the 3-CTA register cap, keep the row count a
+  // compile-time constant: one register less)
+  const int rows = LP == 32 ? a.rows : kGuideRows;
+  for (int i = 0; i < rows; ++i) {
+    const int y = ty * rows + i;
     if (y >= a.H) break;  // the same for the whole CTA
     // depthwise 3x3 convolution, CH quads of this lane at a time in registers
     float s = 0.f;

@@ -101,9 +101,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
-// The same bound (one second) for consumers that may wait long: each poll
-// sleeps up to 2 microseconds inside try_wait, so waiting warps leave the
-// issue slots to the working ones.
+// The same bound (one second) for waits that may be long (a consumer waiting
+// for its box, a producer waiting for a free buffer): each poll sleeps up to 2
+// microseconds inside try_wait, so waiting warps leave the issue slots to the
+// working ones.
 __device__ __forceinline__ bool mbar_wait_bounded_sleep(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();

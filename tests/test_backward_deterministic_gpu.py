@@ -89,6 +89,27 @@ def test_deterministic_backward_matches_oracle(oracle_mod, case, dtype):
     assert torch.equal(goff, ref[1]) and torch.equal(gm, ref[2])
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_offset_and_mask_gradients_have_the_same_raw_bits_in_both_kernels(gen_mod, dtype):
+    """With 2-byte storage the tiled backward forms the corner dot products
+    with the mixed-precision FMA on the raw 16-bit words; the direct kernel
+    widens both operands first.  The products are exact either way, so
+    grad_offset and grad_mask carry the same bits, the sign of zero included
+    (compared as integers).  The batch includes zero grad_out rows."""
+    wl = WORKLOADS[f"internimage_l_stage2_bwd_{ {'bf16': 'bf16', 'f16': 'fp16'}[dtype]}_n32_48x48_c320"]
+    d = gen_mod.make_inputs(wl, n_images=4)
+    d["grad_out"][1, 5:9] = 0.0    # whole rows of zero gradient
+    d["grad_out"][2, :, 7] = -0.0
+    p = dcn.make_problem(4, wl.H, wl.W, wl.G, wl.Cg, offset_scale=wl.offset_scale, dtype=dtype)
+    args = [to_dev(d[k], dtype) for k in ("x", "offset", "mask", "grad_out")]
+    tiled = gpu_backward(p, *args)
+    with env(DCN_CORE_BACKWARD="direct"):
+        direct = gpu_backward(p, *args)
+    torch.cuda.synchronize()
+    for a, b in ((tiled[1], direct[1]), (tiled[2], direct[2])):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 def test_deterministic_backward_is_bitwise_reproducible(gen_mod, dtype):
     """Reruns, another stream, other tile shapes and the direct kernel all

@@ -194,6 +194,39 @@ def test_fused_guide_projection_at_stage1_size():
     assert torch.equal(off1, off2) and torch.equal(msk1, msk2)
 
 
+def test_fused_block_path_chain(oracle_mod):
+    """The block's forward around the core operator with the fused branch,
+    bf16, C = 160: guide + projection in one kernel -> core forward ->
+    output_proj.  Each GPU stage is checked against the oracle fed that stage's
+    GPU inputs (the query the branch keeps on chip is the standalone guide's,
+    bit for bit)."""
+    N, H, W, G = 2, 20, 18, 10
+    C = G * 16
+    p, xd, (w, b, g, be), pw, pb = fused_inputs(N, H, W, G, "bf16")
+    dev = lambda a: torch.from_numpy(a).cuda()
+    off, msk = projection_outputs(p, "bf16")
+    dcn.dcn_core_offset_mask_guide_projection(p, xd, dev(w), dev(b), dev(g), dev(be), 1e-6, pw,
+                                              pb, off, msk)
+    core = gpu_forward(p, xd, off, msk)
+    w_out = torch.from_numpy((RNG.standard_normal((C, C)) / np.sqrt(C)).astype(np.float32))
+    w_out = w_out.to(torch.bfloat16)
+    b_out = torch.from_numpy((0.1 * RNG.standard_normal(C)).astype(np.float32))
+    y = torch.empty((N * H * W, C), dtype=torch.bfloat16, device="cuda")
+    dcn.dcn_core_linear_bf16(core, N * H * W, C, w_out.cuda(), C, b_out.cuda(), y, "bf16")
+    q = run_guide(p, xd, w, b, g, be, 1e-6)
+    torch.cuda.synchronize()
+    dcn.dcn_core_sync_status()
+    assert gate(f64(q), oracle_mod.guide(f64(xd), w, b, g, be, 1e-6)).all()
+    ro, rm = oracle_mod.projection(f64(q), f64(pw), f64(pb.cpu()), G=G)
+    tol = 4 * C * 2.0 ** -24 * 8 + 2.0 ** -8
+    assert np.abs(f64(off) - ro).max() <= tol * max(1.0, np.abs(ro).max())
+    assert np.abs(f64(msk) - rm).max() <= tol * max(1.0, np.abs(rm).max())
+    ref_core = oracle_mod.forward(f64(xd), f64(off), f64(msk), **problem_kwargs(p))
+    assert np.abs(f64(core) - ref_core).max() <= 1e-2 * np.abs(ref_core).max()
+    ref_y = oracle_mod.linear(f64(core).reshape(-1, C), f64(w_out), b_out.numpy())
+    assert np.abs(f64(y) - ref_y).max() <= 1e-2 * np.abs(ref_y).max()
+
+
 def test_fused_guide_projection_rejects_before_launch():
     """Shapes the fused kernel does not serve are refused on the host."""
     fake = 1 << 20

@@ -62,6 +62,14 @@ def test_bench_reference_arm_two_ranks():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the reference arm's config is the GPU arm's, key for key (the sample note
+    # lives in cpu_baseline)
+    sys.path.insert(0, ROOT)
+    import bench
+    import gen
+    wl = gen.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    assert d["config"] == bench.workload_config(wl, wl.backward or wl.dtype == "f32", 2)
+    assert "sample" not in d["config"] and "sample" in d["cpu_baseline"]
 
 
 def test_bench_module_resolves_every_name():
