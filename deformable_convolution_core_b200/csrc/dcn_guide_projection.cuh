@@ -32,7 +32,7 @@
 namespace dcn {
 
 constexpr int kGpGuideWarps = 16;
-constexpr int kGpEpiWarps = kPjEpiWarps;  // 8
+constexpr int kGpEpiWarps = 8;  // two per TMEM lane quarter, each draining 64 columns
 constexpr int kGpFirstGuideWarp = 2 + kGpEpiWarps;
 constexpr int kGpThreads = (kGpFirstGuideWarp + kGpGuideWarps) * 32;
 constexpr uint32_t kGpABlockBytes = kPjBM * kPjBK * 2;  // 128 rows x 64 bf16

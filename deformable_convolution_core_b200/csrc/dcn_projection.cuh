@@ -14,11 +14,13 @@
 // streams 64-wide K blocks of the query and weight tiles into a 4-stage
 // shared-memory ring with TMA (128-byte swizzle); warp 1 allocates 256 TMEM
 // columns (two 128-column accumulators) and one of its threads issues
-// tcgen05.mma (M = 128, N = 128, K = 16) and tcgen05.commit; warps 2-9 drain
-// an accumulator with tcgen05.ld (two warps per 32-lane quarter of TMEM, each
-// taking 64 of the 128 columns), add the bias and store, staging each 32x32
+// tcgen05.mma (M = 128, N = 128, K = 16) and tcgen05.commit; warps 2-17 drain
+// an accumulator with tcgen05.ld (four warps per 32-lane quarter of TMEM, each
+// taking 32 of the 128 columns), add the bias and store, staging each 32x32
 // block through shared memory so that every store instruction writes one
-// pixel's contiguous columns.  The epilogue of one tile overlaps the MMAs of
+// pixel's contiguous columns.  The epilogue is latency-bound (a dependent
+// load / add / store chain per row), so it runs in as many warps as the
+// column blocks allow.  The epilogue of one tile overlaps the MMAs of
 // the next.  Every mbarrier wait is bounded; on expiry the kernel sets the
 // device error word, stops issuing work, waits (bounded) for what is in
 // flight and frees its tensor memory.
@@ -34,7 +36,8 @@ constexpr int kPjBM = 128;      // pixels per tile (MMA M, TMEM lanes)
 constexpr int kPjBN = 128;      // columns per tile (MMA N)
 constexpr int kPjBK = 64;       // K block: one 128-byte swizzle atom of bf16
 constexpr int kPjStages = 4;
-constexpr int kPjEpiWarps = 8;   // two per TMEM lane quarter, each draining half the columns
+constexpr int kPjEpiWarps = 16;  // four per TMEM lane quarter, each draining 32 of the columns
+constexpr int kPjEpiChunks = 16 / kPjEpiWarps;  // 32-column blocks per epilogue warp and tile
 constexpr int kPjThreads = (2 + kPjEpiWarps) * 32;  // TMA warp, MMA warp, epilogue warps
 constexpr uint32_t kPjTmemCols = 256;
 constexpr uint32_t kPjStageBytes = (kPjBM + kPjBN) * kPjBK * 2;  // A + B, 32 KB
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       (void)mbar_wait_bounded(mma_done, 0);
     }
   } else {
-    // ---- epilogue: warps 2-9; TMEM lanes 32 * (warp % 4) ... + 31, columns of half h ----
+    // ---- epilogue: warps 2-17; TMEM lanes 32 * (warp % 4) ... + 31, column block(s) h ----
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
     float* st = epi + (warp - 2) * 32 * kPjEpiPitch;
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
       const int row0 = mt * kPjBM + q * 32;
       const int rows = min(a.M - row0, 32);  // rows of this quarter inside the image batch
 #pragma unroll 1
-      for (int c = 2 * h; c < 2 * h + 2; ++c) {
+      for (int c = kPjEpiChunks * h; c < kPjEpiChunks * (h + 1); ++c) {
         // a block with no column below Nout (the padding of the last column
         // tile) or no row inside the batch has nothing to store
         if (nt * kPjBN + c * 32 >= a.Nout || rows <= 0) continue;
