@@ -350,6 +350,10 @@ def run_ours(args, world, rank, local):
                           "GB/s": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
                           "Gsamples/s": round(wl.samples / (bwd_ms * 1e-3) / 1e9, 2),
                           "frac_of_hbm": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peak, 4),
+                          "red_v4_G_per_s": round(red_v4_per_launch(wl) / (bwd_ms * 1e-3) / 1e9, 1),
+                          "frac_of_l2_red_ceiling": round(
+                              red_v4_per_launch(wl) / (bwd_ms * 1e-3) / 1e9 / L2_RED_V4_G_PER_S, 4),
+                          "l2_red_ceiling": L2_RED_CEILING_NOTE,
                           "note": "includes the zero-fill of grad_input"}},
         "roofline": roofline,
         "e2e": e2e,
@@ -504,6 +508,22 @@ def run_projection(gen, peak, launches=20):
         del q, w, b, off, msk
         torch.cuda.empty_cache()
     return out
+
+
+# The backward's binding ceiling: vector fp32 reductions into L2.  A
+# microbenchmark on this B200 (16 warps per SM, four lanes per random 64-byte
+# chunk, four chunks per step, as the grad_input scatter issues them) sustains
+# 331 G red.global.add.v4.f32 per second into an L2-resident buffer (8 or
+# 32 MB) and 108 G/s into a 1 GB one.
+L2_RED_V4_G_PER_S = 331.0
+L2_RED_CEILING_NOTE = ("331 G red.global.add.v4.f32/s: microbenchmark, random 64-byte chunks of "
+                       "an L2-resident buffer, 16 warps per SM")
+
+
+def red_v4_per_launch(wl):
+    """Vector reductions the atomic backward issues for grad_input: four
+    corners x Cg/4 float4s per sample (16 at Cg = 16)."""
+    return wl.samples * 4 * (wl.Cg // 4)
 
 
 NOMINAL_SM_MHZ = 1965.0
@@ -690,6 +710,9 @@ def run_sweep(gen, peak, clocks=None, reps=30, warmup=3):
                     "Gsamples/s": round(gsps, 2), "frac_of_l1_ceiling": None,
                     "MB": round(b / 1e6, 1), "l2": "flushed before every launch",
                     "_wl": wl}
+        if wl.backward and not det:  # the atomic backward's own ceiling: L2 reductions
+            out[key]["frac_of_l2_red_ceiling"] = round(
+                red_v4_per_launch(wl) / (ms * 1e-3) / 1e9 / L2_RED_V4_G_PER_S, 4)
         del step
         torch.cuda.empty_cache()
     del flush
