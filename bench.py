@@ -520,6 +520,21 @@ L2_RED_CEILING_NOTE = ("331 G red.global.add.v4.f32/s: microbenchmark, random 64
                        "an L2-resident buffer, 16 warps per SM")
 
 
+# The deterministic backward's: exact 64-bit fixed-point reductions, one per
+# channel and corner (lane r of a unit adds channels r, r+4, r+8, r+12, one
+# 32-byte sector per instruction across the unit's four lanes).  The same
+# microbenchmark in that pattern sustains 466 G red.global.add.u64 per second
+# into an L2-resident buffer, 2.8x fewer corner contributions per second than
+# the fp32 vector form.
+L2_RED_U64_G_PER_S = 466.0
+
+
+def red_u64_per_launch(wl):
+    """64-bit reductions the deterministic backward issues: four corners x Cg
+    channels per sample."""
+    return wl.samples * 4 * wl.Cg
+
+
 def red_v4_per_launch(wl):
     """Vector reductions the atomic backward issues for grad_input: four
     corners x Cg/4 float4s per sample (16 at Cg = 16)."""
@@ -710,9 +725,10 @@ def run_sweep(gen, peak, clocks=None, reps=30, warmup=3):
                     "Gsamples/s": round(gsps, 2), "frac_of_l1_ceiling": None,
                     "MB": round(b / 1e6, 1), "l2": "flushed before every launch",
                     "_wl": wl}
-        if wl.backward and not det:  # the atomic backward's own ceiling: L2 reductions
-            out[key]["frac_of_l2_red_ceiling"] = round(
-                red_v4_per_launch(wl) / (ms * 1e-3) / 1e9 / L2_RED_V4_G_PER_S, 4)
+        if wl.backward:  # the backward's own ceiling: reductions into L2
+            reds, peak_red = ((red_u64_per_launch(wl), L2_RED_U64_G_PER_S) if det
+                              else (red_v4_per_launch(wl), L2_RED_V4_G_PER_S))
+            out[key]["frac_of_l2_red_ceiling"] = round(reds / (ms * 1e-3) / 1e9 / peak_red, 4)
         del step
         torch.cuda.empty_cache()
     del flush
