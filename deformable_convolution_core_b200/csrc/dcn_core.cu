@@ -20,6 +20,7 @@
 #include "dcn_backward_tiled.cuh"
 #include "dcn_forward.cuh"
 #include "dcn_forward_tiled.cuh"
+#include "dcn_forward_tiled_wide.cuh"
 #include "dcn_guide.cuh"
 #include "dcn_guide_projection.cuh"
 #include "dcn_projection.cuh"
@@ -412,9 +413,10 @@ int env_int(const char* name, int dflt) {
 bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
   const char* mode = std::getenv("DCN_CORE_FORWARD");
   if (mode && std::strcmp(mode, "direct") == 0) return false;
-  // 16 channels per group in either storage type: 32-byte bf16 groups or
-  // 64-byte fp32 groups (eight accumulated values per phase-B lane).
-  if (p->K != 3 || p->Cg != 16) return false;
+  // 16 channels per group in any storage type: 32-byte 2-byte-type groups or
+  // 64-byte fp32 groups (eight accumulated values per phase-B lane); 3x3
+  // windows, and 5x5 and 7x7 ones in the wide-window kernel.
+  if ((p->K != 3 && p->K != 5 && p->K != 7) || p->Cg != 16) return false;
   if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
   return tensor_map_encoder() != nullptr;
 }
@@ -428,9 +430,13 @@ int box_pitch(int bw, int cs) {
   return bw + (bw & 1);
 }
 
+// Units per warp batch of the tiled kernels: 32 for 3x3 windows, 8 in the
+// wide-window kernel (5x5, 7x7).
+int tiled_batch(const dcn_problem* p) { return p->K == 3 ? kTiledBatch : kWideUnits; }
+
 // Box extent along one axis for a tile of `tile` outputs.
-int box_extent(int tile, int stride, int dil, int halo) {
-  return (tile - 1) * stride + 2 * dil + 2 + 2 * halo;
+int box_extent(int tile, int stride, int dil, int halo, int K) {
+  return (tile - 1) * stride + (K - 1) * dil + 2 + 2 * halo;
 }
 
 // Launch a persistent tiled kernel: as many CTAs as fit on the GPU at once,
@@ -535,8 +541,8 @@ bool fwd_tile_geometry(const dcn_problem* p, int TH, int TW, int cs, int halo, s
                        FwdTile* f) {
   f->TH = TH;
   f->TW = TW;
-  f->BH = clamp_extent(box_extent(TH, p->stride, p->dilation, halo), p->H);
-  f->BW = box_pitch(clamp_extent(box_extent(TW, stride_w(p), dil_w(p), halo), p->W), cs);
+  f->BH = clamp_extent(box_extent(TH, p->stride, p->dilation, halo, p->K), p->H);
+  f->BW = box_pitch(clamp_extent(box_extent(TW, stride_w(p), dil_w(p), halo, p->K), p->W), cs);
   if (f->BH > 256 || f->BW > 256) return false;
   f->box_bytes = uint32_t(size_t(f->BH) * f->BW * cs);
   f->box_stride = (f->box_bytes + 1023u) / 1024u * 1024u;
@@ -557,8 +563,8 @@ void choose_fwd_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, siz
       if (!fwd_tile_geometry(p, th, tw, cs, halo, optin, &f)) continue;
       const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * p->N * p->G;
       const int px = th * tw;
-      const double lane_samples = double((px + kTiledBatch - 1) / kTiledBatch) * kTiledBatch *
-                                  taps(p);
+      const int bu = tiled_batch(p);
+      const double lane_samples = double((px + bu - 1) / bu) * bu * taps(p);
       const double far_frac = f.far ? 0.3 * (1.0 / th + 1.0 / tw) : 0.0;
       const double per_item = lane_samples * (1.0 + 10.0 * far_frac) +
                               0.02 * double(f.box_bytes) / cs + 400.0 + (f.nbuf < 3 ? 200.0 : 0.0);
@@ -623,7 +629,7 @@ dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const
   const int64_t items = int64_t(t.N) * t.nTY * t.nTX * t.G;
   if (items > INT_MAX) return DCN_ERR_UNSUPPORTED;
   t.items = int(items);
-  t.batches = (t.TH * t.TW + kTiledBatch - 1) / kTiledBatch;
+  t.batches = (t.TH * t.TW + tiled_batch(p) - 1) / tiled_batch(p);
   t.fd_G = make_fastdiv(uint32_t(t.G));
   t.fd_nTX = make_fastdiv(uint32_t(t.nTX));
   t.fd_tiles = make_fastdiv(uint32_t(t.nTY * t.nTX));
@@ -634,11 +640,44 @@ dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const
   return encode_input_map(p, t, x, &L->map);
 }
 
+// The wide-window kernel: chunk size and record offset in a warp region.
+template <typename T, bool SOFTMAX>
+dcn_status forward_wide_launch(const CUtensorMap& map, const WideArgs& a, bool far, size_t smem,
+                               int sms, cudaStream_t stream) {
+  return far ? launch_persistent(dcn_forward_tiled_wide_kernel<T, SOFTMAX, true>, map, a, smem, sms, stream)
+             : launch_persistent(dcn_forward_tiled_wide_kernel<T, SOFTMAX, false>, map, a, smem, sms, stream);
+}
+
+dcn_status forward_tiled_wide(const dcn_problem* p, const BoxLaunch& L, const void* x,
+                              const void* off, const void* mask, void* out, cudaStream_t stream) {
+  WideArgs a;
+  a.x = x; a.off = off; a.mask = mask; a.out = out;
+  a.error_word = L.dev.error_word;
+  a.t = L.t;
+  a.K = p->K;
+  a.KK = taps(p);
+  a.kc = p->remove_center ? (p->K * p->K) / 2 : -1;
+  a.fd_K = make_fastdiv(uint32_t(p->K));
+  const int pair_bytes = 2 * esize(p->dtype);
+  a.rec = (wide_stage_bytes(a.KK, pair_bytes) + 15) / 16 * 16;
+  // as many taps per chunk as the region holds, then evened out over the chunks
+  const int ch_max = std::min(32, (kFwdRegion - a.rec) / wide_rec_bytes(1));
+  if (a.KK > kWideMaxTaps || ch_max < 1) return DCN_ERR_UNSUPPORTED;
+  const int nch = (a.KK + ch_max - 1) / ch_max;
+  a.CH = (a.KK + nch - 1) / nch;
+  return with_storage(p->dtype, [&](auto tag) {
+    using T = decltype(tag);
+    return p->softmax ? forward_wide_launch<T, true>(L.map, a, L.far, L.smem, L.dev.sms, stream)
+                      : forward_wide_launch<T, false>(L.map, a, L.far, L.smem, L.dev.sms, stream);
+  });
+}
+
 dcn_status forward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
                          const void* off, const void* mask, void* out, cudaStream_t stream) {
   BoxLaunch L;
   dcn_status st = box_tiled_prepare(p, Ho, Wo, x, "DCN_CORE_TILED_TILE", &L);
   if (st != DCN_OK) return st;
+  if (p->K != 3) return forward_tiled_wide(p, L, x, off, mask, out, stream);
   TiledArgs args;
   args.t = L.t;
   args.x = x; args.off = off; args.mask = mask; args.out = out;

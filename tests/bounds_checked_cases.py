@@ -92,6 +92,13 @@ def main():
     case("separate axes K=5", mk(1, 12, 15, 2, 8, K=5, pad=2, stride_w=2, pad_w=1,
                                  offset_scale=2.0))
     case("Cg 32 raw mask", mk(1, 10, 9, 3, 32, softmax=0, offset_scale=2.0))
+    # the wide-window tiled forward (5x5 and 7x7 windows, chunked taps)
+    case("K=5 wide", mk(2, 13, 17, 3, 16, K=5, pad=2, offset_scale=2.0))
+    case("K=7 bf16 dilation 2 remove_center raw mask",
+         mk(1, 15, 14, 2, 16, K=7, pad=6, dilation=2, softmax=0, offset_scale=2.0,
+            dtype="bf16", remove_center=1), dtype="bf16")
+    case("K=7 fp16 offsets +-1e4", mk(1, 9, 12, 2, 16, K=7, pad=3, offset_scale=2.0,
+                                      dtype="f16"), far, dtype="f16")
     # the tensor-core projection, ragged in pixels and columns
     p = mk(1, 7, 9, 5, 16, offset_scale=2.0)
     q = torch.randn(1, 7, 9, 64).to(torch.bfloat16).cuda()

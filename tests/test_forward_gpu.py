@@ -198,6 +198,31 @@ def test_nonfinite_and_border_offsets(oracle_mod):
     check_full(oracle_mod, p, x, off, mask, "f32")
 
 
+@pytest.mark.parametrize("halo,tile", [("0", "1x1"), ("2", "3x5"), ("4", "24x24"), ("5", "9x40")])
+def test_wide_window_tiled_kernel_tile_and_halo_settings(oracle_mod, halo, tile):
+    """The wide-window tiled kernel (5x5 and 7x7 windows: batches of 8 units,
+    taps in chunks) at every tile shape and halo width, in all three storage
+    types: small tiles and no halo send most taps to the far path."""
+    old = {k: os.environ.get(k) for k in ("DCN_CORE_HALO", "DCN_CORE_TILED_TILE")}
+    os.environ["DCN_CORE_HALO"], os.environ["DCN_CORE_TILED_TILE"] = halo, tile
+    try:
+        for dtype in ("f32", "bf16", "f16"):
+            p, x, off, mask = random_case(2, 23, 29, 3, 16, K=5, dtype=dtype, off_sd=2.0)
+            check_full(oracle_mod, p, x, off, mask, dtype)
+            p, x, off, mask = random_case(1, 26, 21, 2, 16, K=7, dtype=dtype, softmax=0,
+                                          remove_center=1)
+            check_full(oracle_mod, p, x, off, mask, dtype)
+            p, x, off, mask = random_case(1, 30, 27, 2, 16, K=5, dtype=dtype, stride=2, dil=2,
+                                          remove_center=1)
+            check_full(oracle_mod, p, x, off, mask, dtype)
+    finally:
+        for k, v in old.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+
+
 def test_forward_is_deterministic_and_stream_safe(oracle_mod):
     p, x, off, mask = random_case(2, 31, 29, 6, 16, dtype="bf16")
     xd, od, md = to_dev(x, "bf16"), to_dev(off, "bf16"), to_dev(mask, "bf16")
