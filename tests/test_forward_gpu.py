@@ -335,13 +335,15 @@ def test_full_size_workload_sampled(gen_mod, oracle_mod, name, path):
     assert torch.isfinite(out).all()
 
 
-def test_bounded_wait_expiry_is_reported_and_recoverable():
+@pytest.mark.parametrize("K", [3, 5])
+def test_bounded_wait_expiry_is_reported_and_recoverable(K):
     """Failure detection without a GPU fault: with the test knob the first TMA
     box of every CTA never arrives, the bounded mbarrier waits give up (about a
     second), the kernel sets the device error word and returns;
     dcn_core_sync_status reports DCN_ERR_TIMEOUT and clears the word, and the
-    next call works normally."""
-    p, x, off, mask = random_case(2, 23, 29, 3, 16, dtype="f32")
+    next call works normally.  K = 5 runs the wide-window kernel, whose
+    consumers also have staging copies in flight when they give up."""
+    p, x, off, mask = random_case(2, 23, 29, 3, 16, K=K, dtype="f32")
     xd, od, md = to_dev(x, "f32"), to_dev(off, "f32"), to_dev(mask, "f32")
     with forward_path("auto"):
         ref = gpu_forward(p, xd, od, md)
