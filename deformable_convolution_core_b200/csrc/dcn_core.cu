@@ -13,7 +13,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <numeric>
 
 #include "dcn_backward.cuh"
@@ -554,21 +556,32 @@ bool fwd_tile_geometry(const dcn_problem* p, int TH, int TW, int cs, int halo, s
   return true;
 }
 
+// Tile choice: the shape that minimises a per-item cost times the rounds of
+// items each persistent CTA runs.  Per item: the lane-samples of its batches,
+// the far taps (about 0.3 (1/TH + 1/TW) of them leave the box), the box pixels
+// the producer loads, and a penalty for fewer than three boxes in flight.  The
+// rounds are counted for a reference batch of 64 images, not the problem's N:
+// the choice, and with it which taps the box serves (the last bits of the
+// forward), then does not depend on how a batch is split.  The weights were
+// fitted to measured times of tile shapes on the InternImage-L stage shapes
+// and the 256 x 256 DCNv4 shape.
 void choose_fwd_tile(const dcn_problem* p, int Ho, int Wo, int cs, int halo, size_t optin,
-                     FwdTile* out) {
+                     int ctas, FwdTile* out) {
   double best = 1e300;
   for (int th = 1; th <= std::min(Ho, 64); ++th) {
     for (int tw = 1; tw <= std::min(Wo, 64); ++tw) {
       FwdTile f;
       if (!fwd_tile_geometry(p, th, tw, cs, halo, optin, &f)) continue;
-      const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * p->N * p->G;
+      constexpr int64_t kRefImages = 64;
+      const int64_t items = int64_t((Ho + th - 1) / th) * ((Wo + tw - 1) / tw) * kRefImages * p->G;
+      const int64_t rounds = (items + ctas - 1) / std::max(ctas, 1);
       const int px = th * tw;
       const int bu = tiled_batch(p);
       const double lane_samples = double((px + bu - 1) / bu) * bu * taps(p);
       const double far_frac = f.far ? 0.3 * (1.0 / th + 1.0 / tw) : 0.0;
-      const double per_item = lane_samples * (1.0 + 10.0 * far_frac) +
-                              0.02 * double(f.box_bytes) / cs + 400.0 + (f.nbuf < 3 ? 200.0 : 0.0);
-      const double cost = double(items) * per_item;
+      const double per_item = lane_samples * (1.0 + far_frac) + 0.5 * double(f.box_bytes) / cs +
+                              (f.nbuf < 3 ? 200.0 : 0.0);
+      const double cost = double(rounds) * per_item;
       if (cost < best) {
         best = cost;
         *out = f;
@@ -607,7 +620,24 @@ dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const
                            optin, &f))
       return DCN_ERR_UNSUPPORTED;
   } else {
-    choose_fwd_tile(p, int(Ho), int(Wo), cs, halo, optin, &f);
+    // The search costs tens of microseconds of host time: remember its answer
+    // for each problem shape (everything the choice depends on is in the key).
+    using Key = std::tuple<int, int, int, int, int, int, int, int, int, int, int, int, int, int,
+                           int, size_t, int>;
+    static std::map<Key, FwdTile> memo;
+    static std::mutex memo_lock;
+    const Key key{0, p->H, p->W, int(Ho), int(Wo), p->G, p->K, p->stride, stride_w(p),
+                  p->dilation, dil_w(p), p->remove_center, cs, halo, tiled_batch(p), optin,
+                  L->dev.sms};
+    std::lock_guard<std::mutex> guard(memo_lock);
+    auto it = memo.find(key);
+    if (it == memo.end()) {
+      f = FwdTile{};
+      choose_fwd_tile(p, int(Ho), int(Wo), cs, halo, optin, L->dev.sms, &f);
+      if (memo.size() > 4096) memo.clear();  // bound the host memory a long run can use
+      it = memo.emplace(key, f).first;
+    }
+    f = it->second;
     if (f.nbuf == 0) return DCN_ERR_UNSUPPORTED;
   }
   if (const int nb = env_int("DCN_CORE_TILED_BUFS", 0); nb >= 2 && nb < f.nbuf) f.nbuf = nb;

@@ -336,31 +336,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           fv[j] = ldg128_pred(pp, in && in_tensor(pp, 16, a.x, x_bytes));
         }
       };
-      // The first far tap of unit u, fetched one step before it is used; fm
-      // returns the unit's other far taps.
-      auto far_first = [&](int u, uint4 (&fv)[NP], float& fw, uint32_t& fm) {
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(fm) : "r"(reg_a + kFwdRegFm + 4u * u));
-        fw = 0.f;
-#pragma unroll
-        for (int j = 0; j < NP; ++j) fv[j] = make_uint4(0u, 0u, 0u, 0u);
-        if (fm != 0u) {
-          far_fetch(u, __ffs(fm) - 1, fv, fw);
-          fm &= fm - 1u;
-        }
-      };
-      // (2-byte storage only: for fp32 the two prefetched pieces sets would cost
-      // more registers than the rare far taps of fp32 workloads gain)
-      constexpr bool kAhead = FAR && NP == 2;
-      uint4 fv_cur[NP], fv_nxt[NP];
-      float fw_cur = 0.f, fw_nxt = 0.f;
-      uint32_t fm_cur = 0u, fm_nxt = 0u;
-      if (kAhead) far_first(u8, fv_cur, fw_cur, fm_cur);
-
       // Phase B: 8 units per step, one lane per corner.
 #pragma unroll 1
       for (int s = 0; s < kTiledBatch / 8; ++s) {
         const int u = s * 8 + u8;
-        if (kAhead && s + 1 < kTiledBatch / 8) far_first(u + 8, fv_nxt, fw_nxt, fm_nxt);
         float2 acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
@@ -379,16 +358,11 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
             IO::fma16(acc + j * (8 / NP), w2, lds128_a(a0 ^ uint32_t(16 * j)));
         }
         if (FAR) {
-          // The unit's first far tap (fetched during the previous step), then
-          // any others in a warp-uniform loop.
-          uint32_t fm = fm_cur;
-          if (kAhead) {
-#pragma unroll
-            for (int j = 0; j < NP; ++j)
-              IO::fma16(acc + j * (8 / NP), make_float2(fw_cur, fw_cur), fv_cur[j]);
-          } else {
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(fm) : "r"(reg_a + kFwdRegFm + 4u * u));
-          }
+          // The unit's far taps, in a warp-uniform loop.  (Fetching the first
+          // one a step ahead cost more in registers and per-step work than it
+          // saved: 4-6% slower at the stage shapes.)
+          uint32_t fm;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(fm) : "r"(reg_a + kFwdRegFm + 4u * u));
           while (__any_sync(0xFFFFFFFFu, fm != 0u)) {
             if (fm != 0u) {
               uint4 fv[NP];
@@ -399,12 +373,6 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
                 IO::fma16(acc + j * (8 / NP), make_float2(fw, fw), fv[j]);
               fm &= fm - 1u;
             }
-          }
-          if (kAhead) {
-#pragma unroll
-            for (int j = 0; j < NP; ++j) fv_cur[j] = fv_nxt[j];
-            fw_cur = fw_nxt;
-            fm_cur = fm_nxt;
           }
         }
         // Reduce-scatter over the unit's four corner lanes, then store.
