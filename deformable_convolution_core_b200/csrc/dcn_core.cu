@@ -446,14 +446,39 @@ int box_extent(int tile, int stride, int dil, int halo, int K) {
 template <typename Kernel, typename Args>
 dcn_status launch_persistent(Kernel k, const CUtensorMap& map, const Args& args, size_t smem,
                              int sms, cudaStream_t stream) {
-  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-      cudaSuccess)
-    return DCN_ERR_CUDA;
+  // Driver calls made once, not per launch: the kernel's dynamic shared-memory
+  // limit (per context and kernel; only ever raised, since a lower limit would
+  // refuse an earlier, larger configuration) and its occupancy (per context,
+  // kernel and byte count).
+  using KernelKey = std::pair<unsigned long long, const void*>;
+  using OccKey = std::tuple<unsigned long long, const void*, size_t>;
+  static std::map<KernelKey, size_t> smem_limit;
+  static std::map<OccKey, int> blocks_per_sm;
+  static std::mutex lock;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kTiledThreads, smem) !=
-          cudaSuccess ||
-      per_sm < 1)
-    return DCN_ERR_UNSUPPORTED;
+  {
+    std::lock_guard<std::mutex> guard(lock);
+    const unsigned long long ctx = current_context_id();
+    const void* kp = reinterpret_cast<const void*>(k);
+    auto lim = smem_limit.find(KernelKey{ctx, kp});
+    if (lim == smem_limit.end() || lim->second < smem) {
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+          cudaSuccess)
+        return DCN_ERR_CUDA;
+      smem_limit[KernelKey{ctx, kp}] = smem;
+    }
+    const OccKey key{ctx, kp, smem};
+    auto it = blocks_per_sm.find(key);
+    if (it == blocks_per_sm.end()) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kTiledThreads, smem) !=
+          cudaSuccess)
+        return DCN_ERR_UNSUPPORTED;
+      if (blocks_per_sm.size() > 4096) blocks_per_sm.clear();
+      it = blocks_per_sm.emplace(key, per_sm).first;
+    }
+    per_sm = it->second;
+  }
+  if (per_sm < 1) return DCN_ERR_UNSUPPORTED;
   const int64_t grid = std::min<int64_t>(args.t.items, int64_t(sms) * per_sm);
   k<<<unsigned(grid), kTiledThreads, smem, stream>>>(map, args);
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;

@@ -14,7 +14,7 @@ import torch
 
 import deformable_convolution_core_b200 as dcn
 from gen.workloads import WORKLOADS
-from tests.dcn_testutil import assert_fwd, f64, gpu_forward, problem_kwargs, to_dev
+from tests.dcn_testutil import assert_bwd, assert_fwd, f64, gpu_backward, gpu_forward, problem_kwargs, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -221,6 +221,24 @@ def test_wide_window_tiled_kernel_tile_and_halo_settings(oracle_mod, halo, tile)
                 os.environ.pop(k, None)
             else:
                 os.environ[k] = v
+
+
+def test_tiled_kernels_alternate_shared_memory_sizes(oracle_mod):
+    """The same tiled kernels launched with a large, a small and again the
+    large shared-memory size (big image, tiny image, big image): the
+    library's once-per-kernel shared-memory limit must only ever grow."""
+    shapes = [(2, 96, 96), (1, 6, 7), (2, 96, 96)]
+    for N, H, W in shapes:
+        p, x, off, mask = random_case(N, H, W, 2, 16, dtype="bf16", off_sd=3.0)
+        check_full(oracle_mod, p, x, off, mask, "bf16")
+        xd, od, md = to_dev(x, "bf16"), to_dev(off, "bf16"), to_dev(mask, "bf16")
+        gd = to_dev(RNG.standard_normal((N, H, W, 32)).astype(np.float32), "bf16")
+        gx, goff, gm = gpu_backward(p, xd, od, md, gd)
+        torch.cuda.synchronize()
+        dcn.dcn_core_sync_status()
+        rx, roff, rm = oracle_mod.backward(f64(xd), f64(od), f64(md), f64(gd), **problem_kwargs(p))
+        assert_bwd(f64(gx), rx, f"grad_input {N}x{H}x{W}", "bf16")
+        assert_bwd(f64(goff), roff, f"grad_offset {N}x{H}x{W}", "bf16")
 
 
 def test_forward_is_deterministic_and_stream_safe(oracle_mod):
