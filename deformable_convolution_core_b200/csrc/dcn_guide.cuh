@@ -151,7 +151,6 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
   const size_t rowE = size_t(a.W) * a.C;  // elements per image row
   const float inv_c = 1.0f / float(a.C);
 
-#pragma unroll 1
   // (the narrow widths, under the 3-CTA register cap, keep the row count a
   // compile-time constant: one register less)
   const int rows = LP == 32 ? a.rows : kGuideRows;
