@@ -251,6 +251,13 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       uint32_t q;
       batch_unit(beta, ho, wo, q);
       const bool valid = q != ~0u;
+      // Phase-B steps that hold pixels of the tile: the last batch of a tile
+      // whose pixel count is not a multiple of 32 is partly empty.  Only the
+      // whole-image boxes (no far taps) get such tiles from the host's choice;
+      // the far-tap kernel keeps a compile-time step count (a runtime one made
+      // the stage-1 bf16 forward 3.5% slower).
+      const int nsteps = FAR ? kTiledBatch / 8
+                             : min(kTiledBatch / 8, (npx - (beta - il * nb) * kTiledBatch + 7) / 8);
       __syncwarp();
 
       // Phase A: this lane's unit -> softmax, then per tap the corner weights
@@ -338,7 +345,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       };
       // Phase B: 8 units per step, one lane per corner.
 #pragma unroll 1
-      for (int s = 0; s < kTiledBatch / 8; ++s) {
+      for (int s = 0; s < nsteps; ++s) {
         const int u = s * 8 + u8;
         float2 acc[8];
 #pragma unroll
