@@ -520,13 +520,13 @@ L2_RED_CEILING_NOTE = ("331 G red.global.add.v4.f32/s: microbenchmark, random 64
                        "an L2-resident buffer, 16 warps per SM")
 
 
-# The deterministic backward's: exact 64-bit fixed-point reductions, one per
-# channel and corner (lane r of a unit adds channels r, r+4, r+8, r+12, one
-# 32-byte sector per instruction across the unit's four lanes).  The same
-# microbenchmark in that pattern sustains 466 G red.global.add.u64 per second
-# into an L2-resident buffer, 2.8x fewer corner contributions per second than
-# the fp32 vector form.
-L2_RED_U64_G_PER_S = 466.0
+# The deterministic backward's: exact 64-bit fixed-point adds, one per channel
+# and corner.  The tiled kernel sends a corner's 16 channels as one 128-byte
+# bulk reduction from shared memory (cp.reduce.async.bulk .add.u64); the same
+# microbenchmark (random 128-byte corners of an L2-resident buffer, 16 warps
+# per SM) sustains 798 G such adds per second.  Scalar red.global.add.u64
+# (the direct kernel's form) sustains 466 G/s.
+L2_RED_U64_G_PER_S = 798.0
 
 
 def red_u64_per_launch(wl):

@@ -230,6 +230,9 @@ struct GxScatter<true> {
     int S = 0;
     scale = det_exponent(hdr, softmax, cbits, &S) ? __int_as_float((S + 127) << 23) : 0.f;
   }
+  // v * 2^S is exact (a power-of-two scaling below 2^62); the conversion rounds
+  // it to the nearest integer.
+  __device__ __forceinline__ long long fixed(float v) const { return __float2ll_rn(v * scale); }
   __device__ __forceinline__ void add(size_t e, float2 lo, float2 hi, bool pred) const {
     if (pred && !in_range(e + 3, n)) pred = false;
     // v * 2^S is exact (a power-of-two scaling below 2^62); the conversion rounds

@@ -183,9 +183,27 @@ __device__ __forceinline__ void piece_widen<__half>(const uint4& v, float2* g) {
   g[3] = f16x2_to_f32x2(v.w);
 }
 
+// Deterministic backward: after the warp regions and the barriers, each warp
+// has a staging slot of [8 units][CPR corners][16 channels] 64-bit fixed-point
+// values.  A tap's contributions go there, CPR corners per round, and lane r
+// of a unit sends its corner r to the accumulator as one 128-byte bulk
+// reduction (cp.reduce.async.bulk .add.u64): 16 channel adds per request
+// instead of 16 scalar red.global.add.u64 (measured on B200: 798 G adds/s
+// against 466 G/s for the scalar reductions on random corners of an
+// L2-resident accumulator).  fp32 takes two corners per round, so that the
+// slots leave its twice larger boxes room for the tiles the fp32 pass needs.
+__host__ __device__ constexpr int det_corners_per_round(int esize) { return esize == 4 ? 2 : 4; }
+__host__ __device__ constexpr int det_stage_bytes(int esize) {  // per warp
+  return 8 * det_corners_per_round(esize) * 16 * 8;
+}
+__host__ __device__ constexpr size_t det_stage_total(int esize) {
+  return size_t(kTiledWarps) * det_stage_bytes(esize);
+}
+
 // KKS: 9 (the 3x3 window) or 8 (the window without its centre).  DET: exact
-// fixed-point accumulation of grad_input (GxScatter).  FAR: some footprint can
-// leave the box.
+// fixed-point accumulation of grad_input (GxScatter), through the staging slots
+// above (the launch adds det_stage_total(sizeof(T)) bytes of shared memory).  FAR: some
+// footprint can leave the box.
 template <typename T, int KKS, bool SOFTMAX, bool DET, bool FAR>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     dcn_backward_tiled_kernel(const __grid_constant__ CUtensorMap xmap, const TiledBwdArgs a) {
@@ -257,6 +275,11 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   // ---- consumer warps ----
   unsigned char* const reg = regions + size_t(warp) * kFwdRegion;
   const uint32_t reg_a = smem_addr(reg);
+  // this warp's staging slot (deterministic backward), 128-byte aligned: the
+  // regions and the barrier tail are multiples of 128 bytes
+  constexpr int CPR = det_corners_per_round(int(sizeof(T)));
+  const uint32_t stage_a = smem_addr(regions + size_t(kTiledWarps) * kFwdRegion + kFwdTailBytes) +
+                           uint32_t(warp) * det_stage_bytes(int(sizeof(T)));
   const uint32_t zero_a = smem_addr(zero);
   const int u8 = lane >> 2, r = lane & 3, dy = r >> 1, dx = r & 1, rho = u8 & 1;
   const int rot = NP == 2 ? rho : 2 * dy + rho;  // piece j ^ rot in read j (as the forward)
@@ -332,7 +355,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const char* const ximg = reinterpret_cast<const char*>(a.x) + img * sizeof(T);
     const GxScatter<DET> gxs(a.gx, a.det_hdr, SOFTMAX, a.det_cbits, n_img);
     // this lane's first accumulator channel of corner (y0, x0) at CE = 0
-    typename GxScatter<DET>::Acc* const gx_lane = gxs.p + img + (DET ? r : 4 * r);
+    typename GxScatter<DET>::Acc* const gx_lane = gxs.p + img + 4 * r;
 
     for (; beta < (il + 1) * nb; beta += kTiledWarps) {
 #pragma unroll
@@ -438,18 +461,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           if constexpr (NP == 4) return piece_dot<T>(v, gs + j * GP);
           else return piece_dot16<T>(v, gw[j]);
         };
-        // scatter channels of this lane: 4r .. 4r+3 (fp32 vector reductions), or
-        // r, r+4, r+8, r+12 (fixed point: one 32-byte sector per instruction)
+        // scatter channels of this lane: 4r .. 4r+3
         float2 gr_lo, gr_hi;
-        if (DET) {
-          float v[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) v[i] = gok ? Storage<T>::to_float(reinterpret_cast<const T*>(gp)[r + 4 * i]) : 0.f;
-          gr_lo = make_float2(v[0], v[1]);
-          gr_hi = make_float2(v[2], v[3]);
-        } else {
-          BwdIO<T>::quad(gp + 4 * r * sizeof(T), gok, gr_lo, gr_hi);
-        }
+        BwdIO<T>::quad(gp + 4 * r * sizeof(T), gok, gr_lo, gr_hi);
         char* const goff_u = reinterpret_cast<char*>(a.goff) +
                              (size_t(uvalid ? pix : 0u) * t.G + c.g) * KK * sizeof(Pair);
         const uint32_t lead_ok = (r == 0 && uvalid) ? 1u : 0u;
@@ -501,18 +515,55 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           bilinear_weights(ly, lx, bw);
           const float wc[4] = {__fmul_rn(m, bw[0]), __fmul_rn(m, bw[1]), __fmul_rn(m, bw[2]),
                                __fmul_rn(m, bw[3])};
+          if constexpr (DET) {
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int e = ce + (cc >> 1) * rowE + (cc & 1) * pixE;
-            const float2 w2 = make_float2(wc[cc], wc[cc]);
-            if constexpr (DET)
-              gxs.add4_strided(gx_lane + e,
-                               kCheckBounds ? img + size_t(r) + size_t(ptrdiff_t(e)) : 0,
-                               __fmul2_rn(w2, gr_lo), __fmul2_rn(w2, gr_hi), (inb >> cc) & 1u);
-            else
+           for (int c0 = 0; c0 < 4; c0 += CPR) {
+            // The previous round's bulk reductions have read the slot (each lane
+            // waits for its own, then the warp), so it can be rewritten.
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
+            // slot (u8, cc - c0) holds corner cc's 16 channels; this lane's four
+            // at 4r, as two 16-byte stores (odd units store the halves in the
+            // other order: the two units of a quarter-warp hit other banks)
+#pragma unroll
+            for (int cc = c0; cc < c0 + CPR; ++cc) {
+              const float2 w2 = make_float2(wc[cc], wc[cc]);
+              const float2 lo = __fmul2_rn(w2, gr_lo), hi = __fmul2_rn(w2, gr_hi);
+              const uint32_t sa = stage_a + uint32_t(((u8 * CPR + cc - c0) * 16 + 4 * r) * 8);
+              const long long f0 = gxs.fixed(lo.x), f1 = gxs.fixed(lo.y);
+              const long long f2 = gxs.fixed(hi.x), f3 = gxs.fixed(hi.y);
+              if (rho) {
+                asm volatile("st.shared.v2.u64 [%0], {%1, %2};" ::"r"(sa + 16u), "l"(f2), "l"(f3) : "memory");
+                asm volatile("st.shared.v2.u64 [%0], {%1, %2};" ::"r"(sa), "l"(f0), "l"(f1) : "memory");
+              } else {
+                asm volatile("st.shared.v2.u64 [%0], {%1, %2};" ::"r"(sa), "l"(f0), "l"(f1) : "memory");
+                asm volatile("st.shared.v2.u64 [%0], {%1, %2};" ::"r"(sa + 16u), "l"(f2), "l"(f3) : "memory");
+              }
+            }
+            // the slot, written through the generic proxy, is read by the bulk copies
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            // lane r: corner r of its unit (in this round), if it lies in the image
+            const int e = ce + (r >> 1) * rowE + (r & 1) * pixE;
+            const size_t ge = img + size_t(ptrdiff_t(e));  // its channel 0
+            if (r >= c0 && r < c0 + CPR && ((inb >> r) & 1u) != 0u && in_range(ge + 15, n_img)) {
+              unsigned long long* const gq = gxs.p + ge;
+              asm volatile(
+                  "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.u64 [%0], [%1], 128;" ::"l"(gq),
+                  "r"(stage_a + uint32_t((u8 * CPR + r - c0) * 128))
+                  : "memory");
+            }
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+           }
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int e = ce + (cc >> 1) * rowE + (cc & 1) * pixE;
+              const float2 w2 = make_float2(wc[cc], wc[cc]);
               gxs.add_at(gx_lane + e,
                          kCheckBounds ? img + size_t(4 * r) + size_t(ptrdiff_t(e)) : 0,
                          __fmul2_rn(w2, gr_lo), __fmul2_rn(w2, gr_hi), (inb >> cc) & 1u);
+            }
           }
         }
         if (lead_ok) {
@@ -537,6 +588,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       ph ^= 1u;
     }
   }
+  // the bulk reductions of this thread are complete before it exits
+  if constexpr (DET) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 }  // namespace dcn

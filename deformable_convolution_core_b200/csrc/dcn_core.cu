@@ -623,8 +623,10 @@ struct BoxLaunch {
   bool far;
 };
 
+// reserve: shared memory the kernel needs beyond the forward's layout (the
+// deterministic backward's staging slots); the boxes get what is left.
 dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const void* x,
-                             const char* tile_env, BoxLaunch* L) {
+                             const char* tile_env, BoxLaunch* L, size_t reserve = 0) {
   dcn_status st = device_info(&L->dev);
   if (st != DCN_OK) return st;
   const int cs = p->Cg * esize(p->dtype);
@@ -634,7 +636,8 @@ dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const
   // InternImage-L stage-1 shapes, 4 is the fastest for fp32 (forward 0.437 ms
   // against 0.459 at 5) and 5 for bf16 and fp16.
   const int halo = std::max(0, env_int("DCN_CORE_HALO", cs == 64 ? 4 : 5));
-  const size_t optin = size_t(L->dev.smem_optin);
+  if (size_t(L->dev.smem_optin) <= reserve) return DCN_ERR_UNSUPPORTED;
+  const size_t optin = size_t(L->dev.smem_optin) - reserve;
   FwdTile f;
   int TH = 0, TW = 0;
   if (const char* s = std::getenv(tile_env)) {  // "THxTW", for tuning sweeps
@@ -692,6 +695,7 @@ dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const
   L->far = f.far;
   L->smem = fwd_tiled_smem(t.nbuf, t.box_stride, t.BW, cs);
   if (L->smem > optin) return DCN_ERR_UNSUPPORTED;
+  L->smem += reserve;
   return encode_input_map(p, t, x, &L->map);
 }
 
@@ -756,7 +760,9 @@ bool backward_tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
 dcn_status backward_tiled(const dcn_problem* p, int64_t Ho, int64_t Wo, const BwdArgs& a,
                           bool det, cudaStream_t stream) {
   BoxLaunch L;
-  dcn_status st = box_tiled_prepare(p, Ho, Wo, a.x, "DCN_CORE_BWD_TILED_TILE", &L);
+  dcn_status st =
+      box_tiled_prepare(p, Ho, Wo, a.x, "DCN_CORE_BWD_TILED_TILE", &L,
+                        det ? det_stage_total(esize(p->dtype)) : 0);
   if (st != DCN_OK) return st;
   TiledBwdArgs args;
   args.t = L.t;
