@@ -417,8 +417,10 @@ bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
   if (mode && std::strcmp(mode, "direct") == 0) return false;
   // 16 channels per group in any storage type: 32-byte 2-byte-type groups or
   // 64-byte fp32 groups (eight accumulated values per phase-B lane); 3x3
-  // windows, and 5x5 and 7x7 ones in the wide-window kernel.
-  if ((p->K != 3 && p->K != 5 && p->K != 7) || p->Cg != 16) return false;
+  // windows, and 5x5 and 7x7 ones in the wide-window kernel.  The 3x3 kernel
+  // also takes 8 channels of a 2-byte type (16-byte groups).
+  const bool cg8 = p->K == 3 && p->Cg == 8 && esize(p->dtype) == 2;
+  if (!cg8 && ((p->K != 3 && p->K != 5 && p->K != 7) || p->Cg != 16)) return false;
   if (p->H > 16000 || p->W > 16000 || Ho > 16000 || Wo > 16000) return false;
   return tensor_map_encoder() != nullptr;
 }
@@ -426,9 +428,13 @@ bool tiled_eligible(const dcn_problem* p, int64_t Ho, int64_t Wo) {
 // Box row pitch (pixels) that makes the footprint reads conflict-free: for
 // 32-byte groups the two rows of a footprint must fall into complementary
 // halves of the 32 banks (pitch = 2 mod 4); for 64-byte groups the pitch
-// must be even (the lanes' piece rotation does the rest).
+// must be even (the lanes' piece rotation does the rest).  16-byte groups
+// take pitch = 4 mod 8: a unit's four corners then sit in four distinct
+// 16-byte bank groups, and the two units of a quarter-warp meet at most two
+// to a bank group (no pitch keeps every random pair apart).
 int box_pitch(int bw, int cs) {
   if (cs == 32) return bw + (2 - bw % 4 + 4) % 4;
+  if (cs == 16) return bw + (4 - bw % 8 + 8) % 8;
   return bw + (bw & 1);
 }
 
@@ -484,17 +490,26 @@ dcn_status launch_persistent(Kernel k, const CUtensorMap& map, const Args& args,
   return cudaGetLastError() == cudaSuccess ? DCN_OK : DCN_ERR_CUDA;
 }
 
+template <typename T, bool FAR, int CG>
+dcn_status forward_tiled_dispatch_cg(const dcn_problem* p, const CUtensorMap& map,
+                                     const TiledArgs& args, size_t smem, int sms,
+                                     cudaStream_t stream) {
+  if (p->remove_center)
+    return p->softmax
+               ? launch_persistent(dcn_forward_tiled_kernel<T, 8, true, FAR, CG>, map, args, smem, sms, stream)
+               : launch_persistent(dcn_forward_tiled_kernel<T, 8, false, FAR, CG>, map, args, smem, sms, stream);
+  return p->softmax
+             ? launch_persistent(dcn_forward_tiled_kernel<T, 9, true, FAR, CG>, map, args, smem, sms, stream)
+             : launch_persistent(dcn_forward_tiled_kernel<T, 9, false, FAR, CG>, map, args, smem, sms, stream);
+}
+
 template <typename T, bool FAR>
 dcn_status forward_tiled_dispatch_far(const dcn_problem* p, const CUtensorMap& map,
                                       const TiledArgs& args, size_t smem, int sms,
                                       cudaStream_t stream) {
-  if (p->remove_center)
-    return p->softmax
-               ? launch_persistent(dcn_forward_tiled_kernel<T, 8, true, FAR>, map, args, smem, sms, stream)
-               : launch_persistent(dcn_forward_tiled_kernel<T, 8, false, FAR>, map, args, smem, sms, stream);
-  return p->softmax
-             ? launch_persistent(dcn_forward_tiled_kernel<T, 9, true, FAR>, map, args, smem, sms, stream)
-             : launch_persistent(dcn_forward_tiled_kernel<T, 9, false, FAR>, map, args, smem, sms, stream);
+  if constexpr (sizeof(T) == 2)
+    if (p->Cg == 8) return forward_tiled_dispatch_cg<T, FAR, 8>(p, map, args, smem, sms, stream);
+  return forward_tiled_dispatch_cg<T, FAR, 16>(p, map, args, smem, sms, stream);
 }
 
 template <typename T>
@@ -631,11 +646,12 @@ dcn_status box_tiled_prepare(const dcn_problem* p, int64_t Ho, int64_t Wo, const
   if (st != DCN_OK) return st;
   const int cs = p->Cg * esize(p->dtype);
   // Default halo (pixels of box around the tile's sampling window): 4 for
-  // 64-byte groups, 5 for 32-byte ones.  A wider halo turns more far taps into
-  // box reads but shrinks the tile the shared memory allows; measured on the
-  // InternImage-L stage-1 shapes, 4 is the fastest for fp32 (forward 0.437 ms
-  // against 0.459 at 5) and 5 for bf16 and fp16.
-  const int halo = std::max(0, env_int("DCN_CORE_HALO", cs == 64 ? 4 : 5));
+  // 64-byte groups, 5 for 32-byte ones, 3 for 16-byte ones.  A wider halo
+  // turns more far taps into box reads but shrinks the tile the shared memory
+  // allows; measured on the InternImage-L stage-1 shapes, 4 is the fastest for
+  // fp32 (forward 0.437 ms against 0.459 at 5), 5 for bf16 and fp16, and 3 for
+  // 8 bf16 channels (1.039 ms against 1.092 at 4 and 1.208 at 5).
+  const int halo = std::max(0, env_int("DCN_CORE_HALO", cs == 64 ? 4 : (cs == 16 ? 3 : 5)));
   if (size_t(L->dev.smem_optin) <= reserve) return DCN_ERR_UNSUPPORTED;
   const size_t optin = size_t(L->dev.smem_optin) - reserve;
   FwdTile f;

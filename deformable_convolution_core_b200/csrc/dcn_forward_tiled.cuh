@@ -81,8 +81,10 @@ __host__ __device__ constexpr size_t fwd_tiled_smem(int nbuf, uint32_t box_strid
 }
 
 // KKS: 9 (the 3x3 window) or 8 (the window without its centre).  FAR: some
-// footprint can leave the box (the box does not cover the whole image).
-template <typename T, int KKS, bool SOFTMAX, bool FAR>
+// footprint can leave the box (the box does not cover the whole image).  CG:
+// channels per group, 16, or 8 with 2-byte storage (a 16-byte pixel: one
+// piece per corner lane, and the reduce-scatter ends with two channels a lane).
+template <typename T, int KKS, bool SOFTMAX, bool FAR, int CG = 16>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     dcn_forward_tiled_kernel(const __grid_constant__ CUtensorMap xmap, const TiledArgs a) {
   using IO = TiledIO<T>;
@@ -90,8 +92,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   using One = typename IO::One;
   constexpr int KK = KKS, K = tap_side(KKS);
   static_assert(K == 3 && KK <= kTiledMaxTaps, "the tiled kernel serves 3x3 tap sets");
-  constexpr int CS = 16 * int(sizeof(T));  // bytes of one pixel of the group
-  constexpr int NP = CS / 16;              // 16-byte pieces per corner: 2 (bf16) or 4 (fp32)
+  static_assert(CG == 16 || (CG == 8 && sizeof(T) == 2), "16 channels, or 8 of a 2-byte type");
+  constexpr int CS = CG * int(sizeof(T));  // bytes of one pixel of the group
+  constexpr int NP = CS / 16;              // 16-byte pieces per corner: 1, 2 (bf16) or 4 (fp32)
+  constexpr int PA = CG / 2 / NP;          // accumulator pairs per piece
 
   const TiledParams& t = a.t;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -158,8 +162,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   // phase-B roles: unit u8 of the step, corner r = (dy, dx), unit parity rho
   const int u8 = lane >> 2, r = lane & 3, dy = r >> 1, dx = r & 1, rho = u8 & 1;
   // piece rotation: bf16 lanes read pieces rho, 1 - rho; fp32 lanes read piece
-  // j ^ rot in their j-th read, rot = 2 dy + rho
-  const int rot = NP == 2 ? rho : 2 * dy + rho;
+  // j ^ rot in their j-th read, rot = 2 dy + rho; a one-piece pixel has none
+  const int rot = NP == 1 ? 0 : (NP == 2 ? rho : 2 * dy + rho);
   const uint32_t corner_b = uint32_t((dy * t.BW + dx) * CS + 16 * rot);
   const int npx = t.TH * t.TW;
   const int nb = t.batches;
@@ -347,9 +351,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll 1
       for (int s = 0; s < nsteps; ++s) {
         const int u = s * 8 + u8;
-        float2 acc[8];
+        float2 acc[CG / 2];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = make_float2(0.f, 0.f);
+        for (int i = 0; i < CG / 2; ++i) acc[i] = make_float2(0.f, 0.f);
         const uint32_t wa = reg_a + kFwdRegW + uint32_t(u) * 16u + uint32_t(r) * 4u;
         const uint32_t oa = reg_a + kFwdRegOff + uint32_t(u) * 4u;
 #pragma unroll
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           const uint32_t a0 = lane_base + off;
 #pragma unroll
           for (int j = 0; j < NP; ++j)
-            IO::fma16(acc + j * (8 / NP), w2, lds128_a(a0 ^ uint32_t(16 * j)));
+            IO::fma16(acc + j * PA, w2, lds128_a(a0 ^ uint32_t(16 * j)));
         }
         if (FAR) {
           // The unit's far taps, in a warp-uniform loop.  (Fetching the first
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
               far_fetch(u, __ffs(fm) - 1, fv, fw);
 #pragma unroll
               for (int j = 0; j < NP; ++j)
-                IO::fma16(acc + j * (8 / NP), make_float2(fw, fw), fv[j]);
+                IO::fma16(acc + j * PA, make_float2(fw, fw), fv[j]);
               fm &= fm - 1u;
             }
           }
@@ -385,7 +389,28 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         // Reduce-scatter over the unit's four corner lanes, then store.
         uint32_t ob;
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(ob) : "r"(reg_a + kFwdRegOut + 4u * u));
-        if constexpr (NP == 2) {
+        if constexpr (NP == 1) {
+          // acc[0..3]: the 8 channels.  dx partner: keep channels 4 dx ..
+          // 4 dx + 3, then dy partner: keep the pair 4 dx + 2 dy.
+          float2 k2[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float2 keep = dx ? acc[2 + i] : acc[i];
+            const float2 send = dx ? acc[i] : acc[2 + i];
+            k2[i].x = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, 1);
+            k2[i].y = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, 1);
+          }
+          const float2 keep = dy ? k2[1] : k2[0];
+          const float2 send = dy ? k2[0] : k2[1];
+          const float o0 = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, 2);
+          const float o1 = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, 2);
+          if (ob != ~0u) {
+            char* op = reinterpret_cast<char*>(a.out) +
+                       (size_t(ob) + size_t(4 * dx + 2 * dy)) * sizeof(T);
+            if (in_tensor(op, 4, a.out, out_bytes))
+              asm volatile("st.global.b32 [%0], %1;" ::"l"(op), "r"(pack2<T>(o0, o1)) : "memory");
+          }
+        } else if constexpr (NP == 2) {
           // acc[0..3]: piece rho (channels 8 rho ..), acc[4..7]: piece 1 - rho.
           // dx partner: keep piece rho ^ dx, then dy partner: keep half dy of it.
           float2 k4[4];

@@ -92,6 +92,11 @@ def main():
     case("separate axes K=5", mk(1, 12, 15, 2, 8, K=5, pad=2, stride_w=2, pad_w=1,
                                  offset_scale=2.0))
     case("Cg 32 raw mask", mk(1, 10, 9, 3, 32, softmax=0, offset_scale=2.0))
+    # the 3x3 tiled forward with 8 channels of a 2-byte type (16-byte groups)
+    case("Cg 8 bf16 offsets +-1e4", mk(2, 11, 13, 3, 8, offset_scale=2.0, dtype="bf16"), far,
+         dtype="bf16")
+    case("Cg 8 fp16 borders remove_center", mk(1, 9, 10, 2, 8, offset_scale=2.0, dtype="f16",
+                                               remove_center=1), borders(10), dtype="f16")
     # the wide-window tiled forward (5x5 and 7x7 windows, chunked taps)
     case("K=5 wide", mk(2, 13, 17, 3, 16, K=5, pad=2, offset_scale=2.0))
     case("K=7 bf16 dilation 2 remove_center raw mask",

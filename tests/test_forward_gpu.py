@@ -141,6 +141,12 @@ def test_tiled_kernel_tile_and_halo_settings(oracle_mod, halo, tile):
             p, x, off, mask = random_case(2, 29, 31, 3, 16, dtype=dtype, off_sd=3.0,
                                           remove_center=1)
             check_full(oracle_mod, p, x, off, mask, dtype)
+            if dtype != "f32":  # 8 channels of a 2-byte type: 16-byte groups
+                p, x, off, mask = random_case(2, 37, 41, 3, 8, dtype=dtype, off_sd=3.0)
+                check_full(oracle_mod, p, x, off, mask, dtype)
+                p, x, off, mask = random_case(1, 40, 36, 4, 8, dtype=dtype, stride=2, softmax=0,
+                                              remove_center=1)
+                check_full(oracle_mod, p, x, off, mask, dtype)
     finally:
         for k, v in old.items():
             if v is None:
@@ -353,16 +359,18 @@ def test_full_size_workload_sampled(gen_mod, oracle_mod, name, path):
     assert torch.isfinite(out).all()
 
 
-@pytest.mark.parametrize("K", [3, 5])
-def test_bounded_wait_expiry_is_reported_and_recoverable(K):
+@pytest.mark.parametrize("K,Cg,dtype", [(3, 16, "f32"), (5, 16, "f32"), (3, 8, "bf16")])
+def test_bounded_wait_expiry_is_reported_and_recoverable(K, Cg, dtype):
     """Failure detection without a GPU fault: with the test knob the first TMA
     box of every CTA never arrives, the bounded mbarrier waits give up (about a
     second), the kernel sets the device error word and returns;
     dcn_core_sync_status reports DCN_ERR_TIMEOUT and clears the word, and the
     next call works normally.  K = 5 runs the wide-window kernel, whose
-    consumers also have staging copies in flight when they give up."""
-    p, x, off, mask = random_case(2, 23, 29, 3, 16, K=K, dtype="f32")
-    xd, od, md = to_dev(x, "f32"), to_dev(off, "f32"), to_dev(mask, "f32")
+    consumers also have staging copies in flight when they give up; 8 bf16
+    channels run the 3x3 tiled kernel's 16-byte-group form (the timeout also
+    shows that such a problem takes the tiled path)."""
+    p, x, off, mask = random_case(2, 23, 29, 3, Cg, K=K, dtype=dtype)
+    xd, od, md = to_dev(x, dtype), to_dev(off, dtype), to_dev(mask, dtype)
     with forward_path("auto"):
         ref = gpu_forward(p, xd, od, md)
         dcn.dcn_core_sync_status()
