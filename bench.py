@@ -238,7 +238,10 @@ class Step:
             self.bwd()
 
     def launches_per_step(self):
-        return (0 if (self.wl.backward and self.backward) else 1) + (1 if self.backward else 0)
+        # the deterministic backward is three kernels (bound pre-pass, the
+        # backward, the rounding pass) after its zero-fill
+        bwd = (3 if self.deterministic else 1) if self.backward else 0
+        return (0 if (self.wl.backward and self.backward) else 1) + bwd
 
 
 def timed(step, steps, warmup, barrier=None, ev_kernels=True):
@@ -283,7 +286,8 @@ def run_ours(args, world, rank, local):
     wl = gen.WORKLOADS[args.workload]
     backward = wl.backward or wl.dtype == "f32"
     inputs = gen.make_inputs(wl, with_grad_out=backward)
-    step = Step(wl, inputs, backward)
+    det = bool(args.deterministic and backward)
+    step = Step(wl, inputs, backward, deterministic=det)
 
     barrier = None
     if world > 1:
@@ -309,10 +313,14 @@ def run_ours(args, world, rank, local):
     # dominant launch: the longer of forward and backward
     kernels = []
     if fwd_ms > 0:
-        tiled = (os.environ.get("DCN_CORE_FORWARD") != "direct" and wl.K == 3
-                 and wl.Cg == 16)
-        kernels.append(("dcn_forward_tiled_kernel" if tiled else "dcn_forward_kernel",
-                        fwd_bytes, fwd_ms))
+        tiled = os.environ.get("DCN_CORE_FORWARD") != "direct"
+        if tiled and wl.K == 3 and (wl.Cg == 16 or (wl.Cg == 8 and wl.esize == 2)):
+            fname = "dcn_forward_tiled_kernel"
+        elif tiled and wl.K in (5, 7) and wl.Cg == 16:
+            fname = "dcn_forward_tiled_wide_kernel"
+        else:
+            fname = "dcn_forward_kernel"
+        kernels.append((fname, fwd_bytes, fwd_ms))
     if bwd_ms > 0:
         tiled_bwd = (os.environ.get("DCN_CORE_BACKWARD") != "direct" and wl.K == 3
                      and wl.Cg == 16)
@@ -327,7 +335,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API: pinned host inputs -> device, step, results -> host
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not det:  # the host entry points run the atomic backward
         e2e = run_e2e(step, inputs, args, barrier, world)
 
     result = {
@@ -335,7 +343,7 @@ def run_ours(args, world, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": wl.dtype, "data": "synthetic (seeded counter-based generator)",
-        "config": workload_config(wl, backward, world),
+        "config": workload_config(wl, backward, world, det),
         "gsamples_per_s": round(world * samples / (ms_per_step * 1e-3) / 1e9, 3),
         "breakdown": {"forward": None if fwd_ms == 0 else {
                           "ms": round(fwd_ms, 4),
@@ -350,11 +358,17 @@ def run_ours(args, world, rank, local):
                           "GB/s": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
                           "Gsamples/s": round(wl.samples / (bwd_ms * 1e-3) / 1e9, 2),
                           "frac_of_hbm": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peak, 4),
-                          "red_v4_G_per_s": round(red_v4_per_launch(wl) / (bwd_ms * 1e-3) / 1e9, 1),
-                          "frac_of_l2_red_ceiling": round(
-                              red_v4_per_launch(wl) / (bwd_ms * 1e-3) / 1e9 / L2_RED_V4_G_PER_S, 4),
-                          "l2_red_ceiling": L2_RED_CEILING_NOTE,
-                          "note": "includes the zero-fill of grad_input"}},
+                          **({"u64_adds_G_per_s": round(red_u64_per_launch(wl) / (bwd_ms * 1e-3) / 1e9, 1),
+                              "frac_of_l2_red_ceiling": round(
+                                  red_u64_per_launch(wl) / (bwd_ms * 1e-3) / 1e9 / L2_RED_U64_G_PER_S, 4),
+                              "l2_red_ceiling": L2_RED_U64_CEILING_NOTE,
+                              "note": "deterministic: includes the zero-fill, the bound pre-pass "
+                                      "and the rounding pass"} if det else
+                           {"red_v4_G_per_s": round(red_v4_per_launch(wl) / (bwd_ms * 1e-3) / 1e9, 1),
+                            "frac_of_l2_red_ceiling": round(
+                                red_v4_per_launch(wl) / (bwd_ms * 1e-3) / 1e9 / L2_RED_V4_G_PER_S, 4),
+                            "l2_red_ceiling": L2_RED_CEILING_NOTE,
+                            "note": "includes the zero-fill of grad_input"})}},
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": step.launches_per_step() * args.steps,
@@ -527,6 +541,8 @@ L2_RED_CEILING_NOTE = ("331 G red.global.add.v4.f32/s: microbenchmark, random 64
 # per SM) sustains 798 G such adds per second.  Scalar red.global.add.u64
 # (the direct kernel's form) sustains 466 G/s.
 L2_RED_U64_G_PER_S = 798.0
+L2_RED_U64_CEILING_NOTE = ("798 G 64-bit adds/s: microbenchmark, random 128-byte bulk reductions "
+                           "(cp.reduce.async.bulk .add.u64) into an L2-resident buffer, 16 warps per SM")
 
 
 def red_u64_per_launch(wl):
@@ -809,10 +825,12 @@ def step_bytes_of(wl, backward):
     return (wl.forward_bytes() if not wl.backward else 0) + (wl.backward_bytes() if backward else 0)
 
 
-def workload_config(wl, backward, world):
+def workload_config(wl, backward, world, deterministic=False):
     """The `config` object of the JSON line, the same for both arms: the
-    workload, its shape and how the timed steps treat L2."""
-    return {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else ""),
+    workload, its shape, how grad_input is summed and how the timed steps
+    treat L2."""
+    return {"workload": wl.name + (" fwd+bwd" if backward and not wl.backward else "")
+                        + (" (deterministic grad_input)" if deterministic else ""),
             "N": wl.N, "H": wl.H, "W": wl.W, "G": wl.G, "Cg": wl.Cg, "K": wl.K,
             "stride": wl.stride, "offset_scale": wl.offset_scale, "softmax": wl.softmax,
             "remove_center": wl.remove_center, "per_gpu_batch": wl.N,
@@ -849,7 +867,7 @@ def run_reference(args, world, rank):
             "ms_per_step": round(1e3 * statistics.median(secs), 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded counter-based generator)",
-            "config": workload_config(wl, backward, world),
+            "config": workload_config(wl, backward, world, bool(args.deterministic and backward)),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"1 of {wl.N} images of {wl.name} per step"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -866,6 +884,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time dcn_core_backward_deterministic as the step's backward")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
