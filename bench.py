@@ -329,7 +329,10 @@ def run_ours(args, world, rank, local):
     kname, kbytes, kms = max(kernels, key=lambda k: k[2])
     achieved = kbytes / (kms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(kname),
+                "frac": round(achieved / peak, 4),
+                # the recorded DRAM bytes are the default step's (its workload, atomic backward)
+                "traffic": (recorded_traffic(kname)
+                            if args.workload == DEFAULT_WORKLOAD and not det else None),
                 "kernel": kname, "peak_source": peak_kind,
                 "algorithmic_bytes_per_launch": kbytes, "avg_launch_ms": round(kms, 4)}
 
