@@ -122,3 +122,20 @@ def test_bench_module_resolves_every_name():
                 missing.add((fn.name, n.id))
     assert not missing, sorted(missing)
 
+
+
+def test_bench_config_names_the_deterministic_backward():
+    """`--deterministic` changes what the step's backward is, so the config
+    object (the same for both arms) says so; without it the config is the
+    default one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import gen
+    wl = gen.WORKLOADS["internimage_l_stage2_bwd_bf16_n32_48x48_c320"]
+    plain = bench.workload_config(wl, True, 1)
+    det = bench.workload_config(wl, True, 1, True)
+    assert "deterministic" not in plain["workload"] and "deterministic" in det["workload"]
+    assert {k: v for k, v in det.items() if k != "workload"} == \
+        {k: v for k, v in plain.items() if k != "workload"}
+    ap_src = open(os.path.join(ROOT, "bench.py")).read()
+    assert '"--deterministic"' in ap_src
