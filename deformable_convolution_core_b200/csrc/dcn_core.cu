@@ -1415,8 +1415,9 @@ template <typename T, int LP, int NJS>
 dcn_status guide_launch_nj(const GuideArgs& a, cudaStream_t stream) {
   const unsigned grid = unsigned(int64_t(a.N) * a.tiles_y * a.tiles_x);
   const unsigned block = kGuideWarps * 32;
-  // parameters (12 quads per channel quad) and the conv results: at most 160 KB
-  const size_t smem = (size_t(12) * a.Q + size_t(a.NJ) * block) * sizeof(float4);
+  // parameters (12 quads per channel quad) and the conv results of R rows
+  constexpr int R = guide_rows_per_pass<T, LP, NJS>();  // output rows per pass
+  const size_t smem = (size_t(12) * a.Q + size_t(a.NJ) * block * R) * sizeof(float4);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(dcn_guide_kernel<T, LP, NJS>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)

@@ -89,14 +89,23 @@ __device__ __forceinline__ float gelu_erf(float z) {
   return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f));
 }
 
+// Output rows a CTA computes per pass (see the kernel).
+template <typename T, int LP, int NJS>
+__host__ __device__ constexpr int guide_rows_per_pass() {
+  return (NJS > 0 && LP <= 16 && sizeof(T) == 4) ? 2 : 1;
+}
+
 // Three CTAs per SM for groups of 8 or 16 lanes (more warps to cover the
-// load latency; measured 10% faster at C = 160); 32-lane groups are
-// left to the compiler (their spills at three cost more than the warps gain).
+// load latency; measured 10% faster at C = 160), two for the two-row fp32
+// passes (their second accumulator set would spill at three); 32-lane groups
+// are left to the compiler (their spills at three cost more than the warps
+// gain).
 // NJS > 0: the quads fill the lane groups exactly (Q = LP * NJS, the channel
 // widths of the InternImage stages), so the quad count is a compile-time
 // constant and no quad needs a bounds predicate; NJS = 0: any C.
 template <typename T, int LP, int NJS>
-__global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
+__global__ void __launch_bounds__(kGuideWarps * 32,
+                                  LP <= 16 ? (guide_rows_per_pass<T, LP, NJS>() == 2 ? 2 : 3) : 1)
     dcn_guide_kernel(const GuideArgs a) {
   constexpr int PPW = 32 / LP;  // pixels per warp
   constexpr int kThreads = kGuideWarps * 32;
@@ -153,83 +162,193 @@ __global__ void __launch_bounds__(kGuideWarps * 32, LP <= 16 ? 3 : 1)
 
   // (the narrow widths, under the 3-CTA register cap, keep the row count a
   // compile-time constant: one register less)
-  const int rows = LP == 32 ? a.rows : kGuideRows;
-  for (int i = 0; i < rows; ++i) {
-    const int y = ty * rows + i;
-    if (y >= a.H) break;  // the same for the whole CTA
-    // depthwise 3x3 convolution, CH quads of this lane at a time in registers
-    float s = 0.f;
+  // fp32 input at the stage widths: two output rows per pass, which share each
+  // weight read from shared memory (a 16-byte weight load serves 8 pixels
+  // instead of 4); measured 23% faster at stage 1 (two CTAs per SM), while the
+  // 2-byte types lose 5% and keep one row per pass
+  constexpr int R = guide_rows_per_pass<T, LP, NJS>();
+  if constexpr (R == 2) {
+    const int rows = LP == 32 ? a.rows : kGuideRows;
+    for (int i = 0; i < rows; i += R) {
+      const int y = ty * rows + i;
+      if (y >= a.H) break;  // the same for the whole CTA
+      float s[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) s[r] = 0.f;
 #pragma unroll(FULL ? 4 : 1)
-    for (int j0 = 0; j0 < NJ; j0 += CH) {
-      float2 acc[2 * CH];  // quad u: channels (x, y) in acc[2u], (z, w) in acc[2u + 1]
+      for (int j0 = 0; j0 < NJ; j0 += CH) {
+        float2 acc[R][2 * CH];
 #pragma unroll
-      for (int u = 0; u < CH; ++u) {
-        const int q = sub + LP * (j0 + u);
-        const float4 b = ((FULL || (j0 + u < NJ && q < a.Q)) && col_ok)
-                             ? bias_s[FULL && CH > NJS ? (u < NJS ? q : sub) : q]
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        acc[2 * u] = make_float2(b.x, b.y);
-        acc[2 * u + 1] = make_float2(b.z, b.w);
-      }
+        for (int u = 0; u < CH; ++u) {
+          const int q = sub + LP * (j0 + u);
+          const float4 b = ((FULL || (j0 + u < NJ && q < a.Q)) && col_ok)
+                               ? bias_s[FULL && CH > NJS ? (u < NJS ? q : sub) : q]
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int ta = 0; ta < 3; ++ta) {
-        const int yy = y + ta - 1;
-        if (yy < 0 || yy >= a.H) continue;  // the same for the whole CTA
-        const T* row = xs + size_t(n * a.H + yy) * rowE;
+          for (int r = 0; r < R; ++r) {
+            acc[r][2 * u] = make_float2(b.x, b.y);
+            acc[r][2 * u + 1] = make_float2(b.z, b.w);
+          }
+        }
 #pragma unroll
-        for (int tb = 0; tb < 3; ++tb) {
-          const int xx = col + tb - 1;
-          if (!(col_ok && xx >= 0 && xx < a.W)) continue;
-          const T* px = row + xx * a.C + 4 * sub;
-          const float4* wq = w_s + (ta * 3 + tb) * a.Q + sub;
+        for (int ta = 0; ta < 3; ++ta) {
+          bool ok[R];
+          const T* rowp[R];
 #pragma unroll
-          for (int u = 0; u < CH; ++u) {
-            const int j = j0 + u;
-            if ((FULL ? j < NJS : (j < NJ && sub + LP * j < a.Q)) &&
-                in_tensor(px + 4 * LP * j, 4 * sizeof(T), a.x, a.x_bytes)) {
-              const float4 v = guide_ld4<T>(px + 4 * LP * j);
+          for (int r = 0; r < R; ++r) {
+            const int yy = y + r + ta - 1;
+            ok[r] = y + r < a.H && yy >= 0 && yy < a.H;  // the same for the whole CTA
+            rowp[r] = xs + size_t(n * a.H + (ok[r] ? yy : 0)) * rowE;
+          }
+          bool any = false;
+#pragma unroll
+          for (int r = 0; r < R; ++r) any = any || ok[r];
+          if (!any) continue;
+#pragma unroll
+          for (int tb = 0; tb < 3; ++tb) {
+            const int xx = col + tb - 1;
+            if (!(col_ok && xx >= 0 && xx < a.W)) continue;
+            const float4* wq = w_s + (ta * 3 + tb) * a.Q + sub;
+#pragma unroll
+            for (int u = 0; u < CH; ++u) {
+              const int j = j0 + u;
+              if (!(FULL ? j < NJS : (j < NJ && sub + LP * j < a.Q))) continue;
               const float4 wv = wq[LP * j];
-              acc[2 * u] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(v.x, v.y), acc[2 * u]);
-              acc[2 * u + 1] =
-                  __ffma2_rn(make_float2(wv.z, wv.w), make_float2(v.z, v.w), acc[2 * u + 1]);
+#pragma unroll
+              for (int r = 0; r < R; ++r) {
+                const T* pq = rowp[r] + xx * a.C + 4 * sub + 4 * LP * j;
+                if (ok[r] && in_tensor(pq, 4 * sizeof(T), a.x, a.x_bytes)) {
+                  const float4 v = guide_ld4<T>(pq);
+                  acc[r][2 * u] =
+                      __ffma2_rn(make_float2(wv.x, wv.y), make_float2(v.x, v.y), acc[r][2 * u]);
+                  acc[r][2 * u + 1] =
+                      __ffma2_rn(make_float2(wv.z, wv.w), make_float2(v.z, v.w), acc[r][2 * u + 1]);
+                }
+              }
             }
           }
         }
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+          for (int u = 0; u < CH; ++u) {
+            if (j0 + u < NJ) {
+              const float2 lo = acc[r][2 * u], hi = acc[r][2 * u + 1];
+              s[r] += (lo.x + lo.y) + (hi.x + hi.y);  // quads outside C hold 0
+              conv_buf[(r * NJ + j0 + u) * kThreads + tid] = make_float4(lo.x, lo.y, hi.x, hi.y);
+            }
+          }
       }
 #pragma unroll
-      for (int u = 0; u < CH; ++u) {
-        if (j0 + u < NJ) {
-          const float2 lo = acc[2 * u], hi = acc[2 * u + 1];
-          s += (lo.x + lo.y) + (hi.x + hi.y);  // quads outside C hold 0
-          conv_buf[(j0 + u) * kThreads + tid] = make_float4(lo.x, lo.y, hi.x, hi.y);
+      for (int r = 0; r < R; ++r) {
+        if (y + r >= a.H) break;  // the same for the whole CTA
+        // LayerNorm over the pixel's channels: the mean, then the mean squared deviation
+        const float mean = group_sum<LP>(s[r]) * inv_c;
+        float ss = 0.f;
+#pragma unroll(FULL ? 16 : 1)
+        for (int j = 0; j < NJ; ++j) {
+          if (!FULL && sub + LP * j >= a.Q) break;
+          const float4 v = conv_buf[(r * NJ + j) * kThreads + tid];
+          const float d0 = v.x - mean, d1 = v.y - mean, d2 = v.z - mean, d3 = v.w - mean;
+          ss = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, ss))));
+        }
+        const float rstd = 1.0f / sqrtf(group_sum<LP>(ss) * inv_c + a.eps);
+        if (!col_ok) continue;
+        __nv_bfloat16* op = a.out + (size_t(n * a.H + y + r) * a.W + col) * a.C;
+#pragma unroll(FULL ? 16 : 1)
+        for (int j = 0; j < NJ; ++j) {
+          const int q = sub + LP * j;
+          if (!FULL && q >= a.Q) break;
+          const float4 v = conv_buf[(r * NJ + j) * kThreads + tid];
+          const float4 g = gamma_s[q], b = beta_s[q];
+          const float o0 = gelu_erf((v.x - mean) * rstd * g.x + b.x);
+          const float o1 = gelu_erf((v.y - mean) * rstd * g.y + b.y);
+          const float o2 = gelu_erf((v.z - mean) * rstd * g.z + b.z);
+          const float o3 = gelu_erf((v.w - mean) * rstd * g.w + b.w);
+          if (in_tensor(op + 4 * q, 8, a.out, a.out_bytes))
+            *reinterpret_cast<uint2*>(op + 4 * q) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
         }
       }
     }
-    // LayerNorm over the pixel's channels: the mean, then the mean squared deviation
-    const float mean = group_sum<LP>(s) * inv_c;
-    float ss = 0.f;
+  } else {
+    const int rows = LP == 32 ? a.rows : kGuideRows;
+    for (int i = 0; i < rows; ++i) {
+      const int y = ty * rows + i;
+      if (y >= a.H) break;  // the same for the whole CTA
+      // depthwise 3x3 convolution, CH quads of this lane at a time in registers
+      float s = 0.f;
+#pragma unroll(FULL ? 4 : 1)
+      for (int j0 = 0; j0 < NJ; j0 += CH) {
+        float2 acc[2 * CH];  // quad u: channels (x, y) in acc[2u], (z, w) in acc[2u + 1]
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          const int q = sub + LP * (j0 + u);
+          const float4 b = ((FULL || (j0 + u < NJ && q < a.Q)) && col_ok)
+                               ? bias_s[FULL && CH > NJS ? (u < NJS ? q : sub) : q]
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          acc[2 * u] = make_float2(b.x, b.y);
+          acc[2 * u + 1] = make_float2(b.z, b.w);
+        }
+#pragma unroll
+        for (int ta = 0; ta < 3; ++ta) {
+          const int yy = y + ta - 1;
+          if (yy < 0 || yy >= a.H) continue;  // the same for the whole CTA
+          const T* row = xs + size_t(n * a.H + yy) * rowE;
+#pragma unroll
+          for (int tb = 0; tb < 3; ++tb) {
+            const int xx = col + tb - 1;
+            if (!(col_ok && xx >= 0 && xx < a.W)) continue;
+            const T* px = row + xx * a.C + 4 * sub;
+            const float4* wq = w_s + (ta * 3 + tb) * a.Q + sub;
+#pragma unroll
+            for (int u = 0; u < CH; ++u) {
+              const int j = j0 + u;
+              if ((FULL ? j < NJS : (j < NJ && sub + LP * j < a.Q)) &&
+                  in_tensor(px + 4 * LP * j, 4 * sizeof(T), a.x, a.x_bytes)) {
+                const float4 v = guide_ld4<T>(px + 4 * LP * j);
+                const float4 wv = wq[LP * j];
+                acc[2 * u] = __ffma2_rn(make_float2(wv.x, wv.y), make_float2(v.x, v.y), acc[2 * u]);
+                acc[2 * u + 1] =
+                    __ffma2_rn(make_float2(wv.z, wv.w), make_float2(v.z, v.w), acc[2 * u + 1]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < CH; ++u) {
+          if (j0 + u < NJ) {
+            const float2 lo = acc[2 * u], hi = acc[2 * u + 1];
+            s += (lo.x + lo.y) + (hi.x + hi.y);  // quads outside C hold 0
+            conv_buf[(j0 + u) * kThreads + tid] = make_float4(lo.x, lo.y, hi.x, hi.y);
+          }
+        }
+      }
+      // LayerNorm over the pixel's channels: the mean, then the mean squared deviation
+      const float mean = group_sum<LP>(s) * inv_c;
+      float ss = 0.f;
 #pragma unroll(FULL ? 16 : 1)
-    for (int j = 0; j < NJ; ++j) {
-      if (!FULL && sub + LP * j >= a.Q) break;
-      const float4 v = conv_buf[j * kThreads + tid];
-      const float d0 = v.x - mean, d1 = v.y - mean, d2 = v.z - mean, d3 = v.w - mean;
-      ss = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, ss))));
-    }
-    const float rstd = 1.0f / sqrtf(group_sum<LP>(ss) * inv_c + a.eps);
-    if (!col_ok) continue;
-    __nv_bfloat16* op = a.out + (size_t(n * a.H + y) * a.W + col) * a.C;
+      for (int j = 0; j < NJ; ++j) {
+        if (!FULL && sub + LP * j >= a.Q) break;
+        const float4 v = conv_buf[j * kThreads + tid];
+        const float d0 = v.x - mean, d1 = v.y - mean, d2 = v.z - mean, d3 = v.w - mean;
+        ss = fmaf(d0, d0, fmaf(d1, d1, fmaf(d2, d2, fmaf(d3, d3, ss))));
+      }
+      const float rstd = 1.0f / sqrtf(group_sum<LP>(ss) * inv_c + a.eps);
+      if (!col_ok) continue;
+      __nv_bfloat16* op = a.out + (size_t(n * a.H + y) * a.W + col) * a.C;
 #pragma unroll(FULL ? 16 : 1)
-    for (int j = 0; j < NJ; ++j) {
-      const int q = sub + LP * j;
-      if (!FULL && q >= a.Q) break;
-      const float4 v = conv_buf[j * kThreads + tid];
-      const float4 g = gamma_s[q], b = beta_s[q];
-      const float o0 = gelu_erf((v.x - mean) * rstd * g.x + b.x);
-      const float o1 = gelu_erf((v.y - mean) * rstd * g.y + b.y);
-      const float o2 = gelu_erf((v.z - mean) * rstd * g.z + b.z);
-      const float o3 = gelu_erf((v.w - mean) * rstd * g.w + b.w);
-      if (in_tensor(op + 4 * q, 8, a.out, a.out_bytes))
-        *reinterpret_cast<uint2*>(op + 4 * q) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+      for (int j = 0; j < NJ; ++j) {
+        const int q = sub + LP * j;
+        if (!FULL && q >= a.Q) break;
+        const float4 v = conv_buf[j * kThreads + tid];
+        const float4 g = gamma_s[q], b = beta_s[q];
+        const float o0 = gelu_erf((v.x - mean) * rstd * g.x + b.x);
+        const float o1 = gelu_erf((v.y - mean) * rstd * g.y + b.y);
+        const float o2 = gelu_erf((v.z - mean) * rstd * g.z + b.z);
+        const float o3 = gelu_erf((v.w - mean) * rstd * g.w + b.w);
+        if (in_tensor(op + 4 * q, 8, a.out, a.out_bytes))
+          *reinterpret_cast<uint2*>(op + 4 * q) = make_uint2(pack_bf16x2(o0, o1), pack_bf16x2(o2, o3));
+      }
     }
   }
 }
