@@ -45,7 +45,8 @@ def run_guide(p, x_dev, w, b, g, be, eps, stream=None):
 # column and row tiles; a one-pixel image
 CASES = [(2, 13, 11, 10, 16, "f32"), (1, 9, 37, 4, 16, "bf16"), (2, 5, 70, 20, 16, "bf16"),
          (1, 3, 3, 80, 16, "f32"), (1, 1, 1, 2, 4, "f32"), (2, 17, 9, 3, 4, "f32"),
-         (1, 4, 5, 49, 4, "f32"), (1, 6, 7, 128, 16, "bf16"), (3, 10, 33, 12, 16, "bf16")]
+         (1, 4, 5, 49, 4, "f32"), (1, 6, 7, 128, 16, "bf16"), (3, 10, 33, 12, 16, "bf16"),
+         (2, 7, 19, 20, 16, "f32")]  # fp32 at C = 320: two rows per pass, an odd row count
 
 
 @pytest.mark.parametrize("case", CASES, ids=[f"N{c[0]}_{c[1]}x{c[2]}_C{c[3] * c[4]}_{c[5]}"
